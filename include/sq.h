@@ -1,0 +1,209 @@
+/*
+ * sq.h -- C ABI of libsq, the B200 (sm_100a) SmoothQuant W8A8 linear layer.
+ *
+ * The method ("SmoothQuant: Accurate and Efficient Post-Training Quantization
+ * for Large Language Models", Xiao et al., as explained on the abeam.tech
+ * page):
+ *   1. calibration   a_j = max_t |X[t,j]|, b_j = max_n |W[n,j]|
+ *                    (glossary "Calibration"; section "how is the smoothing
+ *                    factor chosen")
+ *   2. smoothing     s_j = a_j^alpha / b_j^(1-alpha), folded offline into the
+ *                    preceding LayerNorm (gamma/s, beta/s) and into diag(s) W
+ *                    (section "what it does mathematically")
+ *   3. runtime       per-token dynamic INT8 quantization of the activations
+ *                    (section "inference", level O1), INT8 x INT8 -> INT32
+ *                    GEMM (glossary "INT8 GEMM") against per-output-channel
+ *                    INT8 weights, dequantized to fp16 by multiplying the
+ *                    scales back (itmedia quantization tutorial, section 3).
+ *
+ * Conventions for every entry point:
+ *   - All pointers except the sizes are DEVICE pointers on the current CUDA
+ *     device, owned by the caller.  The library never allocates or frees.
+ *   - fp16 tensors are passed as `const void*` (IEEE binary16).
+ *   - Matrices are row-major.  Activations are [tokens, K]; the weight is the
+ *     nn.Linear layout [N, K]; the output is [M, N].  K is contiguous.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Arguments are checked on the host first: a bad
+ *     argument returns an error code and launches nothing.
+ *   - Requirements: 1 <= K <= SQ_MAX_K, K % 16 == 0; rows/M/N >= 1;
+ *     every pointer 16-byte aligned; leading dimensions (in elements) a
+ *     multiple of 8 and >= K.  The device must be compute capability 10.0
+ *     (B200); the library is built for sm_100a only and has no CPU path.
+ *   - Numerics: every fp32 operation is IEEE round-to-nearest-even in the
+ *     order written below, with no fused multiply-add; rint is ties-to-even.
+ *     INT8 codes and int32 accumulators are therefore bit-identical to any
+ *     implementation that follows the same order.
+ *   - Device-side waits are bounded (default 2 s, see sq_set_wait_budget_ns).
+ *     A wait that runs out records SQ_ERR_TIMEOUT in a per-device status word
+ *     and the kernel returns early (its outputs are then undefined); read it
+ *     with sq_poll_status.
+ */
+#ifndef SQ_H
+#define SQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Largest K for which a sum of K products of two int8 codes in [-127, 127]
+ * cannot leave the int32 range: 133144 * 127^2 = 2147479576 <= 2^31 - 1. */
+#define SQ_MAX_K 133144
+
+/* Largest token count served by the weight-streaming (swap-AB, stream-K)
+ * GEMM path; larger M uses the tiled path. */
+#define SQ_SPLITK_MAX_M 32
+
+typedef enum sq_status {
+  SQ_OK = 0,
+  SQ_ERR_INVALID_ARG = 1,       /* null pointer, size <= 0, ld < K, bad path */
+  SQ_ERR_MISALIGNED = 2,        /* pointer not 16-byte aligned or ld % 8 != 0 */
+  SQ_ERR_UNSUPPORTED_SHAPE = 3, /* K % 16 != 0, or M too large for a forced path */
+  SQ_ERR_K_OVERFLOW = 4,        /* K > SQ_MAX_K */
+  SQ_ERR_WORKSPACE = 5,         /* workspace NULL or smaller than required */
+  SQ_ERR_ARCH = 6,              /* current device is not compute capability 10.0 */
+  SQ_ERR_CUDA = 7,              /* a CUDA runtime call or launch failed */
+  SQ_ERR_TIMEOUT = 8            /* a device-side bounded wait ran out */
+} sq_status;
+
+/* A cudaStream_t, passed as an opaque pointer. */
+typedef void* sq_stream_t;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* sq_status_string(int status);
+
+/* ABI version of this header (major * 100 + minor). */
+int sq_abi_version(void);
+
+/*
+ * Calibration (step 1): per-input-channel running absmax.
+ *   amax_inout[j] = max(amax_inout[j], max_{r < rows} |x_hat[r, j]|)
+ * where x_hat = x (ln_gamma == NULL) or the LayerNorm of each row of x:
+ *   x_hat = ((x - mu) * rstd) * ln_gamma + ln_beta   (ln_beta may be NULL)
+ * with mu, var the exact mean and biased variance of the row (integer sums of
+ * the fp16 values scaled by 2^24, converted to fp64 by a fixed sequence of
+ * correctly rounded operations) and rstd = 1 / sqrt(var + ln_eps), both
+ * rounded to fp32.  Call it on the calibration activations to get a (the
+ * LayerNorm output is what feeds the linear), and on W [N, K] (ln_gamma NULL)
+ * to get b.
+ *   x           fp16 [rows, ld], first K columns used
+ *   amax_inout  fp32 [K]; the caller zero-fills it before the first batch;
+ *               max is exact, so the result does not depend on call order
+ */
+sq_status sq_calibrate_absmax(const void* x_f16, int64_t rows, int64_t K, int64_t ld,
+                              const float* ln_gamma, const float* ln_beta, float ln_eps,
+                              float* amax_inout, sq_stream_t stream);
+
+/*
+ * Smoothing factor and offline fold (step 2).
+ *   s_j     = fp32( pow(max(a_j, 1e-5f), alpha) / pow(max(b_j, 1e-5f), 1 - alpha) )
+ *             evaluated in fp64 (1e-5f floors dead channels)
+ *   inv_s_j = 1.0f / s_j
+ *   gamma_out_j = gamma_j * inv_s_j, beta_out_j = beta_j * inv_s_j      (fp32)
+ *   w_out[n, j] = fp16(fp32(w[n, j]) * s_j)                             (fp16)
+ * gamma/beta (and their outputs) may be NULL; gamma_out may alias gamma.
+ * w may be NULL (then w_out is ignored and N is unused); w_out may alias w.
+ *   amax_x, amax_w, s_out, inv_s_out, gamma*, beta*   fp32 [K]
+ *   w, w_out                                          fp16 [N, K]
+ */
+sq_status sq_smooth_fold(const float* amax_x, const float* amax_w, int64_t K, float alpha,
+                         float* s_out, float* inv_s_out, const float* gamma, const float* beta,
+                         float* gamma_out, float* beta_out, const void* w_f16, void* w_out_f16,
+                         int64_t N, sq_stream_t stream);
+
+/*
+ * Per-output-channel symmetric INT8 weight quantization (step 2, weight side).
+ * With s == NULL the row is w itself; with s given it is the folded weight
+ * fp16(fp32(w[n, k]) * s_k), computed on the fly (the fold and the
+ * quantization in one pass over w, without writing the folded fp16 weight).
+ *   w_scale[n] = max_k |w'[n, k]| / 127
+ *   wq[n, k]   = clamp(rint(fp32(w'[n, k]) * (1 / w_scale[n])), -127, 127)
+ * An all-zero row gets scale 0 and codes 0.
+ *   w   fp16 [N, K]; s fp32 [K] or NULL; wq int8 [N, K]; w_scale fp32 [N]
+ */
+sq_status sq_quantize_weight(const void* w_f16, int64_t N, int64_t K, const float* s,
+                             int8_t* wq, float* w_scale, sq_stream_t stream);
+
+/*
+ * Runtime activation path (step 3a): optional LayerNorm, optional smoothing,
+ * per-token dynamic INT8 quantization, one pass over h.
+ *   x_hat      = gamma ? ((h - mu) * rstd) * gamma + beta : h      (as in calibration)
+ *   x_hat      = inv_s ? x_hat * inv_s : x_hat
+ *   x_scale[t] = max_k |x_hat[t, k]| / 127
+ *   xq[t, k]   = clamp(rint(x_hat[t, k] * (1 / x_scale[t])), -127, 127)
+ * With the smoothing folded into the LayerNorm pass gamma' / beta' and
+ * inv_s = NULL; for an input with no preceding LayerNorm pass gamma = NULL
+ * and inv_s.  beta may be NULL.
+ *   h fp16 [M, ld]; gamma, beta, inv_s fp32 [K]; xq int8 [M, K]; x_scale fp32 [M]
+ */
+sq_status sq_ln_quant_act(const void* h_f16, int64_t M, int64_t K, int64_t ld,
+                          const float* gamma, const float* beta, const float* inv_s, float eps,
+                          int8_t* xq, float* x_scale, sq_stream_t stream);
+
+/* Bytes of workspace sq_w8a8_linear needs for this shape (0 if none).  The
+ * workspace holds int32 partial sums and per-tile arrival counters of the
+ * stream-K path.  The caller zero-fills it once before its first use; every
+ * call that completes leaves the counters at zero again.  After a call that
+ * reported SQ_ERR_TIMEOUT, zero-fill it again.  Calls that share a workspace
+ * must not overlap on the GPU. */
+size_t sq_w8a8_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * The W8A8 linear (step 3b): INT8 GEMM with the dequant epilogue fused.
+ *   acc[t, n] = sum_k xq[t, k] * wq[n, k]                       (exact int32)
+ *   y[t, n]   = fp16( (fp32(acc) * x_scale[t]) * w_scale[n] + fp32(bias[n]) )
+ * (no add when bias is NULL).  Per-tensor weight scaling (level O1 of the
+ * explainer) is the special case of a w_scale array filled with one value.
+ *   xq int8 [M, K]; x_scale fp32 [M]; wq int8 [N, K]; w_scale fp32 [N];
+ *   bias fp16 [N] or NULL; y fp16 [M, N]
+ * M <= SQ_SPLITK_MAX_M runs the weight-streaming stream-K kernel and needs
+ * sq_w8a8_workspace_bytes(M, N, K) bytes of workspace; larger M runs the
+ * tiled tensor-core kernel (workspace may be NULL).
+ */
+sq_status sq_w8a8_linear(const int8_t* xq, const float* x_scale, const int8_t* wq,
+                         const float* w_scale, const void* bias_f16, void* y_f16, int64_t M,
+                         int64_t N, int64_t K, void* workspace, size_t ws_bytes,
+                         sq_stream_t stream);
+
+/* Kernel choice for sq_w8a8_linear_path. */
+typedef enum sq_gemm_path {
+  SQ_PATH_AUTO = 0,   /* what sq_w8a8_linear does */
+  SQ_PATH_TILED = 1,  /* tiled tcgen05 kernel, any M */
+  SQ_PATH_SPLITK = 2  /* weight-streaming stream-K kernel, M <= SQ_SPLITK_MAX_M */
+} sq_gemm_path;
+
+/* sq_w8a8_linear with the kernel chosen by the caller (testing and
+ * benchmarking both kernels on one shape).  Same contract otherwise. */
+sq_status sq_w8a8_linear_path(const int8_t* xq, const float* x_scale, const int8_t* wq,
+                              const float* w_scale, const void* bias_f16, void* y_f16,
+                              int64_t M, int64_t N, int64_t K, void* workspace,
+                              size_t ws_bytes, int path, sq_stream_t stream);
+
+/* The INT8 GEMM alone: acc int32 [M, N] = xq @ wq^T, written without the
+ * epilogue, through the same kernels (for checking the accumulators). */
+sq_status sq_w8a8_gemm_s32(const int8_t* xq, const int8_t* wq, int32_t* acc, int64_t M,
+                           int64_t N, int64_t K, void* workspace, size_t ws_bytes, int path,
+                           sq_stream_t stream);
+
+/* Synchronizes `stream`, then reports and clears the current device's status
+ * word: SQ_ERR_TIMEOUT if a bounded device wait ran out since the last poll,
+ * SQ_ERR_CUDA if the stream reported an error, else SQ_OK. */
+sq_status sq_poll_status(sq_stream_t stream);
+
+/* Budget of every device-side bounded wait launched after this call, in
+ * nanoseconds (default 2e9; values below 1000 are raised to 1000).  Process
+ * wide. */
+void sq_set_wait_budget_ns(uint64_t ns);
+
+/* Self-test of the bounded-wait machinery: launches one kernel that waits on
+ * a barrier nothing completes, for `budget_ns`; the wait runs out, the kernel
+ * records SQ_ERR_TIMEOUT and returns.  Follow with sq_poll_status. */
+sq_status sq_selftest_wait_timeout(uint64_t budget_ns, sq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_H */

@@ -1,0 +1,105 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point the
+header declares, and rejects bad arguments on the host before touching a
+device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sq.h")
+
+
+def _lib():
+    import w8a8_int8_linear_channel_b200 as sq
+    return sq._L
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_five_stage_entry_points():
+    names = declared_functions()
+    for n in ["sq_calibrate_absmax", "sq_smooth_fold", "sq_quantize_weight", "sq_ln_quant_act",
+              "sq_w8a8_linear"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(os.path.join(ROOT, "w8a8_int8_linear_channel_b200", "libsq.so"))
+    missing = [n for n in declared_functions() if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_status_strings():
+    L = _lib()
+    assert L.sq_status_string(0) == b"SQ_OK"
+    assert L.sq_status_string(8) == b"SQ_ERR_TIMEOUT"
+    assert L.sq_status_string(99) == b"SQ_ERR_UNKNOWN"
+    assert L.sq_abi_version() == 100
+
+
+FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
+FAKE_ODD = ctypes.c_void_p(0x10004)  # misaligned
+
+
+def test_linear_rejects_bad_arguments_on_the_host():
+    L = _lib()
+    f = L.sq_w8a8_linear
+    ok = dict(M=64, N=64, K=64)
+    # null operand
+    assert f(None, FAKE, FAKE, FAKE, None, FAKE, 64, 64, 64, None, 0, None) == 1
+    # non-positive sizes
+    assert f(FAKE, FAKE, FAKE, FAKE, None, FAKE, 0, 64, 64, None, 0, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, None, FAKE, 64, -1, 64, None, 0, None) == 1
+    # K must be a multiple of 16 and at most 133144
+    assert f(FAKE, FAKE, FAKE, FAKE, None, FAKE, 64, 64, 40, None, 0, None) == 3
+    assert f(FAKE, FAKE, FAKE, FAKE, None, FAKE, 64, 64, 133152, None, 0, None) == 4
+    # misaligned pointer
+    assert f(FAKE_ODD, FAKE, FAKE, FAKE, None, FAKE, 64, 64, 64, None, 0, None) == 2
+    # forced stream-K path for too many tokens
+    assert L.sq_w8a8_linear_path(FAKE, FAKE, FAKE, FAKE, None, FAKE, 33, 64, 64, FAKE, 1 << 20, 2, None) == 3
+    # unknown path
+    assert L.sq_w8a8_linear_path(FAKE, FAKE, FAKE, FAKE, None, FAKE, 8, 64, 64, FAKE, 1 << 20, 7, None) == 1
+    del ok
+
+
+def test_other_entry_points_reject_bad_arguments():
+    L = _lib()
+    assert L.sq_calibrate_absmax(None, 4, 64, 64, None, None, 1e-5, FAKE, None) == 1
+    assert L.sq_calibrate_absmax(FAKE, 4, 64, 60, None, None, 1e-5, FAKE, None) == 1   # ld < K
+    assert L.sq_calibrate_absmax(FAKE, 4, 64, 68, None, None, 1e-5, FAKE, None) == 2   # ld % 8
+    assert L.sq_calibrate_absmax(FAKE, 4, 64, 64, None, FAKE, 1e-5, FAKE, None) == 1   # beta w/o gamma
+    assert L.sq_smooth_fold(FAKE, FAKE, 64, ctypes.c_float(1.5), FAKE, FAKE, None, None, None, None,
+                            None, None, 0, None) == 1  # alpha out of [0, 1]
+    assert L.sq_smooth_fold(FAKE, FAKE, 64, ctypes.c_float(0.5), FAKE, FAKE, FAKE, None, None, None,
+                            None, None, 0, None) == 1  # gamma without gamma_out
+    assert L.sq_quantize_weight(FAKE, 0, 64, None, FAKE, FAKE, None) == 1
+    assert L.sq_quantize_weight(FAKE, 8, 24, None, FAKE, FAKE, None) == 3
+    assert L.sq_ln_quant_act(FAKE, 8, 64, 64, None, None, FAKE_ODD, 1e-5, FAKE, FAKE, None) == 2
+    assert L.sq_w8a8_gemm_s32(FAKE, FAKE, None, 8, 8, 64, None, 0, 0, None) == 1
+
+
+def test_workspace_size_formula():
+    L = _lib()
+    assert L.sq_w8a8_workspace_bytes(64, 4096, 4096) == 0       # tiled path needs none
+    assert L.sq_w8a8_workspace_bytes(0, 4096, 4096) == 0
+    n = L.sq_w8a8_workspace_bytes(32, 49152, 12288)
+    # counters for 384 channel tiles (rounded to 256 B) + 2 int32 [128 x 32] slots per SM
+    assert n >= 1536 + 2 * 148 * 128 * 32 * 4
+
+
+def _has_gpu():
+    import torch
+    return torch.cuda.is_available()
+
+
+@pytest.mark.skipif(_has_gpu(), reason="a GPU is present")
+def test_valid_call_without_a_device_reports_cuda_error():
+    L = _lib()
+    r = L.sq_w8a8_linear(FAKE, FAKE, FAKE, FAKE, None, FAKE, 64, 64, 64, None, 0, None)
+    assert r == 7  # SQ_ERR_CUDA: no device; nothing was launched

@@ -1,0 +1,304 @@
+"""SmoothQuant W8A8 linear layer for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over ``libsq.so`` (C ABI in ``include/sq.h``).  The
+functions below carry the C names and only marshal arguments: every step of
+the method runs in the library's CUDA kernels; PyTorch provides device memory
+and the current stream.  There is no CPU path: importing this package fails
+if the library has not been built (``python -m
+w8a8_int8_linear_channel_b200.build``).
+
+The method ("SmoothQuant: Accurate and Efficient Post-Training Quantization
+for Large Language Models", abeam.tech explainer):
+  calibrate  a_j = max|X_j| over calibration tokens, b_j = max|W_j|
+  smooth     s_j = a_j^alpha / b_j^(1-alpha), folded into LayerNorm and W
+  run        per-token INT8 activations x per-channel INT8 weights -> int32
+             -> fp16 with the scales multiplied back.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "SQError", "sq_calibrate_absmax", "sq_smooth_fold", "sq_quantize_weight", "sq_ln_quant_act",
+    "sq_w8a8_workspace_bytes", "sq_w8a8_linear", "sq_w8a8_linear_path", "sq_w8a8_gemm_s32",
+    "sq_poll_status", "sq_set_wait_budget_ns", "sq_selftest_wait_timeout", "SmoothQuantLinear",
+    "PATH_AUTO", "PATH_TILED", "PATH_SPLITK", "SPLITK_MAX_M", "MAX_K", "library_path",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libsq.so")
+
+PATH_AUTO, PATH_TILED, PATH_SPLITK = 0, 1, 2
+SPLITK_MAX_M = 32
+MAX_K = 133144
+
+STATUS = {0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_MISALIGNED", 3: "SQ_ERR_UNSUPPORTED_SHAPE",
+          4: "SQ_ERR_K_OVERFLOW", 5: "SQ_ERR_WORKSPACE", 6: "SQ_ERR_ARCH", 7: "SQ_ERR_CUDA",
+          8: "SQ_ERR_TIMEOUT"}
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"{_LIB_PATH} is missing: build it with `python -m w8a8_int8_linear_channel_b200.build` "
+            "(nvcc, sm_100a).  There is no CPU fallback.")
+    L = ctypes.CDLL(_LIB_PATH)
+    P, I, F, Z, S = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t, ctypes.c_int
+    sigs = {
+        "sq_status_string": ([S], ctypes.c_char_p),
+        "sq_abi_version": ([], S),
+        "sq_calibrate_absmax": ([P, I, I, I, P, P, F, P, P], S),
+        "sq_smooth_fold": ([P, P, I, F, P, P, P, P, P, P, P, P, I, P], S),
+        "sq_quantize_weight": ([P, I, I, P, P, P, P], S),
+        "sq_ln_quant_act": ([P, I, I, I, P, P, P, F, P, P, P], S),
+        "sq_w8a8_workspace_bytes": ([I, I, I], Z),
+        "sq_w8a8_linear": ([P, P, P, P, P, P, I, I, I, P, Z, P], S),
+        "sq_w8a8_linear_path": ([P, P, P, P, P, P, I, I, I, P, Z, S, P], S),
+        "sq_w8a8_gemm_s32": ([P, P, P, I, I, I, P, Z, S, P], S),
+        "sq_poll_status": ([P], S),
+        "sq_set_wait_budget_ns": ([ctypes.c_uint64], None),
+        "sq_selftest_wait_timeout": ([ctypes.c_uint64, P], S),
+    }
+    for name, (args, res) in sigs.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    return L
+
+
+_L = _load()
+
+
+class SQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise SQError(status, where)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _rows(t: torch.Tensor, dtype, name: str):
+    if t.dtype != dtype or t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name}: need a 2-D {dtype} tensor with unit inner stride")
+    return t.shape[0], t.shape[1], t.stride(0)
+
+
+def _vec(t: Optional[torch.Tensor], n: int, dtype, name: str):
+    if t is None:
+        return
+    if t.dtype != dtype or t.numel() != n or not t.is_contiguous():
+        raise ValueError(f"{name}: need a contiguous {dtype} vector of {n} elements")
+
+
+# --------------------------------------------------------------- C names ----
+def sq_calibrate_absmax(x: torch.Tensor, amax: torch.Tensor, gamma=None, beta=None,
+                        eps: float = 1e-5, stream=None) -> torch.Tensor:
+    """Running per-column absmax of x (or of its LayerNorm with gamma/beta) into amax (fp32 [K])."""
+    rows, K, ld = _rows(x, torch.float16, "x")
+    _vec(amax, K, torch.float32, "amax")
+    _vec(gamma, K, torch.float32, "gamma")
+    _vec(beta, K, torch.float32, "beta")
+    _check(_L.sq_calibrate_absmax(_p(x), rows, K, ld, _p(gamma), _p(beta), eps, _p(amax),
+                                  _stream(stream)), "sq_calibrate_absmax")
+    return amax
+
+
+def sq_smooth_fold(amax_x, amax_w, alpha: float, s_out, inv_s_out, gamma=None, beta=None,
+                   gamma_out=None, beta_out=None, w=None, w_out=None, stream=None):
+    """s = a^alpha / b^(1-alpha), inv_s = 1/s; optional fold into gamma/beta and W."""
+    K = amax_x.numel()
+    for t, n in ((amax_x, "amax_x"), (amax_w, "amax_w"), (s_out, "s_out"), (inv_s_out, "inv_s_out"),
+                 (gamma, "gamma"), (beta, "beta"), (gamma_out, "gamma_out"), (beta_out, "beta_out")):
+        _vec(t, K, torch.float32, n)
+    N = 0
+    if w is not None:
+        N, Kw, ld = _rows(w, torch.float16, "w")
+        if Kw != K or ld != K or w_out is None or w_out.shape != w.shape or not w_out.is_contiguous():
+            raise ValueError("w / w_out: need contiguous fp16 [N, K] tensors")
+    _check(_L.sq_smooth_fold(_p(amax_x), _p(amax_w), K, alpha, _p(s_out), _p(inv_s_out), _p(gamma),
+                             _p(beta), _p(gamma_out), _p(beta_out), _p(w), _p(w_out), N,
+                             _stream(stream)), "sq_smooth_fold")
+
+
+def sq_quantize_weight(w: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor, s=None,
+                       stream=None):
+    """Per-output-channel INT8 of w (folded by s on the fly when given)."""
+    N, K, ld = _rows(w, torch.float16, "w")
+    if ld != K:
+        raise ValueError("w must be contiguous")
+    if wq.dtype != torch.int8 or wq.shape != w.shape or not wq.is_contiguous():
+        raise ValueError("wq: need a contiguous int8 [N, K] tensor")
+    _vec(w_scale, N, torch.float32, "w_scale")
+    _vec(s, K, torch.float32, "s")
+    _check(_L.sq_quantize_weight(_p(w), N, K, _p(s), _p(wq), _p(w_scale), _stream(stream)),
+           "sq_quantize_weight")
+
+
+def sq_ln_quant_act(h: torch.Tensor, xq: torch.Tensor, x_scale: torch.Tensor, gamma=None,
+                    beta=None, inv_s=None, eps: float = 1e-5, stream=None):
+    """Optional LayerNorm and smoothing, then per-token INT8 of h."""
+    M, K, ld = _rows(h, torch.float16, "h")
+    if xq.dtype != torch.int8 or tuple(xq.shape) != (M, K) or not xq.is_contiguous():
+        raise ValueError("xq: need a contiguous int8 [M, K] tensor")
+    _vec(x_scale, M, torch.float32, "x_scale")
+    for t, n in ((gamma, "gamma"), (beta, "beta"), (inv_s, "inv_s")):
+        _vec(t, K, torch.float32, n)
+    _check(_L.sq_ln_quant_act(_p(h), M, K, ld, _p(gamma), _p(beta), _p(inv_s), eps, _p(xq),
+                              _p(x_scale), _stream(stream)), "sq_ln_quant_act")
+
+
+def sq_w8a8_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_L.sq_w8a8_workspace_bytes(M, N, K))
+
+
+def _gemm_shapes(xq, wq):
+    M, K, ldx = _rows(xq, torch.int8, "xq")
+    N, Kw, ldw = _rows(wq, torch.int8, "wq")
+    if Kw != K or ldx != K or ldw != K:
+        raise ValueError("xq / wq: need contiguous int8 [M, K] and [N, K]")
+    return M, N, K
+
+
+def sq_w8a8_linear(xq, x_scale, wq, w_scale, y, bias=None, workspace=None, path: int = PATH_AUTO,
+                   stream=None):
+    """y fp16 [M, N] = fp16((xq @ wq^T) * x_scale[:, None] * w_scale[None, :] + bias)."""
+    M, N, K = _gemm_shapes(xq, wq)
+    _vec(x_scale, M, torch.float32, "x_scale")
+    _vec(w_scale, N, torch.float32, "w_scale")
+    _vec(bias, N, torch.float16, "bias")
+    if y.dtype != torch.float16 or tuple(y.shape) != (M, N) or not y.is_contiguous():
+        raise ValueError("y: need a contiguous fp16 [M, N] tensor")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_L.sq_w8a8_linear_path(_p(xq), _p(x_scale), _p(wq), _p(w_scale), _p(bias), _p(y), M, N, K,
+                                  _p(workspace), ws_bytes, path, _stream(stream)), "sq_w8a8_linear")
+    return y
+
+
+sq_w8a8_linear_path = sq_w8a8_linear
+
+
+def sq_w8a8_gemm_s32(xq, wq, acc, workspace=None, path: int = PATH_AUTO, stream=None):
+    """acc int32 [M, N] = xq @ wq^T (the accumulators, no epilogue)."""
+    M, N, K = _gemm_shapes(xq, wq)
+    if acc.dtype != torch.int32 or tuple(acc.shape) != (M, N) or not acc.is_contiguous():
+        raise ValueError("acc: need a contiguous int32 [M, N] tensor")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_L.sq_w8a8_gemm_s32(_p(xq), _p(wq), _p(acc), M, N, K, _p(workspace), ws_bytes, path,
+                               _stream(stream)), "sq_w8a8_gemm_s32")
+    return acc
+
+
+def sq_poll_status(stream=None) -> int:
+    """Synchronize the stream; return the status code of the device's bounded waits (and clear it)."""
+    return int(_L.sq_poll_status(_stream(stream)))
+
+
+def sq_set_wait_budget_ns(ns: int) -> None:
+    _L.sq_set_wait_budget_ns(int(ns))
+
+
+def sq_selftest_wait_timeout(budget_ns: int, stream=None) -> None:
+    _check(_L.sq_selftest_wait_timeout(int(budget_ns), _stream(stream)), "sq_selftest_wait_timeout")
+
+
+def new_workspace(M: int, N: int, K: int, device=None) -> Optional[torch.Tensor]:
+    """A zero-filled workspace tensor for sq_w8a8_linear (None if the shape needs none)."""
+    n = sq_w8a8_workspace_bytes(M, N, K)
+    if n == 0:
+        return None
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+# ------------------------------------------------------------- layer API ----
+class SmoothQuantLinear:
+    """A quantized nn.Linear with its smoothing folded in.
+
+    Built from an fp16 weight, its input's calibration tokens and (optionally)
+    the LayerNorm that precedes it; ``forward`` runs the per-token quantization
+    and the INT8 GEMM.  All work happens in libsq kernels on the current
+    stream."""
+
+    def __init__(self, wq, w_scale, bias, gamma_f, beta_f, inv_s, s, eps):
+        self.wq, self.w_scale, self.bias = wq, w_scale, bias
+        self.gamma_f, self.beta_f, self.inv_s, self.s = gamma_f, beta_f, inv_s, s
+        self.eps = eps
+        self._ws = {}
+
+    @classmethod
+    def from_float(cls, w: torch.Tensor, calib: torch.Tensor, alpha: float = 0.5, gamma=None,
+                   beta=None, bias=None, eps: float = 1e-5, amax_x: Optional[torch.Tensor] = None,
+                   process_group=None):
+        """Calibrate on ``calib`` (the LayerNorm input when gamma is given, else the
+        linear's input), smooth with ``alpha`` and quantize ``w`` [N, K].  With a
+        process group, the activation ranges are max-reduced over its ranks so
+        every rank derives the same smoothing (data-parallel calibration)."""
+        N, K = w.shape
+        dev = w.device
+        if amax_x is None:
+            amax_x = torch.zeros(K, dtype=torch.float32, device=dev)
+            sq_calibrate_absmax(calib, amax_x, gamma, beta, eps)
+        if process_group is not None:
+            import torch.distributed as dist
+            dist.all_reduce(amax_x, op=dist.ReduceOp.MAX, group=process_group)
+        amax_w = torch.zeros(K, dtype=torch.float32, device=dev)
+        sq_calibrate_absmax(w, amax_w)
+        s = torch.empty(K, dtype=torch.float32, device=dev)
+        inv_s = torch.empty_like(s)
+        gamma_f = torch.empty_like(s) if gamma is not None else None
+        beta_f = torch.empty_like(s) if beta is not None else None
+        sq_smooth_fold(amax_x, amax_w, alpha, s, inv_s, gamma, beta, gamma_f, beta_f)
+        wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+        w_scale = torch.empty(N, dtype=torch.float32, device=dev)
+        sq_quantize_weight(w, wq, w_scale, s=s)
+        runtime_inv_s = None if gamma is not None else inv_s
+        return cls(wq, w_scale, bias, gamma_f, beta_f, runtime_inv_s, s, eps)
+
+    def workspace(self, M: int) -> Optional[torch.Tensor]:
+        N, K = self.wq.shape
+        need = sq_w8a8_workspace_bytes(M, N, K)
+        if need == 0:
+            return None
+        ws = self._ws.get(self.wq.device)
+        if ws is None or ws.numel() < need:
+            ws = torch.zeros(need, dtype=torch.uint8, device=self.wq.device)
+            self._ws[self.wq.device] = ws
+        return ws
+
+    def quantize_input(self, h: torch.Tensor, xq=None, x_scale=None):
+        M, K = h.shape
+        xq = torch.empty((M, K), dtype=torch.int8, device=h.device) if xq is None else xq
+        x_scale = torch.empty(M, dtype=torch.float32, device=h.device) if x_scale is None else x_scale
+        sq_ln_quant_act(h, xq, x_scale, self.gamma_f, self.beta_f, self.inv_s, self.eps)
+        return xq, x_scale
+
+    def forward(self, h: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """h fp16 [M, K] (the LayerNorm input if a LayerNorm was folded) -> y fp16 [M, N]."""
+        M = h.shape[0]
+        N = self.wq.shape[0]
+        xq, x_scale = self.quantize_input(h)
+        y = torch.empty((M, N), dtype=torch.float16, device=h.device) if y is None else y
+        sq_w8a8_linear(xq, x_scale, self.wq, self.w_scale, y, self.bias, self.workspace(M))
+        return y
+
+    __call__ = forward

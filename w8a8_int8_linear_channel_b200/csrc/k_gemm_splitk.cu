@@ -1,0 +1,323 @@
+// k_gemm_splitk.cu -- the W8A8 linear for decode-sized token counts
+// (M <= 32), where the layer is bound by streaming the INT8 weight from HBM
+// (the explainer's "decoding stage").
+//
+// Swap-AB: the MMA's 128-row M slot takes 128 weight rows (output channels)
+// and its N slot takes the BT (16 or 32) zero-padded tokens, so
+//   TMEM lane = output channel n,  TMEM column = token t.
+// Stream-K: the (channel tile, 128-byte K block) units of the whole problem
+// are cut into one contiguous range per SM (a persistent grid of num_SMs
+// CTAs), so the TMA stream of every CTA never drains at tile boundaries and
+// no wave is left partly empty.  A tile split between CTAs is summed exactly:
+// each contributor writes its int32 partial accumulator to the workspace and
+// the last to arrive (per-tile counter, no waiting) adds the others and runs
+// the epilogue y = fp16((acc * sx[t]) * sw[n] + bias[n]).  int32 addition is
+// associative, so the result is bit-identical to a single-CTA sum.
+//
+// Roles: warp 0 TMA producer (a STAGES-deep ring of 16 KB weight tiles +
+// BT x 128 B token tiles), warp 1 TMEM owner + MMA issuer (double-buffered
+// accumulators), warps 2-5 epilogue.  All waits are bounded.
+#include "sq_internal.h"
+#include "sq_ptx.cuh"
+#include "sq_tmap.h"
+
+namespace sq {
+namespace {
+
+constexpr int BW = 128;  // weight rows (output channels) per tile
+constexpr int BK = 128;  // K bytes per unit
+constexpr int kThreads = 192;
+constexpr int kStages = 10;
+
+template <int BT>
+struct SkLayout {
+  static constexpr int A_BYTES = BW * BK;  // 16 KB weight tile
+  static constexpr int B_BYTES = BT * BK;  // token tile
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int CTRL = kStages * STAGE_BYTES;
+  static constexpr int NBARS = 2 * kStages + 5;  // full, empty, acc_full[2], acc_empty[2], drain
+  static constexpr int SLOT = CTRL + NBARS * 8;  // TMEM address, abort flag, last flag
+  static constexpr int SX = SLOT + 16;           // sx[BT]
+  static constexpr int BYTES = SX + BT * 4;
+  static constexpr size_t SMEM = BYTES + 1024;
+  static constexpr int TMEM_COLS = 2 * BT < 32 ? 32 : 2 * BT;
+};
+
+struct SkGeom {
+  int64_t U;   // total units = tiles * KB
+  int KB;      // K blocks per tile
+  int G;       // CTAs
+  __device__ __forceinline__ int64_t u0(int c) const { return (static_cast<int64_t>(c) * U) / G; }
+  __device__ __forceinline__ int cta_of(int64_t u) const {
+    return static_cast<int>(((u + 1) * G - 1) / U);
+  }
+};
+
+template <int BT>
+__device__ __forceinline__ void tmem_ld_tokens(uint32_t taddr, uint32_t (&v)[BT]);
+
+template <>
+__device__ __forceinline__ void tmem_ld_tokens<32>(uint32_t taddr, uint32_t (&v)[32]) {
+  tmem_ld_32x32b_x32(taddr, v);
+}
+
+template <>
+__device__ __forceinline__ void tmem_ld_tokens<16>(uint32_t taddr, uint32_t (&v)[16]) {
+  tmem_ld_32x32b_x16(taddr, v);
+}
+
+template <int BT, bool OUT_I32>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_splitk(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                  const GemmArgs g, const SkGeom geo, uint32_t* counters, int32_t* partials,
+                  uint32_t* status, uint64_t budget) {
+  using L = SkLayout<BT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sA = sbase;
+  const uint32_t sB = sbase + kStages * L::A_BYTES;
+  const uint32_t bar0 = sbase + L::CTRL;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+  auto accf_bar = [&](int b) { return bar0 + 8u * (2 * kStages + b); };
+  auto acce_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::SLOT);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile uint32_t* last_flag = tmem_slot + 2;
+  float* sx_s = reinterpret_cast<float*>(smem + L::SX);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cta = blockIdx.x;
+  const int64_t ubeg = geo.u0(cta), uend = geo.u0(cta + 1);
+  const int KB = geo.KB;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf_bar(b), 1);
+      mbar_init(acce_bar(b), 4);  // one arrive per epilogue warp
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  int64_t issued = 0;
+  bool mma_any = false;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int64_t u = ubeg; u < uend; ++u) {
+        const int64_t i = u - ubeg;
+        const int s = static_cast<int>(i % kStages);
+        const int64_t r = i / kStages;
+        if (i >= kStages && !mbar_wait(empty_bar(s), static_cast<uint32_t>((r - 1) & 1), budget, status, abort_flag))
+          break;
+        const int64_t t = u / KB;
+        const int kb = static_cast<int>(u % KB);
+        mbar_arrive_expect_tx(full_bar(s), L::STAGE_BYTES);
+        tma_load_2d(sA + s * L::A_BYTES, &tmW, full_bar(s), kb * BK, static_cast<int32_t>(t * BW));
+        tma_load_2d(sB + s * L::B_BYTES, &tmX, full_bar(s), kb * BK, 0);
+        ++issued;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(BW, BT);
+      int seg = 0;
+      int b = 0;
+      for (int64_t u = ubeg; u < uend; ++u) {
+        const int64_t i = u - ubeg;
+        const int s = static_cast<int>(i % kStages);
+        const int64_t r = i / kStages;
+        const int kb = static_cast<int>(u % KB);
+        const bool first = (u == ubeg) || kb == 0;
+        const bool last = (u == uend - 1) || kb == KB - 1;
+        if (first) {
+          b = seg & 1;
+          if (seg >= 2 && !mbar_wait(acce_bar(b), static_cast<uint32_t>(((seg >> 1) - 1) & 1), budget, status, abort_flag))
+            break;
+        }
+        if (!mbar_wait(full_bar(s), static_cast<uint32_t>(r & 1), budget, status, abort_flag)) break;
+        tc_fence_after();
+        const uint64_t ad = sdesc_k_sw128(sA + s * L::A_BYTES);
+        const uint64_t bd = sdesc_k_sw128(sB + s * L::B_BYTES);
+        const uint32_t d = tmem + static_cast<uint32_t>(b * BT);
+#pragma unroll
+        for (int k = 0; k < BK / 32; ++k)
+          mma_i8(d, ad + 2u * k, bd + 2u * k, idesc, (first && k == 0) ? 0u : 1u);
+        mma_any = true;
+        mma_commit(empty_bar(s));
+        if (last) {
+          mma_commit(accf_bar(b));
+          ++seg;
+        }
+      }
+    }
+  } else {
+    const int et = threadIdx.x - 64;
+    const int q = warp & 3;
+    if (!OUT_I32 && et < BT) sx_s[et] = et < g.M ? g.sx[et] : 0.0f;
+    named_bar_sync(1, 128);
+    int seg = 0;
+    for (int64_t u = ubeg; u < uend;) {
+      const int64_t t = u / KB;
+      const int64_t tile_end = (t + 1) * KB;
+      const int64_t seg_end = uend < tile_end ? uend : tile_end;
+      const bool whole = (u == t * KB) && (seg_end == tile_end);
+      const int slot = (u == ubeg) ? 0 : 1;
+      const int b = seg & 1;
+      if (!mbar_wait(accf_bar(b), static_cast<uint32_t>((seg >> 1) & 1), budget, status, abort_flag)) break;
+      tc_fence_after();
+      uint32_t v[BT];
+      tmem_ld_tokens<BT>(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(b * BT), v);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce_bar(b));
+
+      const int64_t nl = 32 * q + lane;  // channel within the tile
+      const int64_t n = t * BW + nl;
+      bool emit = whole;
+      if (!whole) {
+        int32_t* mine = partials + (static_cast<int64_t>(2 * cta + slot) * BW + nl) * BT;
+#pragma unroll
+        for (int j = 0; j < BT; j += 4)
+          *reinterpret_cast<int4*>(mine + j) = make_int4(static_cast<int>(v[j]), static_cast<int>(v[j + 1]),
+                                                         static_cast<int>(v[j + 2]), static_cast<int>(v[j + 3]));
+        __threadfence();
+        named_bar_sync(1, 128);
+        const int c_lo = geo.cta_of(t * KB);
+        const int c_hi = geo.cta_of(tile_end - 1);
+        if (et == 0) {
+          const uint32_t prev = atomicAdd(counters + t, 1u);
+          const bool is_last = prev == static_cast<uint32_t>(c_hi - c_lo);
+          if (is_last) counters[t] = 0;  // every contributor has arrived: reset for the next call
+          *last_flag = is_last ? 1u : 0u;
+        }
+        named_bar_sync(1, 128);
+        emit = *last_flag != 0;
+        if (emit) {
+          __threadfence();
+          for (int cc = c_lo; cc <= c_hi; ++cc) {
+            if (cc == cta) continue;
+            const int first_tile = static_cast<int>(geo.u0(cc) / KB);
+            const int sl = (t == first_tile) ? 0 : 1;
+            const int32_t* other = partials + (static_cast<int64_t>(2 * cc + sl) * BW + nl) * BT;
+#pragma unroll
+            for (int j = 0; j < BT; j += 4) {
+              const int4 p = __ldcg(reinterpret_cast<const int4*>(other + j));
+              v[j] += p.x;
+              v[j + 1] += p.y;
+              v[j + 2] += p.z;
+              v[j + 3] += p.w;
+            }
+          }
+        }
+      }
+      if (emit && n < g.N) {
+        if (OUT_I32) {
+          for (int m = 0; m < BT; ++m)
+            if (m < g.M) g.acc[m * g.N + n] = static_cast<int32_t>(v[m]);
+        } else {
+          const float swn = g.sw[n];
+          const bool has_bias = g.bias != nullptr;
+          const float bn = has_bias ? __half2float(g.bias[n]) : 0.0f;
+#pragma unroll
+          for (int m = 0; m < BT; ++m) {
+            if (m < g.M) {
+              float f = dequant_f32(static_cast<int32_t>(v[m]), sx_s[m], swn);
+              if (has_bias) f = __fadd_rn(f, bn);
+              g.y[m * g.N + n] = __float2half_rn(f);
+            }
+          }
+        }
+      }
+      u = seg_end;
+      ++seg;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    if (warp == 1 && lane == 0 && mma_any) {
+      mma_commit(drain_bar);
+      mbar_drain(drain_bar, 0, budget);
+    }
+    if (warp == 0 && lane == 0) {
+      for (int s = 0; s < kStages && s < issued; ++s) {
+        const int64_t last = ((issued - 1 - s) / kStages) * kStages + s;
+        mbar_drain(full_bar(s), static_cast<uint32_t>((last / kStages) & 1), budget);
+      }
+    }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+int64_t tiles_of(int64_t N) { return (N + BW - 1) / BW; }
+
+template <int BT, bool OUT_I32>
+cudaError_t launch_bt(const GemmArgs& g, const Ctx& c) {
+  using L = SkLayout<BT>;
+  static bool attr_set[64] = {false};
+  const int dev = c.device < 64 ? c.device : 63;
+  if (!attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_splitk<BT, OUT_I32>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(L::SMEM));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  CUtensorMap tmW, tmX;
+  if (!make_tmap_i8(&tmW, g.wq, g.K, g.N, BK, BW)) return cudaErrorInvalidValue;
+  if (!make_tmap_i8(&tmX, g.xq, g.K, g.M, BK, BT)) return cudaErrorInvalidValue;
+  SkGeom geo;
+  geo.KB = static_cast<int>((g.K + BK - 1) / BK);
+  geo.U = tiles_of(g.N) * geo.KB;
+  geo.G = static_cast<int>(geo.U < c.num_sms ? geo.U : c.num_sms);
+  uint8_t* ws = static_cast<uint8_t*>(g.ws);
+  const size_t counter_bytes = ((tiles_of(g.N) * 4 + 255) / 256) * 256;
+  uint32_t* counters = reinterpret_cast<uint32_t*>(ws);
+  int32_t* partials = reinterpret_cast<int32_t*>(ws + counter_bytes);
+  k_gemm_splitk<BT, OUT_I32><<<geo.G, kThreads, L::SMEM, c.stream>>>(
+      tmW, tmX, g, geo, counters, partials, c.status, c.budget_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
+  (void)K;
+  const int64_t bt = M <= 16 ? 16 : 32;
+  const size_t counter_bytes = ((tiles_of(N) * 4 + 255) / 256) * 256;
+  return counter_bytes + static_cast<size_t>(2) * num_sms * BW * bt * 4;
+}
+
+cudaError_t launch_gemm_splitk(const GemmArgs& g, const Ctx& c) {
+  const bool i32 = g.acc != nullptr;
+  if (g.M <= 16) return i32 ? launch_bt<16, true>(g, c) : launch_bt<16, false>(g, c);
+  return i32 ? launch_bt<32, true>(g, c) : launch_bt<32, false>(g, c);
+}
+
+}  // namespace sq

@@ -1,0 +1,71 @@
+// sq_internal.h -- launchers shared between the C-ABI layer (sq_api.cu) and
+// the kernel files.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sq {
+
+// Per-call launch context filled in by the ABI layer.
+struct Ctx {
+  int device;
+  int num_sms;
+  uint32_t* status;    // device address of this device's status word
+  uint64_t budget_ns;  // bound of every device-side wait
+  cudaStream_t stream;
+};
+
+// Row-wise kernels (k_rows.cu).
+struct RowArgs {
+  const __half* x;  // [rows, ld]
+  int64_t rows, K, ld;
+  const float* gamma;  // LayerNorm scale or NULL
+  const float* beta;   // LayerNorm shift or NULL
+  const float* vec;    // inv_s (activation path) or s (weight path) or NULL
+  float eps;
+  int8_t* q;       // codes [rows, K]
+  float* scale;    // per-row scale [rows]
+  float* amax;     // calibration running max [K]
+};
+
+cudaError_t launch_ln_quant_act(const RowArgs& a, const Ctx& c);
+cudaError_t launch_quantize_weight(const RowArgs& a, const Ctx& c);
+cudaError_t launch_calibrate_ln(const RowArgs& a, const Ctx& c);
+
+// Column-wise / elementwise kernels (k_cols.cu).
+cudaError_t launch_absmax_cols(const __half* x, int64_t rows, int64_t K, int64_t ld, float* amax,
+                               const Ctx& c);
+cudaError_t launch_smooth(const float* amax_x, const float* amax_w, int64_t K, float alpha,
+                          float* s, float* inv_s, const float* gamma, const float* beta,
+                          float* gamma_out, float* beta_out, const Ctx& c);
+cudaError_t launch_fold_weight(const __half* w, __half* w_out, int64_t N, int64_t K,
+                               const float* s, const Ctx& c);
+
+// GEMM kernels (k_gemm_tiled.cu, k_gemm_splitk.cu).
+struct GemmArgs {
+  const int8_t* xq;  // [M, K]
+  const float* sx;   // [M]
+  const int8_t* wq;  // [N, K]
+  const float* sw;   // [N]
+  const __half* bias;  // [N] or NULL
+  __half* y;           // [M, N]   (fp16 output) or NULL
+  int32_t* acc;        // [M, N]   (int32 output, no epilogue) or NULL
+  int64_t M, N, K;
+  void* ws;
+  size_t ws_bytes;
+};
+
+cudaError_t launch_gemm_tiled(const GemmArgs& g, const Ctx& c);
+cudaError_t launch_gemm_splitk(const GemmArgs& g, const Ctx& c);
+size_t splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
+
+cudaError_t launch_wait_selftest(uint64_t budget_ns, const Ctx& c);
+
+// Driver entry point for tensor-map encoding (resolved once through the
+// runtime, so the library does not link libcuda directly).
+void* tensor_map_encoder();
+
+}  // namespace sq
