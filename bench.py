@@ -1,0 +1,530 @@
+#!/usr/bin/env python3
+"""Benchmark of the SmoothQuant W8A8 linear hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic inputs:
+  a1 calibrate the activation ranges (LayerNorm output absmax over the
+     calibration tokens)          sq_calibrate_absmax(calib, gamma, beta)
+  a2 weight ranges                sq_calibrate_absmax(W)
+  a3/a4 smoothing factor + fold   sq_smooth_fold(..., gamma, beta -> gamma', beta')
+  a4/a5 fold + quantize W         sq_quantize_weight(W, s)
+  a6 LayerNorm + per-token quant  sq_ln_quant_act(h, gamma', beta')
+  a7/a8 INT8 GEMM + dequant       sq_w8a8_linear(xq, sx, wq, sw, bias)
+With N > 1 GPUs every rank runs its own batch (data parallel, weak scaling);
+the activation ranges are max-all-reduced over the ranks (NCCL) between a1
+and a3 so every rank derives the same smoothing.
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import sq_inputs  # noqa: E402
+
+METRIC = "W8A8 linear TOPS and % of INT8 peak (large M); GB/s % HBM (decode M≤32)"
+DESCR = {
+    "tiny": "tiny: K=N=256, M=16, calib 128, outliers x60 on channels 3/77",
+    "attn": "OPT-6.7B attention projection: K=N=4096, M=2048 tokens, calib 512, 6 outlier channels x40-100, LN folded, alpha 0.5",
+    "ffn_up": "OPT-6.7B FFN up: K=4096, N=16384, M=4096 tokens, calib 512, 4 outlier channels x50, bias, LN folded, alpha 0.5",
+    "decode": "OPT-175B FFN up decode: K=12288, N=49152, M tokens, calib 512, 12 outlier channels x80, LN folded, alpha 0.5",
+    "ffn_down": "OPT-175B FFN down: K=49152, N=12288, M=8192 tokens, calib 1024, 25 outlier channels x100 on X, alpha 0.5",
+}
+STEP = ("calibrate(LN absmax) + weight absmax + smoothing/fold + fold-and-quantize weight + "
+        "LN/per-token quantize + INT8 GEMM with dequant epilogue")
+I8_PER_BF16 = 2.0  # nominal dense INT8 : BF16 tensor throughput on B200 (4.5 : 2.25 POPS)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers --
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def stage_bytes_ops(wl, M):
+    K, N, C = wl.K, wl.N, wl.calib
+    b = {
+        "calibrate_x": 2 * C * K + 4 * K,
+        "calibrate_w": 2 * N * K + 4 * K,
+        "smooth_fold": 4 * K * 6,
+        "quantize_weight": 2 * N * K + N * K + 4 * N + 4 * K,
+        "ln_quant_act": 2 * M * K + M * K + 4 * M + 8 * K,
+        "w8a8_linear": M * K + N * K + 4 * M + 4 * N + 2 * M * N + (2 * N if wl.bias else 0),
+    }
+    return b, 2 * M * N * K
+
+
+def traffic_from_profile(kernel_src: str, profile_md: str):
+    """DRAM bytes per launch from a committed ncu summary, or None if the kernel
+    source changed since the counters were taken."""
+    if not os.path.exists(profile_md):
+        return None
+    sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    got = {}
+    for line in open(profile_md):
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            got[k.strip()] = v.strip().strip("`")
+    if got.get("source_sha256_16") != sha:
+        return None
+    try:
+        return int(float(got["dram_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons of one GPU, sampled every 100 ms."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, uuid: str):
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+        self.uuid = uuid
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(  # noqa: S603
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, TypeError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        rows = [[c.strip() for c in r.split(",")] for r in self.out.read().strip().splitlines() if r.strip()]
+        os.unlink(self.out.name)
+        mine = [r for r in rows if self.uuid and r[0].lower().endswith(self.uuid.lower())]
+        if not mine:  # uuid unknown: keep the first GPU's rows
+            first = rows[0][0] if rows else None
+            mine = [r for r in rows if r[0] == first]
+        sm, mx, reasons = [], [], set()
+        for r in mine:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(self.REASONS, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        load = [x for x in sm if x > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ GPU arm -------
+class Plan:
+    """Device buffers and prepared C-ABI calls of one step (argument
+    marshalling done once, so the per-step host cost is a few C calls)."""
+
+    def __init__(self, wl, M, rank, device, sq, torch):
+        self.torch, self.sq, self.wl, self.M = torch, sq, wl, M
+        dev = device
+        data_wl = sq_inputs.with_(wl, seed=wl.seed + 1000 * rank)  # this rank's tokens
+        w = sq_inputs.weight(wl)
+        calib = sq_inputs.calib_rows(data_wl)
+        h = sq_inputs.run_rows(data_wl, 0, M)
+        g, b, bias = sq_inputs.gamma(wl), sq_inputs.beta(wl), sq_inputs.bias(wl)
+        self.host = {"w": w, "calib": calib, "h": h, "gamma": g, "beta": b, "bias": bias}
+        T = lambda a, dt=None: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+        self.w, self.calib, self.h = T(w), T(calib), T(h)
+        self.gamma, self.beta, self.bias = T(g), T(b), T(bias)
+        K, N = wl.K, wl.N
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.amax = torch.zeros(2 * K, **f32)
+        self.amax_x, self.amax_w = self.amax[:K], self.amax[K:]
+        self.s, self.inv_s = torch.empty(K, **f32), torch.empty(K, **f32)
+        self.gamma_f = torch.empty(K, **f32) if g is not None else None
+        self.beta_f = torch.empty(K, **f32) if b is not None else None
+        self.wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+        self.sw = torch.empty(N, **f32)
+        self.xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        self.sx = torch.empty(M, **f32)
+        self.y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        self.ws = sq.new_workspace(M, N, K, device=dev)
+        L = sq._L
+        p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        eps = ctypes.c_float(1e-5)
+        runtime_inv_s = None if g is not None else self.inv_s
+        ws_bytes = 0 if self.ws is None else self.ws.numel()
+        self.calls = [
+            ("calibrate_x", L.sq_calibrate_absmax, (p(self.calib), calib.shape[0], K, K, p(self.gamma),
+                                                    p(self.beta), eps, p(self.amax_x), stream)),
+            ("calibrate_w", L.sq_calibrate_absmax, (p(self.w), N, K, K, None, None, eps, p(self.amax_w),
+                                                    stream)),
+            ("smooth_fold", L.sq_smooth_fold, (p(self.amax_x), p(self.amax_w), K, ctypes.c_float(wl.alpha),
+                                               p(self.s), p(self.inv_s), p(self.gamma), p(self.beta),
+                                               p(self.gamma_f), p(self.beta_f), None, None, 0, stream)),
+            ("quantize_weight", L.sq_quantize_weight, (p(self.w), N, K, p(self.s), p(self.wq), p(self.sw),
+                                                       stream)),
+            ("ln_quant_act", L.sq_ln_quant_act, (p(self.h), M, K, K, p(self.gamma_f), p(self.beta_f),
+                                                 p(runtime_inv_s), eps, p(self.xq), p(self.sx), stream)),
+            ("w8a8_linear", L.sq_w8a8_linear, (p(self.xq), p(self.sx), p(self.wq), p(self.sw), p(self.bias),
+                                               p(self.y), M, N, K, p(self.ws), ws_bytes, stream)),
+        ]
+        self.launches_per_step = len(self.calls)
+
+    def step(self, events=None, allreduce=None):
+        """Run one step; events (if given) is a list of len(calls)+1 CUDA events
+        recorded before each call and after the last."""
+        self.amax.zero_()
+        for i, (name, fn, args) in enumerate(self.calls):
+            if events is not None:
+                events[i].record()
+            if name == "smooth_fold" and allreduce is not None:
+                allreduce(self.amax_x)
+            st = fn(*args)
+            if st != 0:
+                raise RuntimeError(f"{name}: status {st}")
+        if events is not None:
+            events[-1].record()
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import w8a8_int8_linear_channel_b200 as sq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the product path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    wl = sq_inputs.WORKLOADS[args.workload]
+    M = args.m if args.m else wl.M
+    plan = Plan(wl, M, rank, device, sq, torch)
+    allreduce = None
+    if world > 1:
+        allreduce = lambda t: dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    ncalls = len(plan.calls)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        plan.step(allreduce=allreduce)
+    torch.cuda.synchronize()
+    if sq.sq_poll_status() != 0:
+        raise RuntimeError("device wait timed out during warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(ncalls + 1)] for _ in range(args.steps)]
+    try:
+        uuid = str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:  # no uuid attribute: the sampler falls back to the first GPU
+        uuid = ""
+    sampler = ClockSampler(uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    for i in range(args.steps):
+        flush.zero_()
+        plan.step(events[i], allreduce)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    if sq.sq_poll_status() != 0:
+        raise RuntimeError("device wait timed out in the timed region")
+
+    per_stage = np.zeros(ncalls)
+    total = 0.0
+    for ev in events:
+        for j in range(ncalls):
+            per_stage[j] += ev[j].elapsed_time(ev[j + 1])
+        total += ev[0].elapsed_time(ev[-1])
+    t_local = torch.tensor([total], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
+    total_ms = float(t_local.item())
+    ms_per_step = total_ms / args.steps
+    stage_us = {c[0]: 1e3 * per_stage[j] / args.steps for j, c in enumerate(plan.calls)}
+
+    nbytes, ops = stage_bytes_ops(wl, M)
+    step_bytes = sum(nbytes.values())
+    decode = M <= sq.SPLITK_MAX_M
+    if decode:
+        value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
+        unit = "GB/s"
+    else:
+        value = world * ops * args.steps / (total_ms * 1e-3) / 1e12
+        unit = "TOPS"
+
+    peaks, peak_kind = load_peaks()
+    gemm_s = stage_us["w8a8_linear"] * 1e-6
+    prof = os.path.join(ROOT, "profiles", f"w8a8_linear_{args.workload}{'_m%d' % M if M != wl.M else ''}.md")
+    src = os.path.join(ROOT, "w8a8_int8_linear_channel_b200", "csrc",
+                       "k_gemm_splitk.cu" if decode else "k_gemm_tiled.cu")
+    traffic = traffic_from_profile(src, prof)
+    if decode:
+        ach = nbytes["w8a8_linear"] / gemm_s / 1e9
+        peak = float(peaks["hbm_gbs"])
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(ach / peak, 4), "traffic": traffic,
+                "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"}
+    else:
+        ach = ops / gemm_s / 1e12
+        peak = float(peaks["bf16_tflops"]) * I8_PER_BF16
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(peak, 1), "unit": "TOPS",
+                "frac": round(ach / peak, 4), "traffic": traffic,
+                "peak_source": f"{peak_kind} cuBLAS bf16 burst {peaks['bf16_tflops']} TFLOP/s x 2 "
+                               "(nominal dense INT8:BF16 ratio 4.5:2.25)"}
+    roof["kernel"] = "k_gemm_splitk (swap-AB stream-K)" if decode else "k_gemm_tiled (tcgen05 kind::i8)"
+    roof["per_launch_us"] = round(stage_us["w8a8_linear"], 2)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(plan, sq, torch, world, allreduce, min(args.steps, args.e2e_steps), dist)
+
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
+            "data": "synthetic (seeded PCG64, OPT-shaped with persistent outlier channels)",
+            "config": {"workload": DESCR[args.workload] + ("" if M == wl.M else f" (M={M})"),
+                       "M": M, "N": wl.N, "K": wl.K, "calib_tokens": wl.calib, "alpha": wl.alpha,
+                       "step": STEP, "parallelism": f"dp{world}",
+                       "l2": "flushed: 256 MiB write before every step, outside the timed events",
+                       "timing": "CUDA events around every stage of every step; sum over steps; max over ranks"},
+            "roofline": roof,
+            "stage_us": {k: round(v, 2) for k, v in stage_us.items()},
+            "gpu_launches": plan.launches_per_step * args.steps,
+            "clocks": clocks,
+            "e2e": e2e,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = oracle_baseline(wl, M, budget_s=args.cpu_budget)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def run_e2e(plan, sq, torch, world, allreduce, steps, dist):
+    """The same step through the public Python API (SmoothQuantLinear) with the
+    inputs in pinned host memory: H2D copies, the whole path, D2H of y, all
+    inside the timed events."""
+    dev = plan.w.device
+    hp = {k: (None if v is None else torch.from_numpy(np.ascontiguousarray(v)).pin_memory())
+          for k, v in plan.host.items()}
+    y_host = torch.empty(tuple(plan.y.shape), dtype=torch.float16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in hp.values() if v is not None)
+    d2h = y_host.numel() * 2
+    pg = dist.group.WORLD if world > 1 else None
+
+    def one():
+        d = {k: (None if v is None else v.to(dev, non_blocking=True)) for k, v in hp.items()}
+        layer = sq.SmoothQuantLinear.from_float(d["w"], d["calib"], plan.wl.alpha, d["gamma"], d["beta"],
+                                                d["bias"], process_group=pg)
+        y = layer(d["h"])
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    e1.synchronize()
+    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    M, N, K = plan.M, plan.wl.N, plan.wl.K
+    nbytes, ops = stage_bytes_ops(plan.wl, M)
+    if M <= sq.SPLITK_MAX_M:
+        v, u = world * sum(nbytes.values()) * steps / (ms * 1e-3) / 1e9, "GB/s"
+    else:
+        v, u = world * ops * steps / (ms * 1e-3) / 1e12, "TOPS"
+    return {"value": round(v, 3), "unit": u, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "steps": steps, "ms_per_step": round(ms / steps, 4),
+            "api": "SmoothQuantLinear.from_float + forward, pinned host buffers"}
+
+
+# ------------------------------------------------------ oracle (CPU) arm -----
+def oracle_sample_inputs(wl, M, c_s, n_s, m_s):
+    bias = sq_inputs.bias(wl)
+    return {"calib": sq_inputs.calib_rows(wl, 0, c_s), "w": sq_inputs.weight(wl, 0, n_s),
+            "h": sq_inputs.run_rows(wl, 0, m_s), "g": sq_inputs.gamma(wl), "b": sq_inputs.beta(wl),
+            "bias": None if bias is None else bias[:n_s]}
+
+
+def oracle_stage_times(wl, inp):
+    """Time each oracle stage (as it stands) on one sample; seconds per stage."""
+    import oracle
+    g, b = inp["g"], inp["b"]
+    t0 = time.perf_counter()
+    ax = oracle.calibrate_absmax(inp["calib"], gamma=g, beta=b)
+    t1 = time.perf_counter()
+    aw = oracle.calibrate_absmax(inp["w"])
+    t2 = time.perf_counter()
+    s, inv_s = oracle.smooth(ax, aw, wl.alpha)
+    gf, bf = oracle.fold_ln(g, b, inv_s) if g is not None else (None, None)
+    t3 = time.perf_counter()
+    wq, sw = oracle.quantize_weight(oracle.fold_weight(inp["w"], s))
+    t4 = time.perf_counter()
+    xq, sx = oracle.ln_quant_act(inp["h"], gf, bf, None if g is not None else inv_s)
+    t5 = time.perf_counter()
+    oracle.w8a8_linear(xq, sx, wq, sw, inp["bias"])
+    t6 = time.perf_counter()
+    return {"calibrate_x": t1 - t0, "calibrate_w": t2 - t1, "smooth_fold": t3 - t2,
+            "quantize_weight": t4 - t3, "ln_quant_act": t5 - t4, "w8a8_linear": t6 - t5}
+
+
+def oracle_full_time(wl, M, st, c_s, n_s, m_s):
+    """Extrapolate sampled stage times linearly to the full workload."""
+    return (st["calibrate_x"] * wl.calib / c_s + st["calibrate_w"] * wl.N / n_s
+            + st["smooth_fold"] + st["quantize_weight"] * wl.N / n_s
+            + st["ln_quant_act"] * M / m_s + st["w8a8_linear"] * (M * wl.N) / (m_s * n_s))
+
+
+def pick_sample(wl, M, budget_s):
+    """Sample sizes whose oracle step takes about budget_s seconds."""
+    import oracle
+    c_s, n_s, m_s = min(wl.calib, 16), min(wl.N, 128), min(M, 4)
+    st = oracle_stage_times(wl, oracle_sample_inputs(wl, M, c_s, n_s, m_s))
+    dt = sum(st.values())
+    grow = max(1.0, budget_s / max(dt, 1e-6))
+    # grow the token and weight samples together (the GEMM is ~ m_s * n_s)
+    f = grow ** 0.5
+    n_s = int(min(wl.N, max(n_s, n_s * f)))
+    m_s = int(min(M, max(m_s, m_s * f)))
+    c_s = int(min(wl.calib, max(c_s, c_s * f)))
+    return c_s, n_s, m_s
+
+
+def oracle_baseline(wl, M, budget_s):
+    import oracle
+    c_s, n_s, m_s = pick_sample(wl, M, budget_s)
+    st = oracle_stage_times(wl, oracle_sample_inputs(wl, M, c_s, n_s, m_s))
+    full = oracle_full_time(wl, M, st, c_s, n_s, m_s)
+    nbytes, ops = stage_bytes_ops(wl, M)
+    if M <= 32:
+        v, u = sum(nbytes.values()) / full / 1e9, "GB/s"
+    else:
+        v, u = ops / full / 1e12, "TOPS"
+    return {"value": round(v, 6), "unit": u, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": (f"{c_s}/{wl.calib} calibration rows, {n_s}/{wl.N} weight rows, {m_s}/{M} tokens; "
+                       f"each stage timed on its sample and scaled linearly to the full workload "
+                       f"({sum(st.values()):.2f} s of CPU work; full step estimated {full:.1f} s)")}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step one bounded sample of the
+    workload, sized so the whole run ends within a few minutes."""
+    import oracle
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    wl = sq_inputs.WORKLOADS[args.workload]
+    M = args.m if args.m else wl.M
+    per_step = max(0.02, min(10.0, args.ref_budget / max(1, args.steps + args.warmup)))
+    c_s, n_s, m_s = pick_sample(wl, M, per_step)
+    inp = oracle_sample_inputs(wl, M, c_s, n_s, m_s)
+    for _ in range(args.warmup):
+        oracle_stage_times(wl, inp)
+    fulls = []
+    work = 0.0
+    for _ in range(args.steps):
+        st = oracle_stage_times(wl, inp)
+        work += sum(st.values())
+        fulls.append(oracle_full_time(wl, M, st, c_s, n_s, m_s))
+    full = sum(fulls) / len(fulls)
+    nbytes, ops = stage_bytes_ops(wl, M)
+    if M <= 32:
+        v, u = sum(nbytes.values()) / full / 1e9, "GB/s"
+    else:
+        v, u = ops / full / 1e12, "TOPS"
+    sample = (f"per step {c_s}/{wl.calib} calibration rows, {n_s}/{wl.N} weight rows, {m_s}/{M} tokens; "
+              f"stage times scaled linearly to the full workload")
+    return {"metric": METRIC, "value": round(v, 6), "unit": u, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(full * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": DESCR[args.workload] + ("" if M == wl.M else f" (M={M})"), "M": M,
+                       "N": wl.N, "K": wl.K, "step": STEP, "parallelism": "cpu oracle, rank 0"},
+            "cpu_baseline": {"value": round(v, 6), "unit": u, "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(v, 6), "unit": u, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "cpu_seconds": round(work, 2)}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["sq", "reference"], default="sq")
+    ap.add_argument("--workload", choices=sorted(DESCR), default="attn")
+    ap.add_argument("--m", type=int, default=0, help="token count override (decode sweep)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU work")
+    ap.add_argument("--ref-budget", type=float, default=150.0, help="seconds for the reference arm")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    res = run_reference(args) if args.impl == "reference" else run_gpu(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

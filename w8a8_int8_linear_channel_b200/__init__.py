@@ -239,9 +239,10 @@ class SmoothQuantLinear:
     and the INT8 GEMM.  All work happens in libsq kernels on the current
     stream."""
 
-    def __init__(self, wq, w_scale, bias, gamma_f, beta_f, inv_s, s, eps):
+    def __init__(self, wq, w_scale, bias, gamma_f, beta_f, inv_s, s, eps, smooth_inv=None):
         self.wq, self.w_scale, self.bias = wq, w_scale, bias
         self.gamma_f, self.beta_f, self.inv_s, self.s = gamma_f, beta_f, inv_s, s
+        self.smooth_inv = smooth_inv if smooth_inv is not None else inv_s  # 1/s, always kept
         self.eps = eps
         self._ws = {}
 
@@ -272,7 +273,7 @@ class SmoothQuantLinear:
         w_scale = torch.empty(N, dtype=torch.float32, device=dev)
         sq_quantize_weight(w, wq, w_scale, s=s)
         runtime_inv_s = None if gamma is not None else inv_s
-        return cls(wq, w_scale, bias, gamma_f, beta_f, runtime_inv_s, s, eps)
+        return cls(wq, w_scale, bias, gamma_f, beta_f, runtime_inv_s, s, eps, inv_s)
 
     def workspace(self, M: int) -> Optional[torch.Tensor]:
         N, K = self.wq.shape
