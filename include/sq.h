@@ -187,6 +187,37 @@ sq_status sq_w8a8_gemm_s32(const int8_t* xq, const int8_t* wq, int32_t* acc, int
                            int64_t N, int64_t K, void* workspace, size_t ws_bytes, int path,
                            sq_stream_t stream);
 
+/*
+ * Allocation-free variant of sq_w8a8_linear for M <= SQ_SPLITK_MAX_M (the
+ * stream-K decode kernel).  The paper has no counterpart: this entry point
+ * exists for callers that cannot allocate device memory -- for example a
+ * plug-in inside another runtime that owns every device allocation and hands
+ * over only input and output buffers, or a latency-critical path where a
+ * cudaMalloc (which may synchronize the whole device) is not acceptable.
+ *
+ * Instead of a caller workspace it uses one fixed array of
+ * SQ_NOALLOC_SCRATCH_BYTES in device global memory, owned by the library;
+ * every GPU that loads the library holds that array until the process exits.
+ * The call allocates and frees nothing.  Limits: M <= SQ_SPLITK_MAX_M
+ * (else SQ_ERR_UNSUPPORTED_SHAPE) and at most SQ_NOALLOC_MAX_TILES tiles of
+ * 128 output channels, i.e. N <= 524288 (else SQ_ERR_WORKSPACE, the shape
+ * needs more scratch than the fixed array holds).  Same numerics and the
+ * same output as sq_w8a8_linear.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call shares the array and it keeps the last call's
+ * contents; each call clears the arrival counters it needs before its GEMM
+ * kernel runs, on `stream`.  Calls whose kernels overlap on the GPU (on
+ * different streams or from different host threads) race on the array and
+ * must be serialized by the caller.
+ */
+#define SQ_NOALLOC_MAX_TILES 4096
+#define SQ_NOALLOC_SCRATCH_BYTES (5u * 1024u * 1024u + 4u * SQ_NOALLOC_MAX_TILES)
+sq_status sq_w8a8_linear_noalloc(const int8_t* xq, const float* x_scale, const int8_t* wq,
+                                 const float* w_scale, const void* bias_f16, void* y_f16,
+                                 int64_t M, int64_t N, int64_t K, sq_stream_t stream);
+
 /* Synchronizes `stream`, then reports and clears the current device's status
  * word: SQ_ERR_TIMEOUT if a bounded device wait ran out since the last poll,
  * SQ_ERR_CUDA if the stream reported an error, else SQ_OK. */

@@ -4,8 +4,8 @@ A thin ctypes binding over ``libsq.so`` (C ABI in ``include/sq.h``).  The
 functions below carry the C names and only marshal arguments: every step of
 the method runs in the library's CUDA kernels; PyTorch provides device memory
 and the current stream.  There is no CPU path: importing this package fails
-if the library has not been built (``python -m
-w8a8_int8_linear_channel_b200.build``).
+if the library has not been built (``python
+w8a8_int8_linear_channel_b200/build.py``).
 
 The method ("SmoothQuant: Accurate and Efficient Post-Training Quantization
 for Large Language Models", abeam.tech explainer):
@@ -48,7 +48,7 @@ def library_path() -> str:
 def _load() -> ctypes.CDLL:
     if not os.path.exists(_LIB_PATH):
         raise ImportError(
-            f"{_LIB_PATH} is missing: build it with `python -m w8a8_int8_linear_channel_b200.build` "
+            f"{_LIB_PATH} is missing: build it with `python w8a8_int8_linear_channel_b200/build.py` "
             "(nvcc, sm_100a).  There is no CPU fallback.")
     L = ctypes.CDLL(_LIB_PATH)
     P, I, F, Z, S = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t, ctypes.c_int
@@ -63,6 +63,7 @@ def _load() -> ctypes.CDLL:
         "sq_w8a8_linear": ([P, P, P, P, P, P, I, I, I, P, Z, P], S),
         "sq_w8a8_linear_path": ([P, P, P, P, P, P, I, I, I, P, Z, S, P], S),
         "sq_w8a8_gemm_s32": ([P, P, P, I, I, I, P, Z, S, P], S),
+        "sq_w8a8_linear_noalloc": ([P, P, P, P, P, P, I, I, I, P], S),
         "sq_poll_status": ([P], S),
         "sq_set_wait_budget_ns": ([ctypes.c_uint64], None),
         "sq_selftest_wait_timeout": ([ctypes.c_uint64, P], S),
@@ -207,6 +208,21 @@ def sq_w8a8_gemm_s32(xq, wq, acc, workspace=None, path: int = PATH_AUTO, stream=
     _check(_L.sq_w8a8_gemm_s32(_p(xq), _p(wq), _p(acc), M, N, K, _p(workspace), ws_bytes, path,
                                _stream(stream)), "sq_w8a8_gemm_s32")
     return acc
+
+
+def sq_w8a8_linear_noalloc(xq, x_scale, wq, w_scale, y, bias=None, stream=None):
+    """sq_w8a8_linear for M <= 32 without a workspace: for callers that cannot
+    allocate device memory (the library's own fixed scratch array is used;
+    overlapping calls race on it)."""
+    M, N, K = _gemm_shapes(xq, wq)
+    _vec(x_scale, M, torch.float32, "x_scale")
+    _vec(w_scale, N, torch.float32, "w_scale")
+    _vec(bias, N, torch.float16, "bias")
+    if y.dtype != torch.float16 or tuple(y.shape) != (M, N) or not y.is_contiguous():
+        raise ValueError("y: need a contiguous fp16 [M, N] tensor")
+    _check(_L.sq_w8a8_linear_noalloc(_p(xq), _p(x_scale), _p(wq), _p(w_scale), _p(bias), _p(y),
+                                     M, N, K, _stream(stream)), "sq_w8a8_linear_noalloc")
+    return y
 
 
 def sq_poll_status(stream=None) -> int:

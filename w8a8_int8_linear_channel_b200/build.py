@@ -1,6 +1,6 @@
 """Build libsq.so (the C-ABI library) in-tree for sm_100a with nvcc.
 
-    python -m w8a8_int8_linear_channel_b200.build [--force] [-v]
+    python w8a8_int8_linear_channel_b200/build.py [--force] [-v]
 
 Objects go to _build/ at the repository root; the shared library lands next
 to this file so the Python binding finds it.  The CUDA runtime is linked

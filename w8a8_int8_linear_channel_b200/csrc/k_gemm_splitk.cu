@@ -321,3 +321,132 @@ cudaError_t launch_gemm_splitk(const GemmArgs& g, const Ctx& c) {
 }
 
 }  // namespace sq
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the stream-K linear.
+//
+// Some callers cannot allocate device memory at all: a plug-in running inside
+// another runtime that owns every device allocation and hands the plug-in
+// only its input and output buffers, or a latency-critical path where
+// cudaMalloc (which may synchronize the device) is not acceptable.  This
+// variant keeps the stream-K scratch (per-tile arrival counters and int32
+// partial accumulators) in one fixed array in device global memory, owned by
+// the library: every GPU that loads the library holds it until the process
+// exits.  Calls share the array and it keeps the last call's contents, so the
+// counters are cleared at the start of every call, and two calls whose
+// kernels overlap on the GPU (different streams, or different host threads)
+// race on it.
+#include <mutex>
+
+#include "../../include/sq.h"
+
+namespace sq {
+namespace {
+
+constexpr size_t kNoAllocCounterBytes = 4u * SQ_NOALLOC_MAX_TILES;        // one uint32 per tile
+constexpr size_t kNoAllocPartialBytes = SQ_NOALLOC_SCRATCH_BYTES - kNoAllocCounterBytes;
+static_assert(kNoAllocCounterBytes % 256 == 0, "partials must start 256-byte aligned");
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SQ_NOALLOC_SCRATCH_BYTES];
+
+// The counters must start at zero; the array keeps whatever the last call left.
+__global__ void k_noalloc_clear_counters(uint32_t n) {
+  uint32_t* counters = reinterpret_cast<uint32_t*>(g_noalloc_scratch);
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    counters[i] = 0;
+}
+
+constexpr int kMaxDev = 64;
+std::once_flag g_noalloc_once[kMaxDev];
+uint8_t* g_noalloc_dev_ptr[kMaxDev];
+cudaError_t g_noalloc_setup_err[kMaxDev];
+
+// Device address of the scratch array on the current device.  Host code only
+// knows a host-side stand-in for the array's name, so the address is looked
+// up once per device (with that device current) and handed to the kernels.
+cudaError_t noalloc_scratch(int dev, uint8_t** out) {
+  std::call_once(g_noalloc_once[dev], [dev] {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) cudaGetLastError();
+    g_noalloc_setup_err[dev] = e;
+    g_noalloc_dev_ptr[dev] = static_cast<uint8_t*>(p);
+  });
+  *out = g_noalloc_dev_ptr[dev];
+  return g_noalloc_setup_err[dev];
+}
+
+// Same kernel as launch_bt, with the scratch of the fixed array and the grid
+// capped to the partial-accumulator slots the array holds.
+template <int BT>
+cudaError_t launch_noalloc(const GemmArgs& g, const Ctx& c, uint8_t* scratch) {
+  using L = SkLayout<BT>;
+  cudaError_t e = cudaFuncSetAttribute(k_gemm_splitk<BT, false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(L::SMEM));
+  if (e != cudaSuccess) return e;
+  CUtensorMap tmW, tmX;
+  if (!make_tmap_i8(&tmW, g.wq, g.K, g.N, BK, BW)) return cudaErrorInvalidValue;
+  if (!make_tmap_i8(&tmX, g.xq, g.K, g.M, BK, BT)) return cudaErrorInvalidValue;
+  SkGeom geo;
+  geo.KB = static_cast<int>((g.K + BK - 1) / BK);
+  geo.U = tiles_of(g.N) * geo.KB;
+  const int64_t slots = static_cast<int64_t>(kNoAllocPartialBytes / (2ull * BW * BT * 4));
+  int64_t G = c.num_sms;
+  if (G > slots) G = slots;
+  if (G > geo.U) G = geo.U;
+  geo.G = static_cast<int>(G);
+  uint32_t* counters = reinterpret_cast<uint32_t*>(scratch);
+  int32_t* partials = reinterpret_cast<int32_t*>(scratch + kNoAllocCounterBytes);
+  const uint32_t ntiles = static_cast<uint32_t>(tiles_of(g.N));
+  k_noalloc_clear_counters<<<(ntiles + 255) / 256, 256, 0, c.stream>>>(ntiles);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_gemm_splitk<BT, false><<<geo.G, kThreads, L::SMEM, c.stream>>>(
+      tmW, tmX, g, geo, counters, partials, c.status, c.budget_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace sq
+
+extern "C" sq_status sq_w8a8_linear_noalloc(const int8_t* xq, const float* x_scale,
+                                            const int8_t* wq, const float* w_scale,
+                                            const void* bias_f16, void* y_f16, int64_t M,
+                                            int64_t N, int64_t K, sq_stream_t stream) {
+  using namespace sq;
+  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!xq || !x_scale || !wq || !w_scale || !y_f16) return SQ_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return SQ_ERR_INVALID_ARG;
+  if (K > SQ_MAX_K) return SQ_ERR_K_OVERFLOW;
+  if (K % 16 != 0 || M > SQ_SPLITK_MAX_M) return SQ_ERR_UNSUPPORTED_SHAPE;
+  if (tiles_of(N) > SQ_NOALLOC_MAX_TILES) return SQ_ERR_WORKSPACE;  // beyond the fixed scratch
+  if (!a16(xq) || !a16(wq) || !a16(x_scale) || !a16(w_scale) || !a16(y_f16) ||
+      (bias_f16 && !a16(bias_f16)))
+    return SQ_ERR_MISALIGNED;
+  Ctx ctx;
+  const int st = call_context(stream, &ctx);
+  if (st != SQ_OK) return static_cast<sq_status>(st);
+  if (ctx.device >= kMaxDev) return SQ_ERR_CUDA;
+  uint8_t* scratch = nullptr;
+  if (noalloc_scratch(ctx.device, &scratch) != cudaSuccess || scratch == nullptr) return SQ_ERR_CUDA;
+  GemmArgs g;
+  g.xq = xq;
+  g.sx = x_scale;
+  g.wq = wq;
+  g.sw = w_scale;
+  g.bias = static_cast<const __half*>(bias_f16);
+  g.y = static_cast<__half*>(y_f16);
+  g.acc = nullptr;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.ws = scratch;
+  g.ws_bytes = SQ_NOALLOC_SCRATCH_BYTES;
+  const cudaError_t e = (M <= 16) ? launch_noalloc<16>(g, ctx, scratch) : launch_noalloc<32>(g, ctx, scratch);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return SQ_ERR_CUDA;
+  }
+  return SQ_OK;
+}

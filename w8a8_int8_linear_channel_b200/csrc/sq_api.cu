@@ -160,6 +160,8 @@ sq_status linear_impl(const int8_t* xq, const float* x_scale, const int8_t* wq,
 
 }  // namespace
 
+int call_context(void* stream, Ctx* ctx) { return current_ctx(stream, ctx); }
+
 void* tensor_map_encoder() {
   std::call_once(g_encoder_once, [] {
     cudaDriverEntryPointQueryResult q;

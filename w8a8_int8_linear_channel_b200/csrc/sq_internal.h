@@ -64,6 +64,10 @@ size_t splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
 
 cudaError_t launch_wait_selftest(uint64_t budget_ns, const Ctx& c);
 
+// Launch context of the current device (arch check, status word, wait
+// budget); returns an sq_status code (0 = ok).
+int call_context(void* stream, Ctx* ctx);
+
 // Driver entry point for tensor-map encoding (resolved once through the
 // runtime, so the library does not link libcuda directly).
 void* tensor_map_encoder();
