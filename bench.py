@@ -243,17 +243,28 @@ def run_gpu(args):
     allreduce = None
     if world > 1:
         allreduce = lambda t: dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    # L2 flush between steps: write a 256 MiB buffer (> the 126 MB L2), then
+    # read another one so the flush's dirty lines are written back before the
+    # step starts (outside the timed events); the step then starts cold.
+    flush_w = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    flush_r = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=device)
+
+    def flush():
+        flush_w.zero_()
+        flush_r.sum()
+
     ncalls = len(plan.calls)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         plan.step(allreduce=allreduce)
     torch.cuda.synchronize()
     if sq.sq_poll_status() != 0:
         raise RuntimeError("device wait timed out during warm-up")
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(ncalls + 1)] for _ in range(args.steps)]
+    # timed region: events only at step boundaries, so consecutive kernels of a
+    # step overlap their launches (programmatic dependent launch)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     try:
         uuid = str(torch.cuda.get_device_properties(local).uuid)
     except Exception:  # no uuid attribute: the sampler falls back to the first GPU
@@ -265,8 +276,10 @@ def run_gpu(args):
     if sampler:
         sampler.start()
     for i in range(args.steps):
-        flush.zero_()
-        plan.step(events[i], allreduce)
+        flush()
+        events[i][0].record()
+        plan.step(None, allreduce)
+        events[i][1].record()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -274,19 +287,27 @@ def run_gpu(args):
     clocks = sampler.stop() if sampler else None
     if sq.sq_poll_status() != 0:
         raise RuntimeError("device wait timed out in the timed region")
-
-    per_stage = np.zeros(ncalls)
-    total = 0.0
-    for ev in events:
-        for j in range(ncalls):
-            per_stage[j] += ev[j].elapsed_time(ev[j + 1])
-        total += ev[0].elapsed_time(ev[-1])
+    total = sum(ev[0].elapsed_time(ev[1]) for ev in events)
     t_local = torch.tensor([total], dtype=torch.float64, device=device)
     if world > 1:
         dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
     total_ms = float(t_local.item())
     ms_per_step = total_ms / args.steps
-    stage_us = {c[0]: 1e3 * per_stage[j] / args.steps for j, c in enumerate(plan.calls)}
+
+    # stage breakdown: a second timed loop with an event around every call
+    # (the events serialize the launches, so each stage also carries its own
+    # launch latency; the GEMM's time here is the roofline's launch duration)
+    n_stage = min(args.steps, args.stage_steps)
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(ncalls + 1)] for _ in range(n_stage)]
+    for i in range(n_stage):
+        flush()
+        plan.step(sev[i], allreduce)
+    torch.cuda.synchronize()
+    per_stage = np.zeros(ncalls)
+    for ev in sev:
+        for j in range(ncalls):
+            per_stage[j] += ev[j].elapsed_time(ev[j + 1])
+    stage_us = {c[0]: 1e3 * per_stage[j] / n_stage for j, c in enumerate(plan.calls)}
 
     nbytes, ops = stage_bytes_ops(wl, M)
     step_bytes = sum(nbytes.values())
@@ -334,11 +355,15 @@ def run_gpu(args):
             "config": {"workload": DESCR[args.workload] + ("" if M == wl.M else f" (M={M})"),
                        "M": M, "N": wl.N, "K": wl.K, "calib_tokens": wl.calib, "alpha": wl.alpha,
                        "step": STEP, "parallelism": f"dp{world}",
-                       "l2": "flushed: 256 MiB write before every step, outside the timed events",
-                       "timing": "CUDA events around every stage of every step; sum over steps; max over ranks"},
+                       "l2": "flushed before every step (256 MiB write, then 256 MiB read so no dirty "
+                             "lines remain), outside the timed events",
+                       "timing": "CUDA events at the boundaries of every step, summed over steps, max over "
+                                 "ranks; stage_us and the roofline's launch time from a second loop with "
+                                 "events around every call"},
             "roofline": roof,
             "stage_us": {k: round(v, 2) for k, v in stage_us.items()},
             "gpu_launches": plan.launches_per_step * args.steps,
+            "launch": "every libsq kernel with programmatic dependent launch (prologue overlaps the previous kernel)",
             "clocks": clocks,
             "e2e": e2e,
         }
@@ -515,6 +540,7 @@ def main():
     ap.add_argument("--m", type=int, default=0, help="token count override (decode sweep)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--stage-steps", type=int, default=300, help="steps of the per-stage timing loop")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU work")
     ap.add_argument("--ref-budget", type=float, default=150.0, help="seconds for the reference arm")

@@ -22,58 +22,80 @@ __device__ __forceinline__ __half2 habs2(__half2 v) {
 
 __device__ __forceinline__ __half2 as_h2(uint32_t w) { return *reinterpret_cast<__half2*>(&w); }
 
-// Each thread owns one 8-column chunk and walks a strided set of rows; the
-// fp16 maxima are exact, merged into amax with atomicMax on the float bits.
-__global__ void __launch_bounds__(256) k_absmax_cols(const __half* __restrict__ x, int64_t rows,
-                                                     int64_t Kc, int64_t ld,
-                                                     float* __restrict__ amax) {
-  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (c >= Kc) return;
+// Column maxima of a row-major fp16 matrix.  A CTA covers 256 columns (32
+// chunks of 8) and a band of rows; its 8 warps read 8 rows at a time (each
+// warp 512 contiguous bytes per row), 8 independent 16-byte loads in flight
+// per thread.  The CTA reduces its 8 row lanes in shared memory and merges
+// its 256 maxima with one global atomicMax each (exact: max of non-negative
+// floats, ordered as ints); the number of row bands is kept small so each
+// column sees only a few dozen atomics.
+__global__ void __launch_bounds__(256)
+    k_absmax_cols(const __half* __restrict__ x, int64_t rows, int64_t Kc, int64_t ld,
+                  int64_t rows_per_cta, float* __restrict__ amax) {
+  __shared__ float red[8][257];
+  griddep_wait();
+  griddep_launch_dependents();
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * 32 + tx;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_cta;
+  const int64_t r1 = r0 + rows_per_cta < rows ? r0 + rows_per_cta : rows;
   __half2 m0 = __float2half2_rn(0.0f), m1 = m0, m2 = m0, m3 = m0;
-  int64_t r = blockIdx.y;
-  const int64_t step = gridDim.y;
-  for (; r + 3 * step < rows; r += 4 * step) {
-    uint4 v[4];
+  if (c < Kc) {
+    const uint4* base = reinterpret_cast<const uint4*>(x) + c;
+    const int64_t ldc = ld / 8;  // row stride in 16-byte chunks
+    // batches of 8 rows per thread (64 per CTA), all loads of a batch issued
+    // before any is used; rows past the band read as zeros
+    for (int64_t r = r0 + ty; r < r1; r += 64) {
+      uint4 v[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      v[u] = __ldg(reinterpret_cast<const uint4*>(x + (r + u * step) * ld) + c);
+      for (int u = 0; u < 8; ++u)
+        v[u] = (r + 8 * u < r1) ? __ldg(base + (r + 8 * u) * ldc) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      m0 = __hmax2(m0, habs2(as_h2(v[u].x)));
-      m1 = __hmax2(m1, habs2(as_h2(v[u].y)));
-      m2 = __hmax2(m2, habs2(as_h2(v[u].z)));
-      m3 = __hmax2(m3, habs2(as_h2(v[u].w)));
+      for (int u = 0; u < 8; ++u) {
+        m0 = __hmax2(m0, habs2(as_h2(v[u].x)));
+        m1 = __hmax2(m1, habs2(as_h2(v[u].y)));
+        m2 = __hmax2(m2, habs2(as_h2(v[u].z)));
+        m3 = __hmax2(m3, habs2(as_h2(v[u].w)));
+      }
     }
   }
-  for (; r < rows; r += step) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + r * ld) + c);
-    m0 = __hmax2(m0, habs2(as_h2(v.x)));
-    m1 = __hmax2(m1, habs2(as_h2(v.y)));
-    m2 = __hmax2(m2, habs2(as_h2(v.z)));
-    m3 = __hmax2(m3, habs2(as_h2(v.w)));
-  }
-  int* dst = reinterpret_cast<int*>(amax) + c * 8;
   const __half2 m[4] = {m0, m1, m2, m3};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    atomicMax(dst + 2 * j, __float_as_int(__low2float(m[j])));
-    atomicMax(dst + 2 * j + 1, __float_as_int(__high2float(m[j])));
+    red[ty][tx * 8 + 2 * j] = __low2float(m[j]);
+    red[ty][tx * 8 + 2 * j + 1] = __high2float(m[j]);
+  }
+  __syncthreads();
+  const int col = threadIdx.x;  // 0..255
+  const int64_t k = static_cast<int64_t>(blockIdx.x) * 256 + col;
+  if (k < Kc * 8) {
+    float mm = 0.0f;
+#pragma unroll
+    for (int y = 0; y < 8; ++y) mm = fmaxf(mm, red[y][col]);
+    atomicMax(reinterpret_cast<int*>(amax) + k, __float_as_int(mm));
   }
 }
 
-// s_j in fp64 (both maxima floored at 1e-5f), rounded once to fp32.
+// s_j in fp64 (both maxima floored at 1e-5f), rounded once to fp32.  The
+// two powers of a channel are evaluated by a pair of adjacent threads (even:
+// a^alpha, odd: b^(1-alpha)) to halve the dependent fp64 latency.
 __global__ void k_smooth(const float* __restrict__ amax_x, const float* __restrict__ amax_w,
                          int64_t K, float alpha, float* __restrict__ s, float* __restrict__ inv_s,
                          const float* gamma, const float* beta, float* gamma_out,
                          float* beta_out) {
-  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (j >= K) return;
-  const float ax = amax_x[j], aw = amax_w[j];
-  const double x = ax > 1e-5f ? static_cast<double>(ax) : static_cast<double>(1e-5f);
-  const double w = aw > 1e-5f ? static_cast<double>(aw) : static_cast<double>(1e-5f);
+  griddep_wait();
+  griddep_launch_dependents();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t j = t >> 1;
+  const bool odd = (t & 1) != 0;
+  const bool valid = j < K;
+  const float av = valid ? (odd ? amax_w[j] : amax_x[j]) : 1.0f;
+  const double base = av > 1e-5f ? static_cast<double>(av) : static_cast<double>(1e-5f);
   const double a = static_cast<double>(alpha);
-  const double sj = __ddiv_rn(pow(x, a), pow(w, __dsub_rn(1.0, a)));
-  const float s32 = __double2float_rn(sj);
+  const double p = pow(base, odd ? __dsub_rn(1.0, a) : a);
+  const double den = __shfl_down_sync(0xffffffffu, p, 1);
+  if (!valid || odd) return;
+  const float s32 = __double2float_rn(__ddiv_rn(p, den));
   const float inv = __frcp_rn(s32);
   s[j] = s32;
   inv_s[j] = inv;
@@ -83,13 +105,15 @@ __global__ void k_smooth(const float* __restrict__ amax_x, const float* __restri
 
 // w_out[n, j] = fp16(fp32(w[n, j]) * s_j), one 8-element chunk per thread and
 // iteration (grid-stride).
-__global__ void __launch_bounds__(256) k_fold_weight(const __half* __restrict__ w,
-                                                     __half* __restrict__ w_out, int64_t total_c,
+__global__ void __launch_bounds__(256) k_fold_weight(const __half* w, __half* w_out,
+                                                     int64_t total_c,
                                                      int64_t Kc, const float* __restrict__ s) {
+  griddep_wait();
+  griddep_launch_dependents();
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_c;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t c = i % Kc;
-    uint4 v = __ldg(reinterpret_cast<const uint4*>(w) + i);
+    uint4 v = reinterpret_cast<const uint4*>(w)[i];  // w_out may alias w
     const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + c * 8));
     const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + c * 8 + 4));
     const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
@@ -111,25 +135,25 @@ __global__ void __launch_bounds__(256) k_fold_weight(const __half* __restrict__ 
 cudaError_t launch_absmax_cols(const __half* x, int64_t rows, int64_t K, int64_t ld, float* amax,
                                const Ctx& c) {
   const int64_t Kc = K / 8;
-  int threads = static_cast<int>(Kc < 256 ? ((Kc + 31) / 32) * 32 : 256);
-  const int64_t gx = (Kc + threads - 1) / threads;
-  int64_t gy = (static_cast<int64_t>(c.num_sms) * 2048 + threads * gx - 1) / (threads * gx);
-  if (gy > rows) gy = rows;
-  if (gy > 65535) gy = 65535;
+  const int64_t gx = (Kc + 31) / 32;
+  // about three CTAs per SM, at least 128 rows per CTA, at most 64 bands
+  int64_t gy = (3 * static_cast<int64_t>(c.num_sms) + gx - 1) / gx;
+  const int64_t by_rows = (rows + 127) / 128;
+  if (gy > by_rows) gy = by_rows;
+  if (gy > 64) gy = 64;
   if (gy < 1) gy = 1;
+  const int64_t rows_per_cta = (rows + gy - 1) / gy;
   dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
-  k_absmax_cols<<<grid, threads, 0, c.stream>>>(x, rows, Kc, ld, amax);
-  return cudaGetLastError();
+  return launch_pdl(k_absmax_cols, grid, dim3(256), 0, c.stream, x, rows, Kc, ld, rows_per_cta, amax);
 }
 
 cudaError_t launch_smooth(const float* amax_x, const float* amax_w, int64_t K, float alpha,
                           float* s, float* inv_s, const float* gamma, const float* beta,
                           float* gamma_out, float* beta_out, const Ctx& c) {
-  const int threads = 256;
-  const int64_t blocks = (K + threads - 1) / threads;
-  k_smooth<<<static_cast<unsigned>(blocks), threads, 0, c.stream>>>(
-      amax_x, amax_w, K, alpha, s, inv_s, gamma, beta, gamma_out, beta_out);
-  return cudaGetLastError();
+  const int threads = 64;  // two threads per channel, spread over many SMs
+  const int64_t blocks = (2 * K + threads - 1) / threads;
+  return launch_pdl(k_smooth, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, c.stream, amax_x,
+                    amax_w, K, alpha, s, inv_s, gamma, beta, gamma_out, beta_out);
 }
 
 cudaError_t launch_fold_weight(const __half* w, __half* w_out, int64_t N, int64_t K,
@@ -139,8 +163,8 @@ cudaError_t launch_fold_weight(const __half* w, __half* w_out, int64_t N, int64_
   int64_t blocks = static_cast<int64_t>(c.num_sms) * 8;
   const int64_t need = (total + 255) / 256;
   if (blocks > need) blocks = need;
-  k_fold_weight<<<static_cast<unsigned>(blocks), 256, 0, c.stream>>>(w, w_out, total, Kc, s);
-  return cudaGetLastError();
+  return launch_pdl(k_fold_weight, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, c.stream, w, w_out,
+                    total, Kc, s);
 }
 
 }  // namespace sq

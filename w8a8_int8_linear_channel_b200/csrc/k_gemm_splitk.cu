@@ -36,8 +36,8 @@ struct SkLayout {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int CTRL = kStages * STAGE_BYTES;
   static constexpr int NBARS = 2 * kStages + 5;  // full, empty, acc_full[2], acc_empty[2], drain
-  static constexpr int SLOT = CTRL + NBARS * 8;  // TMEM address, abort flag, last flag
-  static constexpr int SX = SLOT + 16;           // sx[BT]
+  static constexpr int SLOT = CTRL + NBARS * 8;  // TMEM address, abort, last, decision[2]
+  static constexpr int SX = SLOT + 32;           // sx[BT]
   static constexpr int BYTES = SX + BT * 4;
   static constexpr size_t SMEM = BYTES + 1024;
   static constexpr int TMEM_COLS = 2 * BT < 32 ? 32 : 2 * BT;
@@ -87,6 +87,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::SLOT);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* last_flag = tmem_slot + 2;
+  volatile uint32_t* decision = tmem_slot + 3;  // [2]
   float* sx_s = reinterpret_cast<float*>(smem + L::SX);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -117,6 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // inputs and workspace are written by earlier kernels
 
   int64_t issued = 0;
   bool mma_any = false;
@@ -169,6 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++seg;
         }
       }
+      griddep_launch_dependents();
     }
   } else {
     const int et = threadIdx.x - 64;
@@ -183,7 +186,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool whole = (u == t * KB) && (seg_end == tile_end);
       const int slot = (u == ubeg) ? 0 : 1;
       const int b = seg & 1;
-      if (!mbar_wait(accf_bar(b), static_cast<uint32_t>((seg >> 1) & 1), budget, status, abort_flag)) break;
+      mbar_wait(accf_bar(b), static_cast<uint32_t>((seg >> 1) & 1), budget, status, abort_flag);
+      // one thread decides whether to stop and broadcasts it (double-buffered by
+      // segment parity), so every epilogue thread leaves the loop at the same point
+      if (et == 0) decision[seg & 1] = *abort_flag;
+      named_bar_sync(1, 128);
+      if (decision[seg & 1]) break;
       tc_fence_after();
       uint32_t v[BT];
       tmem_ld_tokens<BT>(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(b * BT), v);
@@ -300,9 +308,8 @@ cudaError_t launch_bt(const GemmArgs& g, const Ctx& c) {
   const size_t counter_bytes = ((tiles_of(g.N) * 4 + 255) / 256) * 256;
   uint32_t* counters = reinterpret_cast<uint32_t*>(ws);
   int32_t* partials = reinterpret_cast<int32_t*>(ws + counter_bytes);
-  k_gemm_splitk<BT, OUT_I32><<<geo.G, kThreads, L::SMEM, c.stream>>>(
-      tmW, tmX, g, geo, counters, partials, c.status, c.budget_ns);
-  return cudaGetLastError();
+  return launch_pdl(k_gemm_splitk<BT, OUT_I32>, dim3(geo.G), dim3(kThreads), L::SMEM, c.stream, tmW, tmX, g,
+                    geo, counters, partials, c.status, c.budget_ns);
 }
 
 }  // namespace
@@ -351,6 +358,8 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[SQ_NOALLOC_SCRATCH_BY
 
 // The counters must start at zero; the array keeps whatever the last call left.
 __global__ void k_noalloc_clear_counters(uint32_t n) {
+  griddep_wait();  // the previous call's kernels may still be reading them
+  griddep_launch_dependents();
   uint32_t* counters = reinterpret_cast<uint32_t*>(g_noalloc_scratch);
   for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
     counters[i] = 0;
@@ -399,12 +408,10 @@ cudaError_t launch_noalloc(const GemmArgs& g, const Ctx& c, uint8_t* scratch) {
   uint32_t* counters = reinterpret_cast<uint32_t*>(scratch);
   int32_t* partials = reinterpret_cast<int32_t*>(scratch + kNoAllocCounterBytes);
   const uint32_t ntiles = static_cast<uint32_t>(tiles_of(g.N));
-  k_noalloc_clear_counters<<<(ntiles + 255) / 256, 256, 0, c.stream>>>(ntiles);
-  e = cudaGetLastError();
+  e = launch_pdl(k_noalloc_clear_counters, dim3((ntiles + 255) / 256), dim3(256), 0, c.stream, ntiles);
   if (e != cudaSuccess) return e;
-  k_gemm_splitk<BT, false><<<geo.G, kThreads, L::SMEM, c.stream>>>(
-      tmW, tmX, g, geo, counters, partials, c.status, c.budget_ns);
-  return cudaGetLastError();
+  return launch_pdl(k_gemm_splitk<BT, false>, dim3(geo.G), dim3(kThreads), L::SMEM, c.stream, tmW, tmX, g,
+                    geo, counters, partials, c.status, c.budget_ns);
 }
 
 }  // namespace

@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // inputs of this kernel are written by the previous one
 
   int issued = 0;        // producer: stages issued
   bool mma_any = false;  // MMA thread: issued at least one MMA
@@ -122,6 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(empty_bar(s));
       }
       if (ok) mma_commit(acc_bar);
+      griddep_launch_dependents();
     }
   } else {
     // epilogue warps 2..5: TMEM lane quarter (warp % 4) = token rows 32q .. 32q+31
@@ -213,9 +215,8 @@ cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
   if (!make_tmap_i8(&tmA, g.xq, g.K, g.M, BK, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_i8(&tmB, g.wq, g.K, g.N, BK, BN)) return cudaErrorInvalidValue;
   dim3 grid(static_cast<unsigned>((g.N + BN - 1) / BN), static_cast<unsigned>((g.M + BM - 1) / BM));
-  k_gemm_tiled<BN, STAGES, OUT_I32><<<grid, kThreads, L::SMEM, c.stream>>>(tmA, tmB, g, c.status,
-                                                                           c.budget_ns);
-  return cudaGetLastError();
+  return launch_pdl(k_gemm_tiled<BN, STAGES, OUT_I32>, grid, dim3(kThreads), L::SMEM, c.stream, tmA, tmB, g,
+                    c.status, c.budget_ns);
 }
 
 }  // namespace

@@ -5,83 +5,49 @@
 //     diag(s) on the fly (section "what it does mathematically");
 //   * calibration absmax of the LayerNorm output (glossary "Calibration").
 //
-// One CTA of 256 threads owns one row at a time (grid-stride over rows); the
-// row is read once from HBM with 16-byte loads and held in registers (8 fp16
-// values per chunk, NCH chunks per thread).  Rows too long for registers
-// re-read their chunks (the row then sits in L2).  Reductions are warp
-// shuffles plus one shared-memory step.
+// Two shapes of the same computation:
+//   * K <= 4096: one warp per row (no block barrier at all; many rows in
+//     flight per SM).  The row and its transformed values live in registers.
+//   * larger K: one CTA of 256 threads per row, warp shuffles plus one
+//     shared-memory step per reduction.
+// Rows are read once from HBM with 16-byte loads.
 //
-// The LayerNorm statistics are exact: every fp16 value h equals v * 2^-24 for
-// an integer v (|v| < 2^40); S1 = sum v is kept in int64 and S2 = sum v^2 in
-// 128 bits, so the sums -- and hence mu, rstd and every INT8 code -- do not
-// depend on the reduction order.
+// LayerNorm statistics are exact and order-independent: every fp16 value h
+// equals v * 2^-24 for an integer v (|v| < 2^40).  Per 8-element chunk the
+// sums of h and of h^2 are formed exactly in fp64 (h^2 has a 22-bit
+// significand; it is split exactly into a multiple of 2^-13 and a remainder
+// below 2^-13 so both partial sums stay within 53 bits), then converted to
+// int64 in units of 2^-24 (S1) and 2^-13 / 2^-48 (S2), and summed as
+// integers.  S1 = sum v and S2 = sum v^2 are therefore the exact integers,
+// whatever the reduction order.
+//
+// Calibration merges its per-column maxima across a cluster of 8 CTAs
+// through distributed shared memory, so each column receives one global
+// atomicMax per cluster instead of one per CTA.
+#include <cooperative_groups.h>
+
 #include "sq_internal.h"
 #include "sq_ptx.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace sq {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+constexpr int kCtaThreads = 256;
+constexpr int kWarpThreads = 128;  // 4 row-warps per CTA in the warp-per-row kernels
+constexpr int kCluster = 8;
 
 enum RowMode { MODE_ACT = 0, MODE_WEIGHT = 1, MODE_CALIB = 2 };
 
 typedef unsigned __int128 u128;
 
-struct RowShared {
-  long long s1[kWarps];
-  unsigned long long s2_hi[kWarps];
-  unsigned long long s2_lo[kWarps];
-  float mx[kWarps];
-  float mu, rstd, inv;
+// ------------------------------------------------------- exact LN sums ---
+struct Sums {
+  long long s1;   // sum v            (units 2^-24 of h)
+  long long s2h;  // sum of h^2 parts that are multiples of 2^-13, in units 2^-13
+  long long s2l;  // sum of the remainders below 2^-13, in units 2^-48
 };
-
-__device__ __forceinline__ void stats_add(uint32_t b, long long& s1, u128& s2) {
-  const uint32_t e = (b >> 10) & 31u;
-  const uint32_t m = b & 1023u;
-  const uint32_t sig = e ? (m | 1024u) : m;
-  const uint32_t sh = e ? e - 1u : 0u;
-  const unsigned long long mag = static_cast<unsigned long long>(sig) << sh;
-  s1 += (b & 0x8000u) ? -static_cast<long long>(mag) : static_cast<long long>(mag);
-  s2 += static_cast<u128>(static_cast<unsigned long long>(sig * sig)) << (2u * sh);
-}
-
-// mu and rstd from the exact sums, by the fixed sequence of correctly rounded
-// fp64 operations documented in sq.h.
-__device__ __forceinline__ void ln_finalize(long long s1, u128 s2, int64_t K, float eps,
-                                            float& mu, float& rstd) {
-  const double two64 = 18446744073709551616.0;
-  const double d1 = __ll2double_rn(s1);
-  const double d2 = __dadd_rn(
-      __dmul_rn(__ull2double_rn(static_cast<unsigned long long>(s2 >> 64)), two64),
-      __ull2double_rn(static_cast<unsigned long long>(s2)));
-  const double Kd = static_cast<double>(K);
-  const double mean = __ddiv_rn(d1, __dmul_rn(Kd, 16777216.0));
-  const double ex2 = __ddiv_rn(d2, __dmul_rn(Kd, 281474976710656.0));
-  double var = __dsub_rn(ex2, __dmul_rn(mean, mean));
-  if (var < 0.0) var = 0.0;
-  const double r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(var, static_cast<double>(eps))));
-  mu = __double2float_rn(mean);
-  rstd = __double2float_rn(r);
-}
-
-__device__ __forceinline__ int8_t quant_code(float x, float inv) {
-  // cvt.rni: nearest, ties to even; NaN -> 0; saturates, then the symmetric clamp
-  int q = __float2int_rn(__fmul_rn(x, inv));
-  q = q > 127 ? 127 : q;
-  q = q < -127 ? -127 : q;
-  return static_cast<int8_t>(q);
-}
-
-__device__ __forceinline__ float4 ld_f4(const float* p) {
-  return __ldg(reinterpret_cast<const float4*>(p));
-}
-
-__device__ __forceinline__ void load8f(const float* p, float (&o)[8]) {
-  const float4 a = ld_f4(p), b = ld_f4(p + 4);
-  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
-  o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
-}
 
 __device__ __forceinline__ uint32_t half_bits(const uint4& v, int j) {
   const uint32_t w = (j < 2) ? v.x : (j < 4) ? v.y : (j < 6) ? v.z : v.w;
@@ -92,19 +58,88 @@ __device__ __forceinline__ float bits_to_f(uint32_t b) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(b)));
 }
 
+__device__ __forceinline__ void chunk_sums(const uint4& v, Sums& s) {
+  const double kSplit = 824633720832.0;  // 1.5 * 2^39: (t + kSplit) - kSplit rounds t to 2^-13
+  double c1 = 0.0, c2h = 0.0, c2l = 0.0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const double d = static_cast<double>(bits_to_f(half_bits(v, j)));
+    c1 = __dadd_rn(c1, d);
+    const double t = __dmul_rn(d, d);
+    const double th = __dsub_rn(__dadd_rn(t, kSplit), kSplit);
+    c2h = __dadd_rn(c2h, th);
+    c2l = __dadd_rn(c2l, __dsub_rn(t, th));
+  }
+  s.s1 += __double2ll_rn(__dmul_rn(c1, 16777216.0));            // * 2^24
+  s.s2h += __double2ll_rn(__dmul_rn(c2h, 8192.0));              // * 2^13
+  s.s2l += __double2ll_rn(__dmul_rn(c2l, 281474976710656.0));   // * 2^48
+}
+
+__device__ __forceinline__ void warp_sum(Sums& s) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s.s1 += __shfl_xor_sync(0xffffffffu, s.s1, o);
+    s.s2h += __shfl_xor_sync(0xffffffffu, s.s2h, o);
+    s.s2l += __shfl_xor_sync(0xffffffffu, s.s2l, o);
+  }
+}
+
+// mu and rstd from the exact sums S1 = s1 and S2 = s2h * 2^35 + s2l, by the
+// fixed sequence of correctly rounded fp64 operations documented in sq.h.
+__device__ __forceinline__ void ln_finalize(const Sums& s, int64_t K, float eps, float& mu,
+                                            float& rstd) {
+  const u128 S2 = (static_cast<u128>(static_cast<unsigned long long>(s.s2h)) << 35) +
+                  static_cast<u128>(static_cast<__int128>(s.s2l));
+  const double two64 = 18446744073709551616.0;
+  const double d1 = __ll2double_rn(s.s1);
+  const double d2 = __dadd_rn(
+      __dmul_rn(__ull2double_rn(static_cast<unsigned long long>(S2 >> 64)), two64),
+      __ull2double_rn(static_cast<unsigned long long>(S2)));
+  const double Kd = static_cast<double>(K);
+  const double mean = __ddiv_rn(d1, __dmul_rn(Kd, 16777216.0));
+  const double ex2 = __ddiv_rn(d2, __dmul_rn(Kd, 281474976710656.0));
+  double var = __dsub_rn(ex2, __dmul_rn(mean, mean));
+  if (var < 0.0) var = 0.0;
+  const double r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(var, static_cast<double>(eps))));
+  mu = __double2float_rn(mean);
+  rstd = __double2float_rn(r);
+}
+
+// ------------------------------------------------------- element math ---
+__device__ __forceinline__ void load8f(const float* p, float (&o)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+  o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+
 // The 8 transformed fp32 values of chunk c (elements 8c..8c+7) of a row.
+__device__ __forceinline__ void unpack8(const uint4& v, float (&x)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[j]));
+    x[2 * j] = f.x;
+    x[2 * j + 1] = f.y;
+  }
+}
+
 template <int MODE>
 __device__ __forceinline__ void transform8(const uint4& v, int64_t c, const RowArgs& a, float mu,
                                            float rstd, float (&x)[8]) {
-#pragma unroll
-  for (int j = 0; j < 8; ++j) x[j] = bits_to_f(half_bits(v, j));
+  unpack8(v, x);
   const int64_t k0 = c * 8;
   if (MODE == MODE_WEIGHT) {
     if (a.vec) {
       float s[8];
       load8f(a.vec + k0, s);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) x[j] = __half2float(__float2half_rn(__fmul_rn(x[j], s[j])));
+      for (int j = 0; j < 8; j += 2) {
+        // fold diag(s) and round once to fp16, two lanes per instruction
+        const float2 f = __half22float2(__floats2half2_rn(__fmul_rn(x[j], s[j]), __fmul_rn(x[j + 1], s[j + 1])));
+        x[j] = f.x;
+        x[j + 1] = f.y;
+      }
     }
     return;
   }
@@ -128,210 +163,428 @@ __device__ __forceinline__ void transform8(const uint4& v, int64_t c, const RowA
   }
 }
 
-// NCH > 0: the thread's chunks of the row live in registers.
-// NCH == 0: chunks are re-read from global memory in every pass.
-template <int MODE, int NCH>
-__global__ void __launch_bounds__(kThreads) k_rows(const RowArgs a) {
-  constexpr bool REG = NCH > 0;
-  __shared__ RowShared sh;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t Kc = a.K / 8;
-  const int nch = REG ? NCH : static_cast<int>((Kc + kThreads - 1) / kThreads);
-  const bool use_ln = (MODE != MODE_WEIGHT) && a.gamma != nullptr;
+// Eight codes packed into 8 bytes.  p = x * inv (rounded), then
+// p + 1.5 * 2^23 rounds p to the nearest integer, ties to even, and leaves
+// that integer in the low mantissa bits: the low byte of the sum is the
+// two's-complement code (a NaN product gives byte 0).  No clamp is needed:
+// inv = RN(1 / RN(amax / 127)) and |x| <= amax bound |p| by 127 (1 + 3 * 2^-24)
+// < 127.5, so the rounded value is already inside [-127, 127] -- the same
+// codes as clamp(rint(p), -127, 127).
+__device__ __forceinline__ uint32_t quant4(float x0, float x1, float x2, float x3, float inv) {
+  const float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const uint32_t b0 = __float_as_uint(__fadd_rn(__fmul_rn(x0, inv), kMagic));
+  const uint32_t b1 = __float_as_uint(__fadd_rn(__fmul_rn(x1, inv), kMagic));
+  const uint32_t b2 = __float_as_uint(__fadd_rn(__fmul_rn(x2, inv), kMagic));
+  const uint32_t b3 = __float_as_uint(__fadd_rn(__fmul_rn(x3, inv), kMagic));
+  return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
 
-  // calibration: running column maxima of this thread's chunks
-  constexpr bool CALIB_REG = (MODE == MODE_CALIB) && REG && NCH <= 8;
-  float cmax[CALIB_REG ? NCH * 8 : 1];
-  if (CALIB_REG) {
-#pragma unroll
-    for (int i = 0; i < (CALIB_REG ? NCH * 8 : 1); ++i) cmax[i] = 0.0f;
-  }
+__device__ __forceinline__ uint2 pack8(const float (&x)[8], float inv) {
+  return make_uint2(quant4(x[0], x[1], x[2], x[3], inv), quant4(x[4], x[5], x[6], x[7], inv));
+}
 
-  uint4 v[REG ? NCH : 1];
-  for (int64_t r = blockIdx.x; r < a.rows; r += gridDim.x) {
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// =========================================================================
+// Warp per row (K <= 32 * 8 * NW).
+// =========================================================================
+template <int MODE, int NW>
+__global__ void __launch_bounds__(kWarpThreads) k_rows_warp(const RowArgs a) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * kWarpThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kWarpThreads) >> 5;
+  const int64_t Kc = a.K >> 3;
+  const bool use_ln = (MODE == MODE_ACT) && a.gamma != nullptr;
+  for (int64_t r = wid; r < a.rows; r += nwarps) {
     const uint4* src = reinterpret_cast<const uint4*>(a.x + r * a.ld);
-    if (REG) {
+    uint4 v[NW];
 #pragma unroll
-      for (int i = 0; i < (REG ? NCH : 1); ++i) {
-        const int64_t c = tid + static_cast<int64_t>(i) * kThreads;
-        v[i] = c < Kc ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-      }
+    for (int i = 0; i < NW; ++i) {
+      const int64_t c = lane + 32 * i;
+      v[i] = c < Kc ? ld_stream(src + c) : make_uint4(0, 0, 0, 0);
     }
-    auto chunk = [&](int i, int64_t c) -> uint4 {
-      if constexpr (REG) return v[i];
-      else return __ldg(src + c);
-    };
-
     float mu = 0.0f, rstd = 0.0f;
     if (use_ln) {
-      long long s1 = 0;
-      u128 s2 = 0;
+      Sums s{0, 0, 0};
 #pragma unroll
-      for (int i = 0; i < (REG ? NCH : 1); ++i) {
-        const int iters = REG ? 1 : nch;
-        for (int ii = 0; ii < iters; ++ii) {
-          const int ci = REG ? i : ii;
-          const int64_t c = tid + static_cast<int64_t>(ci) * kThreads;
-          if (c < Kc) {
-            const uint4 q = chunk(ci, c);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) stats_add(half_bits(q, j), s1, s2);
-          }
-        }
-      }
-      unsigned long long hi = static_cast<unsigned long long>(s2 >> 64);
-      unsigned long long lo = static_cast<unsigned long long>(s2);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const long long t1 = __shfl_xor_sync(0xffffffffu, s1, o);
-        const unsigned long long th = __shfl_xor_sync(0xffffffffu, hi, o);
-        const unsigned long long tl = __shfl_xor_sync(0xffffffffu, lo, o);
-        s1 += t1;
-        const u128 sum = ((static_cast<u128>(hi) << 64) | lo) + ((static_cast<u128>(th) << 64) | tl);
-        hi = static_cast<unsigned long long>(sum >> 64);
-        lo = static_cast<unsigned long long>(sum);
-      }
-      if (lane == 0) {
-        sh.s1[warp] = s1;
-        sh.s2_hi[warp] = hi;
-        sh.s2_lo[warp] = lo;
-      }
-      __syncthreads();
-      if (tid == 0) {
-        long long t1 = 0;
-        u128 t2 = 0;
-        for (int w = 0; w < kWarps; ++w) {
-          t1 += sh.s1[w];
-          t2 += (static_cast<u128>(sh.s2_hi[w]) << 64) | sh.s2_lo[w];
-        }
-        float m_, r_;
-        ln_finalize(t1, t2, a.K, a.eps, m_, r_);
-        sh.mu = m_;
-        sh.rstd = r_;
-      }
-      __syncthreads();
-      mu = sh.mu;
-      rstd = sh.rstd;
+      for (int i = 0; i < NW; ++i)
+        if (lane + 32 * i < Kc) chunk_sums(v[i], s);
+      warp_sum(s);
+      ln_finalize(s, a.K, a.eps, mu, rstd);
     }
-
-    if (MODE == MODE_CALIB) {
-#pragma unroll
-      for (int i = 0; i < (REG ? NCH : 1); ++i) {
-        const int iters = REG ? 1 : nch;
-        for (int ii = 0; ii < iters; ++ii) {
-          const int ci = REG ? i : ii;
-          const int64_t c = tid + static_cast<int64_t>(ci) * kThreads;
-          if (c < Kc) {
-            float x[8];
-            transform8<MODE>(chunk(ci, c), c, a, mu, rstd, x);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float ax = fabsf(x[j]);
-              if constexpr (CALIB_REG) {
-                cmax[ci * 8 + j] = fmaxf(cmax[ci * 8 + j], ax);
-              } else {
-                atomicMax(reinterpret_cast<int*>(a.amax) + c * 8 + j, __float_as_int(ax));
-              }
-            }
-          }
-        }
-      }
-      continue;
-    }
-
-    // row absmax of the transformed values
+    float x[NW][8];
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < (REG ? NCH : 1); ++i) {
-      const int iters = REG ? 1 : nch;
-      for (int ii = 0; ii < iters; ++ii) {
-        const int ci = REG ? i : ii;
-        const int64_t c = tid + static_cast<int64_t>(ci) * kThreads;
-        if (c < Kc) {
-          float x[8];
-          transform8<MODE>(chunk(ci, c), c, a, mu, rstd, x);
+    for (int i = 0; i < NW; ++i) {
+      const int64_t c = lane + 32 * i;
+      if (c < Kc) {
+        transform8<MODE>(v[i], c, a, mu, rstd, x[i]);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(x[j]));
-        }
+        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(x[i][j]));
       }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if (lane == 0) sh.mx[warp] = amax;
-    __syncthreads();
-    if (tid == 0) {
-      float m = 0.0f;
-      for (int w = 0; w < kWarps; ++w) m = fmaxf(m, sh.mx[w]);
-      const float sc = __fdiv_rn(m, 127.0f);
-      sh.inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
-      a.scale[r] = sc;
-    }
-    __syncthreads();
-    const float inv = sh.inv;
-
-    // quantize and store 8 codes (8 bytes) per chunk
+    const float sc = __fdiv_rn(amax, 127.0f);
+    const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+    if (lane == 0) a.scale[r] = sc;
     int8_t* dst = a.q + r * a.K;
 #pragma unroll
-    for (int i = 0; i < (REG ? NCH : 1); ++i) {
-      const int iters = REG ? 1 : nch;
-      for (int ii = 0; ii < iters; ++ii) {
-        const int ci = REG ? i : ii;
-        const int64_t c = tid + static_cast<int64_t>(ci) * kThreads;
-        if (c < Kc) {
-          float x[8];
-          transform8<MODE>(chunk(ci, c), c, a, mu, rstd, x);
-          uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            w0 |= (static_cast<uint32_t>(static_cast<uint8_t>(quant_code(x[j], inv)))) << (8 * j);
-            w1 |= (static_cast<uint32_t>(static_cast<uint8_t>(quant_code(x[j + 4], inv)))) << (8 * j);
-          }
-          *reinterpret_cast<uint2*>(dst + c * 8) = make_uint2(w0, w1);
-        }
-      }
-    }
-  }
-
-  if constexpr (CALIB_REG) {
-#pragma unroll
-    for (int i = 0; i < (CALIB_REG ? NCH : 1); ++i) {
-      const int64_t c = tid + static_cast<int64_t>(i) * kThreads;
-      if (c < Kc) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          atomicMax(reinterpret_cast<int*>(a.amax) + c * 8 + j, __float_as_int(cmax[i * 8 + j]));
-      }
+    for (int i = 0; i < NW; ++i) {
+      const int64_t c = lane + 32 * i;
+      if (c < Kc) *reinterpret_cast<uint2*>(dst + c * 8) = pack8(x[i], inv);
     }
   }
 }
 
-template <int MODE, int NCH>
-cudaError_t launch_nch(const RowArgs& a, const Ctx& c) {
-  static int occ[64] = {0};  // CTAs per SM, per device
-  int dev = c.device < 64 ? c.device : 63;
-  if (occ[dev] == 0) {
-    int n = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_rows<MODE, NCH>, kThreads, 0);
-    if (e != cudaSuccess) return e;
-    occ[dev] = n > 0 ? n : 1;
+// LayerNorm calibration, warp per row: per-lane running maxima of the
+// lane's columns in registers, merged per CTA in shared memory and across
+// the cluster of 8 CTAs through distributed shared memory.
+template <int NW>
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kWarpThreads)
+    k_calib_warp(const RowArgs a) {
+  extern __shared__ int colmax_s[];  // K float bits (non-negative floats order as ints)
+  cg::cluster_group cluster = cg::this_cluster();
+  const int lane = threadIdx.x & 31;
+  const int64_t Kc = a.K >> 3;
+  for (int64_t j = threadIdx.x; j < a.K; j += kWarpThreads) colmax_s[j] = 0;
+  __syncthreads();
+  griddep_wait();
+  griddep_launch_dependents();
+
+  float cm[NW][8];
+#pragma unroll
+  for (int i = 0; i < NW; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) cm[i][j] = 0.0f;
+
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * kWarpThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kWarpThreads) >> 5;
+  for (int64_t r = wid; r < a.rows; r += nwarps) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + r * a.ld);
+    uint4 v[NW];
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+      const int64_t c = lane + 32 * i;
+      v[i] = c < Kc ? ld_stream(src + c) : make_uint4(0, 0, 0, 0);
+    }
+    Sums s{0, 0, 0};
+#pragma unroll
+    for (int i = 0; i < NW; ++i)
+      if (lane + 32 * i < Kc) chunk_sums(v[i], s);
+    warp_sum(s);
+    float mu, rstd;
+    ln_finalize(s, a.K, a.eps, mu, rstd);
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+      const int64_t c = lane + 32 * i;
+      if (c < Kc) {
+        float x[8];
+        transform8<MODE_CALIB>(v[i], c, a, mu, rstd, x);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) cm[i][j] = fmaxf(cm[i][j], fabsf(x[j]));
+      }
+    }
   }
+#pragma unroll
+  for (int i = 0; i < NW; ++i) {
+    const int64_t c = lane + 32 * i;
+    if (c < Kc)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) atomicMax(colmax_s + c * 8 + j, __float_as_int(cm[i][j]));
+  }
+  __syncthreads();
+  cluster.sync();
+  const int64_t slice = (a.K + kCluster - 1) / kCluster;
+  const int64_t j0 = static_cast<int64_t>(cluster.block_rank()) * slice;
+  const int64_t j1 = j0 + slice < a.K ? j0 + slice : a.K;
+  for (int64_t j = j0 + threadIdx.x; j < j1; j += kWarpThreads) {
+    int m = 0;
+#pragma unroll
+    for (int q = 0; q < kCluster; ++q) m = max(m, cluster.map_shared_rank(colmax_s, q)[j]);
+    atomicMax(reinterpret_cast<int*>(a.amax) + j, m);
+  }
+  cluster.sync();  // peers may still be reading this CTA's maxima
+}
+
+// =========================================================================
+// CTA per row (K > 1024): T threads, NCH 16-byte chunks per thread held in
+// registers (NCH == 0: re-read from global in every pass), optionally
+// prefetching the CTA's next row while the current one is processed.
+// Per-row partial sums and maxima go through shared memory double-buffered
+// by row parity, so each row costs one barrier (two with the LayerNorm).
+// =========================================================================
+template <int T>
+struct RowSharedT {
+  long long s1[2][T / 32], s2h[2][T / 32], s2l[2][T / 32];
+  float mx[2][T / 32];
+};
+
+template <int MODE, int T, int NCH, bool PF, int CM>
+__device__ __forceinline__ void cta_rows(const RowArgs& a, RowSharedT<T>& sh, float (&cmax)[CM]) {
+  constexpr bool REG = NCH > 0;
+  constexpr bool KEEPX = REG && NCH <= 8;  // transformed values stay in registers
+  constexpr int W = T / 32;
+  constexpr bool CALIB_REG = (MODE == MODE_CALIB) && REG && CM == NCH * 8;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t Kc = a.K / 8;
+  const int nch = REG ? NCH : static_cast<int>((Kc + T - 1) / T);
+  const bool use_ln = (MODE != MODE_WEIGHT) && a.gamma != nullptr;
+
+  uint4 v[REG ? NCH : 1];
+  uint4 nv[(REG && PF) ? NCH : 1];
+  auto load_row = [&](int64_t row, uint4* dst) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + row * a.ld);
+#pragma unroll
+    for (int i = 0; i < (REG ? NCH : 1); ++i) {
+      const int64_t c = tid + static_cast<int64_t>(i) * T;
+      dst[i] = c < Kc ? ld_stream(src + c) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  if (REG && PF && static_cast<int64_t>(blockIdx.x) < a.rows) load_row(blockIdx.x, v);
+  int par = 0;
+  for (int64_t r = blockIdx.x; r < a.rows; r += gridDim.x, par ^= 1) {
+    if (REG && !PF) load_row(r, v);
+    if (REG && PF) {
+      const int64_t rn = r + gridDim.x;
+      if (rn < a.rows) load_row(rn, nv);
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + r * a.ld);
+    auto chunk = [&](int i, int64_t c) -> uint4 {
+      if constexpr (REG) return v[i];
+      else return __ldg(src + c);
+    };
+    const int iters = REG ? NCH : nch;
+
+    float mu = 0.0f, rstd = 0.0f;
+    if (use_ln) {
+      Sums s{0, 0, 0};
+#pragma unroll
+      for (int i = 0; i < iters; ++i) {
+        const int64_t c = tid + static_cast<int64_t>(i) * T;
+        if (c < Kc) chunk_sums(chunk(i, c), s);
+      }
+      warp_sum(s);
+      if (lane == 0) {
+        sh.s1[par][warp] = s.s1;
+        sh.s2h[par][warp] = s.s2h;
+        sh.s2l[par][warp] = s.s2l;
+      }
+      __syncthreads();
+      Sums t{0, 0, 0};
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        t.s1 += sh.s1[par][w];
+        t.s2h += sh.s2h[par][w];
+        t.s2l += sh.s2l[par][w];
+      }
+      ln_finalize(t, a.K, a.eps, mu, rstd);  // every thread, same inputs, same result
+    }
+
+    if (MODE == MODE_CALIB) {
+#pragma unroll
+      for (int i = 0; i < iters; ++i) {
+        const int64_t c = tid + static_cast<int64_t>(i) * T;
+        if (c < Kc) {
+          float x[8];
+          transform8<MODE>(chunk(i, c), c, a, mu, rstd, x);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float ax = fabsf(x[j]);
+            if constexpr (CALIB_REG) cmax[i * 8 + j] = fmaxf(cmax[i * 8 + j], ax);
+            else atomicMax(reinterpret_cast<int*>(a.amax) + c * 8 + j, __float_as_int(ax));
+          }
+        }
+      }
+    } else {
+      float amax = 0.0f;
+      float xs[KEEPX ? NCH : 1][8];
+#pragma unroll
+      for (int i = 0; i < iters; ++i) {
+        const int64_t c = tid + static_cast<int64_t>(i) * T;
+        if (c < Kc) {
+          float x[8];
+          transform8<MODE>(chunk(i, c), c, a, mu, rstd, x);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(x[j]));
+          if constexpr (KEEPX) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) xs[i][j] = x[j];
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      if (lane == 0) sh.mx[par][warp] = amax;
+      __syncthreads();
+      float m = 0.0f;
+#pragma unroll
+      for (int w = 0; w < W; ++w) m = fmaxf(m, sh.mx[par][w]);
+      const float sc = __fdiv_rn(m, 127.0f);
+      const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+      if (tid == 0) a.scale[r] = sc;
+      int8_t* dst = a.q + r * a.K;
+#pragma unroll
+      for (int i = 0; i < iters; ++i) {
+        const int64_t c = tid + static_cast<int64_t>(i) * T;
+        if (c < Kc) {
+          if constexpr (KEEPX) {
+            *reinterpret_cast<uint2*>(dst + c * 8) = pack8(xs[i], inv);
+          } else {
+            float x[8];
+            transform8<MODE>(chunk(i, c), c, a, mu, rstd, x);
+            *reinterpret_cast<uint2*>(dst + c * 8) = pack8(x, inv);
+          }
+        }
+      }
+    }
+    if (REG && PF) {
+#pragma unroll
+      for (int i = 0; i < (REG ? NCH : 1); ++i) v[i] = nv[i];
+    }
+  }
+}
+
+template <int MODE, int T, int NCH, bool PF>
+__global__ void __launch_bounds__(T) k_rows_cta(const RowArgs a) {
+  __shared__ RowSharedT<T> sh;
+  griddep_wait();
+  griddep_launch_dependents();
+  float none[1];
+  cta_rows<MODE, T, NCH, PF, 1>(a, sh, none);
+}
+
+// CTA-per-row calibration with register maxima, merged across a cluster of 8
+// CTAs through distributed shared memory.
+template <int T, int NCH>
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(T) k_calib_cta(const RowArgs a) {
+  __shared__ RowSharedT<T> sh;
+  extern __shared__ int colmax_s[];
+  cg::cluster_group cluster = cg::this_cluster();
+  float cmax[NCH * 8];
+#pragma unroll
+  for (int i = 0; i < NCH * 8; ++i) cmax[i] = 0.0f;
+  griddep_wait();
+  griddep_launch_dependents();
+  cta_rows<MODE_CALIB, T, NCH, true, NCH * 8>(a, sh, cmax);
+  const int64_t Kc = a.K / 8;
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    const int64_t c = threadIdx.x + static_cast<int64_t>(i) * T;
+    if (c < Kc)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) colmax_s[c * 8 + j] = __float_as_int(cmax[i * 8 + j]);
+  }
+  __syncthreads();
+  cluster.sync();
+  const int64_t slice = (a.K + kCluster - 1) / kCluster;
+  const int64_t j0 = static_cast<int64_t>(cluster.block_rank()) * slice;
+  const int64_t j1 = j0 + slice < a.K ? j0 + slice : a.K;
+  for (int64_t j = j0 + threadIdx.x; j < j1; j += T) {
+    int m = 0;
+#pragma unroll
+    for (int q = 0; q < kCluster; ++q) m = max(m, cluster.map_shared_rank(colmax_s, q)[j]);
+    atomicMax(reinterpret_cast<int*>(a.amax) + j, m);
+  }
+  cluster.sync();  // peers may still be reading this CTA's maxima
+}
+
+// Per-row global atomics: calibration with K too large for register maxima.
+__global__ void __launch_bounds__(kCtaThreads) k_calib_cta_atomic(const RowArgs a) {
+  __shared__ RowSharedT<kCtaThreads> sh;
+  griddep_wait();
+  griddep_launch_dependents();
+  float none[1];
+  cta_rows<MODE_CALIB, kCtaThreads, 0, false, 1>(a, sh, none);
+}
+
+// ------------------------------------------------------------- launch ----
+template <typename Kern>
+int occupancy(Kern k, int threads, size_t smem) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem) != cudaSuccess) {
+    cudaGetLastError();
+    n = 1;
+  }
+  return n > 0 ? n : 1;
+}
+
+template <int MODE, int NW>
+cudaError_t launch_warp(const RowArgs& a, const Ctx& c) {
+  static int occ[64] = {0};
+  const int dev = c.device < 64 ? c.device : 63;
+  if (occ[dev] == 0) occ[dev] = occupancy(k_rows_warp<MODE, NW>, kWarpThreads, 0);
+  int64_t grid = static_cast<int64_t>(c.num_sms) * occ[dev];
+  const int64_t need = (a.rows + 3) / 4;  // 4 row-warps per CTA
+  if (grid > need) grid = need;
+  return launch_pdl(k_rows_warp<MODE, NW>, dim3(static_cast<unsigned>(grid)), dim3(kWarpThreads), 0,
+                    c.stream, a);
+}
+
+template <int MODE, int T, int NCH, bool PF>
+cudaError_t launch_cta(const RowArgs& a, const Ctx& c) {
+  static int occ[64] = {0};
+  const int dev = c.device < 64 ? c.device : 63;
+  if (occ[dev] == 0) occ[dev] = occupancy(k_rows_cta<MODE, T, NCH, PF>, T, 0);
   int64_t grid = static_cast<int64_t>(c.num_sms) * occ[dev];
   if (grid > a.rows) grid = a.rows;
-  k_rows<MODE, NCH><<<static_cast<unsigned>(grid), kThreads, 0, c.stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(k_rows_cta<MODE, T, NCH, PF>, dim3(static_cast<unsigned>(grid)), dim3(T), 0, c.stream, a);
 }
 
 template <int MODE>
 cudaError_t launch_mode(const RowArgs& a, const Ctx& c) {
-  const int64_t per_thread = (a.K / 8 + kThreads - 1) / kThreads;  // chunks per thread
-  if (per_thread <= 1) return launch_nch<MODE, 1>(a, c);
-  if (per_thread <= 2) return launch_nch<MODE, 2>(a, c);
-  if (per_thread <= 4) return launch_nch<MODE, 4>(a, c);
-  if (per_thread <= 6) return launch_nch<MODE, 6>(a, c);
-  if (per_thread <= 8) return launch_nch<MODE, 8>(a, c);
-  if (per_thread <= 12) return launch_nch<MODE, 12>(a, c);
-  if (per_thread <= 24) return launch_nch<MODE, 24>(a, c);
-  return launch_nch<MODE, 0>(a, c);
+  const int64_t Kc = a.K / 8;
+  if (Kc <= 32) return launch_warp<MODE, 1>(a, c);
+  if (Kc <= 64) return launch_warp<MODE, 2>(a, c);
+  if (Kc <= 128) return launch_warp<MODE, 4>(a, c);
+  if (Kc <= 256) return launch_cta<MODE, 64, 4, true>(a, c);
+  if (Kc <= 512) return launch_cta<MODE, 128, 4, true>(a, c);
+  if (Kc <= 1024) return launch_cta<MODE, 256, 4, true>(a, c);
+  if (Kc <= 1536) return launch_cta<MODE, 256, 6, true>(a, c);
+  if (Kc <= 2048) return launch_cta<MODE, 256, 8, true>(a, c);
+  if (Kc <= 3072) return launch_cta<MODE, 256, 12, false>(a, c);
+  if (Kc <= 6144) return launch_cta<MODE, 256, 24, false>(a, c);
+  return launch_cta<MODE, 256, 0, false>(a, c);
+}
+
+// Calibration grids: a multiple of the cluster size.
+int64_t calib_grid(int64_t want, int64_t cap) {
+  cap = (cap / kCluster) * kCluster;
+  if (cap < kCluster) cap = kCluster;
+  if (want > cap) want = cap;
+  return ((want + kCluster - 1) / kCluster) * kCluster;
+}
+
+template <int NW>
+cudaError_t launch_calib_warp(const RowArgs& a, const Ctx& c) {
+  const size_t smem = static_cast<size_t>(a.K) * 4;
+  const int64_t grid = calib_grid((a.rows + 3) / 4, 4 * static_cast<int64_t>(c.num_sms));
+  return launch_pdl(k_calib_warp<NW>, dim3(static_cast<unsigned>(grid)), dim3(kWarpThreads), smem,
+                    c.stream, a);
+}
+
+template <int T, int NCH>
+cudaError_t launch_calib_cta(const RowArgs& a, const Ctx& c) {
+  const size_t smem = static_cast<size_t>(a.K) * 4;
+  static bool attr[64] = {false};
+  const int dev = c.device < 64 ? c.device : 63;
+  if (!attr[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_calib_cta<T, NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         NCH * 8 * T * 4);
+    if (e != cudaSuccess) return e;
+    attr[dev] = true;
+  }
+  // one or two rows per CTA, at most a few CTAs per SM
+  const int64_t grid = calib_grid((a.rows + 1) / 2, 4 * static_cast<int64_t>(c.num_sms));
+  return launch_pdl(k_calib_cta<T, NCH>, dim3(static_cast<unsigned>(grid)), dim3(T), smem, c.stream, a);
 }
 
 }  // namespace
@@ -343,7 +596,20 @@ cudaError_t launch_quantize_weight(const RowArgs& a, const Ctx& c) {
 }
 
 cudaError_t launch_calibrate_ln(const RowArgs& a, const Ctx& c) {
-  return launch_mode<MODE_CALIB>(a, c);
+  const int64_t Kc = a.K / 8;
+  if (Kc <= 32) return launch_calib_warp<1>(a, c);
+  if (Kc <= 64) return launch_calib_warp<2>(a, c);
+  if (Kc <= 128) return launch_calib_warp<4>(a, c);
+  if (Kc <= 256) return launch_calib_cta<64, 4>(a, c);
+  if (Kc <= 512) return launch_calib_cta<128, 4>(a, c);
+  if (Kc <= 1024) return launch_calib_cta<256, 4>(a, c);
+  if (Kc <= 2048) return launch_calib_cta<256, 8>(a, c);
+  static int occ[64] = {0};
+  const int dev = c.device < 64 ? c.device : 63;
+  if (occ[dev] == 0) occ[dev] = occupancy(k_calib_cta_atomic, kCtaThreads, 0);
+  int64_t grid = static_cast<int64_t>(c.num_sms) * occ[dev];
+  if (grid > a.rows) grid = a.rows;
+  return launch_pdl(k_calib_cta_atomic, dim3(static_cast<unsigned>(grid)), dim3(kCtaThreads), 0, c.stream, a);
 }
 
 }  // namespace sq

@@ -155,7 +155,8 @@ sq_status linear_impl(const int8_t* xq, const float* x_scale, const int8_t* wq,
     if (workspace == nullptr || ws_bytes < need || !aligned16(workspace)) return SQ_ERR_WORKSPACE;
     return launched(launch_gemm_splitk(g, ctx));
   }
-  return launched(launch_gemm_tiled(g, ctx));
+  // 256-row tiles once the token count fills them; 128-row tiles below that
+  return launched(M > 128 ? launch_gemm_wide(g, ctx) : launch_gemm_tiled(g, ctx));
 }
 
 }  // namespace

@@ -9,6 +9,24 @@
 
 namespace sq {
 
+// Launch with programmatic stream serialization (see griddep_wait): the
+// kernel's launch and prologue overlap the tail of the previous kernel.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Per-call launch context filled in by the ABI layer.
 struct Ctx {
   int device;
@@ -58,7 +76,8 @@ struct GemmArgs {
   size_t ws_bytes;
 };
 
-cudaError_t launch_gemm_tiled(const GemmArgs& g, const Ctx& c);
+cudaError_t launch_gemm_tiled(const GemmArgs& g, const Ctx& c);  // 128 x 256 tiles
+cudaError_t launch_gemm_wide(const GemmArgs& g, const Ctx& c);   // 256 x 256 tiles, persistent
 cudaError_t launch_gemm_splitk(const GemmArgs& g, const Ctx& c);
 size_t splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
 

@@ -206,6 +206,20 @@ __host__ __device__ constexpr uint32_t idesc_i8(int m, int n) {
          (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with programmatic stream serialization: it may be scheduled while the
+// previous kernel on the stream is still running, runs only its prologue
+// (shared-memory and barrier setup, TMEM allocation), and waits here, before
+// its first global-memory access, until the previous grid has completed and
+// its writes are visible.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next kernel on the stream be scheduled (it still waits in
+// griddep_wait for this grid to complete).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Named barrier among `count` threads (ids 1..15; 0 is __syncthreads).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
