@@ -155,8 +155,9 @@ class Plan:
     """Device buffers and prepared C-ABI calls of one step (argument
     marshalling done once, so the per-step host cost is a few C calls)."""
 
-    def __init__(self, wl, M, rank, device, sq, torch):
+    def __init__(self, wl, M, rank, device, sq, torch, two_streams=False):
         self.torch, self.sq, self.wl, self.M = torch, sq, wl, M
+        self.two_streams = two_streams
         dev = device
         data_wl = sq_inputs.with_(wl, seed=wl.seed + 1000 * rank)  # this rank's tokens
         w = sq_inputs.weight(wl)
@@ -180,43 +181,116 @@ class Plan:
         self.sx = torch.empty(M, **f32)
         self.y = torch.empty((M, N), dtype=torch.float16, device=dev)
         self.ws = sq.new_workspace(M, N, K, device=dev)
-        L = sq._L
+        self.main = torch.cuda.current_stream()
+        self.side = torch.cuda.Stream()
+        self.runtime_inv_s = None if g is not None else self.inv_s
+        self.ws_bytes = 0 if self.ws is None else self.ws.numel()
+        self.calib_rows = calib.shape[0]
+        self.bind(self.main)
+        self.launches_per_step = len(self.calls)
+
+    def bind(self, main_stream):
+        """(Re)build the prepared C calls for the given main stream."""
+        torch, wl, M = self.torch, self.wl, self.M
+        K, N = wl.K, wl.N
+        L = self.sq._L
         p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
-        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        stream = ctypes.c_void_p(main_stream.cuda_stream)
+        side = ctypes.c_void_p(self.side.cuda_stream) if self.two_streams else stream
         eps = ctypes.c_float(1e-5)
-        runtime_inv_s = None if g is not None else self.inv_s
-        ws_bytes = 0 if self.ws is None else self.ws.numel()
+        runtime_inv_s, ws_bytes = self.runtime_inv_s, self.ws_bytes
         self.calls = [
-            ("calibrate_x", L.sq_calibrate_absmax, (p(self.calib), calib.shape[0], K, K, p(self.gamma),
+            ("calibrate_x", L.sq_calibrate_absmax, (p(self.calib), self.calib_rows, K, K, p(self.gamma),
                                                     p(self.beta), eps, p(self.amax_x), stream)),
             ("calibrate_w", L.sq_calibrate_absmax, (p(self.w), N, K, K, None, None, eps, p(self.amax_w),
-                                                    stream)),
+                                                    side)),
             ("smooth_fold", L.sq_smooth_fold, (p(self.amax_x), p(self.amax_w), K, ctypes.c_float(wl.alpha),
                                                p(self.s), p(self.inv_s), p(self.gamma), p(self.beta),
                                                p(self.gamma_f), p(self.beta_f), None, None, 0, stream)),
             ("quantize_weight", L.sq_quantize_weight, (p(self.w), N, K, p(self.s), p(self.wq), p(self.sw),
-                                                       stream)),
+                                                       side)),
             ("ln_quant_act", L.sq_ln_quant_act, (p(self.h), M, K, K, p(self.gamma_f), p(self.beta_f),
                                                  p(runtime_inv_s), eps, p(self.xq), p(self.sx), stream)),
             ("w8a8_linear", L.sq_w8a8_linear, (p(self.xq), p(self.sx), p(self.wq), p(self.sw), p(self.bias),
                                                p(self.y), M, N, K, p(self.ws), ws_bytes, stream)),
         ]
-        self.launches_per_step = len(self.calls)
 
     def step(self, events=None, allreduce=None):
-        """Run one step; events (if given) is a list of len(calls)+1 CUDA events
-        recorded before each call and after the last."""
+        """Run one step.  With two streams the independent stages overlap:
+            main: calibrate_x            | smooth_fold | ln_quant_act    | w8a8_linear
+            side:          calibrate_w   |             | quantize_weight |
+        with events joining them where a stage needs the other stream's output.
+        With `events` (one per call + 1), the stages instead run one after the
+        other on the main stream timing order (for the per-stage breakdown)."""
+        torch = self.torch
         self.amax.zero_()
-        for i, (name, fn, args) in enumerate(self.calls):
-            if events is not None:
-                events[i].record()
-            if name == "smooth_fold" and allreduce is not None:
-                allreduce(self.amax_x)
-            st = fn(*args)
-            if st != 0:
-                raise RuntimeError(f"{name}: status {st}")
-        if events is not None:
-            events[-1].record()
+        if events is not None:  # serialized, one event before each call
+            for i, (name, fn, args) in enumerate(self.calls):
+                events[i].record(self.main)
+                if name in ("calibrate_w", "quantize_weight"):
+                    self.side.wait_stream(self.main)
+                if name == "smooth_fold" and allreduce is not None:
+                    allreduce(self.amax_x)
+                self._call(name, fn, args)
+                if name in ("calibrate_w", "quantize_weight"):
+                    self.main.wait_stream(self.side)
+            events[-1].record(self.main)
+            return
+        if not self.two_streams:  # one stream: consecutive kernels overlap their launches (PDL)
+            for name, fn, args in self.calls:
+                if name == "smooth_fold" and allreduce is not None:
+                    allreduce(self.amax_x)
+                self._call(name, fn, args)
+            return
+        c = dict((n, (fn, args)) for n, fn, args in self.calls)
+        self.side.wait_stream(self.main)               # amax zeroed, previous step done
+        self._call("calibrate_x", *c["calibrate_x"])
+        self._call("calibrate_w", *c["calibrate_w"])   # side
+        self.main.wait_stream(self.side)
+        if allreduce is not None:
+            allreduce(self.amax_x)
+        self._call("smooth_fold", *c["smooth_fold"])
+        self.side.wait_stream(self.main)
+        self._call("quantize_weight", *c["quantize_weight"])  # side
+        self._call("ln_quant_act", *c["ln_quant_act"])
+        self.main.wait_stream(self.side)
+        self._call("w8a8_linear", *c["w8a8_linear"])
+
+    def capture(self, world):
+        """Capture the step into CUDA graphs: one graph for N = 1; for N > 1 two
+        graphs around the NCCL all-reduce, which runs eagerly between them."""
+        torch = self.torch
+        cap = torch.cuda.Stream()
+        cap.wait_stream(self.main)
+        names = [c[0] for c in self.calls]
+        cut = names.index("smooth_fold") if world > 1 else len(names)
+        segs = [names[:cut], names[cut:]] if world > 1 else [names]
+        self.graphs = []
+        with torch.cuda.stream(cap):
+            self.bind(cap)
+            for i, seg in enumerate(segs):
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=cap):
+                    if i == 0:
+                        self.amax.zero_()
+                    for name, fn, args in self.calls:
+                        if name in seg:
+                            self._call(name, fn, args)
+                self.graphs.append(gr)
+        self.bind(self.main)
+        self.main.wait_stream(cap)
+
+    def replay(self, allreduce=None):
+        self.graphs[0].replay()
+        if len(self.graphs) > 1:
+            allreduce(self.amax_x)
+            self.graphs[1].replay()
+
+    @staticmethod
+    def _call(name, fn, args):
+        st = fn(*args)
+        if st != 0:
+            raise RuntimeError(f"{name}: status {st}")
 
 
 def run_gpu(args):
@@ -239,7 +313,7 @@ def run_gpu(args):
 
     wl = sq_inputs.WORKLOADS[args.workload]
     M = args.m if args.m else wl.M
-    plan = Plan(wl, M, rank, device, sq, torch)
+    plan = Plan(wl, M, rank, device, sq, torch, two_streams=args.streams == 2)
     allreduce = None
     if world > 1:
         allreduce = lambda t: dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -261,6 +335,19 @@ def run_gpu(args):
     torch.cuda.synchronize()
     if sq.sq_poll_status() != 0:
         raise RuntimeError("device wait timed out during warm-up")
+    use_graph = not args.no_graph and plan.two_streams is False
+    graph_note = None
+    if use_graph:
+        try:
+            plan.capture(world)
+            for _ in range(3):
+                flush()
+                plan.replay(allreduce)
+            torch.cuda.synchronize()
+        except RuntimeError as e:  # capture refused: time the eager launches instead
+            use_graph, graph_note = False, f"capture failed: {str(e)[:200]}"
+            torch.cuda.synchronize()
+    run_step = (lambda: plan.replay(allreduce)) if use_graph else (lambda: plan.step(None, allreduce))
 
     # timed region: events only at step boundaries, so consecutive kernels of a
     # step overlap their launches (programmatic dependent launch)
@@ -278,7 +365,7 @@ def run_gpu(args):
     for i in range(args.steps):
         flush()
         events[i][0].record()
-        plan.step(None, allreduce)
+        run_step()
         events[i][1].record()
     torch.cuda.synchronize()
     if world > 1:
@@ -354,7 +441,9 @@ def run_gpu(args):
             "data": "synthetic (seeded PCG64, OPT-shaped with persistent outlier channels)",
             "config": {"workload": DESCR[args.workload] + ("" if M == wl.M else f" (M={M})"),
                        "M": M, "N": wl.N, "K": wl.K, "calib_tokens": wl.calib, "alpha": wl.alpha,
-                       "step": STEP, "parallelism": f"dp{world}",
+                       "step": STEP, "streams": args.streams, "cuda_graph": use_graph,
+                       **({"cuda_graph_note": graph_note} if graph_note else {}),
+                       "parallelism": f"dp{world}",
                        "l2": "flushed before every step (256 MiB write, then 256 MiB read so no dirty "
                              "lines remain), outside the timed events",
                        "timing": "CUDA events at the boundaries of every step, summed over steps, max over "
@@ -363,7 +452,10 @@ def run_gpu(args):
             "roofline": roof,
             "stage_us": {k: round(v, 2) for k, v in stage_us.items()},
             "gpu_launches": plan.launches_per_step * args.steps,
-            "launch": "every libsq kernel with programmatic dependent launch (prologue overlaps the previous kernel)",
+            "launch": ("the step captured once into a CUDA graph and replayed (the C-ABI calls are "
+                       "capture-safe); every libsq kernel uses programmatic dependent launch"
+                       if use_graph else "eager C-ABI calls; every libsq kernel uses programmatic "
+                       "dependent launch"),
             "clocks": clocks,
             "e2e": e2e,
         }
@@ -541,6 +633,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--stage-steps", type=int, default=300, help="steps of the per-stage timing loop")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the step's kernels eagerly instead of replaying a captured CUDA graph")
+    ap.add_argument("--streams", type=int, choices=[1, 2], default=1,
+                    help="2: run the independent stages of a step on two streams")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU work")
     ap.add_argument("--ref-budget", type=float, default=150.0, help="seconds for the reference arm")

@@ -14,9 +14,12 @@
 //   warp 1      TMEM allocation; lane 0 issues the MMAs
 //   warps 2-9   epilogue: warp w reads TMEM lane quarter w % 4 (32 token
 //               rows of each accumulator) for column half (w - 2) / 4, then
-//               y = fp16((acc * sx[t]) * sw[n] + bias[n])
+//               y = fp16((acc * sx[t]) * sw[n] + bias[n]); each 32 x 32 block
+//               is staged in shared memory and written by a TMA store
 // Every mbarrier wait is bounded; a wait that runs out records a timeout, the
 // CTA drains what it issued, frees TMEM and returns.
+#include <string.h>
+
 #include "sq_internal.h"
 #include "sq_ptx.cuh"
 #include "sq_tmap.h"
@@ -33,7 +36,9 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int A_BYTES = BM * BK;              // 32 KB
 constexpr int B_BYTES = BN * BK;              // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int CTRL = STAGES * STAGE_BYTES;
+constexpr int STG = STAGES * STAGE_BYTES;     // per-epilogue-warp output staging, 2 KB each
+constexpr int STG_BYTES = 2048;               // 32 rows x 32 fp16, 64-byte swizzle
+constexpr int CTRL = STG + kEpiWarps * STG_BYTES;
 constexpr int NBARS = 2 * STAGES + 3;         // full, empty, acc_full, acc_empty, drain
 constexpr int SLOT = CTRL + NBARS * 8;        // TMEM address, abort flag, decision[2]
 constexpr int VEC = SLOT + 16;                // sw[BN], bias[BN]
@@ -44,7 +49,8 @@ constexpr uint32_t TMEM_COLS = 512;
 template <bool OUT_I32>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_wide(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const GemmArgs g, int tiles_m, int tiles, uint32_t* status, uint64_t budget) {
+                const __grid_constant__ CUtensorMap tmY, const GemmArgs g, int tiles_m, int tiles,
+                int tma_store, uint32_t* status, uint64_t budget) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -152,6 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int et = threadIdx.x - 64;
     const int q = warp & 3;            // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;  // column half of the tile
+    const uint32_t stg = sbase + STG + static_cast<uint32_t>(warp - 2) * STG_BYTES;
     const bool vec_ok = (g.N % 8) == 0;
     int tl = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tl) {
@@ -162,6 +169,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         sw_s[et] = n < g.N ? g.sw[n] : 0.0f;
         bias_s[et] = (g.bias != nullptr && n < g.N) ? __half2float(g.bias[n]) : 0.0f;
       }
+      float sxr[2] = {0.0f, 0.0f};
+      if (!OUT_I32) {
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          const int64_t row = m0 + 128 * a + 32 * q + lane;
+          sxr[a] = row < g.M ? g.sx[row] : 0.0f;
+        }
+      }
       named_bar_sync(1, 32 * kEpiWarps);
       mbar_wait(accf_bar, static_cast<uint32_t>(tl & 1), budget, status, abort_flag);
       // one thread decides whether to stop and broadcasts it (double-buffered by
@@ -170,48 +185,84 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar_sync(1, 32 * kEpiWarps);
       if (decision[tl & 1]) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int a = 0; a < 2; ++a) {
-        const int64_t row = m0 + 128 * a + 32 * q + lane;
-        const bool row_ok = row < g.M;
-        const float sxr = (!OUT_I32 && row_ok) ? g.sx[row] : 0.0f;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          const int cl = 128 * half + 32 * cc;  // column within the tile
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(256 * a + cl), v);
-          tmem_ld_wait();
-          const int64_t col0 = n0 + cl;
-          if (!row_ok || col0 >= g.N) continue;
-          if (OUT_I32) {
+
+      // 8 chunks of 32 columns: (accumulator a, column group cc); the TMEM load
+      // of the next chunk is in flight while the current one is converted
+      auto taddr = [&](int idx) {
+        return tmem + (static_cast<uint32_t>(32 * q) << 16) +
+               static_cast<uint32_t>(256 * (idx >> 2) + 128 * half + 32 * (idx & 3));
+      };
+      auto emit = [&](int idx, uint32_t (&v)[32]) {
+        const int a = idx >> 2;
+        const int cl = 128 * half + 32 * (idx & 3);  // column within the tile
+        const int64_t row0 = m0 + 128 * a + 32 * q;  // first row of this warp's block
+        const int64_t row = row0 + lane;
+        const int64_t col0 = n0 + cl;
+        if constexpr (OUT_I32) {
+          if (row < g.M && col0 < g.N) {
             int32_t* dst = g.acc + row * g.N + col0;
             for (int j = 0; j < 32; ++j)
               if (col0 + j < g.N) dst[j] = static_cast<int32_t>(v[j]);
+          }
+          return;
+        } else {
+        __align__(16) __half h[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          float f = dequant_f32(static_cast<int32_t>(v[j]), sxr[a], sw_s[cl + j]);
+          if (g.bias != nullptr) f = __fadd_rn(f, bias_s[cl + j]);
+          h[j] = __float2half_rn(f);
+        }
+        if (tma_store) {
+          // stage the 32 x 32 block in the 64-byte-swizzled image and let one
+          // TMA store write it (rows/columns outside y are skipped by the TMA)
+          if (lane == 0) bulk_wait_group_read0();  // previous store done reading
+          __syncwarp();
+          const uint4* hv = reinterpret_cast<const uint4*>(h);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t addr = stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) * 16);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(hv[c].x), "r"(hv[c].y),
+                         "r"(hv[c].z), "r"(hv[c].w)
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < g.M && col0 < g.N) {
+            tma_store_2d(&tmY, stg, static_cast<int32_t>(col0), static_cast<int32_t>(row0));
+            bulk_commit_group();
+          }
+        } else if (row < g.M && col0 < g.N) {
+          __half* dst = g.y + row * g.N + col0;
+          if (vec_ok && col0 + 32 <= g.N) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              reinterpret_cast<uint4*>(dst)[j] = reinterpret_cast<const uint4*>(h)[j];
           } else {
-            __half h[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              float f = dequant_f32(static_cast<int32_t>(v[j]), sxr, sw_s[cl + j]);
-              if (g.bias != nullptr) f = __fadd_rn(f, bias_s[cl + j]);
-              h[j] = __float2half_rn(f);
-            }
-            __half* dst = g.y + row * g.N + col0;
-            if (vec_ok && col0 + 32 <= g.N) {
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                reinterpret_cast<uint4*>(dst)[j] = reinterpret_cast<const uint4*>(h)[j];
-            } else {
-              for (int j = 0; j < 32; ++j)
-                if (col0 + j < g.N) dst[j] = h[j];
-            }
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < g.N) dst[j] = h[j];
           }
         }
+        }
+      };
+      uint32_t va[32], vb[32];
+      tmem_ld_32x32b_x32(taddr(0), va);
+      tmem_ld_wait_regs(va);
+#pragma unroll 1
+      for (int idx = 0; idx < 8; idx += 2) {
+        tmem_ld_32x32b_x32(taddr(idx + 1), vb);
+        emit(idx, va);
+        tmem_ld_wait_regs(vb);
+        if (idx + 2 < 8) tmem_ld_32x32b_x32(taddr(idx + 2), va);
+        emit(idx + 1, vb);
+        tmem_ld_wait_regs(va);
       }
       // every epilogue thread has read its TMEM columns: release the accumulators
       tc_fence_before();
       named_bar_sync(1, 32 * kEpiWarps);
       if (et == 0) mbar_arrive(acce_bar);
     }
+    if (lane == 0) bulk_wait_group0();  // this warp's output stores are complete
   }
 
   // teardown: after an abort, wait (bounded) for the MMAs and TMA loads this
@@ -247,15 +298,19 @@ cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmY;
   if (!make_tmap_i8(&tmA, g.xq, g.K, g.M, BK, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_i8(&tmB, g.wq, g.K, g.N, BK, BN)) return cudaErrorInvalidValue;
+  // TMA stores need 16-byte row strides (N % 8 == 0); otherwise direct stores
+  int tma_store = (!OUT_I32 && g.N % 8 == 0) ? 1 : 0;
+  if (tma_store && !make_tmap_f16_out(&tmY, g.y, g.N, g.M)) return cudaErrorInvalidValue;
+  if (!tma_store) memset(&tmY, 0, sizeof(tmY));
   const int tiles_m = static_cast<int>((g.M + BM - 1) / BM);
   const int tiles_n = static_cast<int>((g.N + BN - 1) / BN);
   const int tiles = tiles_m * tiles_n;
   const int grid = tiles < c.num_sms ? tiles : c.num_sms;
-  return launch_pdl(k_gemm_wide<OUT_I32>, dim3(grid), dim3(kThreads), SMEM, c.stream, tmA, tmB, g, tiles_m,
-                    tiles, c.status, c.budget_ns);
+  return launch_pdl(k_gemm_wide<OUT_I32>, dim3(grid), dim3(kThreads), SMEM, c.stream, tmA, tmB, tmY, g,
+                    tiles_m, tiles, tma_store, c.status, c.budget_ns);
 }
 
 }  // namespace

@@ -326,12 +326,15 @@ template <int T>
 struct RowSharedT {
   long long s1[2][T / 32], s2h[2][T / 32], s2l[2][T / 32];
   float mx[2][T / 32];
+  float mu[2], rstd[2];
 };
 
 template <int MODE, int T, int NCH, bool PF, int CM>
 __device__ __forceinline__ void cta_rows(const RowArgs& a, RowSharedT<T>& sh, float (&cmax)[CM]) {
   constexpr bool REG = NCH > 0;
-  constexpr bool KEEPX = REG && NCH <= 8;  // transformed values stay in registers
+  // weights: the folded values stay in registers between the two passes;
+  // activations recompute them (registers go to occupancy instead)
+  constexpr bool KEEPX = REG && NCH <= 8 && MODE == MODE_WEIGHT;
   constexpr int W = T / 32;
   constexpr bool CALIB_REG = (MODE == MODE_CALIB) && REG && CM == NCH * 8;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -379,14 +382,24 @@ __device__ __forceinline__ void cta_rows(const RowArgs& a, RowSharedT<T>& sh, fl
         sh.s2l[par][warp] = s.s2l;
       }
       __syncthreads();
-      Sums t{0, 0, 0};
+      if (warp == 0) {  // one warp turns the sums into mu / rstd and broadcasts them
+        Sums t{0, 0, 0};
 #pragma unroll
-      for (int w = 0; w < W; ++w) {
-        t.s1 += sh.s1[par][w];
-        t.s2h += sh.s2h[par][w];
-        t.s2l += sh.s2l[par][w];
+        for (int w = 0; w < W; ++w) {
+          t.s1 += sh.s1[par][w];
+          t.s2h += sh.s2h[par][w];
+          t.s2l += sh.s2l[par][w];
+        }
+        float m_, r_;
+        ln_finalize(t, a.K, a.eps, m_, r_);
+        if (lane == 0) {
+          sh.mu[par] = m_;
+          sh.rstd[par] = r_;
+        }
       }
-      ln_finalize(t, a.K, a.eps, mu, rstd);  // every thread, same inputs, same result
+      __syncthreads();
+      mu = sh.mu[par];
+      rstd = sh.rstd[par];
     }
 
     if (MODE == MODE_CALIB) {

@@ -2,6 +2,8 @@
 // device / architecture checks, the per-device status word of the bounded
 // device waits, and dispatch to the kernels.  No entry point allocates
 // device memory.
+#include <stdlib.h>
+
 #include <atomic>
 #include <mutex>
 
@@ -162,6 +164,14 @@ sq_status linear_impl(const int8_t* xq, const float* x_scale, const int8_t* wq,
 }  // namespace
 
 int call_context(void* stream, Ctx* ctx) { return current_ctx(stream, ctx); }
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("SQ_NO_PDL");
+    return !(v && v[0] == '1');
+  }();
+  return on;
+}
 
 void* tensor_map_encoder() {
   std::call_once(g_encoder_once, [] {

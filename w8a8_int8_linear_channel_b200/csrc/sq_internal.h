@@ -9,6 +9,10 @@
 
 namespace sq {
 
+// Programmatic dependent launch is on unless the environment sets
+// SQ_NO_PDL=1 (read once per process).
+bool pdl_enabled();
+
 // Launch with programmatic stream serialization (see griddep_wait): the
 // kernel's launch and prologue overlap the tail of the previous kernel.
 template <typename... KArgs, typename... Args>
@@ -23,7 +27,7 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 

@@ -10,9 +10,11 @@
 namespace sq {
 
 // rows x K int8 matrix at `base` (row stride K bytes); boxes of
-// box_k (bytes along K, <= 128 for the 128-byte swizzle) x box_rows rows.
+// box_k bytes along K x box_rows rows, stored with the swizzle whose span is
+// box_k bytes (128 -> 128-byte swizzle, 64 -> 64-byte swizzle).
 inline bool make_tmap_i8(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows,
                          uint32_t box_k, uint32_t box_rows) {
+  const CUtensorMapSwizzle swz = box_k == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   auto encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
   if (!encode) return false;
   cuuint64_t dims[2] = {K, rows};
@@ -20,8 +22,25 @@ inline bool make_tmap_i8(CUtensorMap* map, const void* base, uint64_t K, uint64_
   cuuint32_t box[2] = {box_k, box_rows};
   cuuint32_t elem[2] = {1, 1};
   CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
-                      box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// rows x cols fp16 matrix (row stride cols * 2 bytes, a multiple of 16), boxes
+// of 32 x 32 elements stored with the 64-byte swizzle (the shared-memory
+// image is 32 rows of 64 bytes, 16-byte chunk c of row r at chunk
+// c ^ ((r >> 1) & 3)).
+inline bool make_tmap_f16_out(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows) {
+  auto encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
+  if (!encode) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t elem[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
+                      box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                      CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
