@@ -36,13 +36,14 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int A_BYTES = BM * BK;              // 32 KB
 constexpr int B_BYTES = BN * BK;              // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int STG = STAGES * STAGE_BYTES;     // per-epilogue-warp output staging, 2 KB each
-constexpr int STG_BYTES = 2048;               // 32 rows x 32 fp16, 64-byte swizzle
-constexpr int CTRL = STG + kEpiWarps * STG_BYTES;
+constexpr int STG = STAGES * STAGE_BYTES;     // per-epilogue-warp output staging
+constexpr int STG_BYTES = 2048;               // one 32 rows x 32 fp16 block, 64-byte swizzle
+constexpr int STG_WARP = 2 * STG_BYTES;       // double-buffered per warp
+constexpr int CTRL = STG + kEpiWarps * STG_WARP;
 constexpr int NBARS = 2 * STAGES + 3;         // full, empty, acc_full, acc_empty, drain
 constexpr int SLOT = CTRL + NBARS * 8;        // TMEM address, abort flag, decision[2]
-constexpr int VEC = SLOT + 16;                // sw[BN], bias[BN]
-constexpr int SMEM_BYTES = VEC + 2 * BN * 4;
+constexpr int VEC = SLOT + 16;                // sw[BN] fp32, bias[BN] fp16 of the current tile
+constexpr int SMEM_BYTES = VEC + BN * 4 + BN * 2;
 constexpr size_t SMEM = SMEM_BYTES + 1024;    // slack for 1024-byte alignment
 constexpr uint32_t TMEM_COLS = 512;
 
@@ -65,7 +66,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* decision = tmem_slot + 2;  // [2]
   float* sw_s = reinterpret_cast<float*>(smem + VEC);
-  float* bias_s = sw_s + BN;
+  __half* bias_s = reinterpret_cast<__half*>(smem + VEC + BN * 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KB = static_cast<int>((g.K + BK - 1) / BK);
@@ -158,7 +159,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int et = threadIdx.x - 64;
     const int q = warp & 3;            // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;  // column half of the tile
-    const uint32_t stg = sbase + STG + static_cast<uint32_t>(warp - 2) * STG_BYTES;
+    const uint32_t stg0 = sbase + STG + static_cast<uint32_t>(warp - 2) * STG_WARP;
+    int nst = 0;  // blocks this warp has staged (selects the buffer; two stores may be in flight)
     const bool vec_ok = (g.N % 8) == 0;
     int tl = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tl) {
@@ -167,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!OUT_I32) {
         const int64_t n = n0 + et;
         sw_s[et] = n < g.N ? g.sw[n] : 0.0f;
-        bias_s[et] = (g.bias != nullptr && n < g.N) ? __half2float(g.bias[n]) : 0.0f;
+        bias_s[et] = (g.bias != nullptr && n < g.N) ? g.bias[n] : __float2half_rn(0.0f);
       }
       float sxr[2] = {0.0f, 0.0f};
       if (!OUT_I32) {
@@ -208,16 +210,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
         __align__(16) __half h[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          float f = dequant_f32(static_cast<int32_t>(v[j]), sxr[a], sw_s[cl + j]);
-          if (g.bias != nullptr) f = __fadd_rn(f, bias_s[cl + j]);
-          h[j] = __float2half_rn(f);
+        for (int j = 0; j < 32; j += 2) {
+          float f0 = dequant_f32(static_cast<int32_t>(v[j]), sxr[a], sw_s[cl + j]);
+          float f1 = dequant_f32(static_cast<int32_t>(v[j + 1]), sxr[a], sw_s[cl + j + 1]);
+          if (g.bias != nullptr) {
+            const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&bias_s[cl + j]));
+            f0 = __fadd_rn(f0, b.x);
+            f1 = __fadd_rn(f1, b.y);
+          }
+          // both lanes of the pair rounded to nearest even in one instruction
+          *reinterpret_cast<__half2*>(&h[j]) = __floats2half2_rn(f0, f1);
         }
         if (tma_store) {
           // stage the 32 x 32 block in the 64-byte-swizzled image and let one
-          // TMA store write it (rows/columns outside y are skipped by the TMA)
-          if (lane == 0) bulk_wait_group_read0();  // previous store done reading
+          // TMA store write it (rows/columns outside y are skipped by the TMA);
+          // two buffers per warp, so the store of the previous block may still
+          // be reading the other one
+          const uint32_t stg = stg0 + static_cast<uint32_t>(nst & 1) * STG_BYTES;
+          if (lane == 0 && nst >= 2) bulk_wait_group_read<1>();  // the store from this buffer is done reading
           __syncwarp();
+          ++nst;
           const uint4* hv = reinterpret_cast<const uint4*>(h);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -228,9 +240,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0 && row0 < g.M && col0 < g.N) {
-            tma_store_2d(&tmY, stg, static_cast<int32_t>(col0), static_cast<int32_t>(row0));
-            bulk_commit_group();
+          if (lane == 0) {
+            if (row0 < g.M && col0 < g.N)
+              tma_store_2d(&tmY, stg, static_cast<int32_t>(col0), static_cast<int32_t>(row0));
+            bulk_commit_group();  // one group per staged block, empty if nothing was stored
           }
         } else if (row < g.M && col0 < g.N) {
           __half* dst = g.y + row * g.N + col0;

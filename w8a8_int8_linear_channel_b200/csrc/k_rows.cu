@@ -75,6 +75,24 @@ __device__ __forceinline__ void chunk_sums(const uint4& v, Sums& s) {
   s.s2l += __double2ll_rn(__dmul_rn(c2l, 281474976710656.0));   // * 2^48
 }
 
+// Same sums from the 8 values already converted to fp32 (exact conversions).
+__device__ __forceinline__ void chunk_sums_f(const float (&x)[8], Sums& s) {
+  const double kSplit = 824633720832.0;  // 1.5 * 2^39: (t + kSplit) - kSplit rounds t to 2^-13
+  double c1 = 0.0, c2h = 0.0, c2l = 0.0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const double d = static_cast<double>(x[j]);
+    c1 = __dadd_rn(c1, d);
+    const double t = __dmul_rn(d, d);
+    const double th = __dsub_rn(__dadd_rn(t, kSplit), kSplit);
+    c2h = __dadd_rn(c2h, th);
+    c2l = __dadd_rn(c2l, __dsub_rn(t, th));
+  }
+  s.s1 += __double2ll_rn(__dmul_rn(c1, 16777216.0));            // * 2^24
+  s.s2h += __double2ll_rn(__dmul_rn(c2h, 8192.0));              // * 2^13
+  s.s2l += __double2ll_rn(__dmul_rn(c2l, 281474976710656.0));   // * 2^48
+}
+
 __device__ __forceinline__ void warp_sum(Sums& s) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -177,6 +195,44 @@ __device__ __forceinline__ uint32_t quant4(float x0, float x1, float x2, float x
   const uint32_t b2 = __float_as_uint(__fadd_rn(__fmul_rn(x2, inv), kMagic));
   const uint32_t b3 = __float_as_uint(__fadd_rn(__fmul_rn(x3, inv), kMagic));
   return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
+
+// transform8 on values already unpacked to fp32, in place.
+template <int MODE>
+__device__ __forceinline__ void transform8f(float (&x)[8], int64_t c, const RowArgs& a, float mu,
+                                            float rstd) {
+  const int64_t k0 = c * 8;
+  if (MODE == MODE_WEIGHT) {
+    if (a.vec) {
+      float s[8];
+      load8f(a.vec + k0, s);
+#pragma unroll
+      for (int j = 0; j < 8; j += 2) {
+        const float2 f = __half22float2(__floats2half2_rn(__fmul_rn(x[j], s[j]), __fmul_rn(x[j + 1], s[j + 1])));
+        x[j] = f.x;
+        x[j + 1] = f.y;
+      }
+    }
+    return;
+  }
+  if (a.gamma) {
+    float g[8];
+    load8f(a.gamma + k0, g);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(__fmul_rn(__fsub_rn(x[j], mu), rstd), g[j]);
+    if (a.beta) {
+      float b[8];
+      load8f(a.beta + k0, b);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[j] = __fadd_rn(x[j], b[j]);
+    }
+  }
+  if (MODE == MODE_ACT && a.vec) {
+    float is[8];
+    load8f(a.vec + k0, is);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(x[j], is[j]);
+  }
 }
 
 __device__ __forceinline__ uint2 pack8(const float (&x)[8], float inv) {
@@ -466,13 +522,120 @@ __device__ __forceinline__ void cta_rows(const RowArgs& a, RowSharedT<T>& sh, fl
   }
 }
 
+// Register-resident rows (NCH <= 8): every value is converted to fp32 once;
+// the statistics, the transform (in place), the absmax and the quantization
+// all work on those registers.
+template <int MODE, int T, int NCH, bool PF, int CM>
+__device__ __forceinline__ void cta_rows_fast(const RowArgs& a, RowSharedT<T>& sh, float (&cmax)[CM]) {
+  constexpr int W = T / 32;
+  constexpr bool CALIB_REG = (MODE == MODE_CALIB) && CM == NCH * 8;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t Kc = a.K / 8;
+  const bool use_ln = (MODE != MODE_WEIGHT) && a.gamma != nullptr;
+
+  uint4 v[NCH];
+  uint4 nv[PF ? NCH : 1];
+  auto load_row = [&](int64_t row, uint4* dst) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + row * a.ld);
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int64_t c = tid + static_cast<int64_t>(i) * T;
+      dst[i] = c < Kc ? ld_stream(src + c) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  if (PF && static_cast<int64_t>(blockIdx.x) < a.rows) load_row(blockIdx.x, v);
+  int par = 0;
+  for (int64_t r = blockIdx.x; r < a.rows; r += gridDim.x, par ^= 1) {
+    if (!PF) load_row(r, v);
+    if (PF) {
+      const int64_t rn = r + gridDim.x;
+      if (rn < a.rows) load_row(rn, nv);
+    }
+    float x[NCH][8];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) unpack8(v[i], x[i]);  // chunks past K are zeros
+
+    float mu = 0.0f, rstd = 0.0f;
+    if (use_ln) {
+      Sums s{0, 0, 0};
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+        if (tid + static_cast<int64_t>(i) * T < Kc) chunk_sums_f(x[i], s);
+      warp_sum(s);
+      if (lane == 0) {
+        sh.s1[par][warp] = s.s1;
+        sh.s2h[par][warp] = s.s2h;
+        sh.s2l[par][warp] = s.s2l;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        Sums t{0, 0, 0};
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+          t.s1 += sh.s1[par][w];
+          t.s2h += sh.s2h[par][w];
+          t.s2l += sh.s2l[par][w];
+        }
+        float m_, r_;
+        ln_finalize(t, a.K, a.eps, m_, r_);
+        if (lane == 0) {
+          sh.mu[par] = m_;
+          sh.rstd[par] = r_;
+        }
+      }
+      __syncthreads();
+      mu = sh.mu[par];
+      rstd = sh.rstd[par];
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int64_t c = tid + static_cast<int64_t>(i) * T;
+      if (c < Kc) {
+        transform8f<MODE>(x[i], c, a, mu, rstd);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if constexpr (MODE == MODE_CALIB) {
+            if constexpr (CALIB_REG) cmax[i * 8 + j] = fmaxf(cmax[i * 8 + j], fabsf(x[i][j]));
+          } else {
+            amax = fmaxf(amax, fabsf(x[i][j]));
+          }
+        }
+      }
+    }
+    if constexpr (MODE != MODE_CALIB) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      if (lane == 0) sh.mx[par][warp] = amax;
+      __syncthreads();
+      float m = 0.0f;
+#pragma unroll
+      for (int w = 0; w < W; ++w) m = fmaxf(m, sh.mx[par][w]);
+      const float sc = __fdiv_rn(m, 127.0f);
+      const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+      if (tid == 0) a.scale[r] = sc;
+      int8_t* dst = a.q + r * a.K;
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        const int64_t c = tid + static_cast<int64_t>(i) * T;
+        if (c < Kc) *reinterpret_cast<uint2*>(dst + c * 8) = pack8(x[i], inv);
+      }
+    }
+    if (PF) {
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) v[i] = nv[i];
+    }
+  }
+}
+
 template <int MODE, int T, int NCH, bool PF>
 __global__ void __launch_bounds__(T) k_rows_cta(const RowArgs a) {
   __shared__ RowSharedT<T> sh;
   griddep_wait();
   griddep_launch_dependents();
   float none[1];
-  cta_rows<MODE, T, NCH, PF, 1>(a, sh, none);
+  if constexpr (NCH > 0 && NCH <= 8) cta_rows_fast<MODE, T, NCH, PF, 1>(a, sh, none);
+  else cta_rows<MODE, T, NCH, PF, 1>(a, sh, none);
 }
 
 // CTA-per-row calibration with register maxima, merged across a cluster of 8
@@ -487,7 +650,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(T) k_calib_ct
   for (int i = 0; i < NCH * 8; ++i) cmax[i] = 0.0f;
   griddep_wait();
   griddep_launch_dependents();
-  cta_rows<MODE_CALIB, T, NCH, true, NCH * 8>(a, sh, cmax);
+  cta_rows_fast<MODE_CALIB, T, NCH, true, NCH * 8>(a, sh, cmax);
   const int64_t Kc = a.K / 8;
 #pragma unroll
   for (int i = 0; i < NCH; ++i) {
