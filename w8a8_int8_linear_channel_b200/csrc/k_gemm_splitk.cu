@@ -5,16 +5,17 @@
 // Swap-AB: the MMA's 128-row M slot takes 128 weight rows (output channels)
 // and its N slot takes the BT (16 or 32) zero-padded tokens, so
 //   TMEM lane = output channel n,  TMEM column = token t.
-// Stream-K: the (channel tile, 128-byte K block) units of the whole problem
-// are cut into one contiguous range per SM (a persistent grid of num_SMs
-// CTAs), so the TMA stream of every CTA never drains at tile boundaries and
-// no wave is left partly empty.  A tile split between CTAs is summed exactly:
+// Persistent grid of one CTA per SM; a unit is a (channel tile, 256-byte K
+// span).  Each CTA streams its units back to back, so its TMA stream never
+// drains at tile boundaries, and the units are balanced across CTAs: equal
+// numbers of whole tiles, plus an equal share (stream-K) of the remaining
+// tiles, which every CTA processes first.  A tile split between CTAs is summed exactly:
 // each contributor writes its int32 partial accumulator to the workspace and
 // the last to arrive (per-tile counter, no waiting) adds the others and runs
 // the epilogue y = fp16((acc * sx[t]) * sw[n] + bias[n]).  int32 addition is
 // associative, so the result is bit-identical to a single-CTA sum.
 //
-// Roles: warp 0 TMA producer (a STAGES-deep ring of 16 KB weight tiles +
+// Roles: warp 0 TMA producer (a 5-deep ring; a stage is two K-consecutive 16 KB weight boxes +
 // BT x 128 B token tiles), warp 1 TMEM owner + MMA issuer (double-buffered
 // accumulators), warps 2-5 epilogue.  All waits are bounded.
 #include "sq_internal.h"
@@ -25,14 +26,15 @@ namespace sq {
 namespace {
 
 constexpr int BW = 128;  // weight rows (output channels) per tile
-constexpr int BK = 128;  // K bytes per unit
+constexpr int BK = 128;  // K bytes per swizzled box
+constexpr int KPS = 2;   // consecutive K boxes per unit (per pipeline stage)
 constexpr int kThreads = 192;
-constexpr int kStages = 10;
+constexpr int kStages = 5;
 
 template <int BT>
 struct SkLayout {
-  static constexpr int A_BYTES = BW * BK;  // 16 KB weight tile
-  static constexpr int B_BYTES = BT * BK;  // token tile
+  static constexpr int A_BYTES = BW * BK * KPS;  // 2 x 16 KB weight boxes
+  static constexpr int B_BYTES = BT * BK * KPS;  // 2 token boxes
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int CTRL = kStages * STAGE_BYTES;
   static constexpr int NBARS = 2 * kStages + 5;  // full, empty, acc_full[2], acc_empty[2], drain
@@ -43,10 +45,19 @@ struct SkLayout {
   static constexpr int TMEM_COLS = 2 * BT < 32 ? 32 : 2 * BT;
 };
 
+// Work split.  With T channel tiles on `grid` CTAs, every CTA owns Wt =
+// T / grid whole tiles (the last tiles, processed last); the remaining R
+// tiles are cut stream-K style: their U = R * KB units are split into equal
+// contiguous ranges over the first G CTAs, which process that share first.
+// Tiles shared between CTAs are therefore summed early in the kernel, and
+// every CTA ends on whole tiles that need no cross-CTA fix-up.
 struct SkGeom {
-  int64_t U;   // total units = tiles * KB
-  int KB;      // K blocks per tile
-  int G;       // CTAs
+  int64_t U;   // stream-K units = R * KB
+  int KB;      // units (KPS boxes of 128 K bytes) per tile
+  int G;       // CTAs sharing the stream-K region (>= 1)
+  int R;       // tiles 0 .. R-1 are split stream-K style
+  int Wt;      // whole tiles per CTA: tiles R + c * Wt .. R + c * Wt + Wt - 1
+  int grid;    // CTAs launched
   __device__ __forceinline__ int64_t u0(int c) const { return (static_cast<int64_t>(c) * U) / G; }
   __device__ __forceinline__ int cta_of(int64_t u) const {
     return static_cast<int>(((u + 1) * G - 1) / U);
@@ -92,8 +103,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
-  const int64_t ubeg = geo.u0(cta), uend = geo.u0(cta + 1);
+  const int64_t ubeg = cta < geo.G ? geo.u0(cta) : 0;
+  const int64_t uend = cta < geo.G ? geo.u0(cta + 1) : 0;
   const int KB = geo.KB;
+  const int64_t n_sk = uend - ubeg;                                 // stream-K units of this CTA
+  const int64_t n_all = n_sk + static_cast<int64_t>(geo.Wt) * KB;  // then its whole tiles
+  const int64_t wt0 = geo.R + static_cast<int64_t>(cta) * geo.Wt;  // first whole tile
+  // position j of this CTA's unit sequence -> (tile, unit within the tile)
+  auto unit_of = [&](int64_t j, int64_t& t, int& kb) {
+    if (j < n_sk) {
+      const int64_t u = ubeg + j;
+      t = u / KB;
+      kb = static_cast<int>(u % KB);
+    } else {
+      const int64_t w = j - n_sk;
+      t = wt0 + w / KB;
+      kb = static_cast<int>(w % KB);
+    }
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -125,17 +152,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int64_t u = ubeg; u < uend; ++u) {
-        const int64_t i = u - ubeg;
+      const uint64_t pol_w = l2_policy_evict_first();  // each weight byte is read once
+      const uint64_t pol_x = l2_policy_evict_last();   // every CTA re-reads the tokens
+      for (int64_t i = 0; i < n_all; ++i) {
         const int s = static_cast<int>(i % kStages);
         const int64_t r = i / kStages;
         if (i >= kStages && !mbar_wait(empty_bar(s), static_cast<uint32_t>((r - 1) & 1), budget, status, abort_flag))
           break;
-        const int64_t t = u / KB;
-        const int kb = static_cast<int>(u % KB);
-        mbar_arrive_expect_tx(full_bar(s), L::STAGE_BYTES);
-        tma_load_2d(sA + s * L::A_BYTES, &tmW, full_bar(s), kb * BK, static_cast<int32_t>(t * BW));
-        tma_load_2d(sB + s * L::B_BYTES, &tmX, full_bar(s), kb * BK, 0);
+        int64_t t;
+        int kb;
+        unit_of(i, t, kb);
+        mbar_arrive_expect_tx(full_bar(s), L::STAGE_BYTES);  // boxes past K arrive zero-filled
+#pragma unroll
+        for (int p = 0; p < KPS; ++p) {
+          const int32_t kx = (kb * KPS + p) * BK;
+          tma_load_2d_hint(sA + s * L::A_BYTES + p * (BW * BK), &tmW, full_bar(s), kx,
+                           static_cast<int32_t>(t * BW), pol_w);
+          tma_load_2d_hint(sB + s * L::B_BYTES + p * (BT * BK), &tmX, full_bar(s), kx, 0, pol_x);
+        }
         ++issued;
       }
     }
@@ -144,13 +178,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_i8(BW, BT);
       int seg = 0;
       int b = 0;
-      for (int64_t u = ubeg; u < uend; ++u) {
-        const int64_t i = u - ubeg;
+      for (int64_t i = 0; i < n_all; ++i) {
         const int s = static_cast<int>(i % kStages);
         const int64_t r = i / kStages;
-        const int kb = static_cast<int>(u % KB);
-        const bool first = (u == ubeg) || kb == 0;
-        const bool last = (u == uend - 1) || kb == KB - 1;
+        int64_t t;
+        int kb;
+        unit_of(i, t, kb);
+        const bool first = i == 0 || i == n_sk || kb == 0;
+        const bool last = i == n_sk - 1 || i == n_all - 1 || kb == KB - 1;
         if (first) {
           b = seg & 1;
           if (seg >= 2 && !mbar_wait(acce_bar(b), static_cast<uint32_t>(((seg >> 1) - 1) & 1), budget, status, abort_flag))
@@ -158,12 +193,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!mbar_wait(full_bar(s), static_cast<uint32_t>(r & 1), budget, status, abort_flag)) break;
         tc_fence_after();
-        const uint64_t ad = sdesc_k_sw128(sA + s * L::A_BYTES);
-        const uint64_t bd = sdesc_k_sw128(sB + s * L::B_BYTES);
         const uint32_t d = tmem + static_cast<uint32_t>(b * BT);
 #pragma unroll
-        for (int k = 0; k < BK / 32; ++k)
-          mma_i8(d, ad + 2u * k, bd + 2u * k, idesc, (first && k == 0) ? 0u : 1u);
+        for (int p = 0; p < KPS; ++p) {
+          const uint64_t ad = sdesc_k_sw128(sA + s * L::A_BYTES + p * (BW * BK));
+          const uint64_t bd = sdesc_k_sw128(sB + s * L::B_BYTES + p * (BT * BK));
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)
+            mma_i8(d, ad + 2u * k, bd + 2u * k, idesc, (first && p == 0 && k == 0) ? 0u : 1u);
+        }
         mma_any = true;
         mma_commit(empty_bar(s));
         if (last) {
@@ -179,12 +217,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!OUT_I32 && et < BT) sx_s[et] = et < g.M ? g.sx[et] : 0.0f;
     named_bar_sync(1, 128);
     int seg = 0;
-    for (int64_t u = ubeg; u < uend;) {
-      const int64_t t = u / KB;
-      const int64_t tile_end = (t + 1) * KB;
-      const int64_t seg_end = uend < tile_end ? uend : tile_end;
-      const bool whole = (u == t * KB) && (seg_end == tile_end);
-      const int slot = (u == ubeg) ? 0 : 1;
+    for (int64_t j = 0; j < n_all;) {
+      int64_t t, tile_end = 0, seglen;
+      bool whole;
+      int slot = 0;
+      if (j < n_sk) {  // a piece of a stream-K tile
+        const int64_t u = ubeg + j;
+        t = u / KB;
+        tile_end = (t + 1) * KB;
+        const int64_t seg_end = uend < tile_end ? uend : tile_end;
+        whole = (u == t * KB) && (seg_end == tile_end);
+        slot = (j == 0) ? 0 : 1;
+        seglen = seg_end - u;
+      } else {  // one of this CTA's whole tiles
+        t = wt0 + (j - n_sk) / KB;
+        whole = true;
+        seglen = KB;
+      }
       const int b = seg & 1;
       mbar_wait(accf_bar(b), static_cast<uint32_t>((seg >> 1) & 1), budget, status, abort_flag);
       // one thread decides whether to stop and broadcasts it (double-buffered by
@@ -257,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      u = seg_end;
+      j += seglen;
       ++seg;
     }
   }
@@ -285,6 +334,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 int64_t tiles_of(int64_t N) { return (N + BW - 1) / BW; }
 
+SkGeom make_geom(int64_t N, int64_t K, int64_t grid_cap) {
+  SkGeom geo;
+  geo.KB = static_cast<int>(((K + BK - 1) / BK + KPS - 1) / KPS);
+  const int64_t T = tiles_of(N);
+  const int64_t total = T * geo.KB;
+  const int64_t grid = total < grid_cap ? total : grid_cap;
+  geo.grid = static_cast<int>(grid);
+  geo.Wt = static_cast<int>(T / grid);
+  geo.R = static_cast<int>(T - static_cast<int64_t>(geo.Wt) * grid);
+  geo.U = static_cast<int64_t>(geo.R) * geo.KB;
+  geo.G = geo.U > 0 ? static_cast<int>(geo.U < grid ? geo.U : grid) : 1;
+  return geo;
+}
+
 template <int BT, bool OUT_I32>
 cudaError_t launch_bt(const GemmArgs& g, const Ctx& c) {
   using L = SkLayout<BT>;
@@ -300,16 +363,13 @@ cudaError_t launch_bt(const GemmArgs& g, const Ctx& c) {
   CUtensorMap tmW, tmX;
   if (!make_tmap_i8(&tmW, g.wq, g.K, g.N, BK, BW)) return cudaErrorInvalidValue;
   if (!make_tmap_i8(&tmX, g.xq, g.K, g.M, BK, BT)) return cudaErrorInvalidValue;
-  SkGeom geo;
-  geo.KB = static_cast<int>((g.K + BK - 1) / BK);
-  geo.U = tiles_of(g.N) * geo.KB;
-  geo.G = static_cast<int>(geo.U < c.num_sms ? geo.U : c.num_sms);
+  const SkGeom geo = make_geom(g.N, g.K, c.num_sms);
   uint8_t* ws = static_cast<uint8_t*>(g.ws);
   const size_t counter_bytes = ((tiles_of(g.N) * 4 + 255) / 256) * 256;
   uint32_t* counters = reinterpret_cast<uint32_t*>(ws);
   int32_t* partials = reinterpret_cast<int32_t*>(ws + counter_bytes);
-  return launch_pdl(k_gemm_splitk<BT, OUT_I32>, dim3(geo.G), dim3(kThreads), L::SMEM, c.stream, tmW, tmX, g,
-                    geo, counters, partials, c.status, c.budget_ns);
+  return launch_pdl(k_gemm_splitk<BT, OUT_I32>, dim3(geo.grid), dim3(kThreads), L::SMEM, c.stream, tmW, tmX,
+                    g, geo, counters, partials, c.status, c.budget_ns);
 }
 
 }  // namespace
@@ -397,20 +457,14 @@ cudaError_t launch_noalloc(const GemmArgs& g, const Ctx& c, uint8_t* scratch) {
   CUtensorMap tmW, tmX;
   if (!make_tmap_i8(&tmW, g.wq, g.K, g.N, BK, BW)) return cudaErrorInvalidValue;
   if (!make_tmap_i8(&tmX, g.xq, g.K, g.M, BK, BT)) return cudaErrorInvalidValue;
-  SkGeom geo;
-  geo.KB = static_cast<int>((g.K + BK - 1) / BK);
-  geo.U = tiles_of(g.N) * geo.KB;
   const int64_t slots = static_cast<int64_t>(kNoAllocPartialBytes / (2ull * BW * BT * 4));
-  int64_t G = c.num_sms;
-  if (G > slots) G = slots;
-  if (G > geo.U) G = geo.U;
-  geo.G = static_cast<int>(G);
+  const SkGeom geo = make_geom(g.N, g.K, c.num_sms < slots ? c.num_sms : slots);
   uint32_t* counters = reinterpret_cast<uint32_t*>(scratch);
   int32_t* partials = reinterpret_cast<int32_t*>(scratch + kNoAllocCounterBytes);
   const uint32_t ntiles = static_cast<uint32_t>(tiles_of(g.N));
   e = launch_pdl(k_noalloc_clear_counters, dim3((ntiles + 255) / 256), dim3(256), 0, c.stream, ntiles);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_gemm_splitk<BT, false>, dim3(geo.G), dim3(kThreads), L::SMEM, c.stream, tmW, tmX, g,
+  return launch_pdl(k_gemm_splitk<BT, false>, dim3(geo.grid), dim3(kThreads), L::SMEM, c.stream, tmW, tmX, g,
                     geo, counters, partials, c.status, c.budget_ns);
 }
 
