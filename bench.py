@@ -280,6 +280,47 @@ class Plan:
         self.bind(self.main)
         self.main.wait_stream(cap)
 
+    def capture_staged(self):
+        """Capture the step once more with an event-record node before every
+        call and after the last (N = 1): replaying it gives each kernel's
+        device time without host launch gaps; the event nodes serialize the
+        kernels, so no stage overlaps its neighbour here."""
+        torch = self.torch
+        self.sev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(self.calls) + 1)]
+        cap = torch.cuda.Stream()
+        cap.wait_stream(self.main)
+        with torch.cuda.stream(cap):
+            self.bind(cap)
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=cap):
+                self.amax.zero_()
+                for i, (name, fn, args) in enumerate(self.calls):
+                    self.sev[i].record(cap)
+                    self._call(name, fn, args)
+                self.sev[-1].record(cap)
+        self.bind(self.main)
+        self.main.wait_stream(cap)
+        self.staged = gr
+
+    def capture_gemm_burst(self, reps):
+        """Capture `reps` back-to-back launches of the step's W8A8 linear (same
+        buffers, main-stream order, launch overlap between them) into one
+        graph: its replay time / reps is the kernel's average launch duration
+        with no host gap and no per-launch event."""
+        torch = self.torch
+        cap = torch.cuda.Stream()
+        cap.wait_stream(self.main)
+        with torch.cuda.stream(cap):
+            self.bind(cap)
+            name, fn, args = self.calls[-1]
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=cap):
+                for _ in range(reps):
+                    self._call(name, fn, args)
+        self.bind(self.main)
+        self.main.wait_stream(cap)
+        self.burst, self.burst_reps = gr, reps
+
     def replay(self, allreduce=None):
         self.graphs[0].replay()
         if len(self.graphs) > 1:
@@ -381,20 +422,70 @@ def run_gpu(args):
     total_ms = float(t_local.item())
     ms_per_step = total_ms / args.steps
 
-    # stage breakdown: a second timed loop with an event around every call
-    # (the events serialize the launches, so each stage also carries its own
-    # launch latency; the GEMM's time here is the roofline's launch duration)
+    # stage breakdown: a second loop with an event around every call.  With a
+    # graph (N = 1) the events are graph nodes, so each stage is its kernel's
+    # device time; otherwise eager launches, and each stage also carries its
+    # own launch latency.  The GEMM's time here is the roofline's launch
+    # duration.
     n_stage = min(args.steps, args.stage_steps)
-    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(ncalls + 1)] for _ in range(n_stage)]
-    for i in range(n_stage):
-        flush()
-        plan.step(sev[i], allreduce)
-    torch.cuda.synchronize()
     per_stage = np.zeros(ncalls)
-    for ev in sev:
-        for j in range(ncalls):
-            per_stage[j] += ev[j].elapsed_time(ev[j + 1])
+    stage_mode = "eager"
+    if use_graph and world == 1:
+        try:
+            plan.capture_staged()
+            for _ in range(3):
+                flush()
+                plan.staged.replay()
+            torch.cuda.synchronize()
+            for i in range(n_stage):
+                flush()
+                plan.staged.replay()
+                torch.cuda.synchronize()
+                for j in range(ncalls):
+                    per_stage[j] += plan.sev[j].elapsed_time(plan.sev[j + 1])
+            stage_mode = "graph"
+        except RuntimeError:
+            torch.cuda.synchronize()
+            per_stage[:] = 0.0
+    if stage_mode == "eager":
+        sev = [[torch.cuda.Event(enable_timing=True) for _ in range(ncalls + 1)] for _ in range(n_stage)]
+        for i in range(n_stage):
+            flush()
+            plan.step(sev[i], allreduce)
+        torch.cuda.synchronize()
+        for ev in sev:
+            for j in range(ncalls):
+                per_stage[j] += ev[j].elapsed_time(ev[j + 1])
+    if sq.sq_poll_status() != 0:
+        raise RuntimeError("device wait timed out in the stage loop")
     stage_us = {c[0]: 1e3 * per_stage[j] / n_stage for j, c in enumerate(plan.calls)}
+
+    # the roofline's launch duration: back-to-back launches of the linear in
+    # one graph (inputs as the step leaves them: L2-warm for the large-M
+    # shapes, far larger than L2 for decode), L2 flushed before each burst
+    gemm_us, gemm_mode = stage_us["w8a8_linear"], "stage loop (one event pair per launch)"
+    if use_graph:
+        try:
+            plan.capture_gemm_burst(args.burst)
+            for _ in range(2):
+                flush()
+                plan.burst.replay()
+            torch.cuda.synchronize()
+            bev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.burst_iters)]
+            for i in range(args.burst_iters):
+                flush()
+                bev[i][0].record()
+                plan.burst.replay()
+                bev[i][1].record()
+            torch.cuda.synchronize()
+            tb = sum(e[0].elapsed_time(e[1]) for e in bev) / args.burst_iters
+            gemm_us = 1e3 * tb / args.burst
+            gemm_mode = (f"{args.burst} back-to-back launches in one CUDA graph, events around the replay, "
+                         f"mean of {args.burst_iters} replays")
+        except RuntimeError:
+            torch.cuda.synchronize()
+    if sq.sq_poll_status() != 0:
+        raise RuntimeError("device wait timed out in the GEMM burst")
 
     nbytes, ops = stage_bytes_ops(wl, M)
     step_bytes = sum(nbytes.values())
@@ -407,10 +498,13 @@ def run_gpu(args):
         unit = "TOPS"
 
     peaks, peak_kind = load_peaks()
-    gemm_s = stage_us["w8a8_linear"] * 1e-6
+    gemm_s = gemm_us * 1e-6
     prof = os.path.join(ROOT, "profiles", f"w8a8_linear_{args.workload}{'_m%d' % M if M != wl.M else ''}.md")
-    src = os.path.join(ROOT, "w8a8_int8_linear_channel_b200", "csrc",
-                       "k_gemm_splitk.cu" if decode else "k_gemm_tiled.cu")
+    gemm_src = "k_gemm_splitk.cu" if decode else ("k_gemm_pair.cu" if M > 128 else "k_gemm_tiled.cu")
+    gemm_name = ("k_gemm_splitk (swap-AB stream-K)" if decode else
+                 "k_gemm_pair (tcgen05 cta_group::2 kind::i8, 256x256 tiles)" if M > 128 else
+                 "k_gemm_tiled (tcgen05 kind::i8, 128x256 tiles)")
+    src = os.path.join(ROOT, "w8a8_int8_linear_channel_b200", "csrc", gemm_src)
     traffic = traffic_from_profile(src, prof)
     if decode:
         ach = nbytes["w8a8_linear"] / gemm_s / 1e9
@@ -425,8 +519,9 @@ def run_gpu(args):
                 "frac": round(ach / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_kind} cuBLAS bf16 burst {peaks['bf16_tflops']} TFLOP/s x 2 "
                                "(nominal dense INT8:BF16 ratio 4.5:2.25)"}
-    roof["kernel"] = "k_gemm_splitk (swap-AB stream-K)" if decode else "k_gemm_tiled (tcgen05 kind::i8)"
-    roof["per_launch_us"] = round(stage_us["w8a8_linear"], 2)
+    roof["kernel"] = gemm_name
+    roof["per_launch_us"] = round(gemm_us, 2)
+    roof["launch_timing"] = gemm_mode
 
     e2e = None
     if not args.no_e2e:
@@ -448,7 +543,8 @@ def run_gpu(args):
                              "lines remain), outside the timed events",
                        "timing": "CUDA events at the boundaries of every step, summed over steps, max over "
                                  "ranks; stage_us and the roofline's launch time from a second loop with "
-                                 "events around every call"},
+                                 "events around every call (" + ("event nodes in a CUDA graph of the step"
+                                 if stage_mode == "graph" else "eager launches") + ")"},
             "roofline": roof,
             "stage_us": {k: round(v, 2) for k, v in stage_us.items()},
             "gpu_launches": plan.launches_per_step * args.steps,
@@ -633,6 +729,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--stage-steps", type=int, default=300, help="steps of the per-stage timing loop")
+    ap.add_argument("--burst", type=int, default=20, help="back-to-back GEMM launches per timed burst")
+    ap.add_argument("--burst-iters", type=int, default=20, help="timed bursts (roofline launch duration)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the step's kernels eagerly instead of replaying a captured CUDA graph")
     ap.add_argument("--streams", type=int, choices=[1, 2], default=1,

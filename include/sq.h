@@ -159,8 +159,10 @@ size_t sq_w8a8_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *   xq int8 [M, K]; x_scale fp32 [M]; wq int8 [N, K]; w_scale fp32 [N];
  *   bias fp16 [N] or NULL; y fp16 [M, N]
  * M <= SQ_SPLITK_MAX_M runs the weight-streaming stream-K kernel and needs
- * sq_w8a8_workspace_bytes(M, N, K) bytes of workspace; larger M runs the
- * tiled tensor-core kernel (workspace may be NULL).
+ * sq_w8a8_workspace_bytes(M, N, K) bytes of workspace; 32 < M <= 128 runs the
+ * tiled tensor-core kernel (128 x 256 tiles) and M > 128 the persistent
+ * CTA-pair kernel (256 x 256 tiles, tcgen05 cta_group::2); neither needs a
+ * workspace (it may be NULL).
  */
 sq_status sq_w8a8_linear(const int8_t* xq, const float* x_scale, const int8_t* wq,
                          const float* w_scale, const void* bias_f16, void* y_f16, int64_t M,
@@ -171,7 +173,9 @@ sq_status sq_w8a8_linear(const int8_t* xq, const float* x_scale, const int8_t* w
 typedef enum sq_gemm_path {
   SQ_PATH_AUTO = 0,   /* what sq_w8a8_linear does */
   SQ_PATH_TILED = 1,  /* tiled tcgen05 kernel, any M */
-  SQ_PATH_SPLITK = 2  /* weight-streaming stream-K kernel, M <= SQ_SPLITK_MAX_M */
+  SQ_PATH_SPLITK = 2, /* weight-streaming stream-K kernel, M <= SQ_SPLITK_MAX_M */
+  SQ_PATH_PAIR = 3,   /* 256 x 256 tiles on CTA pairs (tcgen05 cta_group::2), any M */
+  SQ_PATH_WIDE = 4    /* 256 x 256 tiles on single CTAs, any M */
 } sq_gemm_path;
 
 /* sq_w8a8_linear with the kernel chosen by the caller (testing and

@@ -152,14 +152,18 @@ def _rand_i8(rng, M, N, K):
     return xq, wq, sx, sw, bias
 
 
+_PATHS = {"tiled": lambda m: m.PATH_TILED, "splitk": lambda m: m.PATH_SPLITK,
+          "pair": lambda m: m.PATH_PAIR, "wide": lambda m: m.PATH_WIDE}
+
+
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
-@pytest.mark.parametrize("path", ["tiled", "splitk"])
+@pytest.mark.parametrize("path", ["tiled", "splitk", "pair", "wide"])
 def test_gemm_accumulators_bit_exact(sq, M, N, K, path):
     if path == "splitk" and M > sq.SPLITK_MAX_M:
         pytest.skip("stream-K path serves M <= 32")
     rng = np.random.default_rng(M * 1000003 + N * 101 + K)
     xq, wq, _, _, _ = _rand_i8(rng, M, N, K)
-    p = sq.PATH_TILED if path == "tiled" else sq.PATH_SPLITK
+    p = _PATHS[path](sq)
     ws = sq.new_workspace(M, N, K) if path == "splitk" else None
     acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
     sq.sq_w8a8_gemm_s32(dev(xq), dev(wq), acc, workspace=ws, path=p)
@@ -168,7 +172,7 @@ def test_gemm_accumulators_bit_exact(sq, M, N, K, path):
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
-@pytest.mark.parametrize("path", ["tiled", "splitk"])
+@pytest.mark.parametrize("path", ["tiled", "splitk", "pair", "wide"])
 @pytest.mark.parametrize("with_bias", [False, True])
 def test_linear_output(sq, M, N, K, path, with_bias):
     if path == "splitk" and M > sq.SPLITK_MAX_M:
@@ -176,7 +180,7 @@ def test_linear_output(sq, M, N, K, path, with_bias):
     rng = np.random.default_rng(M * 7919 + N * 31 + K + with_bias)
     xq, wq, sx, sw, bias = _rand_i8(rng, M, N, K)
     bias = bias if with_bias else None
-    p = sq.PATH_TILED if path == "tiled" else sq.PATH_SPLITK
+    p = _PATHS[path](sq)
     ws = sq.new_workspace(M, N, K) if path == "splitk" else None
     y = torch.empty((M, N), dtype=torch.float16, device="cuda")
     sq.sq_w8a8_linear(dev(xq), dev(sx), dev(wq), dev(sw), y, dev(bias), workspace=ws, path=p)
@@ -206,7 +210,7 @@ def test_extreme_codes_do_not_wrap(sq):
     xq[1] = -127
     wq = np.full((3, K), 127, np.int8)
     wq[2] = -127
-    for path in (sq.PATH_TILED, sq.PATH_SPLITK):
+    for path in (sq.PATH_TILED, sq.PATH_SPLITK, sq.PATH_PAIR, sq.PATH_WIDE):
         acc = torch.empty((2, 3), dtype=torch.int32, device="cuda")
         ws = sq.new_workspace(2, 3, K)
         sq.sq_w8a8_gemm_s32(dev(xq), dev(wq), acc, workspace=ws, path=path)

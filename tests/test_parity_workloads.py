@@ -145,8 +145,10 @@ def test_full_size_ffn_down(sq, alpha):
     _check(r, wl, wl.M, alpha, tokens, _weight_sample(wl.N, per_tile=2, seed=3))
 
 
-def test_persistent_gemm_more_tiles_than_sms(sq):
-    # 6 x 26 = 156 tiles of 256 x 256 on 148 SMs, ragged M, N and K
+@pytest.mark.parametrize("path", ["auto", "pair", "wide"])
+def test_persistent_gemm_more_tiles_than_sms(sq, path):
+    # 6 x 26 = 156 tiles of 256 x 256 on 148 SMs (74 CTA pairs), ragged M, N and K
+    p = {"auto": sq.PATH_AUTO, "pair": sq.PATH_PAIR, "wide": sq.PATH_WIDE}[path]
     rng = np.random.default_rng(99)
     M, N, K = 1300, 6500, 272
     xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
@@ -155,8 +157,8 @@ def test_persistent_gemm_more_tiles_than_sms(sq):
     sw = rng.uniform(1e-4, 1e-2, N).astype(np.float32)
     bias = (rng.standard_normal(N) * 0.1).astype(np.float16)
     acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
-    sq.sq_w8a8_gemm_s32(_T(xq), _T(wq), acc)
+    sq.sq_w8a8_gemm_s32(_T(xq), _T(wq), acc, path=p)
     assert np.array_equal(acc.cpu().numpy(), oracle.int_gemm(xq, wq))
     y = torch.empty((M, N), dtype=torch.float16, device="cuda")
-    sq.sq_w8a8_linear(_T(xq), _T(sx), _T(wq), _T(sw), y, _T(bias))
+    sq.sq_w8a8_linear(_T(xq), _T(sx), _T(wq), _T(sw), y, _T(bias), path=p)
     assert bits_equal(y.cpu().numpy(), oracle.w8a8_linear(xq, sx, wq, sw, bias))

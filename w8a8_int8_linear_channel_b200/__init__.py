@@ -26,13 +26,13 @@ __all__ = [
     "SQError", "sq_calibrate_absmax", "sq_smooth_fold", "sq_quantize_weight", "sq_ln_quant_act",
     "sq_w8a8_workspace_bytes", "sq_w8a8_linear", "sq_w8a8_linear_path", "sq_w8a8_gemm_s32",
     "sq_poll_status", "sq_set_wait_budget_ns", "sq_selftest_wait_timeout", "SmoothQuantLinear",
-    "PATH_AUTO", "PATH_TILED", "PATH_SPLITK", "SPLITK_MAX_M", "MAX_K", "library_path",
+    "PATH_AUTO", "PATH_TILED", "PATH_SPLITK", "PATH_PAIR", "PATH_WIDE", "SPLITK_MAX_M", "MAX_K", "library_path",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libsq.so")
 
-PATH_AUTO, PATH_TILED, PATH_SPLITK = 0, 1, 2
+PATH_AUTO, PATH_TILED, PATH_SPLITK, PATH_PAIR, PATH_WIDE = 0, 1, 2, 3, 4
 SPLITK_MAX_M = 32
 MAX_K = 133144
 

@@ -1,0 +1,445 @@
+// k_gemm_pair.cu -- the W8A8 linear for large token counts on CTA pairs: INT8
+// x INT8 -> INT32 GEMM on the 5th-generation tensor cores (tcgen05.mma
+// cta_group::2, kind::i8) with the dequant epilogue fused (glossary "INT8
+// GEMM"; section "inference", O1 scales; the quantization tutorial's
+// "multiply the scale back").
+//
+// A cluster of two CTAs (one TPC) computes 256 x 256 output tiles, walking
+// them persistently.  Per 128-byte K block each CTA loads 128 token rows of
+// xq and 128 of the 256 weight rows of wq (32 KB); one pair MMA of
+// 256 x 256 x 32 reads A from both CTAs and B from both halves, so each CTA's
+// shared memory serves 64 bytes per tensor-core cycle (half of what a
+// single-CTA 128 x 256 MMA reads) and the TMA refill another 64.  Each CTA
+// holds its 128 accumulator rows x 256 int32 columns in TMEM, twice (512
+// columns), so the epilogue of one tile runs under the MMAs of the next.
+//   warp 0      TMA producer of this CTA's halves (6-stage ring); the loads
+//               of both CTAs complete on the leader's barrier of the stage
+//   warp 1      TMEM allocation (both CTAs); in the leader, lane 0 issues the
+//               pair MMAs once both CTAs' halves of a stage have landed
+//   warps 2-9   epilogue of this CTA's 128 rows: warp w reads TMEM lane
+//               quarter w % 4 for column half (w - 2) / 4, computes
+//               y = fp16((acc * sx[t]) * sw[n] + bias[n]) and writes 32 x 32
+//               blocks through shared memory with TMA stores
+// Every mbarrier wait is bounded; a wait that runs out records a timeout,
+// tells the other CTA of the pair to stop, and both CTAs drain what they
+// issued, free TMEM and return.
+#include <string.h>
+
+#include "sq_internal.h"
+#include "sq_ptx.cuh"
+#include "sq_tmap.h"
+
+namespace sq {
+namespace {
+
+constexpr int BM = 128;  // token rows per CTA (the pair covers 256)
+constexpr int BN = 256;  // output channels per tile (each CTA loads 128 weight rows)
+constexpr int BNH = BN / 2;
+constexpr int BK = 128;  // K bytes per stage = one 128-byte swizzle row
+constexpr int STAGES = 6;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int A_BYTES = BM * BK;   // 16 KB
+constexpr int B_BYTES = BNH * BK;  // 16 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int STG = STAGES * STAGE_BYTES;  // per-epilogue-warp output staging
+constexpr int STG_BYTES = 2048;            // one 32 rows x 32 fp16 block, 64-byte swizzle
+constexpr int STG_WARP = 2 * STG_BYTES;    // double-buffered per warp
+constexpr int CTRL = STG + kEpiWarps * STG_WARP;
+// barriers: full[S] (leader: both CTAs' loads landed), empty[S], accf[2],
+// acce[2] (leader: both epilogues done), drain
+constexpr int NBARS = 2 * STAGES + 5;
+// TMEM address, abort flag, decision[2], loads issued by the peer
+constexpr int SLOT = CTRL + NBARS * 8;
+// sw[BN] fp32, bias[BN] fp16 of the current tile, read as 16-byte vectors
+constexpr int VEC = (SLOT + 32 + 15) & ~15;
+static_assert(VEC % 16 == 0 && (VEC + BN * 4) % 16 == 0, "vector loads of sw and bias");
+constexpr int SMEM_BYTES = VEC + BN * 4 + BN * 2;
+constexpr size_t SMEM = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
+static_assert(SMEM <= 232448, "shared memory per CTA");
+constexpr uint32_t TMEM_COLS = 512;
+
+// Bounded wait that, when it runs out, also raises the other CTA's abort
+// flag so the pair stops together.  Barriers completed by the other CTA's
+// threads (cluster_scope) are polled without suspending.
+__device__ __forceinline__ bool pair_wait(uint32_t bar, uint32_t parity, bool cluster_scope,
+                                          uint64_t budget_ns, uint32_t* status,
+                                          volatile uint32_t* abort, uint32_t peer_abort) {
+  auto test = [&]() { return cluster_scope ? mbar_test_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (test()) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (test()) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > budget_ns) {
+      atomicCAS(status, DEV_OK, DEV_TIMEOUT);
+      *abort = 1;
+      st_shared_cluster_u32(peer_abort, 1u);
+      return false;
+    }
+  }
+}
+
+template <bool OUT_I32>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmY, const GemmArgs g, int tiles_m, int tiles,
+                int tma_store, uint32_t* status, uint64_t budget) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + CTRL;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto accf_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
+  auto acce_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SLOT);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile uint32_t* decision = tmem_slot + 2;     // [2]
+  volatile uint32_t* peer_issued = tmem_slot + 4;  // leader: loads the peer issued (teardown)
+  float* sw_s = reinterpret_cast<float*>(smem + VEC);
+  __half* bias_s = reinterpret_cast<__half*>(smem + VEC + BN * 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 = leader (issues the MMAs), 1 = peer
+  const uint32_t peer = rank ^ 1u;
+  const uint32_t peer_abort = mapa_shared(smem_u32(tmem_slot + 1), peer);
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int npairs = static_cast<int>(gridDim.x >> 1);
+  const int KB = static_cast<int>((g.K + BK - 1) / BK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);  // the leader's arrive_expect_tx for both halves
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf_bar(b), 1);
+      mbar_init(acce_bar(b), 2);  // one arrival from each CTA's epilogue
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *peer_issued = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  // barriers of both CTAs initialised and TMEM allocated before any
+  // cross-CTA arrival
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // inputs of this kernel are written by the previous one
+
+  int64_t issued = 0;    // producer: stages issued by this CTA
+  bool mma_any = false;  // leader's MMA thread: issued at least one MMA
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t full_leader0 = mapa_shared(full_bar(0), 0);
+      int64_t it = 0;
+      bool ok = true;
+      for (int t = pair; t < tiles && ok; t += npairs) {
+        const int32_t m0 = (t % tiles_m) * (2 * BM) + static_cast<int32_t>(rank) * BM;
+        const int32_t n0 = (t / tiles_m) * BN + static_cast<int32_t>(rank) * BNH;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = static_cast<int>(it % STAGES);
+          const int64_t r = it / STAGES;
+          if (it >= STAGES &&
+              !pair_wait(empty_bar(s), static_cast<uint32_t>((r - 1) & 1), false, budget, status, abort_flag, peer_abort)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = sbase + s * STAGE_BYTES;
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(s), 2 * STAGE_BYTES);
+          tma_load_2d_pair(st, &tmA, full_leader0 + 8u * s, kb * BK, m0);
+          tma_load_2d_pair(st + A_BYTES, &tmB, full_leader0 + 8u * s, kb * BK, n0);
+          ++issued;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // leader: one pair MMA of 256 x 256 x 32 per 32 bytes of K
+      constexpr uint32_t idesc = idesc_i8(2 * BM, BN);
+      int64_t it = 0;
+      int tl = 0;
+      bool ok = true;
+      for (int t = pair; t < tiles && ok; t += npairs, ++tl) {
+        const int b = tl & 1;
+        if (tl >= 2 &&
+            !pair_wait(acce_bar(b), static_cast<uint32_t>(((tl >> 1) - 1) & 1), true, budget, status, abort_flag, peer_abort))
+          break;
+        tc_fence_after();
+        const uint32_t dacc = tmem + static_cast<uint32_t>(b * BN);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = static_cast<int>(it % STAGES);
+          const uint32_t par = static_cast<uint32_t>((it / STAGES) & 1);
+          if (!pair_wait(full_bar(s), par, false, budget, status, abort_flag, peer_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = sbase + s * STAGE_BYTES;
+          const uint64_t a = sdesc_k_sw128(st);
+          const uint64_t bd = sdesc_k_sw128(st + A_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)
+            mma_i8_pair(dacc, a + 2u * k, bd + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          mma_any = true;
+          mma_commit_pair_mc(empty_bar(s), 0x3);  // frees stage s in both CTAs
+        }
+        if (ok) mma_commit_pair_mc(accf_bar(b), 0x3);  // accumulator b complete in both CTAs
+      }
+      griddep_launch_dependents();
+    } else if (lane == 0) {
+      griddep_launch_dependents();
+    }
+  } else {
+    // epilogue: 256 threads over this CTA's 128 rows x 256 columns
+    const int et = threadIdx.x - 64;
+    const int q = warp & 3;            // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;  // column half of the tile
+    const uint32_t stg0 = sbase + STG + static_cast<uint32_t>(warp - 2) * STG_WARP;
+    const uint32_t acce_leader0 = mapa_shared(acce_bar(0), 0);
+    int nst = 0;  // blocks this warp has staged (selects the buffer; two stores may be in flight)
+    const bool vec_ok = (g.N % 8) == 0;
+    int tl = 0;
+    for (int t = pair; t < tiles; t += npairs, ++tl) {
+      const int b = tl & 1;
+      const int64_t m0 = static_cast<int64_t>(t % tiles_m) * (2 * BM) + static_cast<int64_t>(rank) * BM;
+      const int64_t n0 = static_cast<int64_t>(t / tiles_m) * BN;
+      if (!OUT_I32) {
+        const int64_t n = n0 + et;
+        sw_s[et] = n < g.N ? g.sw[n] : 0.0f;
+        bias_s[et] = (g.bias != nullptr && n < g.N) ? g.bias[n] : __float2half_rn(0.0f);
+      }
+      float sxr = 0.0f;
+      if (!OUT_I32) {
+        const int64_t row = m0 + 32 * q + lane;
+        sxr = row < g.M ? g.sx[row] : 0.0f;
+      }
+      named_bar_sync(1, 32 * kEpiWarps);
+      pair_wait(accf_bar(b), static_cast<uint32_t>((tl >> 1) & 1), false, budget, status, abort_flag, peer_abort);
+      // one thread decides whether to stop and broadcasts it (double-buffered by
+      // tile parity), so every epilogue thread leaves the loop at the same point
+      if (et == 0) decision[tl & 1] = *abort_flag;
+      named_bar_sync(1, 32 * kEpiWarps);
+      if (decision[tl & 1]) break;
+      tc_fence_after();
+
+      auto taddr = [&](int c) {
+        return tmem + (static_cast<uint32_t>(32 * q) << 16) +
+               static_cast<uint32_t>(BN * b + 128 * half + 32 * c);
+      };
+      const int64_t row0 = m0 + 32 * q;  // first row of this warp's blocks
+      const int64_t row = row0 + lane;
+      auto emit = [&](int c, uint32_t (&v)[32]) {
+        const int cl = 128 * half + 32 * c;  // column within the tile
+        const int64_t col0 = n0 + cl;
+        if constexpr (OUT_I32) {
+          if (row < g.M && col0 < g.N) {
+            int32_t* dst = g.acc + row * g.N + col0;
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < g.N) dst[j] = static_cast<int32_t>(v[j]);
+          }
+          return;
+        } else {
+          // ((acc * sx) * sw + bias) in packed fp32 pairs, each lane rounded
+          // like the scalar sequence; scales and bias read as 16-byte vectors
+          __align__(16) __half h[32];
+          const uint64_t sx2 = f2_pack(sxr, sxr);
+          const float4* swv = reinterpret_cast<const float4*>(sw_s + cl);
+          const uint4* bv = reinterpret_cast<const uint4*>(bias_s + cl);
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            const float4 w0 = swv[j / 4], w1 = swv[j / 4 + 1];
+            uint64_t p[4];
+            p[0] = f2_mul_rn(f2_mul_rn(f2_pack(__int2float_rn(static_cast<int32_t>(v[j])),
+                                              __int2float_rn(static_cast<int32_t>(v[j + 1]))), sx2),
+                             f2_pack(w0.x, w0.y));
+            p[1] = f2_mul_rn(f2_mul_rn(f2_pack(__int2float_rn(static_cast<int32_t>(v[j + 2])),
+                                              __int2float_rn(static_cast<int32_t>(v[j + 3]))), sx2),
+                             f2_pack(w0.z, w0.w));
+            p[2] = f2_mul_rn(f2_mul_rn(f2_pack(__int2float_rn(static_cast<int32_t>(v[j + 4])),
+                                              __int2float_rn(static_cast<int32_t>(v[j + 5]))), sx2),
+                             f2_pack(w1.x, w1.y));
+            p[3] = f2_mul_rn(f2_mul_rn(f2_pack(__int2float_rn(static_cast<int32_t>(v[j + 6])),
+                                              __int2float_rn(static_cast<int32_t>(v[j + 7]))), sx2),
+                             f2_pack(w1.z, w1.w));
+            if (g.bias != nullptr) {
+              const uint4 b8 = bv[j / 8];
+              const uint32_t bw[4] = {b8.x, b8.y, b8.z, b8.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float2 bf = __half22float2(*reinterpret_cast<const __half2*>(&bw[u]));
+                p[u] = f2_add_rn(p[u], f2_pack(bf.x, bf.y));
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 f = f2_unpack(p[u]);
+              *reinterpret_cast<__half2*>(&h[j + 2 * u]) = __floats2half2_rn(f.x, f.y);
+            }
+          }
+          if (tma_store) {
+            // stage the 32 x 32 block in the 64-byte-swizzled image; one TMA
+            // store writes it (rows/columns outside y are skipped); two buffers
+            // per warp, so the previous block's store may still be reading one
+            const uint32_t stg = stg0 + static_cast<uint32_t>(nst & 1) * STG_BYTES;
+            if (lane == 0 && nst >= 2) bulk_wait_group_read<1>();
+            __syncwarp();
+            ++nst;
+            const uint4* hv = reinterpret_cast<const uint4*>(h);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const uint32_t addr = stg + lane * 64 + ((cc ^ ((lane >> 1) & 3)) * 16);
+              asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(hv[cc].x), "r"(hv[cc].y),
+                           "r"(hv[cc].z), "r"(hv[cc].w)
+                           : "memory");
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (row0 < g.M && col0 < g.N)
+                tma_store_2d(&tmY, stg, static_cast<int32_t>(col0), static_cast<int32_t>(row0));
+              bulk_commit_group();
+            }
+          } else if (row < g.M && col0 < g.N) {
+            __half* dst = g.y + row * g.N + col0;
+            if (vec_ok && col0 + 32 <= g.N) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                reinterpret_cast<uint4*>(dst)[j] = reinterpret_cast<const uint4*>(h)[j];
+            } else {
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < g.N) dst[j] = h[j];
+            }
+          }
+        }
+      };
+      uint32_t va[32], vb[32];
+      tmem_ld_32x32b_x32(taddr(0), va);
+      tmem_ld_wait_regs(va);
+      tmem_ld_32x32b_x32(taddr(1), vb);
+      emit(0, va);
+      tmem_ld_wait_regs(vb);
+      tmem_ld_32x32b_x32(taddr(2), va);
+      emit(1, vb);
+      tmem_ld_wait_regs(va);
+      tmem_ld_32x32b_x32(taddr(3), vb);
+      emit(2, va);
+      tmem_ld_wait_regs(vb);
+      emit(3, vb);
+      // every epilogue thread of this CTA has read accumulator b: tell the leader
+      tc_fence_before();
+      named_bar_sync(1, 32 * kEpiWarps);
+      if (et == 0) mbar_arrive_cluster(acce_leader0 + 8u * b);
+    }
+    if (lane == 0) bulk_wait_group0();  // this warp's output stores are complete
+  }
+
+  // teardown.  The peer tells the leader how many stages it loaded; after
+  // the cluster barrier both CTAs see the same abort flag (a wait that runs
+  // out raises both).  After an abort the leader waits (bounded) for its
+  // MMAs and for the last phase of every stage: a half the peer never loaded
+  // is settled with complete_tx, a half the leader never armed is armed now.
+  // Without an abort nothing is in flight any more at the first cluster
+  // barrier (every load was consumed by an MMA whose completion both
+  // epilogues waited for); after one, a second barrier keeps both CTAs
+  // resident until the drain is done.  Then TMEM is freed.
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && rank == 1)
+    st_shared_cluster_u32(mapa_shared(smem_u32(const_cast<uint32_t*>(peer_issued)), 0),
+                          static_cast<uint32_t>(issued));
+  cluster_sync_all();
+  const bool aborted = *abort_flag != 0;  // the same in both CTAs after the barrier
+  if (aborted && rank == 0) {
+    if (warp == 1 && lane == 0 && mma_any) {
+      mma_commit_pair(drain_bar);
+      mbar_drain(drain_bar, 0, budget);
+    }
+    if (threadIdx.x == 0) {
+      const int64_t pi = static_cast<int64_t>(*peer_issued);
+      for (int s = 0; s < STAGES; ++s) {
+        const int64_t lr = issued > s ? (issued - 1 - s) / STAGES + 1 : 0;  // rounds of stage s armed
+        const int64_t pr = pi > s ? (pi - 1 - s) / STAGES + 1 : 0;          // rounds the peer loaded
+        if (lr == 0 && pr == 0) continue;
+        if (lr == pr + 1) mbar_complete_tx(full_bar(s), STAGE_BYTES);
+        else if (pr == lr + 1) mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
+        const int64_t last = (lr > pr ? lr : pr) - 1;
+        mbar_drain(full_bar(s), static_cast<uint32_t>(last & 1), budget);
+      }
+    }
+  }
+  if (aborted) cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+// Clusters of two CTAs that fit on the device at once (at most one per TPC).
+int max_pairs(int device, int num_sms) {
+  static int cached[64] = {0};
+  const int d = device < 64 ? device : 63;
+  if (cached[d] > 0) return cached[d];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = SMEM;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<false>, &cfg) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    n = num_sms / 2;
+  }
+  if (n > num_sms / 2) n = num_sms / 2;
+  cached[d] = n;
+  return n;
+}
+
+template <bool OUT_I32>
+cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
+  static bool attr_set[64] = {false};
+  const int dev = c.device < 64 ? c.device : 63;
+  if (!attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_pair<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(SMEM));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k_gemm_pair<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(SMEM));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  CUtensorMap tmA, tmB, tmY;
+  if (!make_tmap_i8(&tmA, g.xq, g.K, g.M, BK, BM)) return cudaErrorInvalidValue;
+  if (!make_tmap_i8(&tmB, g.wq, g.K, g.N, BK, BNH)) return cudaErrorInvalidValue;
+  // TMA stores need 16-byte row strides (N % 8 == 0); otherwise direct stores
+  int tma_store = (!OUT_I32 && g.N % 8 == 0) ? 1 : 0;
+  if (tma_store && !make_tmap_f16_out(&tmY, g.y, g.N, g.M)) return cudaErrorInvalidValue;
+  if (!tma_store) memset(&tmY, 0, sizeof(tmY));
+  const int tiles_m = static_cast<int>((g.M + 2 * BM - 1) / (2 * BM));
+  const int tiles_n = static_cast<int>((g.N + BN - 1) / BN);
+  const int tiles = tiles_m * tiles_n;
+  const int mp = max_pairs(c.device, c.num_sms);
+  const int pairs = tiles < mp ? tiles : mp;
+  return launch_pdl(k_gemm_pair<OUT_I32>, dim3(2 * pairs), dim3(kThreads), SMEM, c.stream, tmA, tmB, tmY, g,
+                    tiles_m, tiles, tma_store, c.status, c.budget_ns);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_pair(const GemmArgs& g, const Ctx& c) {
+  if (g.acc != nullptr) return launch_cfg<true>(g, c);
+  return launch_cfg<false>(g, c);
+}
+
+}  // namespace sq

@@ -127,12 +127,12 @@ sq_status linear_impl(const int8_t* xq, const float* x_scale, const int8_t* wq,
   if (M <= 0 || N <= 0) return SQ_ERR_INVALID_ARG;
   sq_status st = check_k(K);
   if (st != SQ_OK) return st;
-  if (path < SQ_PATH_AUTO || path > SQ_PATH_SPLITK) return SQ_ERR_INVALID_ARG;
+  if (path < SQ_PATH_AUTO || path > SQ_PATH_WIDE) return SQ_ERR_INVALID_ARG;
   if (!aligned16(xq) || !aligned16(wq) || !opt_aligned(x_scale) || !opt_aligned(w_scale) ||
       !opt_aligned(bias_f16) || !opt_aligned(y_f16) || !opt_aligned(acc))
     return SQ_ERR_MISALIGNED;
   if (M > 0x7fffffffLL || N > 0x7fffffffLL) return SQ_ERR_UNSUPPORTED_SHAPE;
-  if (path == SQ_PATH_AUTO) path = (M <= SQ_SPLITK_MAX_M) ? SQ_PATH_SPLITK : SQ_PATH_TILED;
+  if (path == SQ_PATH_AUTO && M <= SQ_SPLITK_MAX_M) path = SQ_PATH_SPLITK;
   if (path == SQ_PATH_SPLITK && M > SQ_SPLITK_MAX_M) return SQ_ERR_UNSUPPORTED_SHAPE;
 
   Ctx ctx;
@@ -157,8 +157,12 @@ sq_status linear_impl(const int8_t* xq, const float* x_scale, const int8_t* wq,
     if (workspace == nullptr || ws_bytes < need || !aligned16(workspace)) return SQ_ERR_WORKSPACE;
     return launched(launch_gemm_splitk(g, ctx));
   }
-  // 256-row tiles once the token count fills them; 128-row tiles below that
-  return launched(M > 128 ? launch_gemm_wide(g, ctx) : launch_gemm_tiled(g, ctx));
+  if (path == SQ_PATH_PAIR) return launched(launch_gemm_pair(g, ctx));
+  if (path == SQ_PATH_WIDE) return launched(launch_gemm_wide(g, ctx));
+  if (path == SQ_PATH_TILED) return launched(launch_gemm_tiled(g, ctx));
+  // automatic: 256-row tiles on CTA pairs once the token count fills them,
+  // single-CTA 128-row tiles below that
+  return launched(M > 128 ? launch_gemm_pair(g, ctx) : launch_gemm_tiled(g, ctx));
 }
 
 }  // namespace

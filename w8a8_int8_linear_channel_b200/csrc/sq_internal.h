@@ -82,6 +82,7 @@ struct GemmArgs {
 
 cudaError_t launch_gemm_tiled(const GemmArgs& g, const Ctx& c);  // 128 x 256 tiles
 cudaError_t launch_gemm_wide(const GemmArgs& g, const Ctx& c);   // 256 x 256 tiles, persistent
+cudaError_t launch_gemm_pair(const GemmArgs& g, const Ctx& c);   // 256 x 256 tiles on CTA pairs
 cudaError_t launch_gemm_splitk(const GemmArgs& g, const Ctx& c);
 size_t splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
 
