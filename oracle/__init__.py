@@ -72,6 +72,10 @@ def _declare(L):
         "oracle_fold_weight": [_P, _I, _I, _P, _P],
         "oracle_quantize_weight": [_P, _I, _I, _P, _P],
         "oracle_ln_quant_act": [_P, _I, _I, _I, _P, _P, _P, _F, _P, _P, _P],
+        "oracle_quantize_weight_tensor": [_P, _I, _I, _P, _P, _P],
+        "oracle_ln_quant_act_tensor": [_P, _I, _I, _I, _P, _P, _P, _F, _P, _P, _P, _P],
+        "oracle_ln_quant_act_static": [_P, _I, _I, _I, _P, _P, _P, _F, _F, _P, _P, _P],
+        "oracle_tensor_range": [_P, _P, _I],
         "oracle_int_gemm": [_P, _P, _I, _I, _I, _P],
         "oracle_int_gemm64": [_P, _P, _I, _I, _I, _P],
         "oracle_dequant": [_P, _P, _P, _P, _I, _I, _P],
@@ -82,7 +86,8 @@ def _declare(L):
     for name, args in sig.items():
         fn = getattr(L, name)
         fn.argtypes = args
-        fn.restype = ctypes.c_int if name == "oracle_num_threads" else None
+        fn.restype = (ctypes.c_int if name == "oracle_num_threads" else
+                      ctypes.c_float if name == "oracle_tensor_range" else None)
 
 
 def _ptr(a):
@@ -217,6 +222,53 @@ def ln_quant_act(h, gamma=None, beta=None, inv_s=None, eps: float = 1e-5):
     lib().oracle_ln_quant_act(_ptr(h), M, K, K, _ptr(gamma), _ptr(beta), _ptr(inv_s), eps,
                               _ptr(xq), _ptr(sx), _ptr(scratch))
     return xq, sx
+
+
+def quantize_weight_tensor(w):
+    """[SQ] "inference" levels O1-O3: one scale for the whole weight.
+    Returns (wq [N,K] int8, sw [N] fp32 all equal, range fp32)."""
+    w = _f16(w)
+    N, K = w.shape
+    wq = np.empty((N, K), np.int8)
+    sw = np.empty(N, np.float32)
+    rng = np.zeros(1, np.float32)
+    lib().oracle_quantize_weight_tensor(_ptr(w), N, K, _ptr(wq), _ptr(sw), _ptr(rng))
+    return wq, sw, rng[0]
+
+
+def ln_quant_act_tensor(h, gamma=None, beta=None, inv_s=None, eps: float = 1e-5):
+    """[SQ] level O2: per-tensor dynamic activation scale over the whole batch.
+    Returns (xq [M,K] int8, sx [M] fp32 all equal, range fp32)."""
+    h = _f16(h)
+    M, K = h.shape
+    gamma, beta, inv_s = _f32(gamma), _f32(beta), _f32(inv_s)
+    xq = np.empty((M, K), np.int8)
+    sx = np.empty(M, np.float32)
+    rng = np.zeros(1, np.float32)
+    scratch = np.empty(K, np.float32)
+    lib().oracle_ln_quant_act_tensor(_ptr(h), M, K, K, _ptr(gamma), _ptr(beta), _ptr(inv_s), eps,
+                                     _ptr(xq), _ptr(sx), _ptr(rng), _ptr(scratch))
+    return xq, sx, rng[0]
+
+
+def ln_quant_act_static(h, range_, gamma=None, beta=None, inv_s=None, eps: float = 1e-5):
+    """[SQ] level O3: per-tensor static activation scale range_/127 fixed
+    offline; values beyond the range saturate.  Returns (xq, sx all equal)."""
+    h = _f16(h)
+    M, K = h.shape
+    gamma, beta, inv_s = _f32(gamma), _f32(beta), _f32(inv_s)
+    xq = np.empty((M, K), np.int8)
+    sx = np.empty(M, np.float32)
+    scratch = np.empty(K, np.float32)
+    lib().oracle_ln_quant_act_static(_ptr(h), M, K, K, _ptr(gamma), _ptr(beta), _ptr(inv_s), eps,
+                                     float(np.float32(range_)), _ptr(xq), _ptr(sx), _ptr(scratch))
+    return xq, sx
+
+
+def tensor_range(amax, inv_s=None) -> np.float32:
+    """Static per-tensor range from calibrated per-channel ranges (level O3)."""
+    amax, inv_s = _f32(amax), _f32(inv_s)
+    return np.float32(lib().oracle_tensor_range(_ptr(amax), _ptr(inv_s), amax.size))
 
 
 def int_gemm(xq, wq) -> np.ndarray:

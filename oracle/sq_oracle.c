@@ -254,6 +254,84 @@ void oracle_ln_quant_act(const uint16_t* h, int64_t M, int64_t K, int64_t ld, co
   }
 }
 
+/* ------------------------------------------ per-tensor levels (O1 - O3) --- */
+/* [SQ] "inference": the efficiency levels differ only in how coarse the
+ * scales are.  O1: activations per token, dynamic; weights per tensor.
+ * O2: activations and weights per tensor, dynamic.  O3: both per tensor,
+ * static (the activation scale is fixed offline from calibration).  A
+ * per-tensor scale is the same quantizer with one range for the whole tensor:
+ *   scale = range / 127, q = clamp(rint(x * (1 / scale)), -127, 127).
+ * The scale is returned once per row (sw[n] or sx[t], all equal) so the
+ * INT8 GEMM and its dequant epilogue stay exactly as in O1. */
+
+/* Weights, one scale for all of W' [N, K]: range = max_{n,k} |W'[n, k]|. */
+void oracle_quantize_weight_tensor(const uint16_t* w, int64_t N, int64_t K, int8_t* wq, float* sw,
+                                   float* range_out) {
+  float range = 0.0f;
+  for (int64_t i = 0; i < N * K; ++i) {
+    float a = fabsf(h2f(w[i]));
+    if (a > range) range = a;
+  }
+  float sc = scale_of(range);
+  float inv = inv_of(sc);
+  for (int64_t n = 0; n < N; ++n) sw[n] = sc;
+  for (int64_t i = 0; i < N * K; ++i) wq[i] = quantize_one(h2f(w[i]), inv);
+  *range_out = range;
+}
+
+/* Level O2 activations: one dynamic range over every token of this batch,
+ * range = max_{t,k} |x_hat[t, k]|.  Two passes over the rows (the range must
+ * be known before the first code). */
+void oracle_ln_quant_act_tensor(const uint16_t* h, int64_t M, int64_t K, int64_t ld,
+                                const float* gamma, const float* beta, const float* inv_s, float eps,
+                                int8_t* xq, float* sx, float* range_out,
+                                float* scratch_row /* K floats */) {
+  float range = 0.0f;
+  for (int64_t t = 0; t < M; ++t) {
+    act_row(h + t * ld, K, gamma, beta, inv_s, eps, scratch_row);
+    for (int64_t k = 0; k < K; ++k) {
+      float a = fabsf(scratch_row[k]);
+      if (a > range) range = a;
+    }
+  }
+  float sc = scale_of(range);
+  float inv = inv_of(sc);
+  for (int64_t t = 0; t < M; ++t) {
+    act_row(h + t * ld, K, gamma, beta, inv_s, eps, scratch_row);
+    sx[t] = sc;
+    for (int64_t k = 0; k < K; ++k) xq[t * K + k] = quantize_one(scratch_row[k], inv);
+  }
+  *range_out = range;
+}
+
+/* Level O3 activations: the range was fixed offline; values outside it
+ * saturate at -127 / 127 (the clamp of quantize_one). */
+void oracle_ln_quant_act_static(const uint16_t* h, int64_t M, int64_t K, int64_t ld,
+                                const float* gamma, const float* beta, const float* inv_s, float eps,
+                                float range, int8_t* xq, float* sx, float* scratch_row /* K floats */) {
+  float sc = scale_of(range);
+  float inv = inv_of(sc);
+  for (int64_t t = 0; t < M; ++t) {
+    act_row(h + t * ld, K, gamma, beta, inv_s, eps, scratch_row);
+    sx[t] = sc;
+    for (int64_t k = 0; k < K; ++k) xq[t * K + k] = quantize_one(scratch_row[k], inv);
+  }
+}
+
+/* The static per-tensor range of the smoothed activation from calibrated
+ * per-channel ranges: max_j amax[j] (amax measured on the runtime transform,
+ * e.g. the LayerNorm with the folded gamma' / beta'), or, when the runtime
+ * multiplies by inv_s, max_j fp32(amax[j] * inv_s[j]) -- rounding is
+ * monotonic, so this is the largest |x * inv_s_j| over the calibration set. */
+float oracle_tensor_range(const float* amax, const float* inv_s, int64_t K) {
+  float range = 0.0f;
+  for (int64_t j = 0; j < K; ++j) {
+    float a = inv_s ? amax[j] * inv_s[j] : amax[j];
+    if (a > range) range = a;
+  }
+  return range;
+}
+
 /* ------------------------------------------------------------- INT8 GEMM --- */
 /* [SQ] glossary "INT8 GEMM": acc[t, n] = sum_k xq[t, k] * wq[n, k], int32.
  * K <= 133144 keeps |acc| <= 133144 * 127^2 < 2^31. */

@@ -355,3 +355,96 @@ def test_zero_scale_gives_zero_codes():
     # reciprocal; its codes are 0 and its dequantized values are exactly 0.
     q = oracle.quantize_with_scale(np.array([1.0, -2.0, 0.0], np.float32), 0.0)
     assert list(q) == [0, 0, 0]
+
+
+# ------------------------------------------------- quantization levels O1-O3 --
+def test_hand_example_levels():
+    g = load("levels_2x4.txt")
+    x = f16(g["X"])
+    xq, sx = oracle.ln_quant_act(x)
+    assert np.array_equal(sx, g["o1_sx"]) and np.array_equal(xq, g["o1_qx"])
+    xq, sx, rng_ = oracle.ln_quant_act_tensor(x)
+    assert rng_ == g["o2_range"]
+    assert np.array_equal(sx, g["o2_sx"]) and np.array_equal(xq, g["o2_qx"])
+    xq, sx = oracle.ln_quant_act_static(x, g["o3_range"])
+    assert np.array_equal(sx, g["o3_sx"]) and np.array_equal(xq, g["o3_qx"])
+    wq, sw, wr = oracle.quantize_weight_tensor(f16(g["W"]))
+    assert wr == g["wt_range"]
+    assert np.array_equal(sw, g["wt_sw"]) and np.array_equal(wq, g["wt_qw"])
+    assert oracle.tensor_range(g["cal_amax"], g["cal_inv_s"]) == g["cal_range"]
+    assert oracle.tensor_range(g["cal_amax"]) == 7.0
+
+
+def _ln_batch(seed, M=12, K=96):
+    rng = np.random.default_rng(seed)
+    h = f16(rng.standard_normal((M, K)) * 2)
+    gamma = (1 + rng.uniform(0, 3, K)).astype(np.float32)
+    gamma[rng.integers(0, K, 3)] = 60.0
+    beta = (rng.standard_normal(K) * 0.1).astype(np.float32)
+    inv_s = rng.uniform(0.05, 2.0, K).astype(np.float32)
+    return h, gamma, beta, inv_s
+
+
+def _np_codes(x, range_):
+    """Independent restatement: the same quantizer in numpy float32 arithmetic."""
+    sc = np.float32(range_) / np.float32(127)
+    inv = np.float32(1) / sc if sc > 0 else np.float32(0)
+    p = (np.asarray(x, np.float32) * inv).astype(np.float32)
+    return np.clip(np.rint(p), -127, 127).astype(np.int8), sc
+
+
+@pytest.mark.parametrize("path", ["ln", "inv_s"])
+def test_o2_is_one_range_over_the_batch(path):
+    h, gamma, beta, inv_s = _ln_batch(21)
+    kw = dict(gamma=gamma, beta=beta) if path == "ln" else dict(inv_s=inv_s)
+    xq, sx, rng_ = oracle.ln_quant_act_tensor(h, **kw)
+    x = oracle.act_rows(h, **kw)
+    assert rng_ == np.abs(x).max()
+    codes, sc = _np_codes(x, rng_)
+    assert np.all(sx == sc) and np.array_equal(xq, codes)
+    # a batch of one token: O2 is O1
+    q1, s1 = oracle.ln_quant_act(h[4:5], **kw)
+    q2, s2, _ = oracle.ln_quant_act_tensor(h[4:5], **kw)
+    assert np.array_equal(q1, q2) and np.array_equal(s1, s2)
+
+
+def test_o3_static_equals_o2_when_calibrated_on_the_batch():
+    h, gamma, beta, _ = _ln_batch(22)
+    amax = oracle.calibrate_absmax(h, gamma=gamma, beta=beta)
+    r = oracle.tensor_range(amax)
+    q3, s3 = oracle.ln_quant_act_static(h, r, gamma=gamma, beta=beta)
+    q2, s2, r2 = oracle.ln_quant_act_tensor(h, gamma=gamma, beta=beta)
+    assert r == r2 and np.array_equal(q3, q2) and np.array_equal(s3, s2)
+
+
+def test_o3_saturates_outside_the_static_range():
+    h, gamma, beta, inv_s = _ln_batch(23)
+    x = oracle.act_rows(h, inv_s=inv_s)
+    r = np.float32(np.abs(x).max() * 0.25)  # calibration saw a quarter of this batch's range
+    q, s = oracle.ln_quant_act_static(h, r, inv_s=inv_s)
+    codes, sc = _np_codes(x, r)
+    assert np.all(s == sc) and np.array_equal(q, codes)
+    big = np.abs(x) * (np.float32(1) / sc) > 127.5
+    assert big.any() and np.array_equal(q[big], np.sign(x[big]).astype(np.int8) * 127)
+
+
+def test_static_range_from_inv_s_is_the_smoothed_calibration_max():
+    h, _, _, inv_s = _ln_batch(24)
+    amax = oracle.calibrate_absmax(h)
+    r = oracle.tensor_range(amax, inv_s)
+    assert r == np.abs(oracle.act_rows(h, inv_s=inv_s)).max()
+
+
+def test_per_tensor_weight_quantization():
+    rng = np.random.default_rng(25)
+    w = f16(rng.standard_normal((20, 64)) * rng.uniform(0.1, 5, (20, 1)))
+    wq, sw, r = oracle.quantize_weight_tensor(w)
+    assert r == np.abs(w.astype(np.float32)).max()
+    codes, sc = _np_codes(w.astype(np.float32), r)
+    assert np.all(sw == sc) and np.array_equal(wq, codes)
+    # equal row ranges: per-tensor and per-channel agree
+    w2 = rng.standard_normal((8, 32))
+    w2[np.arange(8), rng.integers(0, 32, 8)] = 4.0
+    a = oracle.quantize_weight(f16(w2))
+    b = oracle.quantize_weight_tensor(f16(w2))
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])

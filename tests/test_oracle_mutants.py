@@ -29,6 +29,10 @@ MUTANTS = {
     "smooth_not_applied": ("for (int64_t k = 0; k < K; ++k) out[k] = out[k] * inv_s[k];",
                            "for (int64_t k = 0; k < K; ++k) out[k] = out[k];"),
     "zero_row_inf": ("return scale > 0.0f ? 1.0f / scale : 0.0f;", "return 1.0f / scale;"),
+    "o2_range_of_last_token": ("  for (int64_t t = 0; t < M; ++t) {\n    act_row(h + t * ld, K, gamma, beta, inv_s, eps, scratch_row);\n    for (int64_t k = 0; k < K; ++k) {",
+                               "  for (int64_t t = 0; t < M; ++t) {\n    act_row(h + t * ld, K, gamma, beta, inv_s, eps, scratch_row);\n    range = 0.0f;\n    for (int64_t k = 0; k < K; ++k) {"),
+    "tensor_range_ignores_inv_s": ("float a = inv_s ? amax[j] * inv_s[j] : amax[j];", "float a = amax[j];"),
+    "weight_tensor_scale_per_row": ("  for (int64_t n = 0; n < N; ++n) sw[n] = sc;", "  for (int64_t n = 0; n < N; ++n) sw[n] = n ? sc : 1.0f;"),
 }
 
 
