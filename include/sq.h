@@ -142,6 +142,54 @@ sq_status sq_ln_quant_act(const void* h_f16, int64_t M, int64_t K, int64_t ld,
                           const float* gamma, const float* beta, const float* inv_s, float eps,
                           int8_t* xq, float* x_scale, sq_stream_t stream);
 
+/*
+ * Per-tensor scales: the efficiency levels of the explainer (section
+ * "inference").  O1 quantizes activations per token (sq_ln_quant_act) and the
+ * weight per tensor; O2 quantizes both per tensor with dynamic scales; O3 per
+ * tensor with static scales fixed offline from calibration.  The quantizer is
+ * the same with one range for the whole tensor:
+ *   scale = range / 127,  q = clamp(rint(x * (1 / scale)), -127, 127)
+ * and the scale is written once per row (w_scale[n] or x_scale[t], all
+ * equal), so sq_w8a8_linear serves every level unchanged.  `range_out` /
+ * `range_in` point to one fp32 in device memory owned by the caller (16-byte
+ * aligned, like every pointer here).
+ */
+
+/* Per-tensor weight quantization: range = max_{n,k} |w'[n, k]| over the
+ * (optionally folded, as in sq_quantize_weight) weight, written to
+ * range_out[0]; w_scale[n] = range / 127 for every n; two passes over w.
+ *   w fp16 [N, K]; s fp32 [K] or NULL; wq int8 [N, K]; w_scale fp32 [N] */
+sq_status sq_quantize_weight_tensor(const void* w_f16, int64_t N, int64_t K, const float* s,
+                                    int8_t* wq, float* w_scale, float* range_out,
+                                    sq_stream_t stream);
+
+/* Level O2 activations: one dynamic scale for the whole batch.  range =
+ * max_{t,k} |x_hat[t, k]| (x_hat as in sq_ln_quant_act) is written to
+ * range_out[0]; x_scale[t] = range / 127 for every t.  Two passes over h
+ * (the range must be known before the first code). */
+sq_status sq_ln_quant_act_tensor(const void* h_f16, int64_t M, int64_t K, int64_t ld,
+                                 const float* gamma, const float* beta, const float* inv_s,
+                                 float eps, int8_t* xq, float* x_scale, float* range_out,
+                                 sq_stream_t stream);
+
+/* Level O3 activations: the range was fixed offline (range_in[0], e.g. from
+ * sq_tensor_range); x_scale[t] = range / 127 for every t, and values beyond
+ * the range saturate at -127 / 127.  One pass over h, no per-row max. */
+sq_status sq_ln_quant_act_static(const void* h_f16, int64_t M, int64_t K, int64_t ld,
+                                 const float* gamma, const float* beta, const float* inv_s,
+                                 float eps, const float* range_in, int8_t* xq, float* x_scale,
+                                 sq_stream_t stream);
+
+/* The static activation range for level O3 from calibrated per-channel
+ * ranges: range_out[0] = max_j amax[j], or max_j fp32(amax[j] * inv_s[j])
+ * when inv_s is given.  With the smoothing folded into a LayerNorm, calibrate
+ * on the folded gamma' / beta' and pass inv_s = NULL; for an input the runtime
+ * multiplies by inv_s, calibrate the raw input and pass inv_s (rounding is
+ * monotonic, so both give the largest |x_hat| over the calibration set).
+ *   amax, inv_s fp32 [K] (inv_s may be NULL); range_out fp32 [1] */
+sq_status sq_tensor_range(const float* amax, const float* inv_s, int64_t K, float* range_out,
+                          sq_stream_t stream);
+
 /* Bytes of workspace sq_w8a8_linear needs for this shape (0 if none).  The
  * workspace holds int32 partial sums and per-tile arrival counters of the
  * stream-K path.  The caller zero-fills it once before its first use; every

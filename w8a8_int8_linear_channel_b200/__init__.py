@@ -26,6 +26,8 @@ __all__ = [
     "SQError", "sq_calibrate_absmax", "sq_smooth_fold", "sq_quantize_weight", "sq_ln_quant_act",
     "sq_w8a8_workspace_bytes", "sq_w8a8_linear", "sq_w8a8_linear_path", "sq_w8a8_gemm_s32",
     "sq_poll_status", "sq_set_wait_budget_ns", "sq_selftest_wait_timeout", "SmoothQuantLinear",
+    "sq_quantize_weight_tensor", "sq_ln_quant_act_tensor", "sq_ln_quant_act_static", "sq_tensor_range",
+    "LEVELS",
     "PATH_AUTO", "PATH_TILED", "PATH_SPLITK", "PATH_PAIR", "PATH_WIDE", "SPLITK_MAX_M", "MAX_K", "library_path",
 ]
 
@@ -59,6 +61,10 @@ def _load() -> ctypes.CDLL:
         "sq_smooth_fold": ([P, P, I, F, P, P, P, P, P, P, P, P, I, P], S),
         "sq_quantize_weight": ([P, I, I, P, P, P, P], S),
         "sq_ln_quant_act": ([P, I, I, I, P, P, P, F, P, P, P], S),
+        "sq_quantize_weight_tensor": ([P, I, I, P, P, P, P, P], S),
+        "sq_ln_quant_act_tensor": ([P, I, I, I, P, P, P, F, P, P, P, P], S),
+        "sq_ln_quant_act_static": ([P, I, I, I, P, P, P, F, P, P, P, P], S),
+        "sq_tensor_range": ([P, P, I, P, P], S),
         "sq_w8a8_workspace_bytes": ([I, I, I], Z),
         "sq_w8a8_linear": ([P, P, P, P, P, P, I, I, I, P, Z, P], S),
         "sq_w8a8_linear_path": ([P, P, P, P, P, P, I, I, I, P, Z, S, P], S),
@@ -156,6 +162,62 @@ def sq_quantize_weight(w: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
            "sq_quantize_weight")
 
 
+def sq_quantize_weight_tensor(w: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
+                              range_out: torch.Tensor, s=None, stream=None):
+    """One INT8 scale for the whole (optionally folded) weight; w_scale [N] all equal,
+    range_out fp32 [1] receives max |w'|."""
+    N, K, ld = _rows(w, torch.float16, "w")
+    if ld != K:
+        raise ValueError("w must be contiguous")
+    if wq.dtype != torch.int8 or wq.shape != w.shape or not wq.is_contiguous():
+        raise ValueError("wq: need a contiguous int8 [N, K] tensor")
+    _vec(w_scale, N, torch.float32, "w_scale")
+    _vec(range_out, 1, torch.float32, "range_out")
+    _vec(s, K, torch.float32, "s")
+    _check(_L.sq_quantize_weight_tensor(_p(w), N, K, _p(s), _p(wq), _p(w_scale), _p(range_out),
+                                        _stream(stream)), "sq_quantize_weight_tensor")
+
+
+def _act_check(h, xq, x_scale, gamma, beta, inv_s):
+    M, K, ld = _rows(h, torch.float16, "h")
+    if xq.dtype != torch.int8 or tuple(xq.shape) != (M, K) or not xq.is_contiguous():
+        raise ValueError("xq: need a contiguous int8 [M, K] tensor")
+    _vec(x_scale, M, torch.float32, "x_scale")
+    for t, n in ((gamma, "gamma"), (beta, "beta"), (inv_s, "inv_s")):
+        _vec(t, K, torch.float32, n)
+    return M, K, ld
+
+
+def sq_ln_quant_act_tensor(h, xq, x_scale, range_out, gamma=None, beta=None, inv_s=None,
+                           eps: float = 1e-5, stream=None):
+    """Level O2: one dynamic INT8 scale for the whole batch (range_out fp32 [1] receives it x 127)."""
+    M, K, ld = _act_check(h, xq, x_scale, gamma, beta, inv_s)
+    _vec(range_out, 1, torch.float32, "range_out")
+    _check(_L.sq_ln_quant_act_tensor(_p(h), M, K, ld, _p(gamma), _p(beta), _p(inv_s), eps, _p(xq),
+                                     _p(x_scale), _p(range_out), _stream(stream)),
+           "sq_ln_quant_act_tensor")
+
+
+def sq_ln_quant_act_static(h, xq, x_scale, range_in, gamma=None, beta=None, inv_s=None,
+                           eps: float = 1e-5, stream=None):
+    """Level O3: INT8 with the static scale range_in / 127 (values beyond it saturate)."""
+    M, K, ld = _act_check(h, xq, x_scale, gamma, beta, inv_s)
+    _vec(range_in, 1, torch.float32, "range_in")
+    _check(_L.sq_ln_quant_act_static(_p(h), M, K, ld, _p(gamma), _p(beta), _p(inv_s), eps,
+                                     _p(range_in), _p(xq), _p(x_scale), _stream(stream)),
+           "sq_ln_quant_act_static")
+
+
+def sq_tensor_range(amax: torch.Tensor, range_out: torch.Tensor, inv_s=None, stream=None):
+    """range_out[0] = max_j amax[j] (* inv_s[j] when given): the static range of level O3."""
+    K = amax.numel()
+    _vec(amax, K, torch.float32, "amax")
+    _vec(inv_s, K, torch.float32, "inv_s")
+    _vec(range_out, 1, torch.float32, "range_out")
+    _check(_L.sq_tensor_range(_p(amax), _p(inv_s), K, _p(range_out), _stream(stream)), "sq_tensor_range")
+    return range_out
+
+
 def sq_ln_quant_act(h: torch.Tensor, xq: torch.Tensor, x_scale: torch.Tensor, gamma=None,
                     beta=None, inv_s=None, eps: float = 1e-5, stream=None):
     """Optional LayerNorm and smoothing, then per-token INT8 of h."""
@@ -247,6 +309,17 @@ def new_workspace(M: int, N: int, K: int, device=None) -> Optional[torch.Tensor]
 
 
 # ------------------------------------------------------------- layer API ----
+# (activation granularity, weight granularity) of each quantization level:
+# "channel" is this library's default (per-token activations, per-output-channel
+# weights); O1-O3 are the explainer's efficiency levels (section "inference").
+LEVELS = {
+    "channel": ("token", "channel"),
+    "O1": ("token", "tensor"),
+    "O2": ("tensor", "tensor"),
+    "O3": ("static", "tensor"),
+}
+
+
 class SmoothQuantLinear:
     """A quantized nn.Linear with its smoothing folded in.
 
@@ -255,21 +328,32 @@ class SmoothQuantLinear:
     and the INT8 GEMM.  All work happens in libsq kernels on the current
     stream."""
 
-    def __init__(self, wq, w_scale, bias, gamma_f, beta_f, inv_s, s, eps, smooth_inv=None):
+    def __init__(self, wq, w_scale, bias, gamma_f, beta_f, inv_s, s, eps, smooth_inv=None,
+                 level: str = "channel", act_range=None):
         self.wq, self.w_scale, self.bias = wq, w_scale, bias
         self.gamma_f, self.beta_f, self.inv_s, self.s = gamma_f, beta_f, inv_s, s
         self.smooth_inv = smooth_inv if smooth_inv is not None else inv_s  # 1/s, always kept
         self.eps = eps
+        self.level = level
+        self.act_mode = LEVELS[level][0]
+        # fp32 [1]: the static range (O3) or the per-batch range written by O2
+        self.act_range = act_range
+        if self.act_mode == "tensor" and act_range is None:
+            self.act_range = torch.zeros(1, dtype=torch.float32, device=wq.device)
         self._ws = {}
 
     @classmethod
     def from_float(cls, w: torch.Tensor, calib: torch.Tensor, alpha: float = 0.5, gamma=None,
                    beta=None, bias=None, eps: float = 1e-5, amax_x: Optional[torch.Tensor] = None,
-                   process_group=None):
+                   process_group=None, level: str = "channel"):
         """Calibrate on ``calib`` (the LayerNorm input when gamma is given, else the
         linear's input), smooth with ``alpha`` and quantize ``w`` [N, K].  With a
         process group, the activation ranges are max-reduced over its ranks so
-        every rank derives the same smoothing (data-parallel calibration)."""
+        every rank derives the same smoothing (data-parallel calibration).
+        ``level`` picks the scale granularities (see LEVELS)."""
+        if level not in LEVELS:
+            raise ValueError(f"level: one of {sorted(LEVELS)}")
+        act_mode, w_mode = LEVELS[level]
         N, K = w.shape
         dev = w.device
         if amax_x is None:
@@ -287,9 +371,27 @@ class SmoothQuantLinear:
         sq_smooth_fold(amax_x, amax_w, alpha, s, inv_s, gamma, beta, gamma_f, beta_f)
         wq = torch.empty((N, K), dtype=torch.int8, device=dev)
         w_scale = torch.empty(N, dtype=torch.float32, device=dev)
-        sq_quantize_weight(w, wq, w_scale, s=s)
+        if w_mode == "tensor":
+            w_range = torch.zeros(1, dtype=torch.float32, device=dev)
+            sq_quantize_weight_tensor(w, wq, w_scale, w_range, s=s)
+        else:
+            sq_quantize_weight(w, wq, w_scale, s=s)
         runtime_inv_s = None if gamma is not None else inv_s
-        return cls(wq, w_scale, bias, gamma_f, beta_f, runtime_inv_s, s, eps, inv_s)
+        act_range = None
+        if act_mode == "static":
+            # the static range of the runtime transform over the calibration set
+            act_range = torch.zeros(1, dtype=torch.float32, device=dev)
+            if gamma is not None:
+                amax_hat = torch.zeros(K, dtype=torch.float32, device=dev)
+                sq_calibrate_absmax(calib, amax_hat, gamma_f, beta_f, eps)
+                sq_tensor_range(amax_hat, act_range)
+            else:
+                sq_tensor_range(amax_x, act_range, inv_s=inv_s)
+            if process_group is not None:
+                import torch.distributed as dist
+                dist.all_reduce(act_range, op=dist.ReduceOp.MAX, group=process_group)
+        return cls(wq, w_scale, bias, gamma_f, beta_f, runtime_inv_s, s, eps, inv_s, level=level,
+                   act_range=act_range)
 
     def workspace(self, M: int) -> Optional[torch.Tensor]:
         N, K = self.wq.shape
@@ -306,7 +408,14 @@ class SmoothQuantLinear:
         M, K = h.shape
         xq = torch.empty((M, K), dtype=torch.int8, device=h.device) if xq is None else xq
         x_scale = torch.empty(M, dtype=torch.float32, device=h.device) if x_scale is None else x_scale
-        sq_ln_quant_act(h, xq, x_scale, self.gamma_f, self.beta_f, self.inv_s, self.eps)
+        if self.act_mode == "tensor":
+            sq_ln_quant_act_tensor(h, xq, x_scale, self.act_range, self.gamma_f, self.beta_f,
+                                   self.inv_s, self.eps)
+        elif self.act_mode == "static":
+            sq_ln_quant_act_static(h, xq, x_scale, self.act_range, self.gamma_f, self.beta_f,
+                                   self.inv_s, self.eps)
+        else:
+            sq_ln_quant_act(h, xq, x_scale, self.gamma_f, self.beta_f, self.inv_s, self.eps)
         return xq, x_scale
 
     def forward(self, h: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:

@@ -130,7 +130,39 @@ __global__ void __launch_bounds__(256) k_fold_weight(const __half* w, __half* w_
   }
 }
 
+// The per-tensor range of calibrated per-channel ranges (level O3 of the
+// explainer): max_j amax[j], or max_j fp32(amax[j] * inv_s[j]) when the
+// runtime multiplies by 1/s.  One CTA (K <= 133144: about 130 values per
+// thread).
+__global__ void __launch_bounds__(1024) k_tensor_range(const float* __restrict__ amax,
+                                                       const float* __restrict__ inv_s, int64_t K,
+                                                       float* __restrict__ range) {
+  __shared__ float red[32];
+  griddep_wait();
+  griddep_launch_dependents();
+  float m = 0.0f;
+  for (int64_t j = threadIdx.x; j < K; j += blockDim.x) {
+    const float v = inv_s ? __fmul_rn(amax[j], inv_s[j]) : amax[j];
+    m = fmaxf(m, v);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (threadIdx.x == 0) range[0] = m;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_tensor_range(const float* amax, const float* inv_s, int64_t K, float* range,
+                                const Ctx& c) {
+  return launch_pdl(k_tensor_range, dim3(1), dim3(1024), 0, c.stream, amax, inv_s, K, range);
+}
 
 cudaError_t launch_absmax_cols(const __half* x, int64_t rows, int64_t K, int64_t ld, float* amax,
                                const Ctx& c) {

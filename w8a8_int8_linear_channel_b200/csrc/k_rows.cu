@@ -239,6 +239,39 @@ __device__ __forceinline__ uint2 pack8(const float (&x)[8], float inv) {
   return make_uint2(quant4(x[0], x[1], x[2], x[3], inv), quant4(x[4], x[5], x[6], x[7], inv));
 }
 
+// The same codes for a scale fixed in advance (per-tensor levels): x * inv
+// may now leave [-127, 127], so it is clamped first (a NaN product passes
+// the clamp unchanged and still gives byte 0 as above).
+__device__ __forceinline__ float clamp127(float p) {
+  p = p > 127.0f ? 127.0f : p;
+  return p < -127.0f ? -127.0f : p;
+}
+
+__device__ __forceinline__ uint32_t quant4c(float x0, float x1, float x2, float x3, float inv) {
+  const float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const uint32_t b0 = __float_as_uint(__fadd_rn(clamp127(__fmul_rn(x0, inv)), kMagic));
+  const uint32_t b1 = __float_as_uint(__fadd_rn(clamp127(__fmul_rn(x1, inv)), kMagic));
+  const uint32_t b2 = __float_as_uint(__fadd_rn(clamp127(__fmul_rn(x2, inv)), kMagic));
+  const uint32_t b3 = __float_as_uint(__fadd_rn(clamp127(__fmul_rn(x3, inv)), kMagic));
+  return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
+
+__device__ __forceinline__ uint2 pack8c(const float (&x)[8], float inv) {
+  return make_uint2(quant4c(x[0], x[1], x[2], x[3], inv), quant4c(x[4], x[5], x[6], x[7], inv));
+}
+
+// Scale and reciprocal of a per-tensor range (same op order as per row).
+__device__ __forceinline__ void range_scale(const float* range, float& sc, float& inv) {
+  sc = __fdiv_rn(*range, 127.0f);
+  inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+}
+
+// Range pass: merge one row's max into the tensor's range (exact and
+// order-free: non-negative floats order as their bit patterns).
+__device__ __forceinline__ void range_merge(float* range, float m) {
+  atomicMax(reinterpret_cast<int*>(range), __float_as_int(m));
+}
+
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -287,12 +320,27 @@ __global__ void __launch_bounds__(kWarpThreads) k_rows_warp(const RowArgs a) {
         for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(x[i][j]));
       }
     }
+    int8_t* dst = a.q + r * a.K;
+    if (a.range_in) {  // per-tensor scale fixed in advance: no row max
+      float sc, inv;
+      range_scale(a.range_in, sc, inv);
+      if (lane == 0) a.scale[r] = sc;
+#pragma unroll
+      for (int i = 0; i < NW; ++i) {
+        const int64_t c = lane + 32 * i;
+        if (c < Kc) *reinterpret_cast<uint2*>(dst + c * 8) = pack8c(x[i], inv);
+      }
+      continue;
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (a.range_out) {  // range pass only
+      if (lane == 0) range_merge(a.range_out, amax);
+      continue;
+    }
     const float sc = __fdiv_rn(amax, 127.0f);
     const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
     if (lane == 0) a.scale[r] = sc;
-    int8_t* dst = a.q + r * a.K;
 #pragma unroll
     for (int i = 0; i < NW; ++i) {
       const int64_t c = lane + 32 * i;
@@ -473,6 +521,20 @@ __device__ __forceinline__ void cta_rows(const RowArgs& a, RowSharedT<T>& sh, fl
           }
         }
       }
+    } else if (a.range_in) {  // per-tensor scale fixed in advance: no row max, one pass
+      float sc, inv;
+      range_scale(a.range_in, sc, inv);
+      if (tid == 0) a.scale[r] = sc;
+      int8_t* dst = a.q + r * a.K;
+#pragma unroll
+      for (int i = 0; i < iters; ++i) {
+        const int64_t c = tid + static_cast<int64_t>(i) * T;
+        if (c < Kc) {
+          float x[8];
+          transform8<MODE>(chunk(i, c), c, a, mu, rstd, x);
+          *reinterpret_cast<uint2*>(dst + c * 8) = pack8c(x, inv);
+        }
+      }
     } else {
       float amax = 0.0f;
       float xs[KEEPX ? NCH : 1][8];
@@ -497,20 +559,24 @@ __device__ __forceinline__ void cta_rows(const RowArgs& a, RowSharedT<T>& sh, fl
       float m = 0.0f;
 #pragma unroll
       for (int w = 0; w < W; ++w) m = fmaxf(m, sh.mx[par][w]);
-      const float sc = __fdiv_rn(m, 127.0f);
-      const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
-      if (tid == 0) a.scale[r] = sc;
-      int8_t* dst = a.q + r * a.K;
+      if (a.range_out) {  // range pass only
+        if (tid == 0) range_merge(a.range_out, m);
+      } else {
+        const float sc = __fdiv_rn(m, 127.0f);
+        const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+        if (tid == 0) a.scale[r] = sc;
+        int8_t* dst = a.q + r * a.K;
 #pragma unroll
-      for (int i = 0; i < iters; ++i) {
-        const int64_t c = tid + static_cast<int64_t>(i) * T;
-        if (c < Kc) {
-          if constexpr (KEEPX) {
-            *reinterpret_cast<uint2*>(dst + c * 8) = pack8(xs[i], inv);
-          } else {
-            float x[8];
-            transform8<MODE>(chunk(i, c), c, a, mu, rstd, x);
-            *reinterpret_cast<uint2*>(dst + c * 8) = pack8(x, inv);
+        for (int i = 0; i < iters; ++i) {
+          const int64_t c = tid + static_cast<int64_t>(i) * T;
+          if (c < Kc) {
+            if constexpr (KEEPX) {
+              *reinterpret_cast<uint2*>(dst + c * 8) = pack8(xs[i], inv);
+            } else {
+              float x[8];
+              transform8<MODE>(chunk(i, c), c, a, mu, rstd, x);
+              *reinterpret_cast<uint2*>(dst + c * 8) = pack8(x, inv);
+            }
           }
         }
       }
@@ -604,21 +670,36 @@ __device__ __forceinline__ void cta_rows_fast(const RowArgs& a, RowSharedT<T>& s
       }
     }
     if constexpr (MODE != MODE_CALIB) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      if (lane == 0) sh.mx[par][warp] = amax;
-      __syncthreads();
-      float m = 0.0f;
-#pragma unroll
-      for (int w = 0; w < W; ++w) m = fmaxf(m, sh.mx[par][w]);
-      const float sc = __fdiv_rn(m, 127.0f);
-      const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
-      if (tid == 0) a.scale[r] = sc;
       int8_t* dst = a.q + r * a.K;
+      if (a.range_in) {  // per-tensor scale fixed in advance: no row max
+        float sc, inv;
+        range_scale(a.range_in, sc, inv);
+        if (tid == 0) a.scale[r] = sc;
 #pragma unroll
-      for (int i = 0; i < NCH; ++i) {
-        const int64_t c = tid + static_cast<int64_t>(i) * T;
-        if (c < Kc) *reinterpret_cast<uint2*>(dst + c * 8) = pack8(x[i], inv);
+        for (int i = 0; i < NCH; ++i) {
+          const int64_t c = tid + static_cast<int64_t>(i) * T;
+          if (c < Kc) *reinterpret_cast<uint2*>(dst + c * 8) = pack8c(x[i], inv);
+        }
+      } else {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (lane == 0) sh.mx[par][warp] = amax;
+        __syncthreads();
+        float m = 0.0f;
+#pragma unroll
+        for (int w = 0; w < W; ++w) m = fmaxf(m, sh.mx[par][w]);
+        if (a.range_out) {  // range pass only
+          if (tid == 0) range_merge(a.range_out, m);
+        } else {
+          const float sc = __fdiv_rn(m, 127.0f);
+          const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+          if (tid == 0) a.scale[r] = sc;
+#pragma unroll
+          for (int i = 0; i < NCH; ++i) {
+            const int64_t c = tid + static_cast<int64_t>(i) * T;
+            if (c < Kc) *reinterpret_cast<uint2*>(dst + c * 8) = pack8(x[i], inv);
+          }
+        }
       }
     }
     if (PF) {

@@ -200,6 +200,32 @@ cudaError_t launch_wait_selftest(uint64_t budget_ns, const Ctx& c) {
 
 using namespace sq;
 
+// Argument checks and row arguments shared by the per-tensor activation entry points.
+static sq_status act_args(const void* h_f16, int64_t M, int64_t K, int64_t ld, const float* gamma,
+                   const float* beta, const float* inv_s, float eps, int8_t* xq, float* x_scale,
+                   const float* range, RowArgs* a) {
+  if (!h_f16 || !xq || !x_scale || !range || M <= 0) return SQ_ERR_INVALID_ARG;
+  if (!gamma && beta) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_k(K);
+  if (st != SQ_OK) return st;
+  if ((st = check_ld(K, ld)) != SQ_OK) return st;
+  if (!aligned16(h_f16) || !aligned16(xq) || !aligned16(x_scale) || !aligned16(range) ||
+      !opt_aligned(gamma) || !opt_aligned(beta) || !opt_aligned(inv_s))
+    return SQ_ERR_MISALIGNED;
+  *a = RowArgs{};
+  a->x = static_cast<const __half*>(h_f16);
+  a->rows = M;
+  a->K = K;
+  a->ld = ld;
+  a->gamma = gamma;
+  a->beta = beta;
+  a->vec = inv_s;
+  a->eps = eps;
+  a->q = xq;
+  a->scale = x_scale;
+  return SQ_OK;
+}
+
 extern "C" {
 
 const char* sq_status_string(int status) {
@@ -217,7 +243,7 @@ const char* sq_status_string(int status) {
   }
 }
 
-int sq_abi_version(void) { return 100; }
+int sq_abi_version(void) { return 101; }
 
 sq_status sq_calibrate_absmax(const void* x_f16, int64_t rows, int64_t K, int64_t ld,
                               const float* ln_gamma, const float* ln_beta, float ln_eps,
@@ -313,6 +339,76 @@ sq_status sq_ln_quant_act(const void* h_f16, int64_t M, int64_t K, int64_t ld, c
   a.q = xq;
   a.scale = x_scale;
   return launched(launch_ln_quant_act(a, ctx));
+}
+
+sq_status sq_quantize_weight_tensor(const void* w_f16, int64_t N, int64_t K, const float* s,
+                                    int8_t* wq, float* w_scale, float* range_out,
+                                    sq_stream_t stream) {
+  if (!w_f16 || !wq || !w_scale || !range_out || N <= 0) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_k(K);
+  if (st != SQ_OK) return st;
+  if (!aligned16(w_f16) || !aligned16(wq) || !aligned16(w_scale) || !aligned16(range_out) ||
+      !opt_aligned(s))
+    return SQ_ERR_MISALIGNED;
+  Ctx ctx;
+  if ((st = current_ctx(stream, &ctx)) != SQ_OK) return st;
+  RowArgs a{};
+  a.x = static_cast<const __half*>(w_f16);
+  a.rows = N;
+  a.K = K;
+  a.ld = K;
+  a.vec = s;
+  a.q = wq;
+  a.scale = w_scale;
+  // pass 1: the range of the (folded) weight; pass 2: codes with one scale
+  if (cudaMemsetAsync(range_out, 0, sizeof(float), ctx.stream) != cudaSuccess) return launched(cudaErrorUnknown);
+  a.range_out = range_out;
+  if ((st = launched(launch_quantize_weight(a, ctx))) != SQ_OK) return st;
+  a.range_out = nullptr;
+  a.range_in = range_out;
+  return launched(launch_quantize_weight(a, ctx));
+}
+
+
+sq_status sq_ln_quant_act_tensor(const void* h_f16, int64_t M, int64_t K, int64_t ld,
+                                 const float* gamma, const float* beta, const float* inv_s,
+                                 float eps, int8_t* xq, float* x_scale, float* range_out,
+                                 sq_stream_t stream) {
+  RowArgs a;
+  sq_status st = act_args(h_f16, M, K, ld, gamma, beta, inv_s, eps, xq, x_scale, range_out, &a);
+  if (st != SQ_OK) return st;
+  Ctx ctx;
+  if ((st = current_ctx(stream, &ctx)) != SQ_OK) return st;
+  if (cudaMemsetAsync(range_out, 0, sizeof(float), ctx.stream) != cudaSuccess) return launched(cudaErrorUnknown);
+  a.range_out = range_out;
+  if ((st = launched(launch_ln_quant_act(a, ctx))) != SQ_OK) return st;
+  a.range_out = nullptr;
+  a.range_in = range_out;
+  return launched(launch_ln_quant_act(a, ctx));
+}
+
+sq_status sq_ln_quant_act_static(const void* h_f16, int64_t M, int64_t K, int64_t ld,
+                                 const float* gamma, const float* beta, const float* inv_s,
+                                 float eps, const float* range_in, int8_t* xq, float* x_scale,
+                                 sq_stream_t stream) {
+  RowArgs a;
+  sq_status st = act_args(h_f16, M, K, ld, gamma, beta, inv_s, eps, xq, x_scale, range_in, &a);
+  if (st != SQ_OK) return st;
+  Ctx ctx;
+  if ((st = current_ctx(stream, &ctx)) != SQ_OK) return st;
+  a.range_in = range_in;
+  return launched(launch_ln_quant_act(a, ctx));
+}
+
+sq_status sq_tensor_range(const float* amax, const float* inv_s, int64_t K, float* range_out,
+                          sq_stream_t stream) {
+  if (!amax || !range_out || K <= 0) return SQ_ERR_INVALID_ARG;
+  if (K > SQ_MAX_K) return SQ_ERR_K_OVERFLOW;
+  if (!aligned16(amax) || !aligned16(range_out) || !opt_aligned(inv_s)) return SQ_ERR_MISALIGNED;
+  Ctx ctx;
+  sq_status st = current_ctx(stream, &ctx);
+  if (st != SQ_OK) return st;
+  return launched(launch_tensor_range(amax, inv_s, K, range_out, ctx));
 }
 
 size_t sq_w8a8_workspace_bytes(int64_t M, int64_t N, int64_t K) {

@@ -51,6 +51,9 @@ struct RowArgs {
   int8_t* q;       // codes [rows, K]
   float* scale;    // per-row scale [rows]
   float* amax;     // calibration running max [K]
+  // per-tensor scales (levels O2 / O3 of the explainer, per-tensor weights):
+  const float* range_in;  // fixed range [1]: scale = range / 127, codes clamped, no row max
+  float* range_out;       // range pass [1]: atomic max of every row's |x_hat|, nothing else written
 };
 
 cudaError_t launch_ln_quant_act(const RowArgs& a, const Ctx& c);
@@ -63,6 +66,8 @@ cudaError_t launch_absmax_cols(const __half* x, int64_t rows, int64_t K, int64_t
 cudaError_t launch_smooth(const float* amax_x, const float* amax_w, int64_t K, float alpha,
                           float* s, float* inv_s, const float* gamma, const float* beta,
                           float* gamma_out, float* beta_out, const Ctx& c);
+cudaError_t launch_tensor_range(const float* amax, const float* inv_s, int64_t K, float* range,
+                                const Ctx& c);
 cudaError_t launch_fold_weight(const __half* w, __half* w_out, int64_t N, int64_t K,
                                const float* s, const Ctx& c);
 
