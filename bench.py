@@ -46,6 +46,12 @@ DESCR = {
 }
 STEP = ("calibrate(LN absmax) + weight absmax + smoothing/fold + fold-and-quantize weight + "
         "LN/per-token quantize + INT8 GEMM with dequant epilogue")
+LEVEL_DESCR = {
+    "channel": "activations per token (dynamic), weights per output channel",
+    "O1": "activations per token (dynamic), weights per tensor",
+    "O2": "activations per tensor (dynamic, two passes), weights per tensor",
+    "O3": "activations per tensor (static range from calibration, one clamped pass), weights per tensor",
+}
 I8_PER_BF16 = 2.0  # nominal dense INT8 : BF16 tensor throughput on B200 (4.5 : 2.25 POPS)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -60,16 +66,30 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def stage_bytes_ops(wl, M):
+# scale granularities of each level: (activations, weights); "channel" is the
+# default (per-token activations, per-output-channel weights), O1-O3 the
+# explainer's efficiency levels (section "inference")
+LEVELS = {"channel": ("token", "channel"), "O1": ("token", "tensor"), "O2": ("tensor", "tensor"),
+          "O3": ("static", "tensor")}
+
+
+def stage_bytes_ops(wl, M, level="channel"):
+    """Algorithmic bytes of every stage of the step (a per-tensor pass reads its
+    input twice) and the GEMM's 2MNK ops."""
     K, N, C = wl.K, wl.N, wl.calib
+    act, wgt = LEVELS[level]
     b = {
         "calibrate_x": 2 * C * K + 4 * K,
         "calibrate_w": 2 * N * K + 4 * K,
         "smooth_fold": 4 * K * 6,
-        "quantize_weight": 2 * N * K + N * K + 4 * N + 4 * K,
-        "ln_quant_act": 2 * M * K + M * K + 4 * M + 8 * K,
-        "w8a8_linear": M * K + N * K + 4 * M + 4 * N + 2 * M * N + (2 * N if wl.bias else 0),
     }
+    if act == "static":
+        if wl.ln:
+            b["static_calib"] = 2 * C * K + 4 * K
+        b["static_range"] = 8 * K + 4
+    b["quantize_weight"] = (2 if wgt == "tensor" else 1) * 2 * N * K + N * K + 4 * N + 4 * K
+    b["ln_quant_act"] = (2 if act == "tensor" else 1) * 2 * M * K + M * K + 4 * M + 8 * K
+    b["w8a8_linear"] = M * K + N * K + 4 * M + 4 * N + 2 * M * N + (2 * N if wl.bias else 0)
     return b, 2 * M * N * K
 
 
@@ -155,8 +175,9 @@ class Plan:
     """Device buffers and prepared C-ABI calls of one step (argument
     marshalling done once, so the per-step host cost is a few C calls)."""
 
-    def __init__(self, wl, M, rank, device, sq, torch, two_streams=False):
+    def __init__(self, wl, M, rank, device, sq, torch, two_streams=False, level="channel"):
         self.torch, self.sq, self.wl, self.M = torch, sq, wl, M
+        self.level = level
         self.two_streams = two_streams
         dev = device
         data_wl = sq_inputs.with_(wl, seed=wl.seed + 1000 * rank)  # this rank's tokens
@@ -170,8 +191,12 @@ class Plan:
         self.gamma, self.beta, self.bias = T(g), T(b), T(bias)
         K, N = wl.K, wl.N
         f32 = dict(dtype=torch.float32, device=dev)
-        self.amax = torch.zeros(2 * K, **f32)
-        self.amax_x, self.amax_w = self.amax[:K], self.amax[K:]
+        # activation ranges, weight ranges and (level O3) the folded transform's
+        # ranges, zeroed together at the start of every step
+        self.amax = torch.zeros(3 * K, **f32)
+        self.amax_x, self.amax_w, self.amax_hat = self.amax[:K], self.amax[K:2 * K], self.amax[2 * K:]
+        self.w_range = torch.zeros(4, **f32)  # per-tensor ranges (16-byte aligned slots)
+        self.a_range = torch.zeros(4, **f32)
         self.s, self.inv_s = torch.empty(K, **f32), torch.empty(K, **f32)
         self.gamma_f = torch.empty(K, **f32) if g is not None else None
         self.beta_f = torch.empty(K, **f32) if b is not None else None
@@ -187,7 +212,8 @@ class Plan:
         self.ws_bytes = 0 if self.ws is None else self.ws.numel()
         self.calib_rows = calib.shape[0]
         self.bind(self.main)
-        self.launches_per_step = len(self.calls)
+        # libsq kernels per step (a per-tensor quantization is two kernels)
+        self.launches_per_step = sum(self.kernels.values())
 
     def bind(self, main_stream):
         """(Re)build the prepared C calls for the given main stream."""
@@ -199,7 +225,8 @@ class Plan:
         side = ctypes.c_void_p(self.side.cuda_stream) if self.two_streams else stream
         eps = ctypes.c_float(1e-5)
         runtime_inv_s, ws_bytes = self.runtime_inv_s, self.ws_bytes
-        self.calls = [
+        act, wgt = LEVELS[self.level]
+        calls = [
             ("calibrate_x", L.sq_calibrate_absmax, (p(self.calib), self.calib_rows, K, K, p(self.gamma),
                                                     p(self.beta), eps, p(self.amax_x), stream)),
             ("calibrate_w", L.sq_calibrate_absmax, (p(self.w), N, K, K, None, None, eps, p(self.amax_w),
@@ -207,13 +234,39 @@ class Plan:
             ("smooth_fold", L.sq_smooth_fold, (p(self.amax_x), p(self.amax_w), K, ctypes.c_float(wl.alpha),
                                                p(self.s), p(self.inv_s), p(self.gamma), p(self.beta),
                                                p(self.gamma_f), p(self.beta_f), None, None, 0, stream)),
-            ("quantize_weight", L.sq_quantize_weight, (p(self.w), N, K, p(self.s), p(self.wq), p(self.sw),
-                                                       side)),
-            ("ln_quant_act", L.sq_ln_quant_act, (p(self.h), M, K, K, p(self.gamma_f), p(self.beta_f),
-                                                 p(runtime_inv_s), eps, p(self.xq), p(self.sx), stream)),
-            ("w8a8_linear", L.sq_w8a8_linear, (p(self.xq), p(self.sx), p(self.wq), p(self.sw), p(self.bias),
-                                               p(self.y), M, N, K, p(self.ws), ws_bytes, stream)),
         ]
+        if act == "static":  # level O3: the static range of the runtime transform
+            if self.gamma is not None:
+                calls.append(("static_calib", L.sq_calibrate_absmax,
+                              (p(self.calib), self.calib_rows, K, K, p(self.gamma_f), p(self.beta_f), eps,
+                               p(self.amax_hat), stream)))
+                calls.append(("static_range", L.sq_tensor_range, (p(self.amax_hat), None, K, p(self.a_range),
+                                                                  stream)))
+            else:
+                calls.append(("static_range", L.sq_tensor_range, (p(self.amax_x), p(self.inv_s), K,
+                                                                  p(self.a_range), stream)))
+        if wgt == "tensor":
+            calls.append(("quantize_weight", L.sq_quantize_weight_tensor,
+                          (p(self.w), N, K, p(self.s), p(self.wq), p(self.sw), p(self.w_range), side)))
+        else:
+            calls.append(("quantize_weight", L.sq_quantize_weight,
+                          (p(self.w), N, K, p(self.s), p(self.wq), p(self.sw), side)))
+        act_common = (p(self.h), M, K, K, p(self.gamma_f), p(self.beta_f), p(runtime_inv_s), eps)
+        if act == "tensor":
+            calls.append(("ln_quant_act", L.sq_ln_quant_act_tensor,
+                          act_common + (p(self.xq), p(self.sx), p(self.a_range), stream)))
+        elif act == "static":
+            calls.append(("ln_quant_act", L.sq_ln_quant_act_static,
+                          act_common + (p(self.a_range), p(self.xq), p(self.sx), stream)))
+        else:
+            calls.append(("ln_quant_act", L.sq_ln_quant_act, act_common + (p(self.xq), p(self.sx), stream)))
+        calls.append(("w8a8_linear", L.sq_w8a8_linear, (p(self.xq), p(self.sx), p(self.wq), p(self.sw),
+                                                        p(self.bias), p(self.y), M, N, K, p(self.ws),
+                                                        ws_bytes, stream)))
+        self.calls = calls
+        self.kernels = {name: (2 if (name == "quantize_weight" and wgt == "tensor") or
+                               (name == "ln_quant_act" and act == "tensor") else 1)
+                        for name, _, _ in calls}
 
     def step(self, events=None, allreduce=None):
         """Run one step.  With two streams the independent stages overlap:
@@ -354,7 +407,7 @@ def run_gpu(args):
 
     wl = sq_inputs.WORKLOADS[args.workload]
     M = args.m if args.m else wl.M
-    plan = Plan(wl, M, rank, device, sq, torch, two_streams=args.streams == 2)
+    plan = Plan(wl, M, rank, device, sq, torch, two_streams=args.streams == 2, level=args.level)
     allreduce = None
     if world > 1:
         allreduce = lambda t: dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -464,9 +517,13 @@ def run_gpu(args):
     # one graph (inputs as the step leaves them: L2-warm for the large-M
     # shapes, far larger than L2 for decode), L2 flushed before each burst
     gemm_us, gemm_mode = stage_us["w8a8_linear"], "stage loop (one event pair per launch)"
+    # about 2 ms of launches per burst: enough to amortize the event pair on a
+    # short kernel, short enough that a long kernel is still timed as a burst
+    # (not under the sustained power cap of a seconds-long loop)
+    reps = int(max(1, min(args.burst, round(2000.0 / max(stage_us["w8a8_linear"], 1.0)))))
     if use_graph:
         try:
-            plan.capture_gemm_burst(args.burst)
+            plan.capture_gemm_burst(reps)
             for _ in range(2):
                 flush()
                 plan.burst.replay()
@@ -479,15 +536,15 @@ def run_gpu(args):
                 bev[i][1].record()
             torch.cuda.synchronize()
             tb = sum(e[0].elapsed_time(e[1]) for e in bev) / args.burst_iters
-            gemm_us = 1e3 * tb / args.burst
-            gemm_mode = (f"{args.burst} back-to-back launches in one CUDA graph, events around the replay, "
+            gemm_us = 1e3 * tb / reps
+            gemm_mode = (f"{reps} back-to-back launches in one CUDA graph, events around the replay, "
                          f"mean of {args.burst_iters} replays")
         except RuntimeError:
             torch.cuda.synchronize()
     if sq.sq_poll_status() != 0:
         raise RuntimeError("device wait timed out in the GEMM burst")
 
-    nbytes, ops = stage_bytes_ops(wl, M)
+    nbytes, ops = stage_bytes_ops(wl, M, args.level)
     step_bytes = sum(nbytes.values())
     decode = M <= sq.SPLITK_MAX_M
     if decode:
@@ -500,9 +557,13 @@ def run_gpu(args):
     peaks, peak_kind = load_peaks()
     gemm_s = gemm_us * 1e-6
     prof = os.path.join(ROOT, "profiles", f"w8a8_linear_{args.workload}{'_m%d' % M if M != wl.M else ''}.md")
-    gemm_src = "k_gemm_splitk.cu" if decode else ("k_gemm_pair.cu" if M > 128 else "k_gemm_tiled.cu")
+    big = M > 128
+    pair = big and wl.K < 16384  # the library's automatic choice (sq_w8a8_linear)
+    gemm_src = ("k_gemm_splitk.cu" if decode else "k_gemm_pair.cu" if pair else
+                "k_gemm_wide.cu" if big else "k_gemm_tiled.cu")
     gemm_name = ("k_gemm_splitk (swap-AB stream-K)" if decode else
-                 "k_gemm_pair (tcgen05 cta_group::2 kind::i8, 256x256 tiles)" if M > 128 else
+                 "k_gemm_pair (tcgen05 cta_group::2 kind::i8, 256x256 tiles)" if pair else
+                 "k_gemm_wide (tcgen05 kind::i8, 256x256 tiles per CTA)" if big else
                  "k_gemm_tiled (tcgen05 kind::i8, 128x256 tiles)")
     src = os.path.join(ROOT, "w8a8_int8_linear_channel_b200", "csrc", gemm_src)
     traffic = traffic_from_profile(src, prof)
@@ -536,6 +597,7 @@ def run_gpu(args):
             "data": "synthetic (seeded PCG64, OPT-shaped with persistent outlier channels)",
             "config": {"workload": DESCR[args.workload] + ("" if M == wl.M else f" (M={M})"),
                        "M": M, "N": wl.N, "K": wl.K, "calib_tokens": wl.calib, "alpha": wl.alpha,
+                       "level": args.level, "granularity": LEVEL_DESCR[args.level],
                        "step": STEP, "streams": args.streams, "cuda_graph": use_graph,
                        **({"cuda_graph_note": graph_note} if graph_note else {}),
                        "parallelism": f"dp{world}",
@@ -556,7 +618,7 @@ def run_gpu(args):
             "e2e": e2e,
         }
         if world == 1 and not args.no_cpu_baseline:
-            result["cpu_baseline"] = oracle_baseline(wl, M, budget_s=args.cpu_budget)
+            result["cpu_baseline"] = oracle_baseline(wl, M, budget_s=args.cpu_budget, level=args.level)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -578,7 +640,7 @@ def run_e2e(plan, sq, torch, world, allreduce, steps, dist):
     def one():
         d = {k: (None if v is None else v.to(dev, non_blocking=True)) for k, v in hp.items()}
         layer = sq.SmoothQuantLinear.from_float(d["w"], d["calib"], plan.wl.alpha, d["gamma"], d["beta"],
-                                                d["bias"], process_group=pg)
+                                                d["bias"], process_group=pg, level=plan.level)
         y = layer(d["h"])
         y_host.copy_(y, non_blocking=True)
 
@@ -599,7 +661,7 @@ def run_e2e(plan, sq, torch, world, allreduce, steps, dist):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms = float(t.item())
     M, N, K = plan.M, plan.wl.N, plan.wl.K
-    nbytes, ops = stage_bytes_ops(plan.wl, M)
+    nbytes, ops = stage_bytes_ops(plan.wl, M, plan.level)
     if M <= sq.SPLITK_MAX_M:
         v, u = world * sum(nbytes.values()) * steps / (ms * 1e-3) / 1e9, "GB/s"
     else:
@@ -617,40 +679,64 @@ def oracle_sample_inputs(wl, M, c_s, n_s, m_s):
             "bias": None if bias is None else bias[:n_s]}
 
 
-def oracle_stage_times(wl, inp):
+def oracle_stage_times(wl, inp, level="channel"):
     """Time each oracle stage (as it stands) on one sample; seconds per stage."""
     import oracle
+    act, wgt = LEVELS[level]
     g, b = inp["g"], inp["b"]
-    t0 = time.perf_counter()
+    st = {}
+    t = time.perf_counter()
+
+    def lap(name):
+        nonlocal t
+        now = time.perf_counter()
+        st[name] = now - t
+        t = now
+
     ax = oracle.calibrate_absmax(inp["calib"], gamma=g, beta=b)
-    t1 = time.perf_counter()
+    lap("calibrate_x")
     aw = oracle.calibrate_absmax(inp["w"])
-    t2 = time.perf_counter()
+    lap("calibrate_w")
     s, inv_s = oracle.smooth(ax, aw, wl.alpha)
     gf, bf = oracle.fold_ln(g, b, inv_s) if g is not None else (None, None)
-    t3 = time.perf_counter()
-    wq, sw = oracle.quantize_weight(oracle.fold_weight(inp["w"], s))
-    t4 = time.perf_counter()
-    xq, sx = oracle.ln_quant_act(inp["h"], gf, bf, None if g is not None else inv_s)
-    t5 = time.perf_counter()
+    lap("smooth_fold")
+    rt_inv = None if g is not None else inv_s
+    if act == "static":
+        if g is not None:
+            ahat = oracle.calibrate_absmax(inp["calib"], gamma=gf, beta=bf)
+            lap("static_calib")
+            rng_ = oracle.tensor_range(ahat)
+        else:
+            rng_ = oracle.tensor_range(ax, inv_s)
+        lap("static_range")
+    w_f = oracle.fold_weight(inp["w"], s)
+    wq, sw = oracle.quantize_weight_tensor(w_f)[:2] if wgt == "tensor" else oracle.quantize_weight(w_f)
+    lap("quantize_weight")
+    if act == "tensor":
+        xq, sx, _ = oracle.ln_quant_act_tensor(inp["h"], gf, bf, rt_inv)
+    elif act == "static":
+        xq, sx = oracle.ln_quant_act_static(inp["h"], rng_, gf, bf, rt_inv)
+    else:
+        xq, sx = oracle.ln_quant_act(inp["h"], gf, bf, rt_inv)
+    lap("ln_quant_act")
     oracle.w8a8_linear(xq, sx, wq, sw, inp["bias"])
-    t6 = time.perf_counter()
-    return {"calibrate_x": t1 - t0, "calibrate_w": t2 - t1, "smooth_fold": t3 - t2,
-            "quantize_weight": t4 - t3, "ln_quant_act": t5 - t4, "w8a8_linear": t6 - t5}
+    lap("w8a8_linear")
+    return st
 
 
 def oracle_full_time(wl, M, st, c_s, n_s, m_s):
     """Extrapolate sampled stage times linearly to the full workload."""
     return (st["calibrate_x"] * wl.calib / c_s + st["calibrate_w"] * wl.N / n_s
-            + st["smooth_fold"] + st["quantize_weight"] * wl.N / n_s
+            + st["smooth_fold"] + st.get("static_calib", 0.0) * wl.calib / c_s + st.get("static_range", 0.0)
+            + st["quantize_weight"] * wl.N / n_s
             + st["ln_quant_act"] * M / m_s + st["w8a8_linear"] * (M * wl.N) / (m_s * n_s))
 
 
-def pick_sample(wl, M, budget_s):
+def pick_sample(wl, M, budget_s, level="channel"):
     """Sample sizes whose oracle step takes about budget_s seconds."""
     import oracle
     c_s, n_s, m_s = min(wl.calib, 16), min(wl.N, 128), min(M, 4)
-    st = oracle_stage_times(wl, oracle_sample_inputs(wl, M, c_s, n_s, m_s))
+    st = oracle_stage_times(wl, oracle_sample_inputs(wl, M, c_s, n_s, m_s), level)
     dt = sum(st.values())
     grow = max(1.0, budget_s / max(dt, 1e-6))
     # grow the token and weight samples together (the GEMM is ~ m_s * n_s)
@@ -661,12 +747,12 @@ def pick_sample(wl, M, budget_s):
     return c_s, n_s, m_s
 
 
-def oracle_baseline(wl, M, budget_s):
+def oracle_baseline(wl, M, budget_s, level="channel"):
     import oracle
-    c_s, n_s, m_s = pick_sample(wl, M, budget_s)
-    st = oracle_stage_times(wl, oracle_sample_inputs(wl, M, c_s, n_s, m_s))
+    c_s, n_s, m_s = pick_sample(wl, M, budget_s, level)
+    st = oracle_stage_times(wl, oracle_sample_inputs(wl, M, c_s, n_s, m_s), level)
     full = oracle_full_time(wl, M, st, c_s, n_s, m_s)
-    nbytes, ops = stage_bytes_ops(wl, M)
+    nbytes, ops = stage_bytes_ops(wl, M, level)
     if M <= 32:
         v, u = sum(nbytes.values()) / full / 1e9, "GB/s"
     else:
@@ -688,18 +774,18 @@ def run_reference(args):
     wl = sq_inputs.WORKLOADS[args.workload]
     M = args.m if args.m else wl.M
     per_step = max(0.02, min(10.0, args.ref_budget / max(1, args.steps + args.warmup)))
-    c_s, n_s, m_s = pick_sample(wl, M, per_step)
+    c_s, n_s, m_s = pick_sample(wl, M, per_step, args.level)
     inp = oracle_sample_inputs(wl, M, c_s, n_s, m_s)
     for _ in range(args.warmup):
-        oracle_stage_times(wl, inp)
+        oracle_stage_times(wl, inp, args.level)
     fulls = []
     work = 0.0
     for _ in range(args.steps):
-        st = oracle_stage_times(wl, inp)
+        st = oracle_stage_times(wl, inp, args.level)
         work += sum(st.values())
         fulls.append(oracle_full_time(wl, M, st, c_s, n_s, m_s))
     full = sum(fulls) / len(fulls)
-    nbytes, ops = stage_bytes_ops(wl, M)
+    nbytes, ops = stage_bytes_ops(wl, M, args.level)
     if M <= 32:
         v, u = sum(nbytes.values()) / full / 1e9, "GB/s"
     else:
@@ -711,7 +797,9 @@ def run_reference(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
             "impl": "reference",
             "config": {"workload": DESCR[args.workload] + ("" if M == wl.M else f" (M={M})"), "M": M,
-                       "N": wl.N, "K": wl.K, "step": STEP, "parallelism": "cpu oracle, rank 0"},
+                       "N": wl.N, "K": wl.K, "calib_tokens": wl.calib, "alpha": wl.alpha,
+                       "level": args.level, "granularity": LEVEL_DESCR[args.level], "step": STEP,
+                       "parallelism": "cpu oracle, rank 0"},
             "cpu_baseline": {"value": round(v, 6), "unit": u, "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(v, 6), "unit": u, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -726,10 +814,13 @@ def main():
     ap.add_argument("--impl", choices=["sq", "reference"], default="sq")
     ap.add_argument("--workload", choices=sorted(DESCR), default="attn")
     ap.add_argument("--m", type=int, default=0, help="token count override (decode sweep)")
+    ap.add_argument("--level", choices=["channel", "O1", "O2", "O3"], default="channel",
+                    help="scale granularities (default: per-token activations, per-channel weights)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--stage-steps", type=int, default=300, help="steps of the per-stage timing loop")
-    ap.add_argument("--burst", type=int, default=20, help="back-to-back GEMM launches per timed burst")
+    ap.add_argument("--burst", type=int, default=20,
+                    help="most back-to-back GEMM launches per timed burst (fewer for long kernels)")
     ap.add_argument("--burst-iters", type=int, default=20, help="timed bursts (roofline launch duration)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the step's kernels eagerly instead of replaying a captured CUDA graph")

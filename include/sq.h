@@ -208,9 +208,9 @@ size_t sq_w8a8_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *   bias fp16 [N] or NULL; y fp16 [M, N]
  * M <= SQ_SPLITK_MAX_M runs the weight-streaming stream-K kernel and needs
  * sq_w8a8_workspace_bytes(M, N, K) bytes of workspace; 32 < M <= 128 runs the
- * tiled tensor-core kernel (128 x 256 tiles) and M > 128 the persistent
- * CTA-pair kernel (256 x 256 tiles, tcgen05 cta_group::2); neither needs a
- * workspace (it may be NULL).
+ * tiled tensor-core kernel (128 x 256 tiles) and M > 128 a persistent kernel
+ * of 256 x 256 tiles: on CTA pairs (tcgen05 cta_group::2) for K < 16384, on
+ * single CTAs for longer K; none of these needs a workspace (it may be NULL).
  */
 sq_status sq_w8a8_linear(const int8_t* xq, const float* x_scale, const int8_t* wq,
                          const float* w_scale, const void* bias_f16, void* y_f16, int64_t M,

@@ -59,6 +59,23 @@ constexpr size_t SMEM = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
 static_assert(SMEM <= 232448, "shared memory per CTA");
 constexpr uint32_t TMEM_COLS = 512;
 
+// Tile t -> (token tile, channel tile), grouped: groups of kGroupM token
+// tiles walk every channel tile, token tile fastest.  The 74 tiles in flight
+// at a time then span about 8 token tiles x 9 channel tiles, so each operand
+// panel they read is shared by several of them in L2 (token-tile-fastest over
+// all token tiles would span 32 x 2.3 tiles for 8192 tokens and re-read every
+// token panel from DRAM for each group of channel tiles).
+constexpr int kGroupM = 8;
+
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn) {
+  const int g = t / (kGroupM * tiles_n);
+  const int first = g * kGroupM;
+  const int gm = tiles_m - first < kGroupM ? tiles_m - first : kGroupM;
+  const int r = t - g * kGroupM * tiles_n;
+  tm = first + r % gm;
+  tn = r / gm;
+}
+
 // Bounded wait that, when it runs out, also raises the other CTA's abort
 // flag so the pair stops together.  Barriers completed by the other CTA's
 // threads (cluster_scope) are polled without suspending.
@@ -109,6 +126,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int pair = static_cast<int>(blockIdx.x >> 1);
   const int npairs = static_cast<int>(gridDim.x >> 1);
   const int KB = static_cast<int>((g.K + BK - 1) / BK);
+  const int tiles_n = tiles / tiles_m;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -147,8 +165,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int64_t it = 0;
       bool ok = true;
       for (int t = pair; t < tiles && ok; t += npairs) {
-        const int32_t m0 = (t % tiles_m) * (2 * BM) + static_cast<int32_t>(rank) * BM;
-        const int32_t n0 = (t / tiles_m) * BN + static_cast<int32_t>(rank) * BNH;
+        int tm, tn;
+        tile_coords(t, tiles_m, tiles_n, tm, tn);
+        const int32_t m0 = tm * (2 * BM) + static_cast<int32_t>(rank) * BM;
+        const int32_t n0 = tn * BN + static_cast<int32_t>(rank) * BNH;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = static_cast<int>(it % STAGES);
           const int64_t r = it / STAGES;
@@ -214,8 +234,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int tl = 0;
     for (int t = pair; t < tiles; t += npairs, ++tl) {
       const int b = tl & 1;
-      const int64_t m0 = static_cast<int64_t>(t % tiles_m) * (2 * BM) + static_cast<int64_t>(rank) * BM;
-      const int64_t n0 = static_cast<int64_t>(t / tiles_m) * BN;
+      int tm, tn;
+      tile_coords(t, tiles_m, tiles_n, tm, tn);
+      const int64_t m0 = static_cast<int64_t>(tm) * (2 * BM) + static_cast<int64_t>(rank) * BM;
+      const int64_t n0 = static_cast<int64_t>(tn) * BN;
       if (!OUT_I32) {
         const int64_t n = n0 + et;
         sw_s[et] = n < g.N ? g.sw[n] : 0.0f;
