@@ -215,14 +215,17 @@ class Plan:
         # libsq kernels per step (a per-tensor quantization is two kernels)
         self.launches_per_step = sum(self.kernels.values())
 
-    def bind(self, main_stream):
-        """(Re)build the prepared C calls for the given main stream."""
+    def bind(self, main_stream, single=False):
+        """(Re)build the prepared C calls for the given main stream (all of them
+        on it when `single`, else the weight stages on the side stream when the
+        plan uses two streams)."""
         torch, wl, M = self.torch, self.wl, self.M
         K, N = wl.K, wl.N
         L = self.sq._L
         p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+        self.cur = main_stream
         stream = ctypes.c_void_p(main_stream.cuda_stream)
-        side = ctypes.c_void_p(self.side.cuda_stream) if self.two_streams else stream
+        side = ctypes.c_void_p(self.side.cuda_stream) if self.two_streams and not single else stream
         eps = ctypes.c_float(1e-5)
         runtime_inv_s, ws_bytes = self.runtime_inv_s, self.ws_bytes
         act, wgt = LEVELS[self.level]
@@ -295,19 +298,18 @@ class Plan:
                     allreduce(self.amax_x)
                 self._call(name, fn, args)
             return
-        c = dict((n, (fn, args)) for n, fn, args in self.calls)
-        self.side.wait_stream(self.main)               # amax zeroed, previous step done
-        self._call("calibrate_x", *c["calibrate_x"])
-        self._call("calibrate_w", *c["calibrate_w"])   # side
-        self.main.wait_stream(self.side)
-        if allreduce is not None:
-            allreduce(self.amax_x)
-        self._call("smooth_fold", *c["smooth_fold"])
-        self.side.wait_stream(self.main)
-        self._call("quantize_weight", *c["quantize_weight"])  # side
-        self._call("ln_quant_act", *c["ln_quant_act"])
-        self.main.wait_stream(self.side)
-        self._call("w8a8_linear", *c["w8a8_linear"])
+        main = self.cur
+        self.side.wait_stream(main)                    # amax zeroed, previous step done
+        for name, fn, args in self.calls:
+            if name == "smooth_fold":                  # needs both ranges
+                main.wait_stream(self.side)
+                if allreduce is not None:
+                    allreduce(self.amax_x)
+            if name == "quantize_weight":              # needs s
+                self.side.wait_stream(main)
+            if name == "w8a8_linear":                  # needs wq and xq
+                main.wait_stream(self.side)
+            self._call(name, fn, args)                 # calibrate_w / quantize_weight run on side
 
     def capture(self, world):
         """Capture the step into CUDA graphs: one graph for N = 1; for N > 1 two
@@ -324,11 +326,14 @@ class Plan:
             for i, seg in enumerate(segs):
                 gr = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(gr, stream=cap):
-                    if i == 0:
-                        self.amax.zero_()
-                    for name, fn, args in self.calls:
-                        if name in seg:
-                            self._call(name, fn, args)
+                    if self.two_streams:  # the side stream forks from and joins the capture
+                        self.step()
+                    else:
+                        if i == 0:
+                            self.amax.zero_()
+                        for name, fn, args in self.calls:
+                            if name in seg:
+                                self._call(name, fn, args)
                 self.graphs.append(gr)
         self.bind(self.main)
         self.main.wait_stream(cap)
@@ -343,7 +348,7 @@ class Plan:
         cap = torch.cuda.Stream()
         cap.wait_stream(self.main)
         with torch.cuda.stream(cap):
-            self.bind(cap)
+            self.bind(cap, single=True)
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr, stream=cap):
                 self.amax.zero_()
@@ -364,7 +369,7 @@ class Plan:
         cap = torch.cuda.Stream()
         cap.wait_stream(self.main)
         with torch.cuda.stream(cap):
-            self.bind(cap)
+            self.bind(cap, single=True)
             name, fn, args = self.calls[-1]
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr, stream=cap):
@@ -429,7 +434,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     if sq.sq_poll_status() != 0:
         raise RuntimeError("device wait timed out during warm-up")
-    use_graph = not args.no_graph and plan.two_streams is False
+    use_graph = not args.no_graph and (not plan.two_streams or world == 1)
     graph_note = None
     if use_graph:
         try:
@@ -609,6 +614,12 @@ def run_gpu(args):
                                  if stage_mode == "graph" else "eager launches") + ")"},
             "roofline": roof,
             "stage_us": {k: round(v, 2) for k, v in stage_us.items()},
+            # side kernels are HBM-bound: algorithmic bytes / stage time, and its
+            # share of the measured copy bandwidth (stage times carry the event
+            # pair's few microseconds, so small stages read low)
+            "stage_gbs": {k: round(nbytes[k] / (v * 1e-6) / 1e9, 1) for k, v in stage_us.items() if v > 0},
+            "stage_hbm_frac": {k: round(nbytes[k] / (v * 1e-6) / 1e9 / float(peaks["hbm_gbs"]), 3)
+                               for k, v in stage_us.items() if v > 0 and (k != "w8a8_linear" or decode)},
             "gpu_launches": plan.launches_per_step * args.steps,
             "launch": ("the step captured once into a CUDA graph and replayed (the C-ABI calls are "
                        "capture-safe); every libsq kernel uses programmatic dependent launch"
@@ -824,7 +835,7 @@ def main():
     ap.add_argument("--burst-iters", type=int, default=20, help="timed bursts (roofline launch duration)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the step's kernels eagerly instead of replaying a captured CUDA graph")
-    ap.add_argument("--streams", type=int, choices=[1, 2], default=1,
+    ap.add_argument("--streams", type=int, choices=[1, 2], default=2,
                     help="2: run the independent stages of a step on two streams")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU work")
