@@ -80,6 +80,7 @@ def _declare(L):
         "oracle_int_gemm64": [_P, _P, _I, _I, _I, _P],
         "oracle_dequant": [_P, _P, _P, _P, _I, _I, _P],
         "oracle_w8a8_linear": [_P, _P, _P, _P, _P, _I, _I, _I, _P],
+        "oracle_w8a8_linear_quant_static": [_P, _P, _P, _P, _P, ctypes.c_int, _P, _F, _I, _I, _I, _P, _P],
         "oracle_num_threads": [],
         "oracle_set_num_threads": [ctypes.c_int],
     }
@@ -314,6 +315,25 @@ def w8a8_linear(xq, sx, wq, sw, bias=None) -> np.ndarray:
     y = np.empty((M, N), np.float16)
     lib().oracle_w8a8_linear(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias), M, N, K, _ptr(y))
     return y
+
+
+def w8a8_linear_quant_static(xq, sx, wq, sw, bias=None, relu=False, inv_s_next=None,
+                             range_next=1.0):
+    """[SQ] producer-side quantization: the linear, an optional ReLU, the next
+    linear's 1/s and its static (level O3) quantization, composed.  Returns
+    (q_next [M,N] int8, sx_next [M] fp32 all equal)."""
+    xq = np.ascontiguousarray(xq, np.int8)
+    wq = np.ascontiguousarray(wq, np.int8)
+    M, K = xq.shape
+    N = wq.shape[0]
+    sx, sw, inv_s_next = _f32(sx), _f32(sw), _f32(inv_s_next)
+    bias = _f16(bias) if bias is not None else None
+    q = np.empty((M, N), np.int8)
+    s_next = np.empty(M, np.float32)
+    lib().oracle_w8a8_linear_quant_static(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias), int(bool(relu)),
+                                          _ptr(inv_s_next), float(np.float32(range_next)), M, N, K,
+                                          _ptr(q), _ptr(s_next))
+    return q, s_next
 
 
 # ------------------------------------------------------- fp64 mathematics ----

@@ -387,6 +387,39 @@ void oracle_w8a8_linear(const int8_t* xq, const float* sx, const int8_t* wq, con
     }
 }
 
+/* ------------------------------------- producer-side quantization (fused) --- */
+/* [SQ] "what it does mathematically" folds s into the layer that produces a
+ * linear's input; with the next linear at level O3 ("inference": one static
+ * activation scale), the producing linear can hand over INT8 codes directly.
+ * The result is defined as the plain composition of the steps above:
+ *   y    = fp16(((float)acc * sx[t]) * sw[n] + bias[n])     (the linear's output)
+ *   a    = relu ? max(y, 0) : y                            (fp16 activation)
+ *   x    = (float)a * inv_s_next[n]                        (the next linear's X diag(s)^-1)
+ *   q    = clamp(rint(x * (1 / scale)), -127, 127),  scale = range_next / 127
+ * and sx_next[t] = scale for every token.  inv_s_next may be NULL (x = a). */
+void oracle_w8a8_linear_quant_static(const int8_t* xq, const float* sx, const int8_t* wq,
+                                     const float* sw, const uint16_t* bias, int relu,
+                                     const float* inv_s_next, float range_next, int64_t M,
+                                     int64_t N, int64_t K, int8_t* q_next, float* sx_next) {
+  float sc = scale_of(range_next);
+  float inv = inv_of(sc);
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < M; ++t) {
+    sx_next[t] = sc;
+    for (int64_t n = 0; n < N; ++n) {
+      int32_t sum = 0;
+      for (int64_t k = 0; k < K; ++k) sum += (int32_t)xq[t * K + k] * (int32_t)wq[n * K + k];
+      float v = (float)sum * sx[t];
+      v = v * sw[n];
+      if (bias) v = v + h2f(bias[n]);
+      float a = h2f(f2h(v));
+      if (relu && !(a > 0.0f)) a = 0.0f;
+      float x = inv_s_next ? a * inv_s_next[n] : a;
+      q_next[t * N + n] = quantize_one(x, inv);
+    }
+  }
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

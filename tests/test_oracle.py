@@ -448,3 +448,35 @@ def test_per_tensor_weight_quantization():
     a = oracle.quantize_weight(f16(w2))
     b = oracle.quantize_weight_tensor(f16(w2))
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+# ------------------------------------------- producer-side quantization ----
+def test_hand_example_producer_quant():
+    g = load("producer_quant_2x3.txt")
+    args = (g["xq"].astype(np.int8), g["sx"], g["wq"].astype(np.int8), g["sw"], f16(g["bias"]))
+    q, s = oracle.w8a8_linear_quant_static(*args, relu=True, inv_s_next=g["inv_s"], range_next=g["range"])
+    assert np.array_equal(q, g["q_relu"]) and np.array_equal(s, g["sx_next"])
+    q, s = oracle.w8a8_linear_quant_static(*args, relu=False, inv_s_next=g["inv_s"], range_next=g["range"])
+    assert np.array_equal(q, g["q_plain"])
+
+
+@pytest.mark.parametrize("relu", [False, True])
+def test_producer_quant_is_linear_then_static_quant(relu):
+    """Independent restatement in numpy float32 of everything after the
+    (separately pinned) fp16 linear output."""
+    rng = np.random.default_rng(31 + relu)
+    M, N, K = 9, 40, 64
+    xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    wq = rng.integers(-127, 128, (N, K)).astype(np.int8)
+    sx = rng.uniform(1e-3, 1e-2, M).astype(np.float32)
+    sw = rng.uniform(1e-3, 1e-2, N).astype(np.float32)
+    bias = f16(rng.standard_normal(N) * 0.1)
+    inv = rng.uniform(0.1, 3.0, N).astype(np.float32)
+    y = oracle.w8a8_linear(xq, sx, wq, sw, bias).astype(np.float32)
+    a = np.where(y > 0, y, np.float32(0)) if relu else y
+    x = (a * inv[None, :]).astype(np.float32)
+    r = np.float32(np.abs(x).max() * 0.7)  # some values saturate
+    codes, sc = _np_codes(x, r)
+    q, s = oracle.w8a8_linear_quant_static(xq, sx, wq, sw, bias, relu=relu, inv_s_next=inv, range_next=r)
+    assert np.all(s == sc) and np.array_equal(q, codes)
+    assert (np.abs(q) == 127).any()

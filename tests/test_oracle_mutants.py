@@ -32,6 +32,9 @@ MUTANTS = {
     "o2_range_of_last_token": ("  for (int64_t t = 0; t < M; ++t) {\n    act_row(h + t * ld, K, gamma, beta, inv_s, eps, scratch_row);\n    for (int64_t k = 0; k < K; ++k) {",
                                "  for (int64_t t = 0; t < M; ++t) {\n    act_row(h + t * ld, K, gamma, beta, inv_s, eps, scratch_row);\n    range = 0.0f;\n    for (int64_t k = 0; k < K; ++k) {"),
     "tensor_range_ignores_inv_s": ("float a = inv_s ? amax[j] * inv_s[j] : amax[j];", "float a = amax[j];"),
+    "producer_relu_dropped": ("if (relu && !(a > 0.0f)) a = 0.0f;", "if (relu && 0) a = 0.0f;"),
+    "producer_no_fp16_round": ("float a = h2f(f2h(v));", "float a = v;"),
+    "producer_inv_s_not_applied": ("float x = inv_s_next ? a * inv_s_next[n] : a;", "float x = a;"),
     "weight_tensor_scale_per_row": ("  for (int64_t n = 0; n < N; ++n) sw[n] = sc;", "  for (int64_t n = 0; n < N; ++n) sw[n] = n ? sc : 1.0f;"),
 }
 
