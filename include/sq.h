@@ -217,6 +217,33 @@ sq_status sq_w8a8_linear(const int8_t* xq, const float* x_scale, const int8_t* w
                          int64_t N, int64_t K, void* workspace, size_t ws_bytes,
                          sq_stream_t stream);
 
+/*
+ * Producer-side quantization: the linear with the NEXT linear's input
+ * quantization fused into its epilogue (the smoothing of the next linear
+ * folded into the layer that produces its input -- section "what it does
+ * mathematically" -- at level O3 of section "inference": one static
+ * activation scale).  Per element, in this order:
+ *   y = fp16( (fp32(acc) * x_scale[t]) * w_scale[n] + fp32(bias[n]) )  (as sq_w8a8_linear)
+ *   a = relu ? max(y, 0) : y
+ *   x = fp32(a) * inv_s_next[n]                  (x = a when inv_s_next is NULL)
+ *   xq_next[t, n] = clamp(rint(x * (1 / scale)), -127, 127),  scale = range_next[0] / 127
+ * and x_scale_next[t] = scale for every t, so (xq_next, x_scale_next) feed
+ * the next sq_w8a8_linear directly: the fp16 y never reaches memory (1 byte
+ * written per output instead of 2 written + 3 moved by a separate
+ * quantization pass).  range_next is the next linear's static input range
+ * (sq_tensor_range).  A per-token dynamic scale cannot be fused this way:
+ * a token's maximum spans every output tile of its row.
+ *   xq int8 [M, K]; x_scale fp32 [M]; wq int8 [N, K]; w_scale fp32 [N];
+ *   bias fp16 [N] or NULL; inv_s_next fp32 [N] or NULL; range_next fp32 [1];
+ *   xq_next int8 [M, N]; x_scale_next fp32 [M].  N % 16 == 0 (the next
+ *   linear's K).  M <= SQ_SPLITK_MAX_M needs the stream-K workspace.
+ */
+sq_status sq_w8a8_linear_quant(const int8_t* xq, const float* x_scale, const int8_t* wq,
+                               const float* w_scale, const void* bias_f16, int relu,
+                               const float* inv_s_next, const float* range_next, int8_t* xq_next,
+                               float* x_scale_next, int64_t M, int64_t N, int64_t K, void* workspace,
+                               size_t ws_bytes, sq_stream_t stream);
+
 /* Kernel choice for sq_w8a8_linear_path. */
 typedef enum sq_gemm_path {
   SQ_PATH_AUTO = 0,   /* what sq_w8a8_linear does */

@@ -27,7 +27,7 @@ __all__ = [
     "sq_w8a8_workspace_bytes", "sq_w8a8_linear", "sq_w8a8_linear_path", "sq_w8a8_gemm_s32",
     "sq_poll_status", "sq_set_wait_budget_ns", "sq_selftest_wait_timeout", "SmoothQuantLinear",
     "sq_quantize_weight_tensor", "sq_ln_quant_act_tensor", "sq_ln_quant_act_static", "sq_tensor_range",
-    "LEVELS",
+    "LEVELS", "sq_w8a8_linear_quant",
     "PATH_AUTO", "PATH_TILED", "PATH_SPLITK", "PATH_PAIR", "PATH_WIDE", "SPLITK_MAX_M", "MAX_K", "library_path",
 ]
 
@@ -70,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "sq_w8a8_linear_path": ([P, P, P, P, P, P, I, I, I, P, Z, S, P], S),
         "sq_w8a8_gemm_s32": ([P, P, P, I, I, I, P, Z, S, P], S),
         "sq_w8a8_linear_noalloc": ([P, P, P, P, P, P, I, I, I, P], S),
+        "sq_w8a8_linear_quant": ([P, P, P, P, P, S, P, P, P, P, I, I, I, P, Z, P], S),
         "sq_poll_status": ([P], S),
         "sq_set_wait_budget_ns": ([ctypes.c_uint64], None),
         "sq_selftest_wait_timeout": ([ctypes.c_uint64, P], S),
@@ -270,6 +271,27 @@ def sq_w8a8_gemm_s32(xq, wq, acc, workspace=None, path: int = PATH_AUTO, stream=
     _check(_L.sq_w8a8_gemm_s32(_p(xq), _p(wq), _p(acc), M, N, K, _p(workspace), ws_bytes, path,
                                _stream(stream)), "sq_w8a8_gemm_s32")
     return acc
+
+
+def sq_w8a8_linear_quant(xq, x_scale, wq, w_scale, range_next, xq_next, x_scale_next, bias=None,
+                         relu: bool = False, inv_s_next=None, workspace=None, stream=None):
+    """The linear with the next linear's static (level O3) input quantization
+    fused into its epilogue: optional ReLU, times inv_s_next, INT8 codes
+    xq_next [M, N] with x_scale_next [M] = range_next / 127."""
+    M, N, K = _gemm_shapes(xq, wq)
+    _vec(x_scale, M, torch.float32, "x_scale")
+    _vec(w_scale, N, torch.float32, "w_scale")
+    _vec(bias, N, torch.float16, "bias")
+    _vec(inv_s_next, N, torch.float32, "inv_s_next")
+    _vec(range_next, 1, torch.float32, "range_next")
+    _vec(x_scale_next, M, torch.float32, "x_scale_next")
+    if xq_next.dtype != torch.int8 or tuple(xq_next.shape) != (M, N) or not xq_next.is_contiguous():
+        raise ValueError("xq_next: need a contiguous int8 [M, N] tensor")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_L.sq_w8a8_linear_quant(_p(xq), _p(x_scale), _p(wq), _p(w_scale), _p(bias), int(bool(relu)),
+                                   _p(inv_s_next), _p(range_next), _p(xq_next), _p(x_scale_next), M, N, K,
+                                   _p(workspace), ws_bytes, _stream(stream)), "sq_w8a8_linear_quant")
+    return xq_next, x_scale_next
 
 
 def sq_w8a8_linear_noalloc(xq, x_scale, wq, w_scale, y, bias=None, stream=None):

@@ -19,7 +19,9 @@
 //   warps 2-9   epilogue of this CTA's 128 rows: warp w reads TMEM lane
 //               quarter w % 4 for column half (w - 2) / 4, computes
 //               y = fp16((acc * sx[t]) * sw[n] + bias[n]) and writes 32 x 32
-//               blocks through shared memory with TMA stores
+//               blocks through shared memory with TMA stores -- or, for
+//               producer-side quantization, turns y into the next linear's
+//               INT8 codes at its static scale and writes 32 bytes per row
 // Every mbarrier wait is bounded; a wait that runs out records a timeout,
 // tells the other CTA of the pair to stop, and both CTAs drain what they
 // issued, free TMEM and return.
@@ -59,6 +61,9 @@ constexpr size_t SMEM = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
 static_assert(SMEM <= 232448, "shared memory per CTA");
 constexpr uint32_t TMEM_COLS = 512;
 
+// What the epilogue writes.
+enum Epi { EPI_F16 = 0, EPI_I32 = 1, EPI_Q8 = 2 };
+
 // Tile t -> (token tile, channel tile), grouped: groups of kGroupM token
 // tiles walk every channel tile, token tile fastest.  The 74 tiles in flight
 // at a time then span about 8 token tiles x 9 channel tiles, so each operand
@@ -97,7 +102,7 @@ __device__ __forceinline__ bool pair_wait(uint32_t bar, uint32_t parity, bool cl
   }
 }
 
-template <bool OUT_I32>
+template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, const GemmArgs g, int tiles_m, int tiles,
@@ -231,6 +236,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t acce_leader0 = mapa_shared(acce_bar(0), 0);
     int nst = 0;  // blocks this warp has staged (selects the buffer; two stores may be in flight)
     const bool vec_ok = (g.N % 8) == 0;
+    // producer-side quantization: the next linear's 1/s of this tile's columns
+    // (in the output staging area, unused in that mode) and its static scale
+    float* inv_s_s = reinterpret_cast<float*>(smem + STG);
+    float q_inv = 0.0f, q_sc = 0.0f;
+    if constexpr (EPI == EPI_Q8) {
+      q_sc = __fdiv_rn(*g.range_next, 127.0f);
+      q_inv = q_sc > 0.0f ? __frcp_rn(q_sc) : 0.0f;
+    }
     int tl = 0;
     for (int t = pair; t < tiles; t += npairs, ++tl) {
       const int b = tl & 1;
@@ -238,15 +251,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tile_coords(t, tiles_m, tiles_n, tm, tn);
       const int64_t m0 = static_cast<int64_t>(tm) * (2 * BM) + static_cast<int64_t>(rank) * BM;
       const int64_t n0 = static_cast<int64_t>(tn) * BN;
-      if (!OUT_I32) {
+      if (EPI != EPI_I32) {
         const int64_t n = n0 + et;
         sw_s[et] = n < g.N ? g.sw[n] : 0.0f;
         bias_s[et] = (g.bias != nullptr && n < g.N) ? g.bias[n] : __float2half_rn(0.0f);
+        if (EPI == EPI_Q8) inv_s_s[et] = (g.inv_s_next != nullptr && n < g.N) ? g.inv_s_next[n] : 1.0f;
       }
       float sxr = 0.0f;
-      if (!OUT_I32) {
+      if (EPI != EPI_I32) {
         const int64_t row = m0 + 32 * q + lane;
         sxr = row < g.M ? g.sx[row] : 0.0f;
+        if (EPI == EPI_Q8 && tn == 0 && half == 0 && row < g.M) g.sx_next[row] = q_sc;
       }
       named_bar_sync(1, 32 * kEpiWarps);
       pair_wait(accf_bar(b), static_cast<uint32_t>((tl >> 1) & 1), false, budget, status, abort_flag, peer_abort);
@@ -266,11 +281,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       auto emit = [&](int c, uint32_t (&v)[32]) {
         const int cl = 128 * half + 32 * c;  // column within the tile
         const int64_t col0 = n0 + cl;
-        if constexpr (OUT_I32) {
+        if constexpr (EPI == EPI_I32) {
           if (row < g.M && col0 < g.N) {
             int32_t* dst = g.acc + row * g.N + col0;
             for (int j = 0; j < 32; ++j)
               if (col0 + j < g.N) dst[j] = static_cast<int32_t>(v[j]);
+          }
+          return;
+        } else if constexpr (EPI == EPI_Q8) {
+          // the composition, per element: y = fp16((acc * sx) * sw + bias),
+          // a = relu ? max(y, 0) : y, x = a * inv_s_next, then the static
+          // quantizer (a NaN product gives code 0, like the scalar quantizer)
+          __align__(16) uint8_t qb[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            float f = dequant_f32(static_cast<int32_t>(v[j]), sxr, sw_s[cl + j]);
+            if (g.bias != nullptr) f = __fadd_rn(f, __half2float(bias_s[cl + j]));
+            float a = __half2float(__float2half_rn(f));
+            if (g.relu && !(a > 0.0f)) a = 0.0f;
+            float p = __fmul_rn(__fmul_rn(a, inv_s_s[cl + j]), q_inv);
+            if (p != p) p = 0.0f;
+            p = p > 127.0f ? 127.0f : p;
+            p = p < -127.0f ? -127.0f : p;
+            qb[j] = static_cast<uint8_t>(__float_as_uint(__fadd_rn(p, 12582912.0f)) & 0xFFu);
+          }
+          if (row < g.M && col0 < g.N) {
+            int8_t* dst = g.q_next + row * g.N + col0;
+            if ((g.N % 16) == 0 && col0 + 32 <= g.N) {
+              reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<const uint4*>(qb)[0];
+              reinterpret_cast<uint4*>(dst)[1] = reinterpret_cast<const uint4*>(qb)[1];
+            } else {
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < g.N) dst[j] = static_cast<int8_t>(qb[j]);
+            }
           }
           return;
         } else {
@@ -419,7 +462,7 @@ int max_pairs(int device, int num_sms) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = SMEM;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<false>, &cfg) != cudaSuccess || n <= 0) {
+  if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<EPI_F16>, &cfg) != cudaSuccess || n <= 0) {
     (void)cudaGetLastError();
     n = num_sms / 2;
   }
@@ -428,24 +471,22 @@ int max_pairs(int device, int num_sms) {
   return n;
 }
 
-template <bool OUT_I32>
+template <int EPI>
 cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
-  static bool attr_set[64] = {false};
+  static bool attr_set[3][64] = {};
   const int dev = c.device < 64 ? c.device : 63;
-  if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_pair<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (!attr_set[EPI][dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_pair<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM));
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(k_gemm_pair<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(SMEM));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[EPI][dev] = true;
   }
   CUtensorMap tmA, tmB, tmY;
   if (!make_tmap_i8(&tmA, g.xq, g.K, g.M, BK, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_i8(&tmB, g.wq, g.K, g.N, BK, BNH)) return cudaErrorInvalidValue;
-  // TMA stores need 16-byte row strides (N % 8 == 0); otherwise direct stores
-  int tma_store = (!OUT_I32 && g.N % 8 == 0) ? 1 : 0;
+  // TMA stores of fp16 y need 16-byte row strides (N % 8 == 0); otherwise
+  // direct stores (always for int32 accumulators and int8 codes)
+  int tma_store = (EPI == EPI_F16 && g.N % 8 == 0) ? 1 : 0;
   if (tma_store && !make_tmap_f16_out(&tmY, g.y, g.N, g.M)) return cudaErrorInvalidValue;
   if (!tma_store) memset(&tmY, 0, sizeof(tmY));
   const int tiles_m = static_cast<int>((g.M + 2 * BM - 1) / (2 * BM));
@@ -453,15 +494,16 @@ cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
   const int tiles = tiles_m * tiles_n;
   const int mp = max_pairs(c.device, c.num_sms);
   const int pairs = tiles < mp ? tiles : mp;
-  return launch_pdl(k_gemm_pair<OUT_I32>, dim3(2 * pairs), dim3(kThreads), SMEM, c.stream, tmA, tmB, tmY, g,
+  return launch_pdl(k_gemm_pair<EPI>, dim3(2 * pairs), dim3(kThreads), SMEM, c.stream, tmA, tmB, tmY, g,
                     tiles_m, tiles, tma_store, c.status, c.budget_ns);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_pair(const GemmArgs& g, const Ctx& c) {
-  if (g.acc != nullptr) return launch_cfg<true>(g, c);
-  return launch_cfg<false>(g, c);
+  if (g.acc != nullptr) return launch_cfg<EPI_I32>(g, c);
+  if (g.q_next != nullptr) return launch_cfg<EPI_Q8>(g, c);
+  return launch_cfg<EPI_F16>(g, c);
 }
 
 }  // namespace sq

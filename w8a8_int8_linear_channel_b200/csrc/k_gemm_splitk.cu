@@ -77,11 +77,14 @@ __device__ __forceinline__ void tmem_ld_tokens<16>(uint32_t taddr, uint32_t (&v)
   tmem_ld_32x32b_x16(taddr, v);
 }
 
-template <int BT, bool OUT_I32>
+// EPI: 0 = fp16 y, 1 = int32 accumulators, 2 = the next linear's INT8 codes
+// at its static scale (producer-side quantization).
+template <int BT, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_splitk(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                   const GemmArgs g, const SkGeom geo, uint32_t* counters, int32_t* partials,
                   uint32_t* status, uint64_t budget) {
+  constexpr bool OUT_I32 = EPI == 1;
   using L = SkLayout<BT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -215,6 +218,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int et = threadIdx.x - 64;
     const int q = warp & 3;
     if (!OUT_I32 && et < BT) sx_s[et] = et < g.M ? g.sx[et] : 0.0f;
+    float q_inv = 0.0f;
+    if constexpr (EPI == 2) {
+      const float q_sc = __fdiv_rn(*g.range_next, 127.0f);
+      q_inv = q_sc > 0.0f ? __frcp_rn(q_sc) : 0.0f;
+      if (blockIdx.x == 0 && et < BT && et < g.M) g.sx_next[et] = q_sc;
+    }
     named_bar_sync(1, 128);
     int seg = 0;
     for (int64_t j = 0; j < n_all;) {
@@ -292,6 +301,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (OUT_I32) {
           for (int m = 0; m < BT; ++m)
             if (m < g.M) g.acc[m * g.N + n] = static_cast<int32_t>(v[m]);
+        } else if (EPI == 2) {
+          // y = fp16((acc * sx) * sw + bias), a = relu ? max(y, 0) : y,
+          // code = clamp(rint(a * inv_s_next[n] * (1 / scale)), -127, 127)
+          const float swn = g.sw[n];
+          const bool has_bias = g.bias != nullptr;
+          const float bn = has_bias ? __half2float(g.bias[n]) : 0.0f;
+          const float isn = g.inv_s_next != nullptr ? g.inv_s_next[n] : 1.0f;
+#pragma unroll
+          for (int m = 0; m < BT; ++m) {
+            if (m < g.M) {
+              float f = dequant_f32(static_cast<int32_t>(v[m]), sx_s[m], swn);
+              if (has_bias) f = __fadd_rn(f, bn);
+              float a = __half2float(__float2half_rn(f));
+              if (g.relu && !(a > 0.0f)) a = 0.0f;
+              float p = __fmul_rn(__fmul_rn(a, isn), q_inv);
+              if (p != p) p = 0.0f;
+              p = p > 127.0f ? 127.0f : p;
+              p = p < -127.0f ? -127.0f : p;
+              g.q_next[m * g.N + n] = static_cast<int8_t>(__float_as_uint(__fadd_rn(p, 12582912.0f)) & 0xFFu);
+            }
+          }
         } else {
           const float swn = g.sw[n];
           const bool has_bias = g.bias != nullptr;
@@ -348,13 +378,13 @@ SkGeom make_geom(int64_t N, int64_t K, int64_t grid_cap) {
   return geo;
 }
 
-template <int BT, bool OUT_I32>
+template <int BT, int EPI>
 cudaError_t launch_bt(const GemmArgs& g, const Ctx& c) {
   using L = SkLayout<BT>;
   static bool attr_set[64] = {false};
   const int dev = c.device < 64 ? c.device : 63;
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_splitk<BT, OUT_I32>,
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_splitk<BT, EPI>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(L::SMEM));
     if (e != cudaSuccess) return e;
@@ -368,7 +398,7 @@ cudaError_t launch_bt(const GemmArgs& g, const Ctx& c) {
   const size_t counter_bytes = ((tiles_of(g.N) * 4 + 255) / 256) * 256;
   uint32_t* counters = reinterpret_cast<uint32_t*>(ws);
   int32_t* partials = reinterpret_cast<int32_t*>(ws + counter_bytes);
-  return launch_pdl(k_gemm_splitk<BT, OUT_I32>, dim3(geo.grid), dim3(kThreads), L::SMEM, c.stream, tmW, tmX,
+  return launch_pdl(k_gemm_splitk<BT, EPI>, dim3(geo.grid), dim3(kThreads), L::SMEM, c.stream, tmW, tmX,
                     g, geo, counters, partials, c.status, c.budget_ns);
 }
 
@@ -382,9 +412,9 @@ size_t splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
 }
 
 cudaError_t launch_gemm_splitk(const GemmArgs& g, const Ctx& c) {
-  const bool i32 = g.acc != nullptr;
-  if (g.M <= 16) return i32 ? launch_bt<16, true>(g, c) : launch_bt<16, false>(g, c);
-  return i32 ? launch_bt<32, true>(g, c) : launch_bt<32, false>(g, c);
+  const int epi = g.acc != nullptr ? 1 : g.q_next != nullptr ? 2 : 0;
+  if (g.M <= 16) return epi == 1 ? launch_bt<16, 1>(g, c) : epi == 2 ? launch_bt<16, 2>(g, c) : launch_bt<16, 0>(g, c);
+  return epi == 1 ? launch_bt<32, 1>(g, c) : epi == 2 ? launch_bt<32, 2>(g, c) : launch_bt<32, 0>(g, c);
 }
 
 }  // namespace sq
@@ -450,7 +480,7 @@ cudaError_t noalloc_scratch(int dev, uint8_t** out) {
 template <int BT>
 cudaError_t launch_noalloc(const GemmArgs& g, const Ctx& c, uint8_t* scratch) {
   using L = SkLayout<BT>;
-  cudaError_t e = cudaFuncSetAttribute(k_gemm_splitk<BT, false>,
+  cudaError_t e = cudaFuncSetAttribute(k_gemm_splitk<BT, 0>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L::SMEM));
   if (e != cudaSuccess) return e;
@@ -464,7 +494,7 @@ cudaError_t launch_noalloc(const GemmArgs& g, const Ctx& c, uint8_t* scratch) {
   const uint32_t ntiles = static_cast<uint32_t>(tiles_of(g.N));
   e = launch_pdl(k_noalloc_clear_counters, dim3((ntiles + 255) / 256), dim3(256), 0, c.stream, ntiles);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_gemm_splitk<BT, false>, dim3(geo.grid), dim3(kThreads), L::SMEM, c.stream, tmW, tmX, g,
+  return launch_pdl(k_gemm_splitk<BT, 0>, dim3(geo.grid), dim3(kThreads), L::SMEM, c.stream, tmW, tmX, g,
                     geo, counters, partials, c.status, c.budget_ns);
 }
 
@@ -491,7 +521,7 @@ extern "C" sq_status sq_w8a8_linear_noalloc(const int8_t* xq, const float* x_sca
   if (ctx.device >= kMaxDev) return SQ_ERR_CUDA;
   uint8_t* scratch = nullptr;
   if (noalloc_scratch(ctx.device, &scratch) != cudaSuccess || scratch == nullptr) return SQ_ERR_CUDA;
-  GemmArgs g;
+  GemmArgs g{};
   g.xq = xq;
   g.sx = x_scale;
   g.wq = wq;

@@ -139,7 +139,7 @@ sq_status linear_impl(const int8_t* xq, const float* x_scale, const int8_t* wq,
   st = current_ctx(stream, &ctx);
   if (st != SQ_OK) return st;
 
-  GemmArgs g;
+  GemmArgs g{};
   g.xq = xq;
   g.sx = x_scale;
   g.wq = wq;
@@ -247,7 +247,7 @@ const char* sq_status_string(int status) {
   }
 }
 
-int sq_abi_version(void) { return 101; }
+int sq_abi_version(void) { return 102; }
 
 sq_status sq_calibrate_absmax(const void* x_f16, int64_t rows, int64_t K, int64_t ld,
                               const float* ln_gamma, const float* ln_beta, float ln_eps,
@@ -413,6 +413,49 @@ sq_status sq_tensor_range(const float* amax, const float* inv_s, int64_t K, floa
   sq_status st = current_ctx(stream, &ctx);
   if (st != SQ_OK) return st;
   return launched(launch_tensor_range(amax, inv_s, K, range_out, ctx));
+}
+
+sq_status sq_w8a8_linear_quant(const int8_t* xq, const float* x_scale, const int8_t* wq,
+                               const float* w_scale, const void* bias_f16, int relu,
+                               const float* inv_s_next, const float* range_next, int8_t* xq_next,
+                               float* x_scale_next, int64_t M, int64_t N, int64_t K, void* workspace,
+                               size_t ws_bytes, sq_stream_t stream) {
+  if (!xq || !x_scale || !wq || !w_scale || !range_next || !xq_next || !x_scale_next)
+    return SQ_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_k(K);
+  if (st != SQ_OK) return st;
+  // the codes are the next linear's input: its K (= N here) follows the same rule
+  if (N % 16 != 0 || N > SQ_MAX_K) return SQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(xq) || !aligned16(x_scale) || !aligned16(wq) || !aligned16(w_scale) ||
+      !opt_aligned(bias_f16) || !opt_aligned(inv_s_next) || !aligned16(range_next) ||
+      !aligned16(xq_next) || !aligned16(x_scale_next))
+    return SQ_ERR_MISALIGNED;
+  if (M > 0x7fffffffLL) return SQ_ERR_UNSUPPORTED_SHAPE;
+  Ctx ctx;
+  if ((st = current_ctx(stream, &ctx)) != SQ_OK) return st;
+  GemmArgs g{};
+  g.xq = xq;
+  g.sx = x_scale;
+  g.wq = wq;
+  g.sw = w_scale;
+  g.bias = static_cast<const __half*>(bias_f16);
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.ws = workspace;
+  g.ws_bytes = ws_bytes;
+  g.q_next = xq_next;
+  g.sx_next = x_scale_next;
+  g.inv_s_next = inv_s_next;
+  g.range_next = range_next;
+  g.relu = relu ? 1 : 0;
+  if (M <= SQ_SPLITK_MAX_M) {
+    const size_t need = splitk_workspace_bytes(M, N, K, ctx.num_sms);
+    if (workspace == nullptr || ws_bytes < need || !aligned16(workspace)) return SQ_ERR_WORKSPACE;
+    return launched(launch_gemm_splitk(g, ctx));
+  }
+  return launched(launch_gemm_pair(g, ctx));
 }
 
 size_t sq_w8a8_workspace_bytes(int64_t M, int64_t N, int64_t K) {

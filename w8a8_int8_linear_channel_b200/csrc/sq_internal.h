@@ -83,6 +83,15 @@ struct GemmArgs {
   int64_t M, N, K;
   void* ws;
   size_t ws_bytes;
+  // producer-side quantization of the next linear's input at a static
+  // per-tensor scale (q_next != NULL; y and acc unused):
+  //   a = fp16(y) (ReLU if relu), x = a * inv_s_next[n] (if given),
+  //   q_next = clamp(rint(x * (1 / scale)), -127, 127), scale = *range_next / 127
+  int8_t* q_next;           // [M, N]
+  float* sx_next;           // [M], every entry = scale
+  const float* inv_s_next;  // [N] or NULL
+  const float* range_next;  // [1]
+  int relu;
 };
 
 cudaError_t launch_gemm_tiled(const GemmArgs& g, const Ctx& c);  // 128 x 256 tiles
