@@ -379,6 +379,23 @@ class Plan:
         self.main.wait_stream(cap)
         self.burst, self.burst_reps = gr, reps
 
+    def capture_burst_of(self, calls, reps):
+        """One graph of `reps` rounds of the given (fn, args-builder) calls on a
+        capture stream; args-builder(stream) returns the C arguments."""
+        torch = self.torch
+        cap = torch.cuda.Stream()
+        cap.wait_stream(self.main)
+        with torch.cuda.stream(cap):
+            st = ctypes.c_void_p(cap.cuda_stream)
+            bound = [(fn, mk(st)) for fn, mk in calls]
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=cap):
+                for _ in range(reps):
+                    for fn, a in bound:
+                        self._call("producer", fn, a)
+        self.main.wait_stream(cap)
+        return gr
+
     def replay(self, allreduce=None):
         self.graphs[0].replay()
         if len(self.graphs) > 1:
@@ -549,6 +566,8 @@ def run_gpu(args):
     if sq.sq_poll_status() != 0:
         raise RuntimeError("device wait timed out in the GEMM burst")
 
+    producer = run_producer(plan, sq, torch, flush, reps, args) if args.producer and use_graph else None
+
     nbytes, ops = stage_bytes_ops(wl, M, args.level)
     step_bytes = sum(nbytes.values())
     decode = M <= sq.SPLITK_MAX_M
@@ -628,12 +647,64 @@ def run_gpu(args):
             "clocks": clocks,
             "e2e": e2e,
         }
+        if producer is not None:
+            result["producer_quant"] = producer
         if world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = oracle_baseline(wl, M, budget_s=args.cpu_budget, level=args.level)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return result
+
+
+def run_producer(plan, sq, torch, flush, reps, args):
+    """Producer-side quantization on the step's linear: the fused linear that
+    emits the next linear's INT8 input at a static scale (times 1/s of the
+    next layer), against the unfused pair (linear to fp16, then the static
+    quantization pass), each as back-to-back launches in one graph."""
+    L = sq._L
+    wl, M = plan.wl, plan.M
+    N, K = wl.N, wl.K
+    dev = plan.y.device
+    p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    g = torch.Generator(device="cpu").manual_seed(5)
+    inv_next = (torch.rand(N, generator=g) * 1.5 + 0.5).to(dev)
+    rng_next = torch.full((4,), 4.0, dtype=torch.float32, device=dev)
+    q_next = torch.empty((M, N), dtype=torch.int8, device=dev)
+    s_next = torch.empty(M, dtype=torch.float32, device=dev)
+    y = plan.y
+    fused = [(L.sq_w8a8_linear_quant, lambda st: (p(plan.xq), p(plan.sx), p(plan.wq), p(plan.sw), p(plan.bias), 0,
+                                                  p(inv_next), p(rng_next), p(q_next), p(s_next), M, N, K,
+                                                  p(plan.ws), plan.ws_bytes, st))]
+    unfused = [(L.sq_w8a8_linear, lambda st: (p(plan.xq), p(plan.sx), p(plan.wq), p(plan.sw), p(plan.bias), p(y),
+                                              M, N, K, p(plan.ws), plan.ws_bytes, st)),
+               (L.sq_ln_quant_act_static, lambda st: (p(y), M, N, N, None, None, p(inv_next), ctypes.c_float(1e-5),
+                                                      p(rng_next), p(q_next), p(s_next), st))]
+    out = {}
+    for name, calls in (("fused", fused), ("unfused", unfused)):
+        gr = plan.capture_burst_of(calls, reps)
+        flush()
+        gr.replay()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.burst_iters)]
+        for e in ev:
+            flush()
+            e[0].record()
+            gr.replay()
+            e[1].record()
+        torch.cuda.synchronize()
+        out[name + "_us"] = round(1e3 * sum(a.elapsed_time(b) for a, b in ev) / len(ev) / reps, 2)
+    if sq.sq_poll_status() != 0:
+        raise RuntimeError("device wait timed out in the producer-quantization loop")
+    # algorithmic bytes: the linear's operands and scales, then its output
+    base = M * K + N * K + 4 * M + 4 * N + (2 * N if plan.bias is not None else 0)
+    out["fused_bytes"] = base + M * N + 4 * N + 4 * M
+    out["unfused_bytes"] = base + 2 * M * N + (2 * M * N + M * N + 4 * M + 4 * N)
+    out["ops"] = 2 * M * N * K
+    out["what"] = ("linear + the next linear's static (level O3) input quantization with its 1/s: fused into "
+                   "the GEMM epilogue (sq_w8a8_linear_quant) vs sq_w8a8_linear then sq_ln_quant_act_static; "
+                   f"{reps} back-to-back launches per graph, L2 flushed before each replay")
+    return out
 
 
 def run_e2e(plan, sq, torch, world, allreduce, steps, dist):
@@ -838,6 +909,8 @@ def main():
     ap.add_argument("--streams", type=int, choices=[1, 2], default=2,
                     help="2: run the independent stages of a step on two streams")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--producer", action="store_true",
+                    help="also time the fused producer-side quantization of the linear's output")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU work")
     ap.add_argument("--ref-budget", type=float, default=150.0, help="seconds for the reference arm")
     args = ap.parse_args()

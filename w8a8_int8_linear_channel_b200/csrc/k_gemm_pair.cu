@@ -291,28 +291,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         } else if constexpr (EPI == EPI_Q8) {
           // the composition, per element: y = fp16((acc * sx) * sw + bias),
           // a = relu ? max(y, 0) : y, x = a * inv_s_next, then the static
-          // quantizer (a NaN product gives code 0, like the scalar quantizer)
-          __align__(16) uint8_t qb[32];
+          // quantizer; fp32 pairs, the ReLU on half2 (max with 0 turns a NaN
+          // into 0, like the scalar test), codes packed 4 per word.  With a
+          // zero range every code is 0 (as the scalar quantizer gives for a
+          // zero reciprocal), so the product x * q_inv below is never NaN.
+          __align__(16) uint32_t qw[8];
+          if (q_inv == 0.0f) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            float f = dequant_f32(static_cast<int32_t>(v[j]), sxr, sw_s[cl + j]);
-            if (g.bias != nullptr) f = __fadd_rn(f, __half2float(bias_s[cl + j]));
-            float a = __half2float(__float2half_rn(f));
-            if (g.relu && !(a > 0.0f)) a = 0.0f;
-            float p = __fmul_rn(__fmul_rn(a, inv_s_s[cl + j]), q_inv);
-            if (p != p) p = 0.0f;
-            p = p > 127.0f ? 127.0f : p;
-            p = p < -127.0f ? -127.0f : p;
-            qb[j] = static_cast<uint8_t>(__float_as_uint(__fadd_rn(p, 12582912.0f)) & 0xFFu);
+            for (int u = 0; u < 8; ++u) qw[u] = 0u;
+          } else {
+            const uint64_t sx2 = f2_pack(sxr, sxr);
+            const uint64_t qi2 = f2_pack(q_inv, q_inv);
+            const float4* swv = reinterpret_cast<const float4*>(sw_s + cl);
+            const float4* isv = reinterpret_cast<const float4*>(inv_s_s + cl);
+            const uint4* bv = reinterpret_cast<const uint4*>(bias_s + cl);
+            const __half2 zero2 = __float2half2_rn(0.0f);
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 w = swv[j / 4];
+              const float4 is = isv[j / 4];
+              uint64_t d0 = f2_mul_rn(f2_mul_rn(f2_pack(__int2float_rn(static_cast<int32_t>(v[j])),
+                                                        __int2float_rn(static_cast<int32_t>(v[j + 1]))), sx2),
+                                      f2_pack(w.x, w.y));
+              uint64_t d1 = f2_mul_rn(f2_mul_rn(f2_pack(__int2float_rn(static_cast<int32_t>(v[j + 2])),
+                                                        __int2float_rn(static_cast<int32_t>(v[j + 3]))), sx2),
+                                      f2_pack(w.z, w.w));
+              if (g.bias != nullptr) {
+                const uint2 b4 = reinterpret_cast<const uint2*>(bv)[j / 4];
+                const float2 b01 = __half22float2(*reinterpret_cast<const __half2*>(&b4.x));
+                const float2 b23 = __half22float2(*reinterpret_cast<const __half2*>(&b4.y));
+                d0 = f2_add_rn(d0, f2_pack(b01.x, b01.y));
+                d1 = f2_add_rn(d1, f2_pack(b23.x, b23.y));
+              }
+              const float2 f0 = f2_unpack(d0), f1 = f2_unpack(d1);
+              __half2 h0 = __floats2half2_rn(f0.x, f0.y), h1 = __floats2half2_rn(f1.x, f1.y);
+              if (g.relu) {
+                h0 = __hmax2(h0, zero2);
+                h1 = __hmax2(h1, zero2);
+              }
+              const float2 a0 = __half22float2(h0), a1 = __half22float2(h1);
+              const float2 p0 = f2_unpack(f2_mul_rn(f2_mul_rn(f2_pack(a0.x, a0.y), f2_pack(is.x, is.y)), qi2));
+              const float2 p1 = f2_unpack(f2_mul_rn(f2_mul_rn(f2_pack(a1.x, a1.y), f2_pack(is.z, is.w)), qi2));
+              const float kMagic = 12582912.0f;  // 1.5 * 2^23: rint, code in the low byte
+              const uint32_t c0 = __float_as_uint(__fadd_rn(fminf(fmaxf(p0.x, -127.0f), 127.0f), kMagic));
+              const uint32_t c1 = __float_as_uint(__fadd_rn(fminf(fmaxf(p0.y, -127.0f), 127.0f), kMagic));
+              const uint32_t c2 = __float_as_uint(__fadd_rn(fminf(fmaxf(p1.x, -127.0f), 127.0f), kMagic));
+              const uint32_t c3 = __float_as_uint(__fadd_rn(fminf(fmaxf(p1.y, -127.0f), 127.0f), kMagic));
+              qw[j / 4] = __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
+            }
           }
           if (row < g.M && col0 < g.N) {
             int8_t* dst = g.q_next + row * g.N + col0;
             if ((g.N % 16) == 0 && col0 + 32 <= g.N) {
-              reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<const uint4*>(qb)[0];
-              reinterpret_cast<uint4*>(dst)[1] = reinterpret_cast<const uint4*>(qb)[1];
+              reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<const uint4*>(qw)[0];
+              reinterpret_cast<uint4*>(dst)[1] = reinterpret_cast<const uint4*>(qw)[1];
             } else {
+              const int8_t* qb = reinterpret_cast<const int8_t*>(qw);
               for (int j = 0; j < 32; ++j)
-                if (col0 + j < g.N) dst[j] = static_cast<int8_t>(qb[j]);
+                if (col0 + j < g.N) dst[j] = qb[j];
             }
           }
           return;
