@@ -244,6 +244,23 @@ sq_status sq_w8a8_linear_quant(const int8_t* xq, const float* x_scale, const int
                                float* x_scale_next, int64_t M, int64_t N, int64_t K, void* workspace,
                                size_t ws_bytes, sq_stream_t stream);
 
+/*
+ * INT8 BMM (the explainer, section "inference": after smoothing, the linear
+ * layers and the BMMs of attention run in INT8): `batch` independent
+ * products, e.g. one per attention head,
+ *   acc[i, m, n] = sum_k a[i, m, k] * b[i, n, k]                      (exact int32)
+ *   y[i, m, n]   = fp16( (fp32(acc) * a_scale[i, m]) * b_scale[i, n] )
+ * a int8 [batch, M, K] (e.g. Q per head, K contiguous); b int8 [batch, N, K]
+ * (K per head for Q K^T; V^T per head for P V, i.e. V stored transposed);
+ * a_scale fp32 [batch, M]; b_scale fp32 [batch, N] (per-head scales: every
+ * entry of a head equal; per-token scales: one per row); y fp16 [batch, M, N].
+ * Items are independent: rows past M or N of one item never mix with the
+ * next (3-D tensor maps, out-of-bounds rows read as zero).  Runs the
+ * CTA-pair tensor-core kernel over batch x 256 x 256 tiles.
+ */
+sq_status sq_w8a8_bmm(const int8_t* a, const float* a_scale, const int8_t* b, const float* b_scale,
+                      void* y_f16, int64_t batch, int64_t M, int64_t N, int64_t K, sq_stream_t stream);
+
 /* Kernel choice for sq_w8a8_linear_path. */
 typedef enum sq_gemm_path {
   SQ_PATH_AUTO = 0,   /* what sq_w8a8_linear does */

@@ -81,6 +81,7 @@ def _declare(L):
         "oracle_dequant": [_P, _P, _P, _P, _I, _I, _P],
         "oracle_w8a8_linear": [_P, _P, _P, _P, _P, _I, _I, _I, _P],
         "oracle_w8a8_linear_quant_static": [_P, _P, _P, _P, _P, ctypes.c_int, _P, _F, _I, _I, _I, _P, _P],
+        "oracle_w8a8_bmm": [_P, _P, _P, _P, _I, _I, _I, _I, _P],
         "oracle_num_threads": [],
         "oracle_set_num_threads": [ctypes.c_int],
     }
@@ -334,6 +335,18 @@ def w8a8_linear_quant_static(xq, sx, wq, sw, bias=None, relu=False, inv_s_next=N
                                           _ptr(inv_s_next), float(np.float32(range_next)), M, N, K,
                                           _ptr(q), _ptr(s_next))
     return q, s_next
+
+
+def w8a8_bmm(a, a_scale, b, b_scale) -> np.ndarray:
+    """[SQ] INT8 BMM: y[i] = fp16((a[i] @ b[i]^T) * a_scale[i][:, None] * b_scale[i][None, :])."""
+    a = np.ascontiguousarray(a, np.int8)
+    b = np.ascontiguousarray(b, np.int8)
+    B, M, K = a.shape
+    N = b.shape[1]
+    a_scale, b_scale = _f32(a_scale), _f32(b_scale)
+    y = np.empty((B, M, N), np.float16)
+    lib().oracle_w8a8_bmm(_ptr(a), _ptr(a_scale), _ptr(b), _ptr(b_scale), B, M, N, K, _ptr(y))
+    return y
 
 
 # ------------------------------------------------------- fp64 mathematics ----

@@ -420,6 +420,28 @@ void oracle_w8a8_linear_quant_static(const int8_t* xq, const float* sx, const in
   }
 }
 
+/* --------------------------------------------------------------- INT8 BMM --- */
+/* [SQ] "inference": with the smoothing in place the attention BMMs run in
+ * INT8 too.  `batch` independent products (one per head):
+ *   acc[i, m, n] = sum_k a[i, m, k] * b[i, n, k]              (int32)
+ *   y[i, m, n]   = fp16((float)acc * a_scale[i, m] * b_scale[i, n])  (in that order) */
+void oracle_w8a8_bmm(const int8_t* a, const float* a_scale, const int8_t* b, const float* b_scale,
+                     int64_t batch, int64_t M, int64_t N, int64_t K, uint16_t* y) {
+  for (int64_t i = 0; i < batch; ++i) {
+    const int8_t* ai = a + i * M * K;
+    const int8_t* bi = b + i * N * K;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+      for (int64_t n = 0; n < N; ++n) {
+        int32_t sum = 0;
+        for (int64_t k = 0; k < K; ++k) sum += (int32_t)ai[m * K + k] * (int32_t)bi[n * K + k];
+        float v = (float)sum * a_scale[i * M + m];
+        v = v * b_scale[i * N + n];
+        y[(i * M + m) * N + n] = f2h(v);
+      }
+  }
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

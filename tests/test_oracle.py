@@ -480,3 +480,27 @@ def test_producer_quant_is_linear_then_static_quant(relu):
     q, s = oracle.w8a8_linear_quant_static(xq, sx, wq, sw, bias, relu=relu, inv_s_next=inv, range_next=r)
     assert np.all(s == sc) and np.array_equal(q, codes)
     assert (np.abs(q) == 127).any()
+
+
+# ------------------------------------------------------------------ INT8 BMM --
+def test_hand_example_bmm():
+    g = load("bmm_2x2x2.txt")
+    a = np.stack([g["a0"], g["a1"]]).astype(np.int8)
+    b = np.stack([g["b0"], g["b1"]]).astype(np.int8)
+    y = oracle.w8a8_bmm(a, np.stack([g["as0"], g["as1"]]), b, np.stack([g["bs0"], g["bs1"]]))
+    assert np.array_equal(y.astype(np.float64), np.stack([g["y0"], g["y1"]]))
+
+
+def test_bmm_items_are_independent_linears():
+    rng = np.random.default_rng(41)
+    B, M, N, K = 3, 7, 9, 48
+    a = rng.integers(-127, 128, (B, M, K)).astype(np.int8)
+    b = rng.integers(-127, 128, (B, N, K)).astype(np.int8)
+    sa = rng.uniform(1e-3, 1e-2, (B, M)).astype(np.float32)
+    sb = rng.uniform(1e-3, 1e-2, (B, N)).astype(np.float32)
+    y = oracle.w8a8_bmm(a, sa, b, sb)
+    for i in range(B):
+        acc = a[i].astype(np.int64) @ b[i].astype(np.int64).T  # numpy brute force
+        exact = acc * sa[i][:, None].astype(np.float64) * sb[i][None, :].astype(np.float64)
+        assert np.all(np.abs(y[i].astype(np.float64) - exact) <= np.spacing(np.abs(exact).astype(np.float16)))
+        assert np.array_equal(y[i], oracle.w8a8_linear(a[i], sa[i], b[i], sb[i]))

@@ -35,6 +35,8 @@ MUTANTS = {
     "producer_relu_dropped": ("if (relu && !(a > 0.0f)) a = 0.0f;", "if (relu && 0) a = 0.0f;"),
     "producer_no_fp16_round": ("float a = h2f(f2h(v));", "float a = v;"),
     "producer_inv_s_not_applied": ("float x = inv_s_next ? a * inv_s_next[n] : a;", "float x = a;"),
+    "bmm_scales_of_item_0": ("float v = (float)sum * a_scale[i * M + m];", "float v = (float)sum * a_scale[m];"),
+    "bmm_b_of_item_0": ("const int8_t* bi = b + i * N * K;", "const int8_t* bi = b;"),
     "weight_tensor_scale_per_row": ("  for (int64_t n = 0; n < N; ++n) sw[n] = sc;", "  for (int64_t n = 0; n < N; ++n) sw[n] = n ? sc : 1.0f;"),
 }
 

@@ -27,7 +27,7 @@ __all__ = [
     "sq_w8a8_workspace_bytes", "sq_w8a8_linear", "sq_w8a8_linear_path", "sq_w8a8_gemm_s32",
     "sq_poll_status", "sq_set_wait_budget_ns", "sq_selftest_wait_timeout", "SmoothQuantLinear",
     "sq_quantize_weight_tensor", "sq_ln_quant_act_tensor", "sq_ln_quant_act_static", "sq_tensor_range",
-    "LEVELS", "sq_w8a8_linear_quant",
+    "LEVELS", "sq_w8a8_linear_quant", "sq_w8a8_bmm",
     "PATH_AUTO", "PATH_TILED", "PATH_SPLITK", "PATH_PAIR", "PATH_WIDE", "SPLITK_MAX_M", "MAX_K", "library_path",
 ]
 
@@ -71,6 +71,7 @@ def _load() -> ctypes.CDLL:
         "sq_w8a8_gemm_s32": ([P, P, P, I, I, I, P, Z, S, P], S),
         "sq_w8a8_linear_noalloc": ([P, P, P, P, P, P, I, I, I, P], S),
         "sq_w8a8_linear_quant": ([P, P, P, P, P, S, P, P, P, P, I, I, I, P, Z, P], S),
+        "sq_w8a8_bmm": ([P, P, P, P, P, I, I, I, I, P], S),
         "sq_poll_status": ([P], S),
         "sq_set_wait_budget_ns": ([ctypes.c_uint64], None),
         "sq_selftest_wait_timeout": ([ctypes.c_uint64, P], S),
@@ -292,6 +293,26 @@ def sq_w8a8_linear_quant(xq, x_scale, wq, w_scale, range_next, xq_next, x_scale_
                                    _p(inv_s_next), _p(range_next), _p(xq_next), _p(x_scale_next), M, N, K,
                                    _p(workspace), ws_bytes, _stream(stream)), "sq_w8a8_linear_quant")
     return xq_next, x_scale_next
+
+
+def sq_w8a8_bmm(a, a_scale, b, b_scale, y, stream=None):
+    """INT8 BMM: y[i] = fp16((a[i] @ b[i]^T) * a_scale[i][:, None] * b_scale[i][None, :]) for every
+    batch item i; a int8 [B, M, K], b int8 [B, N, K], scales fp32 [B, M] / [B, N], y fp16 [B, M, N]."""
+    for t, n in ((a, "a"), (b, "b")):
+        if t.dtype != torch.int8 or t.dim() != 3 or not t.is_contiguous():
+            raise ValueError(f"{n}: need a contiguous int8 [batch, rows, K] tensor")
+    B, M, K = a.shape
+    if b.shape[0] != B or b.shape[2] != K:
+        raise ValueError("b: need [batch, N, K] with the same batch and K as a")
+    N = b.shape[1]
+    for t, n, r in ((a_scale, "a_scale", M), (b_scale, "b_scale", N)):
+        if t.dtype != torch.float32 or tuple(t.shape) != (B, r) or not t.is_contiguous():
+            raise ValueError(f"{n}: need a contiguous fp32 [batch, {r}] tensor")
+    if y.dtype != torch.float16 or tuple(y.shape) != (B, M, N) or not y.is_contiguous():
+        raise ValueError("y: need a contiguous fp16 [batch, M, N] tensor")
+    _check(_L.sq_w8a8_bmm(_p(a), _p(a_scale), _p(b), _p(b_scale), _p(y), B, M, N, K, _stream(stream)),
+           "sq_w8a8_bmm")
+    return y
 
 
 def sq_w8a8_linear_noalloc(xq, x_scale, wq, w_scale, y, bias=None, stream=None):

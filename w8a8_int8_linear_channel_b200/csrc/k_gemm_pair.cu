@@ -61,8 +61,8 @@ constexpr size_t SMEM = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
 static_assert(SMEM <= 232448, "shared memory per CTA");
 constexpr uint32_t TMEM_COLS = 512;
 
-// What the epilogue writes.
-enum Epi { EPI_F16 = 0, EPI_I32 = 1, EPI_Q8 = 2 };
+// What the epilogue writes (EPI_BMM: fp16 y of a batched GEMM, 3-D maps).
+enum Epi { EPI_F16 = 0, EPI_I32 = 1, EPI_Q8 = 2, EPI_BMM = 3 };
 
 // Tile t -> (token tile, channel tile), grouped: groups of kGroupM token
 // tiles walk every channel tile, token tile fastest.  The 74 tiles in flight
@@ -131,7 +131,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int pair = static_cast<int>(blockIdx.x >> 1);
   const int npairs = static_cast<int>(gridDim.x >> 1);
   const int KB = static_cast<int>((g.K + BK - 1) / BK);
-  const int tiles_n = tiles / tiles_m;
+  // tiles of one batch item (the whole grid when not batched)
+  const int per_item = EPI == EPI_BMM ? tiles / static_cast<int>(g.batch) : tiles;
+  const int tiles_n = per_item / tiles_m;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -170,8 +172,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int64_t it = 0;
       bool ok = true;
       for (int t = pair; t < tiles && ok; t += npairs) {
+        const int bi = t / per_item;  // batch item (0 when not batched)
         int tm, tn;
-        tile_coords(t, tiles_m, tiles_n, tm, tn);
+        tile_coords(t - bi * per_item, tiles_m, tiles_n, tm, tn);
         const int32_t m0 = tm * (2 * BM) + static_cast<int32_t>(rank) * BM;
         const int32_t n0 = tn * BN + static_cast<int32_t>(rank) * BNH;
         for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -184,8 +187,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           const uint32_t st = sbase + s * STAGE_BYTES;
           if (rank == 0) mbar_arrive_expect_tx(full_bar(s), 2 * STAGE_BYTES);
-          tma_load_2d_pair(st, &tmA, full_leader0 + 8u * s, kb * BK, m0);
-          tma_load_2d_pair(st + A_BYTES, &tmB, full_leader0 + 8u * s, kb * BK, n0);
+          if constexpr (EPI == EPI_BMM) {
+            tma_load_3d_pair(st, &tmA, full_leader0 + 8u * s, kb * BK, m0, bi);
+            tma_load_3d_pair(st + A_BYTES, &tmB, full_leader0 + 8u * s, kb * BK, n0, bi);
+          } else {
+            tma_load_2d_pair(st, &tmA, full_leader0 + 8u * s, kb * BK, m0);
+            tma_load_2d_pair(st + A_BYTES, &tmB, full_leader0 + 8u * s, kb * BK, n0);
+          }
           ++issued;
         }
       }
@@ -247,20 +255,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int tl = 0;
     for (int t = pair; t < tiles; t += npairs, ++tl) {
       const int b = tl & 1;
+      const int bi = t / per_item;  // batch item (0 when not batched)
       int tm, tn;
-      tile_coords(t, tiles_m, tiles_n, tm, tn);
+      tile_coords(t - bi * per_item, tiles_m, tiles_n, tm, tn);
       const int64_t m0 = static_cast<int64_t>(tm) * (2 * BM) + static_cast<int64_t>(rank) * BM;
       const int64_t n0 = static_cast<int64_t>(tn) * BN;
       if (EPI != EPI_I32) {
         const int64_t n = n0 + et;
-        sw_s[et] = n < g.N ? g.sw[n] : 0.0f;
+        sw_s[et] = n < g.N ? g.sw[static_cast<int64_t>(bi) * g.N + n] : 0.0f;
         bias_s[et] = (g.bias != nullptr && n < g.N) ? g.bias[n] : __float2half_rn(0.0f);
         if (EPI == EPI_Q8) inv_s_s[et] = (g.inv_s_next != nullptr && n < g.N) ? g.inv_s_next[n] : 1.0f;
       }
       float sxr = 0.0f;
       if (EPI != EPI_I32) {
         const int64_t row = m0 + 32 * q + lane;
-        sxr = row < g.M ? g.sx[row] : 0.0f;
+        sxr = row < g.M ? g.sx[static_cast<int64_t>(bi) * g.M + row] : 0.0f;
         if (EPI == EPI_Q8 && tn == 0 && half == 0 && row < g.M) g.sx_next[row] = q_sc;
       }
       named_bar_sync(1, 32 * kEpiWarps);
@@ -409,12 +418,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              if (row0 < g.M && col0 < g.N)
-                tma_store_2d(&tmY, stg, static_cast<int32_t>(col0), static_cast<int32_t>(row0));
+              if (row0 < g.M && col0 < g.N) {
+                if constexpr (EPI == EPI_BMM)
+                  tma_store_3d(&tmY, stg, static_cast<int32_t>(col0), static_cast<int32_t>(row0), bi);
+                else
+                  tma_store_2d(&tmY, stg, static_cast<int32_t>(col0), static_cast<int32_t>(row0));
+              }
               bulk_commit_group();
             }
           } else if (row < g.M && col0 < g.N) {
-            __half* dst = g.y + row * g.N + col0;
+            __half* dst = g.y + (static_cast<int64_t>(bi) * g.M + row) * g.N + col0;
             if (vec_ok && col0 + 32 <= g.N) {
 #pragma unroll
               for (int j = 0; j < 4; ++j)
@@ -509,7 +522,7 @@ int max_pairs(int device, int num_sms) {
 
 template <int EPI>
 cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
-  static bool attr_set[3][64] = {};
+  static bool attr_set[4][64] = {};
   const int dev = c.device < 64 ? c.device : 63;
   if (!attr_set[EPI][dev]) {
     cudaError_t e = cudaFuncSetAttribute(k_gemm_pair<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -518,16 +531,29 @@ cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
     attr_set[EPI][dev] = true;
   }
   CUtensorMap tmA, tmB, tmY;
-  if (!make_tmap_i8(&tmA, g.xq, g.K, g.M, BK, BM)) return cudaErrorInvalidValue;
-  if (!make_tmap_i8(&tmB, g.wq, g.K, g.N, BK, BNH)) return cudaErrorInvalidValue;
+  const bool bmm = EPI == EPI_BMM;
+  const uint64_t items = bmm ? static_cast<uint64_t>(g.batch) : 1;
+  if (bmm) {
+    if (!make_tmap_i8_3d(&tmA, g.xq, g.K, g.M, items, BK, BM)) return cudaErrorInvalidValue;
+    if (!make_tmap_i8_3d(&tmB, g.wq, g.K, g.N, items, BK, BNH)) return cudaErrorInvalidValue;
+  } else {
+    if (!make_tmap_i8(&tmA, g.xq, g.K, g.M, BK, BM)) return cudaErrorInvalidValue;
+    if (!make_tmap_i8(&tmB, g.wq, g.K, g.N, BK, BNH)) return cudaErrorInvalidValue;
+  }
   // TMA stores of fp16 y need 16-byte row strides (N % 8 == 0); otherwise
   // direct stores (always for int32 accumulators and int8 codes)
-  int tma_store = (EPI == EPI_F16 && g.N % 8 == 0) ? 1 : 0;
-  if (tma_store && !make_tmap_f16_out(&tmY, g.y, g.N, g.M)) return cudaErrorInvalidValue;
-  if (!tma_store) memset(&tmY, 0, sizeof(tmY));
+  int tma_store = ((EPI == EPI_F16 || bmm) && g.N % 8 == 0) ? 1 : 0;
+  if (tma_store) {
+    const bool ok = bmm ? make_tmap_f16_out_3d(&tmY, g.y, g.N, g.M, items) : make_tmap_f16_out(&tmY, g.y, g.N, g.M);
+    if (!ok) return cudaErrorInvalidValue;
+  } else {
+    memset(&tmY, 0, sizeof(tmY));
+  }
   const int tiles_m = static_cast<int>((g.M + 2 * BM - 1) / (2 * BM));
   const int tiles_n = static_cast<int>((g.N + BN - 1) / BN);
-  const int tiles = tiles_m * tiles_n;
+  const int64_t tiles64 = static_cast<int64_t>(items) * tiles_m * tiles_n;
+  if (tiles64 > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const int tiles = static_cast<int>(tiles64);
   const int mp = max_pairs(c.device, c.num_sms);
   const int pairs = tiles < mp ? tiles : mp;
   return launch_pdl(k_gemm_pair<EPI>, dim3(2 * pairs), dim3(kThreads), SMEM, c.stream, tmA, tmB, tmY, g,
@@ -535,6 +561,8 @@ cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
 }
 
 }  // namespace
+
+cudaError_t launch_bmm_pair(const GemmArgs& g, const Ctx& c) { return launch_cfg<EPI_BMM>(g, c); }
 
 cudaError_t launch_gemm_pair(const GemmArgs& g, const Ctx& c) {
   if (g.acc != nullptr) return launch_cfg<EPI_I32>(g, c);

@@ -247,7 +247,7 @@ const char* sq_status_string(int status) {
   }
 }
 
-int sq_abi_version(void) { return 102; }
+int sq_abi_version(void) { return 103; }
 
 sq_status sq_calibrate_absmax(const void* x_f16, int64_t rows, int64_t K, int64_t ld,
                               const float* ln_gamma, const float* ln_beta, float ln_eps,
@@ -456,6 +456,30 @@ sq_status sq_w8a8_linear_quant(const int8_t* xq, const float* x_scale, const int
     return launched(launch_gemm_splitk(g, ctx));
   }
   return launched(launch_gemm_pair(g, ctx));
+}
+
+sq_status sq_w8a8_bmm(const int8_t* a, const float* a_scale, const int8_t* b, const float* b_scale,
+                      void* y_f16, int64_t batch, int64_t M, int64_t N, int64_t K, sq_stream_t stream) {
+  if (!a || !a_scale || !b || !b_scale || !y_f16) return SQ_ERR_INVALID_ARG;
+  if (batch <= 0 || M <= 0 || N <= 0) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_k(K);
+  if (st != SQ_OK) return st;
+  if (!aligned16(a) || !aligned16(a_scale) || !aligned16(b) || !aligned16(b_scale) || !aligned16(y_f16))
+    return SQ_ERR_MISALIGNED;
+  if (M > 0x7fffffffLL || N > 0x7fffffffLL || batch > 0x7fffffffLL) return SQ_ERR_UNSUPPORTED_SHAPE;
+  Ctx ctx;
+  if ((st = current_ctx(stream, &ctx)) != SQ_OK) return st;
+  GemmArgs g{};
+  g.xq = a;
+  g.sx = a_scale;
+  g.wq = b;
+  g.sw = b_scale;
+  g.y = static_cast<__half*>(y_f16);
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.batch = batch;
+  return launched(launch_bmm_pair(g, ctx));
 }
 
 size_t sq_w8a8_workspace_bytes(int64_t M, int64_t N, int64_t K) {

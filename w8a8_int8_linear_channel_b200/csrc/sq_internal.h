@@ -92,11 +92,15 @@ struct GemmArgs {
   const float* inv_s_next;  // [N] or NULL
   const float* range_next;  // [1]
   int relu;
+  // batched GEMM (INT8 BMM): batch items of [M, K] x [N, K]^T -> [M, N], the
+  // scales per (item, row) sx [batch, M] and per (item, column) sw [batch, N]
+  int64_t batch;  // 0 = not batched
 };
 
 cudaError_t launch_gemm_tiled(const GemmArgs& g, const Ctx& c);  // 128 x 256 tiles
 cudaError_t launch_gemm_wide(const GemmArgs& g, const Ctx& c);   // 256 x 256 tiles, persistent
 cudaError_t launch_gemm_pair(const GemmArgs& g, const Ctx& c);   // 256 x 256 tiles on CTA pairs
+cudaError_t launch_bmm_pair(const GemmArgs& g, const Ctx& c);    // the same, batched (g.batch items)
 cudaError_t launch_gemm_splitk(const GemmArgs& g, const Ctx& c);
 size_t splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
 
