@@ -567,6 +567,7 @@ def run_gpu(args):
         raise RuntimeError("device wait timed out in the GEMM burst")
 
     producer = run_producer(plan, sq, torch, flush, reps, args) if args.producer and use_graph else None
+    bmm = run_bmm(sq, torch, device, flush, args) if args.bmm and use_graph else None
 
     nbytes, ops = stage_bytes_ops(wl, M, args.level)
     step_bytes = sum(nbytes.values())
@@ -649,6 +650,8 @@ def run_gpu(args):
         }
         if producer is not None:
             result["producer_quant"] = producer
+        if bmm is not None:
+            result["bmm"] = bmm
         if world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = oracle_baseline(wl, M, budget_s=args.cpu_budget, level=args.level)
     if world > 1:
@@ -704,6 +707,58 @@ def run_producer(plan, sq, torch, flush, reps, args):
     out["what"] = ("linear + the next linear's static (level O3) input quantization with its 1/s: fused into "
                    "the GEMM epilogue (sq_w8a8_linear_quant) vs sq_w8a8_linear then sq_ln_quant_act_static; "
                    f"{reps} back-to-back launches per graph, L2 flushed before each replay")
+    return out
+
+
+def run_bmm(sq, torch, device, flush, args):
+    """INT8 BMM on the OPT-6.7B attention shapes (32 heads, 2048 tokens, head
+    dim 128): Q K^T and P V (V stored transposed), per-head scales, random
+    codes; back-to-back launches in one graph, L2 flushed before each replay.
+    Both are HBM-bound (fp16 scores out, or the [2048 x 2048] probabilities
+    in): the roofline is the algorithmic bytes against the measured copy
+    bandwidth, with the tensor-core time beside it."""
+    L = sq._L
+    peaks, kind = load_peaks()
+    out = {}
+    g = torch.Generator(device="cpu").manual_seed(9)
+    for name, (B, M, N, K) in (("qk", (32, 2048, 2048, 128)), ("pv", (32, 2048, 128, 2048))):
+        a = torch.randint(-127, 128, (B, M, K), dtype=torch.int8, generator=g).to(device)
+        b = torch.randint(-127, 128, (B, N, K), dtype=torch.int8, generator=g).to(device)
+        sa = (torch.rand(B, 1, generator=g) * 1e-2).expand(B, M).contiguous().to(device)
+        sb = (torch.rand(B, 1, generator=g) * 1e-2).expand(B, N).contiguous().to(device)
+        y = torch.empty((B, M, N), dtype=torch.float16, device=device)
+        p = lambda t: ctypes.c_void_p(t.data_ptr())
+        reps = 10
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap):
+            st = ctypes.c_void_p(cap.cuda_stream)
+            for _ in range(2):
+                Plan._call("bmm", L.sq_w8a8_bmm, (p(a), p(sa), p(b), p(sb), p(y), B, M, N, K, st))
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=cap):
+                for _ in range(reps):
+                    Plan._call("bmm", L.sq_w8a8_bmm, (p(a), p(sa), p(b), p(sb), p(y), B, M, N, K, st))
+        torch.cuda.current_stream().wait_stream(cap)
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.burst_iters)]
+        for e in ev:
+            flush()
+            e[0].record()
+            gr.replay()
+            e[1].record()
+        torch.cuda.synchronize()
+        us = 1e3 * sum(x.elapsed_time(z) for x, z in ev) / len(ev) / reps
+        nbytes = B * (M * K + N * K + 4 * M + 4 * N + 2 * M * N)
+        ops = 2 * B * M * N * K
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out[name] = {"shape": f"{B} x [{M} x {K}] x [{N} x {K}]^T", "us": round(us, 2),
+                     "tops": round(ops / (us * 1e-6) / 1e12, 1), "gbs": round(gbs, 1), "bound": "hbm",
+                     "frac": round(gbs / float(peaks["hbm_gbs"]), 4),
+                     "tensor_time_us_at_peak": round(ops / (float(peaks["bf16_tflops"]) * I8_PER_BF16 * 1e12) * 1e6, 2)}
+        del a, b, y
+    if sq.sq_poll_status() != 0:
+        raise RuntimeError("device wait timed out in the BMM loop")
     return out
 
 
@@ -909,6 +964,7 @@ def main():
     ap.add_argument("--streams", type=int, choices=[1, 2], default=2,
                     help="2: run the independent stages of a step on two streams")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bmm", action="store_true", help="also time the INT8 BMMs of attention")
     ap.add_argument("--producer", action="store_true",
                     help="also time the fused producer-side quantization of the linear's output")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU work")
