@@ -190,6 +190,43 @@ sq_status sq_ln_quant_act_static(const void* h_f16, int64_t M, int64_t K, int64_
 sq_status sq_tensor_range(const float* amax, const float* inv_s, int64_t K, float* range_out,
                           sq_stream_t stream);
 
+/*
+ * Tensor-parallel building blocks (the explainer runs the quantized models
+ * sharded over several GPUs: sections "how far speed and memory improved",
+ * OPT-175B on 4 GPUs instead of 8, and "does it hold for a 530B model", 8
+ * INT8 GPUs instead of 16 FP16).  A rank that
+ * holds a slice of K (row-parallel: a slice of every token's channels and of
+ * every weight row) must quantize with the ranges of the WHOLE row, so each
+ * rank reports its slice's per-row ranges, the ranks max-reduce them, and
+ * every rank quantizes its slice with the global ranges; the int32 partial
+ * accumulators (sq_w8a8_gemm_s32) are then sum-reduced, exactly, and
+ * dequantized once (sq_dequant).  The result equals the unsharded layer bit
+ * for bit.
+ *
+ * Rows are the activation transform of sq_ln_quant_act (gamma, beta, inv_s,
+ * eps) or, with s_fold given (and gamma, beta, inv_s NULL), the folded weight
+ * fp16(fp32(x) * s_fold[k]) of sq_quantize_weight.
+ */
+
+/* range_out[r] = max_k |x_hat[r, k]| over this slice's K columns.
+ *   x fp16 [rows, ld]; range_out fp32 [rows] */
+sq_status sq_row_ranges(const void* x_f16, int64_t rows, int64_t K, int64_t ld, const float* gamma,
+                        const float* beta, const float* inv_s, const float* s_fold, float eps,
+                        float* range_out, sq_stream_t stream);
+
+/* INT8 codes with given per-row ranges: scale[r] = range_in[r] / 127,
+ * q[r, k] = clamp(rint(x_hat[r, k] * (1 / scale[r])), -127, 127).
+ *   x fp16 [rows, ld]; range_in fp32 [rows]; q int8 [rows, K]; scale fp32 [rows] */
+sq_status sq_quantize_rows_ranged(const void* x_f16, int64_t rows, int64_t K, int64_t ld,
+                                  const float* gamma, const float* beta, const float* inv_s,
+                                  const float* s_fold, float eps, const float* range_in, int8_t* q,
+                                  float* scale, sq_stream_t stream);
+
+/* The linear's epilogue on its own: y[t, n] = fp16((fp32(acc[t, n]) * x_scale[t]) * w_scale[n]
+ * + fp32(bias[n])) (no add when bias is NULL).  acc int32 [M, N]; N % 4 == 0. */
+sq_status sq_dequant(const int32_t* acc, const float* x_scale, const float* w_scale,
+                     const void* bias_f16, void* y_f16, int64_t M, int64_t N, sq_stream_t stream);
+
 /* Bytes of workspace sq_w8a8_linear needs for this shape (0 if none).  The
  * workspace holds int32 partial sums and per-tile arrival counters of the
  * stream-K path.  The caller zero-fills it once before its first use; every

@@ -40,7 +40,7 @@ def test_status_strings():
     assert L.sq_status_string(0) == b"SQ_OK"
     assert L.sq_status_string(8) == b"SQ_ERR_TIMEOUT"
     assert L.sq_status_string(99) == b"SQ_ERR_UNKNOWN"
-    assert L.sq_abi_version() == 103
+    assert L.sq_abi_version() == 104
 
 
 FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced

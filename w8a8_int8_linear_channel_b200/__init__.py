@@ -27,7 +27,8 @@ __all__ = [
     "sq_w8a8_workspace_bytes", "sq_w8a8_linear", "sq_w8a8_linear_path", "sq_w8a8_gemm_s32",
     "sq_poll_status", "sq_set_wait_budget_ns", "sq_selftest_wait_timeout", "SmoothQuantLinear",
     "sq_quantize_weight_tensor", "sq_ln_quant_act_tensor", "sq_ln_quant_act_static", "sq_tensor_range",
-    "LEVELS", "sq_w8a8_linear_quant", "sq_w8a8_bmm",
+    "LEVELS", "sq_w8a8_linear_quant", "sq_w8a8_bmm", "sq_row_ranges", "sq_quantize_rows_ranged",
+    "sq_dequant",
     "PATH_AUTO", "PATH_TILED", "PATH_SPLITK", "PATH_PAIR", "PATH_WIDE", "SPLITK_MAX_M", "MAX_K", "library_path",
 ]
 
@@ -72,6 +73,9 @@ def _load() -> ctypes.CDLL:
         "sq_w8a8_linear_noalloc": ([P, P, P, P, P, P, I, I, I, P], S),
         "sq_w8a8_linear_quant": ([P, P, P, P, P, S, P, P, P, P, I, I, I, P, Z, P], S),
         "sq_w8a8_bmm": ([P, P, P, P, P, I, I, I, I, P], S),
+        "sq_row_ranges": ([P, I, I, I, P, P, P, P, F, P, P], S),
+        "sq_quantize_rows_ranged": ([P, I, I, I, P, P, P, P, F, P, P, P, P], S),
+        "sq_dequant": ([P, P, P, P, P, I, I, P], S),
         "sq_poll_status": ([P], S),
         "sq_set_wait_budget_ns": ([ctypes.c_uint64], None),
         "sq_selftest_wait_timeout": ([ctypes.c_uint64, P], S),
@@ -293,6 +297,48 @@ def sq_w8a8_linear_quant(xq, x_scale, wq, w_scale, range_next, xq_next, x_scale_
                                    _p(inv_s_next), _p(range_next), _p(xq_next), _p(x_scale_next), M, N, K,
                                    _p(workspace), ws_bytes, _stream(stream)), "sq_w8a8_linear_quant")
     return xq_next, x_scale_next
+
+
+def sq_row_ranges(x, range_out, gamma=None, beta=None, inv_s=None, s_fold=None, eps: float = 1e-5,
+                  stream=None):
+    """range_out[r] = max |x_hat[r, :]| over this slice's columns (activation transform, or the
+    folded weight when s_fold is given): a tensor-parallel shard's row ranges."""
+    rows, K, ld = _rows(x, torch.float16, "x")
+    _vec(range_out, rows, torch.float32, "range_out")
+    for t, n in ((gamma, "gamma"), (beta, "beta"), (inv_s, "inv_s"), (s_fold, "s_fold")):
+        _vec(t, K, torch.float32, n)
+    _check(_L.sq_row_ranges(_p(x), rows, K, ld, _p(gamma), _p(beta), _p(inv_s), _p(s_fold), eps,
+                            _p(range_out), _stream(stream)), "sq_row_ranges")
+    return range_out
+
+
+def sq_quantize_rows_ranged(x, range_in, q, scale, gamma=None, beta=None, inv_s=None, s_fold=None,
+                            eps: float = 1e-5, stream=None):
+    """INT8 codes of the rows with given per-row ranges (scale = range / 127, codes clamped)."""
+    rows, K, ld = _rows(x, torch.float16, "x")
+    _vec(range_in, rows, torch.float32, "range_in")
+    _vec(scale, rows, torch.float32, "scale")
+    if q.dtype != torch.int8 or tuple(q.shape) != (rows, K) or not q.is_contiguous():
+        raise ValueError("q: need a contiguous int8 [rows, K] tensor")
+    for t, n in ((gamma, "gamma"), (beta, "beta"), (inv_s, "inv_s"), (s_fold, "s_fold")):
+        _vec(t, K, torch.float32, n)
+    _check(_L.sq_quantize_rows_ranged(_p(x), rows, K, ld, _p(gamma), _p(beta), _p(inv_s), _p(s_fold), eps,
+                                      _p(range_in), _p(q), _p(scale), _stream(stream)), "sq_quantize_rows_ranged")
+    return q, scale
+
+
+def sq_dequant(acc, x_scale, w_scale, y, bias=None, stream=None):
+    """y = fp16((acc * x_scale[:, None]) * w_scale[None, :] + bias) from int32 accumulators."""
+    if acc.dtype != torch.int32 or acc.dim() != 2 or not acc.is_contiguous():
+        raise ValueError("acc: need a contiguous int32 [M, N] tensor")
+    M, N = acc.shape
+    _vec(x_scale, M, torch.float32, "x_scale")
+    _vec(w_scale, N, torch.float32, "w_scale")
+    _vec(bias, N, torch.float16, "bias")
+    if y.dtype != torch.float16 or tuple(y.shape) != (M, N) or not y.is_contiguous():
+        raise ValueError("y: need a contiguous fp16 [M, N] tensor")
+    _check(_L.sq_dequant(_p(acc), _p(x_scale), _p(w_scale), _p(bias), _p(y), M, N, _stream(stream)), "sq_dequant")
+    return y
 
 
 def sq_w8a8_bmm(a, a_scale, b, b_scale, y, stream=None):

@@ -157,7 +157,50 @@ __global__ void __launch_bounds__(1024) k_tensor_range(const float* __restrict__
   }
 }
 
+// y[t, n] = fp16(((float)acc[t, n] * sx[t]) * sw[n] + bias[n]): the linear's
+// epilogue on its own, for int32 accumulators summed across tensor-parallel
+// ranks.  Four outputs per thread and iteration (N % 4 == 0), grid-stride.
+__global__ void __launch_bounds__(256) k_dequant(const int32_t* __restrict__ acc, const float* __restrict__ sx,
+                                                 const float* __restrict__ sw, const __half* __restrict__ bias,
+                                                 __half* __restrict__ y, int64_t M, int64_t N) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int64_t n4 = N / 4;
+  const int64_t total = M * n4;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / n4;
+    const int64_t n = (i - t * n4) * 4;
+    const int4 a = __ldg(reinterpret_cast<const int4*>(acc + t * N + n));
+    const float4 w = __ldg(reinterpret_cast<const float4*>(sw + n));
+    const float x = sx[t];
+    float f[4] = {__fmul_rn(__fmul_rn(__int2float_rn(a.x), x), w.x), __fmul_rn(__fmul_rn(__int2float_rn(a.y), x), w.y),
+                  __fmul_rn(__fmul_rn(__int2float_rn(a.z), x), w.z), __fmul_rn(__fmul_rn(__int2float_rn(a.w), x), w.w)};
+    if (bias != nullptr) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) f[j] = __fadd_rn(f[j], __half2float(bias[n + j]));
+    }
+    const __half2 lo = __floats2half2_rn(f[0], f[1]);
+    const __half2 hi = __floats2half2_rn(f[2], f[3]);
+    uint2 o;
+    o.x = *reinterpret_cast<const uint32_t*>(&lo);
+    o.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(y + t * N + n) = o;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_dequant(const int32_t* acc, const float* sx, const float* sw, const __half* bias, __half* y,
+                           int64_t M, int64_t N, const Ctx& c) {
+  const int64_t total = M * (N / 4);
+  int64_t blocks = static_cast<int64_t>(c.num_sms) * 8;
+  const int64_t need = (total + 255) / 256;
+  if (blocks > need) blocks = need;
+  if (blocks < 1) blocks = 1;
+  return launch_pdl(k_dequant, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, c.stream, acc, sx, sw, bias, y,
+                    M, N);
+}
 
 cudaError_t launch_tensor_range(const float* amax, const float* inv_s, int64_t K, float* range,
                                 const Ctx& c) {

@@ -260,16 +260,19 @@ __device__ __forceinline__ uint2 pack8c(const float (&x)[8], float inv) {
   return make_uint2(quant4c(x[0], x[1], x[2], x[3], inv), quant4c(x[4], x[5], x[6], x[7], inv));
 }
 
-// Scale and reciprocal of a per-tensor range (same op order as per row).
-__device__ __forceinline__ void range_scale(const float* range, float& sc, float& inv) {
-  sc = __fdiv_rn(*range, 127.0f);
+// Scale and reciprocal of a given range (same op order as per row): one
+// range for the tensor, or one per row (range_per_row).
+__device__ __forceinline__ void range_scale(const RowArgs& a, int64_t r, float& sc, float& inv) {
+  sc = __fdiv_rn(a.range_per_row ? a.range_in[r] : *a.range_in, 127.0f);
   inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
 }
 
-// Range pass: merge one row's max into the tensor's range (exact and
-// order-free: non-negative floats order as their bit patterns).
-__device__ __forceinline__ void range_merge(float* range, float m) {
-  atomicMax(reinterpret_cast<int*>(range), __float_as_int(m));
+// Range pass: a row's max goes to its own slot (range_per_row) or is merged
+// into the tensor's range (exact and order-free: non-negative floats order
+// as their bit patterns).
+__device__ __forceinline__ void range_merge(const RowArgs& a, int64_t r, float m) {
+  if (a.range_per_row) a.range_out[r] = m;
+  else atomicMax(reinterpret_cast<int*>(a.range_out), __float_as_int(m));
 }
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
@@ -323,7 +326,7 @@ __global__ void __launch_bounds__(kWarpThreads) k_rows_warp(const RowArgs a) {
     int8_t* dst = a.q + r * a.K;
     if (a.range_in) {  // per-tensor scale fixed in advance: no row max
       float sc, inv;
-      range_scale(a.range_in, sc, inv);
+      range_scale(a, r, sc, inv);
       if (lane == 0) a.scale[r] = sc;
 #pragma unroll
       for (int i = 0; i < NW; ++i) {
@@ -335,7 +338,7 @@ __global__ void __launch_bounds__(kWarpThreads) k_rows_warp(const RowArgs a) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if (a.range_out) {  // range pass only
-      if (lane == 0) range_merge(a.range_out, amax);
+      if (lane == 0) range_merge(a, r, amax);
       continue;
     }
     const float sc = __fdiv_rn(amax, 127.0f);
@@ -523,7 +526,7 @@ __device__ __forceinline__ void cta_rows(const RowArgs& a, RowSharedT<T>& sh, fl
       }
     } else if (a.range_in) {  // per-tensor scale fixed in advance: no row max, one pass
       float sc, inv;
-      range_scale(a.range_in, sc, inv);
+      range_scale(a, r, sc, inv);
       if (tid == 0) a.scale[r] = sc;
       int8_t* dst = a.q + r * a.K;
 #pragma unroll
@@ -560,7 +563,7 @@ __device__ __forceinline__ void cta_rows(const RowArgs& a, RowSharedT<T>& sh, fl
 #pragma unroll
       for (int w = 0; w < W; ++w) m = fmaxf(m, sh.mx[par][w]);
       if (a.range_out) {  // range pass only
-        if (tid == 0) range_merge(a.range_out, m);
+        if (tid == 0) range_merge(a, r, m);
       } else {
         const float sc = __fdiv_rn(m, 127.0f);
         const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
@@ -673,7 +676,7 @@ __device__ __forceinline__ void cta_rows_fast(const RowArgs& a, RowSharedT<T>& s
       int8_t* dst = a.q + r * a.K;
       if (a.range_in) {  // per-tensor scale fixed in advance: no row max
         float sc, inv;
-        range_scale(a.range_in, sc, inv);
+        range_scale(a, r, sc, inv);
         if (tid == 0) a.scale[r] = sc;
 #pragma unroll
         for (int i = 0; i < NCH; ++i) {
@@ -689,7 +692,7 @@ __device__ __forceinline__ void cta_rows_fast(const RowArgs& a, RowSharedT<T>& s
 #pragma unroll
         for (int w = 0; w < W; ++w) m = fmaxf(m, sh.mx[par][w]);
         if (a.range_out) {  // range pass only
-          if (tid == 0) range_merge(a.range_out, m);
+          if (tid == 0) range_merge(a, r, m);
         } else {
           const float sc = __fdiv_rn(m, 127.0f);
           const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;

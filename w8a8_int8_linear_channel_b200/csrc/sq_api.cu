@@ -230,6 +230,33 @@ static sq_status act_args(const void* h_f16, int64_t M, int64_t K, int64_t ld, c
   return SQ_OK;
 }
 
+// Row arguments of the per-row-range entry points: the weight fold (s_fold)
+// or the activation transform (LayerNorm / 1/s), never both.
+static sq_status ranged_args(const void* x_f16, int64_t rows, int64_t K, int64_t ld, const float* gamma,
+                             const float* beta, const float* inv_s, const float* s_fold, float eps,
+                             RowArgs* a) {
+  if (!x_f16 || rows <= 0) return SQ_ERR_INVALID_ARG;
+  if (!gamma && beta) return SQ_ERR_INVALID_ARG;
+  if (s_fold && (gamma || inv_s)) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_k(K);
+  if (st != SQ_OK) return st;
+  if ((st = check_ld(K, ld)) != SQ_OK) return st;
+  if (!aligned16(x_f16) || !opt_aligned(gamma) || !opt_aligned(beta) || !opt_aligned(inv_s) ||
+      !opt_aligned(s_fold))
+    return SQ_ERR_MISALIGNED;
+  *a = RowArgs{};
+  a->x = static_cast<const __half*>(x_f16);
+  a->rows = rows;
+  a->K = K;
+  a->ld = ld;
+  a->gamma = gamma;
+  a->beta = beta;
+  a->vec = s_fold ? s_fold : inv_s;
+  a->eps = eps;
+  a->range_per_row = 1;
+  return SQ_OK;
+}
+
 extern "C" {
 
 const char* sq_status_string(int status) {
@@ -247,7 +274,7 @@ const char* sq_status_string(int status) {
   }
 }
 
-int sq_abi_version(void) { return 103; }
+int sq_abi_version(void) { return 104; }
 
 sq_status sq_calibrate_absmax(const void* x_f16, int64_t rows, int64_t K, int64_t ld,
                               const float* ln_gamma, const float* ln_beta, float ln_eps,
@@ -402,6 +429,50 @@ sq_status sq_ln_quant_act_static(const void* h_f16, int64_t M, int64_t K, int64_
   if ((st = current_ctx(stream, &ctx)) != SQ_OK) return st;
   a.range_in = range_in;
   return launched(launch_ln_quant_act(a, ctx));
+}
+
+sq_status sq_row_ranges(const void* x_f16, int64_t rows, int64_t K, int64_t ld, const float* gamma,
+                        const float* beta, const float* inv_s, const float* s_fold, float eps,
+                        float* range_out, sq_stream_t stream) {
+  RowArgs a;
+  sq_status st = ranged_args(x_f16, rows, K, ld, gamma, beta, inv_s, s_fold, eps, &a);
+  if (st != SQ_OK) return st;
+  if (!range_out) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(range_out)) return SQ_ERR_MISALIGNED;
+  Ctx ctx;
+  if ((st = current_ctx(stream, &ctx)) != SQ_OK) return st;
+  a.range_out = range_out;
+  return launched(s_fold ? launch_quantize_weight(a, ctx) : launch_ln_quant_act(a, ctx));
+}
+
+sq_status sq_quantize_rows_ranged(const void* x_f16, int64_t rows, int64_t K, int64_t ld, const float* gamma,
+                                  const float* beta, const float* inv_s, const float* s_fold, float eps,
+                                  const float* range_in, int8_t* q, float* scale, sq_stream_t stream) {
+  RowArgs a;
+  sq_status st = ranged_args(x_f16, rows, K, ld, gamma, beta, inv_s, s_fold, eps, &a);
+  if (st != SQ_OK) return st;
+  if (!range_in || !q || !scale) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(range_in) || !aligned16(q) || !aligned16(scale)) return SQ_ERR_MISALIGNED;
+  Ctx ctx;
+  if ((st = current_ctx(stream, &ctx)) != SQ_OK) return st;
+  a.range_in = range_in;
+  a.q = q;
+  a.scale = scale;
+  return launched(s_fold ? launch_quantize_weight(a, ctx) : launch_ln_quant_act(a, ctx));
+}
+
+sq_status sq_dequant(const int32_t* acc, const float* x_scale, const float* w_scale, const void* bias_f16,
+                     void* y_f16, int64_t M, int64_t N, sq_stream_t stream) {
+  if (!acc || !x_scale || !w_scale || !y_f16 || M <= 0 || N <= 0) return SQ_ERR_INVALID_ARG;
+  if (N % 4 != 0) return SQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(acc) || !aligned16(x_scale) || !aligned16(w_scale) || !opt_aligned(bias_f16) ||
+      !aligned16(y_f16))
+    return SQ_ERR_MISALIGNED;
+  Ctx ctx;
+  sq_status st = current_ctx(stream, &ctx);
+  if (st != SQ_OK) return st;
+  return launched(launch_dequant(acc, x_scale, w_scale, static_cast<const __half*>(bias_f16),
+                                 static_cast<__half*>(y_f16), M, N, ctx));
 }
 
 sq_status sq_tensor_range(const float* amax, const float* inv_s, int64_t K, float* range_out,

@@ -54,7 +54,12 @@ struct RowArgs {
   // per-tensor scales (levels O2 / O3 of the explainer, per-tensor weights):
   const float* range_in;  // fixed range [1]: scale = range / 127, codes clamped, no row max
   float* range_out;       // range pass [1]: atomic max of every row's |x_hat|, nothing else written
+  int range_per_row;      // range_in / range_out hold one range per row [rows] instead
 };
+
+// Elementwise dequantization of int32 accumulators (k_cols.cu).
+cudaError_t launch_dequant(const int32_t* acc, const float* sx, const float* sw, const __half* bias, __half* y,
+                           int64_t M, int64_t N, const Ctx& c);
 
 cudaError_t launch_ln_quant_act(const RowArgs& a, const Ctx& c);
 cudaError_t launch_quantize_weight(const RowArgs& a, const Ctx& c);
