@@ -55,3 +55,25 @@ def test_bmm_attention_shapes(sq, which):
     got = host(y)
     for i in (0, B - 1):
         assert bits_equal(got[i:i + 1], oracle.w8a8_bmm(a[i:i + 1], sa[i:i + 1], b[i:i + 1], sb[i:i + 1]))
+
+
+@pytest.mark.parametrize("K", [256, 272])
+def test_extreme_codes_short_k(sq, K):
+    """All +-127 codes at short K (|acc| = K * 127^2, 4 129 024 at K = 256,
+    4 386 688 at K = 272: either side of 2^22), through the BMM and the
+    linear on the CTA-pair kernel."""
+    B, M, N = 2, 300, 264
+    a = np.full((B, M, K), 127, np.int8)
+    a[:, 1::2] = -127
+    b = np.full((B, N, K), 127, np.int8)
+    b[:, 3::5] = -127
+    rng = np.random.default_rng(K)
+    sa = rng.uniform(1e-6, 1e-5, (B, M)).astype(np.float32)
+    sb = rng.uniform(1e-6, 1e-5, (B, N)).astype(np.float32)
+    y = torch.empty((B, M, N), dtype=torch.float16, device="cuda")
+    sq.sq_w8a8_bmm(dev(a), dev(sa), dev(b), dev(sb), y)
+    assert bits_equal(host(y), oracle.w8a8_bmm(a, sa, b, sb))
+    # the same through the linear (CTA-pair kernel, M > 128)
+    y2 = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    sq.sq_w8a8_linear(dev(a[0]), dev(sa[0]), dev(b[0]), dev(sb[0]), y2)
+    assert bits_equal(host(y2), oracle.w8a8_linear(a[0], sa[0], b[0], sb[0]))

@@ -252,6 +252,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       q_sc = __fdiv_rn(*g.range_next, 127.0f);
       q_inv = q_sc > 0.0f ? __frcp_rn(q_sc) : 0.0f;
     }
+    // this thread's scale entries of a tile: sw / bias / 1/s of column et and
+    // sx of its row; fetched one tile ahead so their global-load latency
+    // overlaps the previous tile's epilogue instead of stalling every tile
+    struct Vecs {
+      float sw, is, sx;
+      __half bias;
+    };
+    auto fetch = [&](int t) {
+      Vecs v{0.0f, 1.0f, 0.0f, __float2half_rn(0.0f)};
+      if (EPI == EPI_I32 || t >= tiles) return v;
+      const int bi = t / per_item;
+      int tm, tn;
+      tile_coords(t - bi * per_item, tiles_m, tiles_n, tm, tn);
+      const int64_t n = static_cast<int64_t>(tn) * BN + et;
+      const int64_t row = static_cast<int64_t>(tm) * (2 * BM) + static_cast<int64_t>(rank) * BM + 32 * q + lane;
+      if (n < g.N) {
+        v.sw = g.sw[static_cast<int64_t>(bi) * g.N + n];
+        if (g.bias != nullptr) v.bias = g.bias[n];
+        if (EPI == EPI_Q8 && g.inv_s_next != nullptr) v.is = g.inv_s_next[n];
+      }
+      if (row < g.M) v.sx = g.sx[static_cast<int64_t>(bi) * g.M + row];
+      return v;
+    };
+    Vecs nxt = fetch(pair);
     int tl = 0;
     for (int t = pair; t < tiles; t += npairs, ++tl) {
       const int b = tl & 1;
@@ -260,17 +284,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tile_coords(t - bi * per_item, tiles_m, tiles_n, tm, tn);
       const int64_t m0 = static_cast<int64_t>(tm) * (2 * BM) + static_cast<int64_t>(rank) * BM;
       const int64_t n0 = static_cast<int64_t>(tn) * BN;
+      const Vecs cur = nxt;
+      nxt = fetch(t + npairs);
       if (EPI != EPI_I32) {
-        const int64_t n = n0 + et;
-        sw_s[et] = n < g.N ? g.sw[static_cast<int64_t>(bi) * g.N + n] : 0.0f;
-        bias_s[et] = (g.bias != nullptr && n < g.N) ? g.bias[n] : __float2half_rn(0.0f);
-        if (EPI == EPI_Q8) inv_s_s[et] = (g.inv_s_next != nullptr && n < g.N) ? g.inv_s_next[n] : 1.0f;
+        sw_s[et] = cur.sw;
+        bias_s[et] = cur.bias;
+        if (EPI == EPI_Q8) inv_s_s[et] = cur.is;
       }
-      float sxr = 0.0f;
-      if (EPI != EPI_I32) {
+      const float sxr = cur.sx;
+      if (EPI == EPI_Q8) {
         const int64_t row = m0 + 32 * q + lane;
-        sxr = row < g.M ? g.sx[static_cast<int64_t>(bi) * g.M + row] : 0.0f;
-        if (EPI == EPI_Q8 && tn == 0 && half == 0 && row < g.M) g.sx_next[row] = q_sc;
+        if (tn == 0 && half == 0 && row < g.M) g.sx_next[row] = q_sc;
       }
       named_bar_sync(1, 32 * kEpiWarps);
       pair_wait(accf_bar(b), static_cast<uint32_t>((tl >> 1) & 1), false, budget, status, abort_flag, peer_abort);
