@@ -24,6 +24,11 @@ Sources, cited by page title and section:
   [Q]  itmedia LLM quantization tutorial, section 3 (range -> scale -> round,
        the 53 -> 5 -> 50 example).
 
+Beyond the per-token / per-channel layer: the explainer's quantization
+levels O1-O3 (``quantize_weight_tensor``, ``ln_quant_act_tensor``,
+``ln_quant_act_static``, ``tensor_range``), producer-side quantization
+(``w8a8_linear_quant_static``) and the INT8 BMM (``w8a8_bmm``).
+
 Parity status: every function here is pinned by ``tests/test_oracle.py``
 except the quality ranking (naive vs smoothed reconstruction error), which
 the pages predict only qualitatively: parity unpinned for
