@@ -101,10 +101,19 @@ void oracle_quantize_with_scale(const float* x, int64_t n, float scale, int8_t* 
  *   mu    = (double)S1 / (K * 2^24)
  *   var   = max(d(S2) / (K * 2^48) - mu * mu, 0)
  *   rstd  = 1 / sqrt(var + (double)eps)
- * and then rounded to float. */
+ * and then rounded to float.  A row holding an Inf or a NaN has no finite
+ * mean or variance; as in the usual LayerNorm's IEEE arithmetic, both are
+ * then NaN (so is every value of the row's LayerNorm output). */
 static void ln_stats(const uint16_t* h, int64_t K, float eps, float* mu32, float* rstd32) {
   i128 s1 = 0;
   u128 s2 = 0;
+  for (int64_t k = 0; k < K; ++k) {
+    if (!isfinite(h2f(h[k]))) {
+      *mu32 = NAN;
+      *rstd32 = NAN;
+      return;
+    }
+  }
   for (int64_t k = 0; k < K; ++k) {
     double hv = (double)h2f(h[k]);
     int64_t v = (int64_t)(hv * 16777216.0); /* exact: hv * 2^24 is an integer */

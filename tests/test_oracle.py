@@ -504,3 +504,55 @@ def test_bmm_items_are_independent_linears():
         exact = acc * sa[i][:, None].astype(np.float64) * sb[i][None, :].astype(np.float64)
         assert np.all(np.abs(y[i].astype(np.float64) - exact) <= np.spacing(np.abs(exact).astype(np.float16)))
         assert np.array_equal(y[i], oracle.w8a8_linear(a[i], sa[i], b[i], sb[i]))
+
+
+# ------------------------------------------------------- non-finite inputs ----
+# IEEE arithmetic fixes these: a mean or variance over a row that holds an Inf
+# or a NaN is NaN, a NaN never wins a maximum taken with ">", and a NaN
+# product has no nearest integer level (the quantizer gives 0 for it).
+@pytest.mark.parametrize("bad", [np.inf, -np.inf, np.nan])
+def test_ln_stats_of_a_non_finite_row_are_nan(bad):
+    h = f16(np.linspace(-2, 2, 64)).reshape(2, 32)
+    h[1, 7] = bad
+    mu, rstd = oracle.ln_stats(h)
+    assert np.isfinite(mu[0]) and np.isfinite(rstd[0])
+    assert np.isnan(mu[1]) and np.isnan(rstd[1])
+    g = np.ones(32, np.float32)
+    x = oracle.act_rows(h, g, g)
+    assert np.isfinite(x[0]).all() and np.isnan(x[1]).all()
+
+
+@pytest.mark.parametrize("bad", [np.inf, np.nan])
+def test_ln_quantization_of_a_non_finite_row(bad):
+    rng = np.random.default_rng(3)
+    h = f16(rng.standard_normal((3, 48)))
+    h[1, 5] = bad
+    g = (rng.random(48) + 0.5).astype(np.float32)
+    b = rng.standard_normal(48).astype(np.float32)
+    xq, sx = oracle.ln_quant_act(h, g, b)
+    # the NaN row: no level wins the maximum, scale 0, every code 0
+    assert sx[1] == 0.0 and not xq[1].any()
+    # the finite rows are what they are alone
+    for r in (0, 2):
+        q1, s1 = oracle.ln_quant_act(h[r:r + 1], g, b)
+        assert np.array_equal(xq[r], q1[0]) and sx[r] == s1[0]
+    # calibration: the NaN row adds nothing to the running maxima
+    a_all = oracle.calibrate_absmax(h, gamma=g, beta=b)
+    a_fin = oracle.calibrate_absmax(h[[0, 2]], gamma=g, beta=b)
+    assert np.array_equal(a_all, a_fin)
+
+
+def test_nan_values_quantize_to_zero_and_inf_saturates():
+    rng = np.random.default_rng(4)
+    h = f16(rng.standard_normal((2, 40)))
+    h[0, 3] = np.nan
+    h[1, 9] = np.inf
+    xq, sx = oracle.ln_quant_act(h)  # no LayerNorm: x_hat = h
+    # row 0: the NaN is ignored by the maximum and gets code 0
+    assert sx[0] == np.float32(np.abs(np.delete(h[0], 3).astype(np.float32)).max() / np.float32(127))
+    assert xq[0, 3] == 0 and np.abs(xq[0]).max() == 127
+    # row 1: an infinite range makes the scale Inf and 1/scale 0, so every
+    # product is 0 (finite values) or NaN (Inf * 0): all codes 0
+    assert np.isinf(sx[1]) and not xq[1].any()
+    wq, sw = oracle.quantize_weight(h)
+    assert np.array_equal(wq, xq) and np.array_equal(sw, sx)
