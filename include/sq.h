@@ -33,6 +33,13 @@
  *     order written below, with no fused multiply-add; rint is ties-to-even.
  *     INT8 codes and int32 accumulators are therefore bit-identical to any
  *     implementation that follows the same order.
+ *   - Non-finite inputs follow IEEE arithmetic: a NaN never sets a range
+ *     (maxima ignore it) and is coded 0; an Inf sets an infinite range (scale
+ *     Inf, reciprocal 0, so every code of that row or tensor is 0); a
+ *     LayerNorm row holding an Inf or a NaN has NaN mean and rstd, so all of
+ *     its values are NaN (scale 0, codes 0, no effect on calibration).  With
+ *     a range fixed in advance (level O3, producer-side quantization) +-Inf
+ *     saturate to +-127 and NaN is coded 0.
  *   - Device-side waits are bounded (default 2 s, see sq_set_wait_budget_ns).
  *     A wait that runs out records SQ_ERR_TIMEOUT in a per-device status word
  *     and the kernel returns early (its outputs are then undefined); read it

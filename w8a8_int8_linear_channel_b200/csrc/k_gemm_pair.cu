@@ -325,9 +325,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // the composition, per element: y = fp16((acc * sx) * sw + bias),
           // a = relu ? max(y, 0) : y, x = a * inv_s_next, then the static
           // quantizer; fp32 pairs, the ReLU on half2 (max with 0 turns a NaN
-          // into 0, like the scalar test), codes packed 4 per word.  With a
-          // zero range every code is 0 (as the scalar quantizer gives for a
-          // zero reciprocal), so the product x * q_inv below is never NaN.
+          // into 0, like the scalar test), codes packed 4 per word, a NaN
+          // product coded 0 (q8_code_bits).  With a zero range every code is
+          // 0, as the scalar quantizer gives for a zero reciprocal.
           __align__(16) uint32_t qw[8];
           if (q_inv == 0.0f) {
 #pragma unroll
@@ -365,11 +365,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               const float2 a0 = __half22float2(h0), a1 = __half22float2(h1);
               const float2 p0 = f2_unpack(f2_mul_rn(f2_mul_rn(f2_pack(a0.x, a0.y), f2_pack(is.x, is.y)), qi2));
               const float2 p1 = f2_unpack(f2_mul_rn(f2_mul_rn(f2_pack(a1.x, a1.y), f2_pack(is.z, is.w)), qi2));
-              const float kMagic = 12582912.0f;  // 1.5 * 2^23: rint, code in the low byte
-              const uint32_t c0 = __float_as_uint(__fadd_rn(fminf(fmaxf(p0.x, -127.0f), 127.0f), kMagic));
-              const uint32_t c1 = __float_as_uint(__fadd_rn(fminf(fmaxf(p0.y, -127.0f), 127.0f), kMagic));
-              const uint32_t c2 = __float_as_uint(__fadd_rn(fminf(fmaxf(p1.x, -127.0f), 127.0f), kMagic));
-              const uint32_t c3 = __float_as_uint(__fadd_rn(fminf(fmaxf(p1.y, -127.0f), 127.0f), kMagic));
+              const uint32_t c0 = q8_code_bits(p0.x);
+              const uint32_t c1 = q8_code_bits(p0.y);
+              const uint32_t c2 = q8_code_bits(p1.x);
+              const uint32_t c3 = q8_code_bits(p1.y);
               qw[j / 4] = __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
             }
           }

@@ -26,6 +26,8 @@
 // atomicMax per cluster instead of one per CTA.
 #include <cooperative_groups.h>
 
+#include <type_traits>
+
 #include "sq_internal.h"
 #include "sq_ptx.cuh"
 
@@ -47,6 +49,7 @@ struct Sums {
   long long s1;   // sum v            (units 2^-24 of h)
   long long s2h;  // sum of h^2 parts that are multiples of 2^-13, in units 2^-13
   long long s2l;  // sum of the remainders below 2^-13, in units 2^-48
+  int bad;        // the row holds an Inf or a NaN (its statistics are NaN)
 };
 
 __device__ __forceinline__ uint32_t half_bits(const uint4& v, int j) {
@@ -73,6 +76,9 @@ __device__ __forceinline__ void chunk_sums(const uint4& v, Sums& s) {
   s.s1 += __double2ll_rn(__dmul_rn(c1, 16777216.0));            // * 2^24
   s.s2h += __double2ll_rn(__dmul_rn(c2h, 8192.0));              // * 2^13
   s.s2l += __double2ll_rn(__dmul_rn(c2l, 281474976710656.0));   // * 2^48
+  // eight finite fp16 values sum to a finite double; an Inf or a NaN among
+  // them leaves c1 infinite or NaN
+  s.bad |= !(fabs(c1) <= 1.7976931348623157e308);
 }
 
 // Same sums from the 8 values already converted to fp32 (exact conversions).
@@ -91,6 +97,7 @@ __device__ __forceinline__ void chunk_sums_f(const float (&x)[8], Sums& s) {
   s.s1 += __double2ll_rn(__dmul_rn(c1, 16777216.0));            // * 2^24
   s.s2h += __double2ll_rn(__dmul_rn(c2h, 8192.0));              // * 2^13
   s.s2l += __double2ll_rn(__dmul_rn(c2l, 281474976710656.0));   // * 2^48
+  s.bad |= !(fabs(c1) <= 1.7976931348623157e308);
 }
 
 __device__ __forceinline__ void warp_sum(Sums& s) {
@@ -100,12 +107,18 @@ __device__ __forceinline__ void warp_sum(Sums& s) {
     s.s2h += __shfl_xor_sync(0xffffffffu, s.s2h, o);
     s.s2l += __shfl_xor_sync(0xffffffffu, s.s2l, o);
   }
+  s.bad = __any_sync(0xffffffffu, s.bad);
 }
 
 // mu and rstd from the exact sums S1 = s1 and S2 = s2h * 2^35 + s2l, by the
 // fixed sequence of correctly rounded fp64 operations documented in sq.h.
 __device__ __forceinline__ void ln_finalize(const Sums& s, int64_t K, float eps, float& mu,
                                             float& rstd) {
+  if (s.bad) {  // a row with an Inf or a NaN: NaN statistics
+    mu = __int_as_float(0x7fc00000);
+    rstd = mu;
+    return;
+  }
   const u128 S2 = (static_cast<u128>(static_cast<unsigned long long>(s.s2h)) << 35) +
                   static_cast<u128>(static_cast<__int128>(s.s2l));
   const double two64 = 18446744073709551616.0;
@@ -184,16 +197,27 @@ __device__ __forceinline__ void transform8(const uint4& v, int64_t c, const RowA
 // Eight codes packed into 8 bytes.  p = x * inv (rounded), then
 // p + 1.5 * 2^23 rounds p to the nearest integer, ties to even, and leaves
 // that integer in the low mantissa bits: the low byte of the sum is the
-// two's-complement code (a NaN product gives byte 0).  No clamp is needed:
+// two's-complement code (code_bits maps a NaN sum to byte 0).  No clamp is needed:
 // inv = RN(1 / RN(amax / 127)) and |x| <= amax bound |p| by 127 (1 + 3 * 2^-24)
 // < 127.5, so the rounded value is already inside [-127, 127] -- the same
 // codes as clamp(rint(p), -127, 127).
-__device__ __forceinline__ uint32_t quant4(float x0, float x1, float x2, float x3, float inv) {
+// SAFE: a NaN sum (any NaN bit pattern) is mapped by an unsigned min onto
+// 1.5 * 2^23 + 256, whose low byte is 0, while every in-range sum
+// (0x4B3FFF81 .. 0x4B40007F) is below it.  Rows whose range is finite have
+// no NaN product and skip it.
+template <bool SAFE>
+__device__ __forceinline__ uint32_t code_bits(float p) {
   const float kMagic = 12582912.0f;  // 1.5 * 2^23
-  const uint32_t b0 = __float_as_uint(__fadd_rn(__fmul_rn(x0, inv), kMagic));
-  const uint32_t b1 = __float_as_uint(__fadd_rn(__fmul_rn(x1, inv), kMagic));
-  const uint32_t b2 = __float_as_uint(__fadd_rn(__fmul_rn(x2, inv), kMagic));
-  const uint32_t b3 = __float_as_uint(__fadd_rn(__fmul_rn(x3, inv), kMagic));
+  const uint32_t b = __float_as_uint(__fadd_rn(p, kMagic));
+  return SAFE ? min(b, 0x4B400100u) : b;
+}
+
+template <bool SAFE>
+__device__ __forceinline__ uint32_t quant4(float x0, float x1, float x2, float x3, float inv) {
+  const uint32_t b0 = code_bits<SAFE>(__fmul_rn(x0, inv));
+  const uint32_t b1 = code_bits<SAFE>(__fmul_rn(x1, inv));
+  const uint32_t b2 = code_bits<SAFE>(__fmul_rn(x2, inv));
+  const uint32_t b3 = code_bits<SAFE>(__fmul_rn(x3, inv));
   return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
 }
 
@@ -235,9 +259,20 @@ __device__ __forceinline__ void transform8f(float (&x)[8], int64_t c, const RowA
   }
 }
 
+template <bool SAFE = false>
 __device__ __forceinline__ uint2 pack8(const float (&x)[8], float inv) {
-  return make_uint2(quant4(x[0], x[1], x[2], x[3], inv), quant4(x[4], x[5], x[6], x[7], inv));
+  return make_uint2(quant4<SAFE>(x[0], x[1], x[2], x[3], inv), quant4<SAFE>(x[4], x[5], x[6], x[7], inv));
 }
+
+// max(a, |b|) for a >= 0 (or NaN), propagating a NaN.  A row maximum taken
+// with it is finite exactly when the row holds no NaN and no Inf.
+__device__ __forceinline__ float absmax_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(fabsf(b)));
+  return d;
+}
+
+__device__ __forceinline__ bool finite_f(float m) { return fabsf(m) <= 3.402823466e38f; }
 
 // The same codes for a scale fixed in advance (per-tensor levels): x * inv
 // may now leave [-127, 127], so it is clamped first (a NaN product passes
@@ -248,11 +283,10 @@ __device__ __forceinline__ float clamp127(float p) {
 }
 
 __device__ __forceinline__ uint32_t quant4c(float x0, float x1, float x2, float x3, float inv) {
-  const float kMagic = 12582912.0f;  // 1.5 * 2^23
-  const uint32_t b0 = __float_as_uint(__fadd_rn(clamp127(__fmul_rn(x0, inv)), kMagic));
-  const uint32_t b1 = __float_as_uint(__fadd_rn(clamp127(__fmul_rn(x1, inv)), kMagic));
-  const uint32_t b2 = __float_as_uint(__fadd_rn(clamp127(__fmul_rn(x2, inv)), kMagic));
-  const uint32_t b3 = __float_as_uint(__fadd_rn(clamp127(__fmul_rn(x3, inv)), kMagic));
+  const uint32_t b0 = code_bits<true>(clamp127(__fmul_rn(x0, inv)));
+  const uint32_t b1 = code_bits<true>(clamp127(__fmul_rn(x1, inv)));
+  const uint32_t b2 = code_bits<true>(clamp127(__fmul_rn(x2, inv)));
+  const uint32_t b3 = code_bits<true>(clamp127(__fmul_rn(x3, inv)));
   return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
 }
 
@@ -305,7 +339,7 @@ __global__ void __launch_bounds__(kWarpThreads) k_rows_warp(const RowArgs a) {
     }
     float mu = 0.0f, rstd = 0.0f;
     if (use_ln) {
-      Sums s{0, 0, 0};
+      Sums s{0, 0, 0, 0};
 #pragma unroll
       for (int i = 0; i < NW; ++i)
         if (lane + 32 * i < Kc) chunk_sums(v[i], s);
@@ -320,7 +354,7 @@ __global__ void __launch_bounds__(kWarpThreads) k_rows_warp(const RowArgs a) {
       if (c < Kc) {
         transform8<MODE>(v[i], c, a, mu, rstd, x[i]);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(x[i][j]));
+        for (int j = 0; j < 8; ++j) amax = absmax_nan(amax, x[i][j]);
       }
     }
     int8_t* dst = a.q + r * a.K;
@@ -336,7 +370,19 @@ __global__ void __launch_bounds__(kWarpThreads) k_rows_warp(const RowArgs a) {
       continue;
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    for (int o = 16; o > 0; o >>= 1) amax = absmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const bool safe = !finite_f(amax);  // warp-uniform
+    if (safe) {  // a NaN or an Inf in the row: the range ignores NaN
+      amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < NW; ++i)
+        if (lane + 32 * i < Kc)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(x[i][j]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    }
+    amax = fabsf(amax);
     if (a.range_out) {  // range pass only
       if (lane == 0) range_merge(a, r, amax);
       continue;
@@ -344,11 +390,15 @@ __global__ void __launch_bounds__(kWarpThreads) k_rows_warp(const RowArgs a) {
     const float sc = __fdiv_rn(amax, 127.0f);
     const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
     if (lane == 0) a.scale[r] = sc;
+    auto store = [&](auto safe_t) {
 #pragma unroll
-    for (int i = 0; i < NW; ++i) {
-      const int64_t c = lane + 32 * i;
-      if (c < Kc) *reinterpret_cast<uint2*>(dst + c * 8) = pack8(x[i], inv);
-    }
+      for (int i = 0; i < NW; ++i) {
+        const int64_t c = lane + 32 * i;
+        if (c < Kc) *reinterpret_cast<uint2*>(dst + c * 8) = pack8<decltype(safe_t)::value>(x[i], inv);
+      }
+    };
+    if (safe) store(std::true_type{});
+    else store(std::false_type{});
   }
 }
 
@@ -383,7 +433,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kWarpThreads)
       const int64_t c = lane + 32 * i;
       v[i] = c < Kc ? ld_stream(src + c) : make_uint4(0, 0, 0, 0);
     }
-    Sums s{0, 0, 0};
+    Sums s{0, 0, 0, 0};
 #pragma unroll
     for (int i = 0; i < NW; ++i)
       if (lane + 32 * i < Kc) chunk_sums(v[i], s);
@@ -432,7 +482,9 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kWarpThreads)
 template <int T>
 struct RowSharedT {
   long long s1[2][T / 32], s2h[2][T / 32], s2l[2][T / 32];
+  int bad[2][T / 32];
   float mx[2][T / 32];
+  float mx2[2][T / 32];  // NaN-free row maxima (rows holding a NaN or an Inf)
   float mu[2], rstd[2];
 };
 
@@ -476,7 +528,7 @@ __device__ __forceinline__ void cta_rows(const RowArgs& a, RowSharedT<T>& sh, fl
 
     float mu = 0.0f, rstd = 0.0f;
     if (use_ln) {
-      Sums s{0, 0, 0};
+      Sums s{0, 0, 0, 0};
 #pragma unroll
       for (int i = 0; i < iters; ++i) {
         const int64_t c = tid + static_cast<int64_t>(i) * T;
@@ -487,15 +539,17 @@ __device__ __forceinline__ void cta_rows(const RowArgs& a, RowSharedT<T>& sh, fl
         sh.s1[par][warp] = s.s1;
         sh.s2h[par][warp] = s.s2h;
         sh.s2l[par][warp] = s.s2l;
+        sh.bad[par][warp] = s.bad;
       }
       __syncthreads();
       if (warp == 0) {  // one warp turns the sums into mu / rstd and broadcasts them
-        Sums t{0, 0, 0};
+        Sums t{0, 0, 0, 0};
 #pragma unroll
         for (int w = 0; w < W; ++w) {
           t.s1 += sh.s1[par][w];
           t.s2h += sh.s2h[par][w];
           t.s2l += sh.s2l[par][w];
+          t.bad |= sh.bad[par][w];
         }
         float m_, r_;
         ln_finalize(t, a.K, a.eps, m_, r_);
@@ -520,7 +574,7 @@ __device__ __forceinline__ void cta_rows(const RowArgs& a, RowSharedT<T>& sh, fl
           for (int j = 0; j < 8; ++j) {
             const float ax = fabsf(x[j]);
             if constexpr (CALIB_REG) cmax[i * 8 + j] = fmaxf(cmax[i * 8 + j], ax);
-            else atomicMax(reinterpret_cast<int*>(a.amax) + c * 8 + j, __float_as_int(ax));
+            else atomicMax(reinterpret_cast<int*>(a.amax) + c * 8 + j, __float_as_int(fmaxf(ax, 0.0f)));  // NaN: 0
           }
         }
       }
@@ -548,7 +602,7 @@ __device__ __forceinline__ void cta_rows(const RowArgs& a, RowSharedT<T>& sh, fl
           float x[8];
           transform8<MODE>(chunk(i, c), c, a, mu, rstd, x);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(x[j]));
+          for (int j = 0; j < 8; ++j) amax = absmax_nan(amax, x[j]);
           if constexpr (KEEPX) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) xs[i][j] = x[j];
@@ -556,12 +610,39 @@ __device__ __forceinline__ void cta_rows(const RowArgs& a, RowSharedT<T>& sh, fl
         }
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      for (int o = 16; o > 0; o >>= 1) amax = absmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, o));
       if (lane == 0) sh.mx[par][warp] = amax;
       __syncthreads();
       float m = 0.0f;
 #pragma unroll
-      for (int w = 0; w < W; ++w) m = fmaxf(m, sh.mx[par][w]);
+      for (int w = 0; w < W; ++w) m = absmax_nan(m, sh.mx[par][w]);
+      const bool safe = !finite_f(m);  // CTA-uniform
+      if (safe) {  // a NaN or an Inf in the row: the range ignores NaN
+        float a2 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < iters; ++i) {
+          const int64_t c = tid + static_cast<int64_t>(i) * T;
+          if (c < Kc) {
+            float x[8];
+            if constexpr (KEEPX) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) x[j] = xs[i][j];
+            } else {
+              transform8<MODE>(chunk(i, c), c, a, mu, rstd, x);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) a2 = fmaxf(a2, fabsf(x[j]));
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a2 = fmaxf(a2, __shfl_xor_sync(0xffffffffu, a2, o));
+        if (lane == 0) sh.mx2[par][warp] = a2;
+        __syncthreads();
+        m = 0.0f;
+#pragma unroll
+        for (int w = 0; w < W; ++w) m = fmaxf(m, sh.mx2[par][w]);
+      }
+      m = fabsf(m);
       if (a.range_out) {  // range pass only
         if (tid == 0) range_merge(a, r, m);
       } else {
@@ -569,19 +650,24 @@ __device__ __forceinline__ void cta_rows(const RowArgs& a, RowSharedT<T>& sh, fl
         const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
         if (tid == 0) a.scale[r] = sc;
         int8_t* dst = a.q + r * a.K;
+        auto store = [&](auto safe_t) {
 #pragma unroll
-        for (int i = 0; i < iters; ++i) {
-          const int64_t c = tid + static_cast<int64_t>(i) * T;
-          if (c < Kc) {
-            if constexpr (KEEPX) {
-              *reinterpret_cast<uint2*>(dst + c * 8) = pack8(xs[i], inv);
-            } else {
+          for (int i = 0; i < iters; ++i) {
+            const int64_t c = tid + static_cast<int64_t>(i) * T;
+            if (c < Kc) {
               float x[8];
-              transform8<MODE>(chunk(i, c), c, a, mu, rstd, x);
-              *reinterpret_cast<uint2*>(dst + c * 8) = pack8(x, inv);
+              if constexpr (KEEPX) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) x[j] = xs[i][j];
+              } else {
+                transform8<MODE>(chunk(i, c), c, a, mu, rstd, x);
+              }
+              *reinterpret_cast<uint2*>(dst + c * 8) = pack8<decltype(safe_t)::value>(x, inv);
             }
           }
-        }
+        };
+        if (safe) store(std::true_type{});
+        else store(std::false_type{});
       }
     }
     if (REG && PF) {
@@ -626,7 +712,7 @@ __device__ __forceinline__ void cta_rows_fast(const RowArgs& a, RowSharedT<T>& s
 
     float mu = 0.0f, rstd = 0.0f;
     if (use_ln) {
-      Sums s{0, 0, 0};
+      Sums s{0, 0, 0, 0};
 #pragma unroll
       for (int i = 0; i < NCH; ++i)
         if (tid + static_cast<int64_t>(i) * T < Kc) chunk_sums_f(x[i], s);
@@ -635,15 +721,17 @@ __device__ __forceinline__ void cta_rows_fast(const RowArgs& a, RowSharedT<T>& s
         sh.s1[par][warp] = s.s1;
         sh.s2h[par][warp] = s.s2h;
         sh.s2l[par][warp] = s.s2l;
+        sh.bad[par][warp] = s.bad;
       }
       __syncthreads();
       if (warp == 0) {
-        Sums t{0, 0, 0};
+        Sums t{0, 0, 0, 0};
 #pragma unroll
         for (int w = 0; w < W; ++w) {
           t.s1 += sh.s1[par][w];
           t.s2h += sh.s2h[par][w];
           t.s2l += sh.s2l[par][w];
+          t.bad |= sh.bad[par][w];
         }
         float m_, r_;
         ln_finalize(t, a.K, a.eps, m_, r_);
@@ -667,7 +755,7 @@ __device__ __forceinline__ void cta_rows_fast(const RowArgs& a, RowSharedT<T>& s
           if constexpr (MODE == MODE_CALIB) {
             if constexpr (CALIB_REG) cmax[i * 8 + j] = fmaxf(cmax[i * 8 + j], fabsf(x[i][j]));
           } else {
-            amax = fmaxf(amax, fabsf(x[i][j]));
+            amax = absmax_nan(amax, x[i][j]);
           }
         }
       }
@@ -685,23 +773,44 @@ __device__ __forceinline__ void cta_rows_fast(const RowArgs& a, RowSharedT<T>& s
         }
       } else {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        for (int o = 16; o > 0; o >>= 1) amax = absmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         if (lane == 0) sh.mx[par][warp] = amax;
         __syncthreads();
         float m = 0.0f;
 #pragma unroll
-        for (int w = 0; w < W; ++w) m = fmaxf(m, sh.mx[par][w]);
+        for (int w = 0; w < W; ++w) m = absmax_nan(m, sh.mx[par][w]);
+        const bool safe = !finite_f(m);  // CTA-uniform
+        if (safe) {  // a NaN or an Inf in the row: the range ignores NaN
+          float a2 = 0.0f;
+#pragma unroll
+          for (int i = 0; i < NCH; ++i)
+            if (tid + static_cast<int64_t>(i) * T < Kc)
+#pragma unroll
+              for (int j = 0; j < 8; ++j) a2 = fmaxf(a2, fabsf(x[i][j]));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) a2 = fmaxf(a2, __shfl_xor_sync(0xffffffffu, a2, o));
+          if (lane == 0) sh.mx2[par][warp] = a2;
+          __syncthreads();
+          m = 0.0f;
+#pragma unroll
+          for (int w = 0; w < W; ++w) m = fmaxf(m, sh.mx2[par][w]);
+        }
+        m = fabsf(m);
         if (a.range_out) {  // range pass only
           if (tid == 0) range_merge(a, r, m);
         } else {
           const float sc = __fdiv_rn(m, 127.0f);
           const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
           if (tid == 0) a.scale[r] = sc;
+          auto store = [&](auto safe_t) {
 #pragma unroll
-          for (int i = 0; i < NCH; ++i) {
-            const int64_t c = tid + static_cast<int64_t>(i) * T;
-            if (c < Kc) *reinterpret_cast<uint2*>(dst + c * 8) = pack8(x[i], inv);
-          }
+            for (int i = 0; i < NCH; ++i) {
+              const int64_t c = tid + static_cast<int64_t>(i) * T;
+              if (c < Kc) *reinterpret_cast<uint2*>(dst + c * 8) = pack8<decltype(safe_t)::value>(x[i], inv);
+            }
+          };
+          if (safe) store(std::true_type{});
+          else store(std::false_type{});
         }
       }
     }

@@ -485,6 +485,18 @@ __device__ __forceinline__ uint64_t f2_add_rn(uint64_t a, uint64_t b) {
 
 namespace sq {
 
+// The INT8 code of p for a static scale, in the low byte of the result:
+// clamp to [-127, 127] keeping a NaN (max/min.NaN), round to the nearest
+// integer (ties to even) by adding 1.5 * 2^23, and map a NaN sum (any NaN bit
+// pattern) by an unsigned min onto 1.5 * 2^23 + 256, whose low byte is 0
+// (every in-range sum, 0x4B3FFF81 .. 0x4B40007F, is below it).
+__device__ __forceinline__ uint32_t q8_code_bits(float p) {
+  float c;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(c) : "f"(p), "f"(-127.0f));
+  asm("min.NaN.f32 %0, %0, %1;" : "+f"(c) : "f"(127.0f));
+  return min(__float_as_uint(__fadd_rn(c, 12582912.0f)), 0x4B400100u);
+}
+
 // 3-D tiled load (c2 = batch item), completion counted on a barrier of
 // either CTA of the pair; no multicast.
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
