@@ -204,6 +204,31 @@ def test_splitk_many_contributors_per_tile(sq):
     assert sq.sq_poll_status() == 0
 
 
+@pytest.mark.parametrize("path", ["tiled", "splitk", "pair", "wide"])
+def test_linear_large_accumulators(sq, path):
+    # rows of +-127 codes against +-127 weight rows make |acc| = 127^2 K, far
+    # above 2^22 (beyond exact conversion through 1.5 * 2^23 + acc); the other
+    # rows stay small, so one tile holds both kinds of 32-value chunks
+    M = 16 if path == "splitk" else 300
+    N, K = 520, 8192
+    rng = np.random.default_rng(17)
+    xq = rng.integers(-3, 4, (M, K)).astype(np.int8)
+    wq = rng.integers(-127, 128, (N, K)).astype(np.int8)
+    big = rng.choice(M, M // 3, replace=False)
+    xq[big] = rng.choice([-127, 127], (big.size, 1)).astype(np.int8)
+    wq[::7] = rng.choice([-127, 127], (len(range(0, N, 7)), 1)).astype(np.int8)
+    sx = rng.uniform(1e-7, 1e-6, M).astype(np.float32)
+    sw = rng.uniform(1e-4, 1e-3, N).astype(np.float32)
+    bias = (rng.standard_normal(N) * 0.5).astype(np.float16)
+    acc = oracle.int_gemm(xq, wq)
+    assert (np.abs(acc) >= 2 ** 22).any() and (np.abs(acc) < 2 ** 22).any()
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    sq.sq_w8a8_linear(dev(xq), dev(sx), dev(wq), dev(sw), y, dev(bias), workspace=sq.new_workspace(M, N, K),
+                      path=_PATHS[path](sq))
+    assert bits_equal(host(y), oracle.dequant(acc, sx, sw, bias))
+    assert sq.sq_poll_status() == 0
+
+
 def test_extreme_codes_do_not_wrap(sq):
     K = 133136  # the largest multiple of 16 <= 133144
     xq = np.full((2, K), 127, np.int8)
