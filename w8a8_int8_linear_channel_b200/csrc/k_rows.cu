@@ -5,12 +5,19 @@
 //     diag(s) on the fly (section "what it does mathematically");
 //   * calibration absmax of the LayerNorm output (glossary "Calibration").
 //
-// Two shapes of the same computation:
-//   * K <= 4096: one warp per row (no block barrier at all; many rows in
+// Shapes of the same computation (chosen by K):
+//   * K <= 1024: one warp per row (no block barrier at all; many rows in
 //     flight per SM).  The row and its transformed values live in registers.
-//   * larger K: one CTA of 256 threads per row, warp shuffles plus one
-//     shared-memory step per reduction.
-// Rows are read once from HBM with 16-byte loads.
+//   * K <= 16384: one CTA of 64 to 256 threads per row, up to 8 16-byte
+//     chunks per thread held in registers (converted to fp32 once), the
+//     CTA's next row prefetched; warp shuffles plus one shared-memory step
+//     per reduction.
+//   * larger K: the same CTA shape with 12 or 24 chunks per thread in
+//     registers, or (K > 49152) the row re-read from global in every pass.
+// Rows are read once from HBM with 16-byte loads (except the last shape).
+// A row maximum is taken NaN-propagating; a row whose maximum is not finite
+// (it holds a NaN or an Inf) recomputes its NaN-free maximum and quantizes
+// through the NaN-safe path.
 //
 // LayerNorm statistics are exact and order-independent: every fp16 value h
 // equals v * 2^-24 for an integer v (|v| < 2^40).  Per 8-element chunk the
