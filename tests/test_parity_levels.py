@@ -156,3 +156,25 @@ def test_o2_full_size_attention_batch(sq):
     assert bits_equal(host(r), np.float32(r_ref).reshape(1))
     assert bits_equal(host(sx), s_ref)
     assert bits_equal(host(xq), q_ref)
+
+
+def test_layer_batch_shapes(sq):
+    """Leading dimensions are flattened into tokens (same bits as the 2-D call);
+    an empty batch returns an empty output and launches nothing."""
+    wl = sq_inputs.WORKLOADS["tiny_ln"]
+    w, calib = sq_inputs.weight(wl), sq_inputs.calib_rows(wl)
+    g, b, bias = sq_inputs.gamma(wl), sq_inputs.beta(wl), sq_inputs.bias(wl)
+    layer = sq.SmoothQuantLinear.from_float(dev(w), dev(calib), alpha=wl.alpha, gamma=dev(g), beta=dev(b),
+                                            bias=dev(bias))
+    h = sq_inputs.run_rows(wl, 0, 12)
+    y2 = host(layer(dev(h)))
+    y3 = layer(dev(h).view(3, 4, wl.K))
+    assert tuple(y3.shape) == (3, 4, wl.N) and bits_equal(host(y3).reshape(12, wl.N), y2)
+    out = torch.empty((3, 4, wl.N), dtype=torch.float16, device="cuda")
+    assert layer(dev(h).view(3, 4, wl.K), out) is out and bits_equal(host(out).reshape(12, wl.N), y2)
+    for shape in [(0, wl.K), (2, 0, wl.K)]:
+        e = layer(torch.empty(shape, dtype=torch.float16, device="cuda"))
+        assert tuple(e.shape) == shape[:-1] + (wl.N,)
+    with pytest.raises(ValueError):
+        layer(dev(h)[:, :16])
+    assert sq.sq_poll_status() == 0

@@ -508,12 +508,22 @@ class SmoothQuantLinear:
         return xq, x_scale
 
     def forward(self, h: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
-        """h fp16 [M, K] (the LayerNorm input if a LayerNorm was folded) -> y fp16 [M, N]."""
-        M = h.shape[0]
-        N = self.wq.shape[0]
-        xq, x_scale = self.quantize_input(h)
-        y = torch.empty((M, N), dtype=torch.float16, device=h.device) if y is None else y
-        sq_w8a8_linear(xq, x_scale, self.wq, self.w_scale, y, self.bias, self.workspace(M))
+        """h fp16 [..., K] (the LayerNorm input if a LayerNorm was folded) -> y fp16 [..., N].
+        Leading dimensions are flattened into tokens; an empty batch launches nothing."""
+        N, K = self.wq.shape
+        if h.dim() < 1 or h.shape[-1] != K:
+            raise ValueError(f"h: need [..., {K}], got {tuple(h.shape)}")
+        lead = tuple(h.shape[:-1])
+        h2 = h if h.dim() == 2 else h.reshape(-1, K)
+        M = h2.shape[0]
+        if y is None:
+            y = torch.empty(lead + (N,), dtype=torch.float16, device=h.device)
+        elif tuple(y.shape) not in (lead + (N,), (M, N)) or not y.is_contiguous():
+            raise ValueError(f"y: need a contiguous fp16 {lead + (N,)} tensor")
+        if M == 0:
+            return y
+        xq, x_scale = self.quantize_input(h2)
+        sq_w8a8_linear(xq, x_scale, self.wq, self.w_scale, y.view(M, N), self.bias, self.workspace(M))
         return y
 
     __call__ = forward
