@@ -102,11 +102,14 @@ __device__ __forceinline__ bool pair_wait(uint32_t bar, uint32_t parity, bool cl
   }
 }
 
-template <int EPI>
+// TMAS: fp16 blocks leave through TMA stores (rows 16-byte aligned); without
+// it they go through the warp's staging, row by row (a separate
+// instantiation, so the TMA-store kernel keeps its own registers).
+template <int EPI, bool TMAS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, const GemmArgs g, int tiles_m, int tiles,
-                int tma_store, uint32_t* status, uint64_t budget) {
+                uint32_t* status, uint64_t budget) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -243,7 +246,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t stg0 = sbase + STG + static_cast<uint32_t>(warp - 2) * STG_WARP;
     const uint32_t acce_leader0 = mapa_shared(acce_bar(0), 0);
     int nst = 0;  // blocks this warp has staged (selects the buffer; two stores may be in flight)
-    const bool vec_ok = (g.N % 8) == 0;
     // producer-side quantization: the next linear's 1/s of this tile's columns
     // (in the output staging area, unused in that mode) and its static scale
     float* inv_s_s = reinterpret_cast<float*>(smem + STG);
@@ -314,12 +316,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       auto emit = [&](int c, uint32_t (&v)[32]) {
         const int cl = 128 * half + 32 * c;  // column within the tile
         const int64_t col0 = n0 + cl;
+        // rows / columns of this warp's 32 x 32 block inside the output (warp-uniform)
+        const int brows = g.M - row0 < 32 ? static_cast<int>(g.M - row0) : 32;
+        const int bcols = g.N - col0 < 32 ? static_cast<int>(g.N - col0) : 32;
         if constexpr (EPI == EPI_I32) {
-          if (row < g.M && col0 < g.N) {
-            int32_t* dst = g.acc + row * g.N + col0;
-            for (int j = 0; j < 32; ++j)
-              if (col0 + j < g.N) dst[j] = static_cast<int32_t>(v[j]);
-          }
+          if (brows > 0 && bcols > 0)  // through the warp's 4 KB staging, row by row
+            warp_store_rows_i32(stg0, v, g.acc + row0 * g.N + col0, g.N, brows, bcols);
           return;
         } else if constexpr (EPI == EPI_Q8) {
           // the composition, per element: y = fp16((acc * sx) * sw + bias),
@@ -422,7 +424,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               *reinterpret_cast<__half2*>(&h[j + 2 * u]) = __floats2half2_rn(f.x, f.y);
             }
           }
-          if (tma_store) {
+          if constexpr (TMAS) {
             // stage the 32 x 32 block in the 64-byte-swizzled image; one TMA
             // store writes it (rows/columns outside y are skipped); two buffers
             // per warp, so the previous block's store may still be reading one
@@ -449,16 +451,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               }
               bulk_commit_group();
             }
-          } else if (row < g.M && col0 < g.N) {
-            __half* dst = g.y + (static_cast<int64_t>(bi) * g.M + row) * g.N + col0;
-            if (vec_ok && col0 + 32 <= g.N) {
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                reinterpret_cast<uint4*>(dst)[j] = reinterpret_cast<const uint4*>(h)[j];
-            } else {
-              for (int j = 0; j < 32; ++j)
-                if (col0 + j < g.N) dst[j] = h[j];
-            }
+          } else if (brows > 0 && bcols > 0) {
+            // rows not 16-byte aligned (N % 8 != 0): through the staging, row by row
+            warp_store_rows_f16(stg0, h, g.y + (static_cast<int64_t>(bi) * g.M + row0) * g.N + col0, g.N, brows,
+                                bcols);
           }
         }
       };
@@ -534,7 +530,7 @@ int max_pairs(int device, int num_sms) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = SMEM;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<EPI_F16>, &cfg) != cudaSuccess || n <= 0) {
+  if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<EPI_F16, true>, &cfg) != cudaSuccess || n <= 0) {
     (void)cudaGetLastError();
     n = num_sms / 2;
   }
@@ -543,16 +539,21 @@ int max_pairs(int device, int num_sms) {
   return n;
 }
 
-template <int EPI>
-cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
-  static bool attr_set[4][64] = {};
-  const int dev = c.device < 64 ? c.device : 63;
-  if (!attr_set[EPI][dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_pair<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <int EPI, bool TMAS>
+cudaError_t smem_attr(int device) {
+  static bool attr_set[64] = {};
+  const int dev = device < 64 ? device : 63;
+  if (!attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_pair<EPI, TMAS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM));
     if (e != cudaSuccess) return e;
-    attr_set[EPI][dev] = true;
+    attr_set[dev] = true;
   }
+  return cudaSuccess;
+}
+
+template <int EPI>
+cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
   CUtensorMap tmA, tmB, tmY;
   const bool bmm = EPI == EPI_BMM;
   const uint64_t items = bmm ? static_cast<uint64_t>(g.batch) : 1;
@@ -564,8 +565,9 @@ cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
     if (!make_tmap_i8(&tmB, g.wq, g.K, g.N, BK, BNH)) return cudaErrorInvalidValue;
   }
   // TMA stores of fp16 y need 16-byte row strides (N % 8 == 0); otherwise
-  // direct stores (always for int32 accumulators and int8 codes)
-  int tma_store = ((EPI == EPI_F16 || bmm) && g.N % 8 == 0) ? 1 : 0;
+  // row-by-row stores through the staging (always for int32 accumulators;
+  // int8 codes are written 32 bytes per row)
+  const bool tma_store = (EPI == EPI_F16 || bmm) && g.N % 8 == 0;
   if (tma_store) {
     const bool ok = bmm ? make_tmap_f16_out_3d(&tmY, g.y, g.N, g.M, items) : make_tmap_f16_out(&tmY, g.y, g.N, g.M);
     if (!ok) return cudaErrorInvalidValue;
@@ -579,8 +581,18 @@ cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
   const int tiles = static_cast<int>(tiles64);
   const int mp = max_pairs(c.device, c.num_sms);
   const int pairs = tiles < mp ? tiles : mp;
-  return launch_pdl(k_gemm_pair<EPI>, dim3(2 * pairs), dim3(kThreads), SMEM, c.stream, tmA, tmB, tmY, g,
-                    tiles_m, tiles, tma_store, c.status, c.budget_ns);
+  if (tma_store) {
+    if constexpr (EPI == EPI_F16 || EPI == EPI_BMM) {
+      cudaError_t e = smem_attr<EPI, true>(c.device);
+      if (e != cudaSuccess) return e;
+      return launch_pdl(k_gemm_pair<EPI, true>, dim3(2 * pairs), dim3(kThreads), SMEM, c.stream, tmA, tmB, tmY, g,
+                        tiles_m, tiles, c.status, c.budget_ns);
+    }
+  }
+  cudaError_t e = smem_attr<EPI, false>(c.device);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_gemm_pair<EPI, false>, dim3(2 * pairs), dim3(kThreads), SMEM, c.stream, tmA, tmB, tmY, g,
+                    tiles_m, tiles, c.status, c.budget_ns);
 }
 
 }  // namespace

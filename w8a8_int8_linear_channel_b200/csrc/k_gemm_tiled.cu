@@ -26,7 +26,7 @@ constexpr int BM = 128;  // token rows per tile (TMEM lanes)
 constexpr int BK = 128;  // K bytes per stage = one 128-byte swizzle row
 constexpr int kThreads = 192;
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool ROWS>
 struct TiledLayout {
   static constexpr int A_BYTES = BM * BK;
   static constexpr int B_BYTES = BN * BK;
@@ -35,15 +35,20 @@ struct TiledLayout {
   static constexpr int NBARS = 2 * STAGES + 2;           // full, empty, acc_full, drain
   static constexpr int SLOT = CTRL + NBARS * 8;          // TMEM address, abort flag
   static constexpr int VEC = SLOT + 16;                  // sw[BN], bias[BN]
-  static constexpr int BYTES = VEC + 2 * BN * 4;
+  static constexpr int STG = VEC + 2 * BN * 4;           // 4 KB output staging per epilogue warp (ROWS)
+  static constexpr int BYTES = STG + (ROWS ? 4 * 4096 : 0);
   static constexpr size_t SMEM = BYTES + 1024;           // slack for 1024-byte alignment
+  static_assert(STG % 16 == 0 && SMEM <= 232448, "staging alignment, shared memory per CTA");
 };
 
-template <int BN, int STAGES, bool OUT_I32>
+// ROWS: the output blocks go through the warp's staging, row by row (int32,
+// or fp16 rows that are not 16-byte aligned); otherwise each lane stores its
+// fp16 row as 16-byte vectors.
+template <int BN, int STAGES, bool OUT_I32, bool ROWS>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_tiled(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const GemmArgs g, uint32_t* status, uint64_t budget) {
-  using L = TiledLayout<BN, STAGES>;
+  using L = TiledLayout<BN, STAGES, ROWS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -142,34 +147,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t row = m0 + 32 * q + lane;
       const bool row_ok = row < g.M;
       const float sxr = (!OUT_I32 && row_ok) ? g.sx[row] : 0.0f;
-      const bool vec_ok = (g.N % 8) == 0;
+      // this warp's 32 x 32 blocks go out through its 4 KB staging, row by
+      // row (coalesced row segments instead of one row per lane)
+      const uint32_t stg = sbase + L::STG + static_cast<uint32_t>(warp - 2) * 4096u;
+      const int64_t row0 = m0 + 32 * q;
+      const int brows = g.M - row0 < 32 ? static_cast<int>(g.M - row0) : 32;  // warp-uniform
 #pragma unroll 1
       for (int cc = 0; cc < BN / 32; ++cc) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 32u * cc, v);
         tmem_ld_wait();
         const int64_t col0 = n0 + 32 * cc;
-        if (!row_ok || col0 >= g.N) continue;
-        if (OUT_I32) {
-          int32_t* dst = g.acc + row * g.N + col0;
-          for (int j = 0; j < 32; ++j)
-            if (col0 + j < g.N) dst[j] = static_cast<int32_t>(v[j]);
+        if (brows <= 0 || col0 >= g.N) continue;  // warp-uniform
+        const int bcols = g.N - col0 < 32 ? static_cast<int>(g.N - col0) : 32;
+        if constexpr (OUT_I32) {
+          warp_store_rows_i32(stg, v, g.acc + row0 * g.N + col0, g.N, brows, bcols);
         } else {
-          __half h[32];
+          __align__(16) __half h[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             float f = dequant_f32(static_cast<int32_t>(v[j]), sxr, sw_s[32 * cc + j]);
             if (g.bias != nullptr) f = __fadd_rn(f, bias_s[32 * cc + j]);
             h[j] = __float2half_rn(f);
           }
-          __half* dst = g.y + row * g.N + col0;
-          if (vec_ok && col0 + 32 <= g.N) {
+          if constexpr (ROWS) {
+            warp_store_rows_f16(stg, h, g.y + row0 * g.N + col0, g.N, brows, bcols);
+          } else if (lane < brows) {
+            __half* dst = g.y + (row0 + lane) * g.N + col0;
+            if (bcols == 32) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              reinterpret_cast<uint4*>(dst)[j] = reinterpret_cast<const uint4*>(h)[j];
-          } else {
-            for (int j = 0; j < 32; ++j)
-              if (col0 + j < g.N) dst[j] = h[j];
+              for (int j = 0; j < 4; ++j)
+                reinterpret_cast<uint4*>(dst)[j] = reinterpret_cast<const uint4*>(h)[j];
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < bcols) dst[j] = h[j];
+            }
           }
         }
       }
@@ -199,13 +212,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BN, int STAGES, bool OUT_I32>
+template <int BN, int STAGES, bool OUT_I32, bool ROWS>
 cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
-  using L = TiledLayout<BN, STAGES>;
+  using L = TiledLayout<BN, STAGES, ROWS>;
   static bool attr_set[64] = {false};
   const int dev = c.device < 64 ? c.device : 63;
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tiled<BN, STAGES, OUT_I32>,
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tiled<BN, STAGES, OUT_I32, ROWS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(L::SMEM));
     if (e != cudaSuccess) return e;
@@ -215,15 +228,16 @@ cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
   if (!make_tmap_i8(&tmA, g.xq, g.K, g.M, BK, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_i8(&tmB, g.wq, g.K, g.N, BK, BN)) return cudaErrorInvalidValue;
   dim3 grid(static_cast<unsigned>((g.N + BN - 1) / BN), static_cast<unsigned>((g.M + BM - 1) / BM));
-  return launch_pdl(k_gemm_tiled<BN, STAGES, OUT_I32>, grid, dim3(kThreads), L::SMEM, c.stream, tmA, tmB, g,
+  return launch_pdl(k_gemm_tiled<BN, STAGES, OUT_I32, ROWS>, grid, dim3(kThreads), L::SMEM, c.stream, tmA, tmB, g,
                     c.status, c.budget_ns);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_tiled(const GemmArgs& g, const Ctx& c) {
-  if (g.acc != nullptr) return launch_cfg<256, 4, true>(g, c);
-  return launch_cfg<256, 4, false>(g, c);
+  if (g.acc != nullptr) return launch_cfg<256, 4, true, true>(g, c);
+  if (g.N % 8 != 0) return launch_cfg<256, 4, false, true>(g, c);  // fp16 rows not 16-byte aligned
+  return launch_cfg<256, 4, false, false>(g, c);
 }
 
 }  // namespace sq

@@ -47,11 +47,14 @@ constexpr int SMEM_BYTES = VEC + BN * 4 + BN * 2;
 constexpr size_t SMEM = SMEM_BYTES + 1024;    // slack for 1024-byte alignment
 constexpr uint32_t TMEM_COLS = 512;
 
-template <bool OUT_I32>
+// TMAS: fp16 blocks leave through TMA stores (rows 16-byte aligned); without
+// it (and for int32) through the warp's staging, row by row -- a separate
+// instantiation, so the TMA-store kernel keeps its own registers.
+template <bool OUT_I32, bool TMAS>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_wide(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, const GemmArgs g, int tiles_m, int tiles,
-                int tma_store, uint32_t* status, uint64_t budget) {
+                uint32_t* status, uint64_t budget) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -161,7 +164,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = (warp - 2) >> 2;  // column half of the tile
     const uint32_t stg0 = sbase + STG + static_cast<uint32_t>(warp - 2) * STG_WARP;
     int nst = 0;  // blocks this warp has staged (selects the buffer; two stores may be in flight)
-    const bool vec_ok = (g.N % 8) == 0;
     int tl = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tl) {
       const int64_t m0 = static_cast<int64_t>(t % tiles_m) * BM;
@@ -198,14 +200,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int a = idx >> 2;
         const int cl = 128 * half + 32 * (idx & 3);  // column within the tile
         const int64_t row0 = m0 + 128 * a + 32 * q;  // first row of this warp's block
-        const int64_t row = row0 + lane;
         const int64_t col0 = n0 + cl;
+        // rows / columns of this warp's 32 x 32 block inside the output (warp-uniform)
+        const int brows = g.M - row0 < 32 ? static_cast<int>(g.M - row0) : 32;
+        const int bcols = g.N - col0 < 32 ? static_cast<int>(g.N - col0) : 32;
         if constexpr (OUT_I32) {
-          if (row < g.M && col0 < g.N) {
-            int32_t* dst = g.acc + row * g.N + col0;
-            for (int j = 0; j < 32; ++j)
-              if (col0 + j < g.N) dst[j] = static_cast<int32_t>(v[j]);
-          }
+          if (brows > 0 && bcols > 0)  // through the warp's 4 KB staging, row by row
+            warp_store_rows_i32(stg0, v, g.acc + row0 * g.N + col0, g.N, brows, bcols);
           return;
         } else {
         __align__(16) __half h[32];
@@ -221,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // both lanes of the pair rounded to nearest even in one instruction
           *reinterpret_cast<__half2*>(&h[j]) = __floats2half2_rn(f0, f1);
         }
-        if (tma_store) {
+        if constexpr (TMAS) {
           // stage the 32 x 32 block in the 64-byte-swizzled image and let one
           // TMA store write it (rows/columns outside y are skipped by the TMA);
           // two buffers per warp, so the store of the previous block may still
@@ -245,16 +246,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_store_2d(&tmY, stg, static_cast<int32_t>(col0), static_cast<int32_t>(row0));
             bulk_commit_group();  // one group per staged block, empty if nothing was stored
           }
-        } else if (row < g.M && col0 < g.N) {
-          __half* dst = g.y + row * g.N + col0;
-          if (vec_ok && col0 + 32 <= g.N) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              reinterpret_cast<uint4*>(dst)[j] = reinterpret_cast<const uint4*>(h)[j];
-          } else {
-            for (int j = 0; j < 32; ++j)
-              if (col0 + j < g.N) dst[j] = h[j];
-          }
+        } else if (brows > 0 && bcols > 0) {
+          // rows not 16-byte aligned (N % 8 != 0): through the staging, row by row
+          warp_store_rows_f16(stg0, h, g.y + row0 * g.N + col0, g.N, brows, bcols);
         }
         }
       };
@@ -301,29 +295,39 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool OUT_I32>
-cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
+template <bool OUT_I32, bool TMAS>
+cudaError_t launch_kernel(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY,
+                          const GemmArgs& g, int tiles_m, int tiles, const Ctx& c) {
   static bool attr_set[64] = {false};
   const int dev = c.device < 64 ? c.device : 63;
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_wide<OUT_I32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_wide<OUT_I32, TMAS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM));
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
+  const int grid = tiles < c.num_sms ? tiles : c.num_sms;
+  return launch_pdl(k_gemm_wide<OUT_I32, TMAS>, dim3(grid), dim3(kThreads), SMEM, c.stream, tmA, tmB, tmY, g,
+                    tiles_m, tiles, c.status, c.budget_ns);
+}
+
+template <bool OUT_I32>
+cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
   CUtensorMap tmA, tmB, tmY;
   if (!make_tmap_i8(&tmA, g.xq, g.K, g.M, BK, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_i8(&tmB, g.wq, g.K, g.N, BK, BN)) return cudaErrorInvalidValue;
-  // TMA stores need 16-byte row strides (N % 8 == 0); otherwise direct stores
-  int tma_store = (!OUT_I32 && g.N % 8 == 0) ? 1 : 0;
+  // TMA stores need 16-byte row strides (N % 8 == 0); otherwise row-by-row
+  // stores through the staging
+  const bool tma_store = !OUT_I32 && g.N % 8 == 0;
   if (tma_store && !make_tmap_f16_out(&tmY, g.y, g.N, g.M)) return cudaErrorInvalidValue;
   if (!tma_store) memset(&tmY, 0, sizeof(tmY));
   const int tiles_m = static_cast<int>((g.M + BM - 1) / BM);
   const int tiles_n = static_cast<int>((g.N + BN - 1) / BN);
   const int tiles = tiles_m * tiles_n;
-  const int grid = tiles < c.num_sms ? tiles : c.num_sms;
-  return launch_pdl(k_gemm_wide<OUT_I32>, dim3(grid), dim3(kThreads), SMEM, c.stream, tmA, tmB, tmY, g,
-                    tiles_m, tiles, tma_store, c.status, c.budget_ns);
+  if (tma_store) {
+    if constexpr (!OUT_I32) return launch_kernel<false, true>(tmA, tmB, tmY, g, tiles_m, tiles, c);
+  }
+  return launch_kernel<OUT_I32, false>(tmA, tmB, tmY, g, tiles_m, tiles, c);
 }
 
 }  // namespace

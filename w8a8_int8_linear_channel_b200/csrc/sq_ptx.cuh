@@ -485,6 +485,76 @@ __device__ __forceinline__ uint64_t f2_add_rn(uint64_t a, uint64_t b) {
 
 namespace sq {
 
+// Coalesced output of a warp's 32 x 32 block when no tensor-map store fits
+// (rows not 16-byte aligned, or int32 accumulators): lane l holds row l's 32
+// values.  Each lane writes its row into the warp's shared staging area in
+// 16-byte pieces, XOR-swizzled so the eight lanes of a phase hit distinct
+// banks; then the warp writes the block back row by row, so every store
+// instruction covers one contiguous segment of a row (instead of 32 rows).
+// dst0 points at element (row0, col0) of the row-major output with row pitch
+// ld; rows / cols (<= 32) are how many of the block's rows / columns exist.
+// Warp-collective: all 32 lanes call it; staging is reusable on return.
+
+// fp16: 2 KB staging (32 rows x 64 bytes).
+__device__ __forceinline__ void warp_store_rows_f16(uint32_t stg, const __half (&h)[32], __half* dst0, int64_t ld,
+                                                    int rows, int cols) {
+  const int lane = threadIdx.x & 31;
+  const uint4* hv = reinterpret_cast<const uint4*>(h);
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const uint32_t addr = stg + lane * 64 + ((cc ^ ((lane >> 1) & 3)) * 16);
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(hv[cc].x), "r"(hv[cc].y),
+                 "r"(hv[cc].z), "r"(hv[cc].w)
+                 : "memory");
+  }
+  __syncwarp();
+  if ((ld & 1) == 0) {
+    // even pitch (so cols is even too): two columns per lane, two rows per store
+    const int jc = 2 * (lane & 15);
+    const uint32_t off = ((jc >> 3) * 16) + (jc & 7) * 2;
+    for (int r = lane >> 4; r < rows; r += 2) {
+      if (jc < cols) {
+        uint32_t w;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(stg + r * 64 + (off ^ ((((r >> 1) & 3)) * 16))));
+        *reinterpret_cast<uint32_t*>(dst0 + r * ld + jc) = w;
+      }
+    }
+  } else {
+    const uint32_t off = ((lane >> 3) * 16) + (lane & 7) * 2;
+    for (int r = 0; r < rows; ++r) {
+      if (lane < cols) {
+        unsigned short w;
+        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(w) : "r"(stg + r * 64 + (off ^ ((((r >> 1) & 3)) * 16))));
+        dst0[r * ld + lane] = __ushort_as_half(w);
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// int32: 4 KB staging (32 rows x 128 bytes).
+__device__ __forceinline__ void warp_store_rows_i32(uint32_t stg, const uint32_t (&v)[32], int32_t* dst0,
+                                                    int64_t ld, int rows, int cols) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int cc = 0; cc < 8; ++cc) {
+    const uint32_t addr = stg + lane * 128 + ((cc ^ (lane & 7)) * 16);
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[4 * cc]), "r"(v[4 * cc + 1]),
+                 "r"(v[4 * cc + 2]), "r"(v[4 * cc + 3])
+                 : "memory");
+  }
+  __syncwarp();
+  const uint32_t off = ((lane >> 2) * 16) + (lane & 3) * 4;
+  for (int r = 0; r < rows; ++r) {
+    if (lane < cols) {
+      uint32_t w;
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(stg + r * 128 + (off ^ ((r & 7) * 16))));
+      dst0[r * ld + lane] = static_cast<int32_t>(w);
+    }
+  }
+  __syncwarp();
+}
+
 // The INT8 code of p for a static scale, in the low byte of the result:
 // clamp to [-127, 127] keeping a NaN (max/min.NaN), round to the nearest
 // integer (ties to even) by adding 1.5 * 2^23, and map a NaN sum (any NaN bit
