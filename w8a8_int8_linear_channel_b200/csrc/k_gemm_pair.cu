@@ -312,7 +312,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                static_cast<uint32_t>(BN * b + 128 * half + 32 * c);
       };
       const int64_t row0 = m0 + 32 * q;  // first row of this warp's blocks
-      const int64_t row = row0 + lane;
       auto emit = [&](int c, uint32_t (&v)[32]) {
         const int cl = 128 * half + 32 * c;  // column within the tile
         const int64_t col0 = n0 + cl;
@@ -374,8 +373,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               qw[j / 4] = __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
             }
           }
-          if (row < g.M && col0 < g.N) {
-            int8_t* dst = g.q_next + row * g.N + col0;
+          if (row0 + lane < g.M && col0 < g.N) {
+            // each lane writes its row's 32 codes, one full 32-byte sector
+            int8_t* dst = g.q_next + (row0 + lane) * g.N + col0;
             if ((g.N % 16) == 0 && col0 + 32 <= g.N) {
               reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<const uint4*>(qw)[0];
               reinterpret_cast<uint4*>(dst)[1] = reinterpret_cast<const uint4*>(qw)[1];
