@@ -261,12 +261,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t nl = 32 * q + lane;  // channel within the tile
       const int64_t n = t * BW + nl;
       bool emit = whole;
+      // a partial slot holds BW x BT int32 as BT/4 groups of [channel][4 tokens]:
+      // a warp's 16-byte stores and loads of one group cover 512 contiguous bytes
+      auto part = [&](int64_t sl, int j) { return partials + (sl * BT + j) * BW + nl * 4; };
       if (!whole) {
-        int32_t* mine = partials + (static_cast<int64_t>(2 * cta + slot) * BW + nl) * BT;
 #pragma unroll
         for (int j = 0; j < BT; j += 4)
-          *reinterpret_cast<int4*>(mine + j) = make_int4(static_cast<int>(v[j]), static_cast<int>(v[j + 1]),
-                                                         static_cast<int>(v[j + 2]), static_cast<int>(v[j + 3]));
+          *reinterpret_cast<int4*>(part(2 * cta + slot, j)) =
+              make_int4(static_cast<int>(v[j]), static_cast<int>(v[j + 1]), static_cast<int>(v[j + 2]),
+                        static_cast<int>(v[j + 3]));
         __threadfence();
         named_bar_sync(1, 128);
         const int c_lo = geo.cta_of(t * KB);
@@ -285,10 +288,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (cc == cta) continue;
             const int first_tile = static_cast<int>(geo.u0(cc) / KB);
             const int sl = (t == first_tile) ? 0 : 1;
-            const int32_t* other = partials + (static_cast<int64_t>(2 * cc + sl) * BW + nl) * BT;
 #pragma unroll
             for (int j = 0; j < BT; j += 4) {
-              const int4 p = __ldcg(reinterpret_cast<const int4*>(other + j));
+              const int4 p = __ldcg(reinterpret_cast<const int4*>(part(2 * cc + sl, j)));
               v[j] += p.x;
               v[j + 1] += p.y;
               v[j + 2] += p.z;
@@ -369,7 +371,13 @@ SkGeom make_geom(int64_t N, int64_t K, int64_t grid_cap) {
   geo.KB = static_cast<int>(((K + BK - 1) / BK + KPS - 1) / KPS);
   const int64_t T = tiles_of(N);
   const int64_t total = T * geo.KB;
-  const int64_t grid = total < grid_cap ? total : grid_cap;
+  // at least half a tile of K per CTA, so a split tile has at most three
+  // contributors and its last arrival adds at most two partials (on small
+  // layers fewer CTAs then stream the weight; each still keeps a deep ring)
+  const int64_t min_units = (geo.KB + 1) / 2;
+  const int64_t by_units = (total + min_units - 1) / min_units;
+  int64_t grid = total < grid_cap ? total : grid_cap;
+  if (grid > by_units) grid = by_units;
   geo.grid = static_cast<int>(grid);
   geo.Wt = static_cast<int>(T / grid);
   geo.R = static_cast<int>(T - static_cast<int64_t>(geo.Wt) * grid);
