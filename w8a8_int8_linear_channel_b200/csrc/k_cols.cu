@@ -90,17 +90,22 @@ __global__ void k_smooth(const float* __restrict__ amax_x, const float* __restri
   const bool odd = (t & 1) != 0;
   const bool valid = j < K;
   const float av = valid ? (odd ? amax_w[j] : amax_x[j]) : 1.0f;
+  // gamma / beta do not depend on the powers: load them now, so their
+  // latency overlaps the fp64 work instead of following it
+  const bool even_ok = valid && !odd;
+  const float gj = (even_ok && gamma) ? gamma[j] : 0.0f;
+  const float bj = (even_ok && beta) ? beta[j] : 0.0f;
   const double base = av > 1e-5f ? static_cast<double>(av) : static_cast<double>(1e-5f);
   const double a = static_cast<double>(alpha);
   const double p = pow(base, odd ? __dsub_rn(1.0, a) : a);
   const double den = __shfl_down_sync(0xffffffffu, p, 1);
-  if (!valid || odd) return;
+  if (!even_ok) return;
   const float s32 = __double2float_rn(__ddiv_rn(p, den));
   const float inv = __frcp_rn(s32);
   s[j] = s32;
   inv_s[j] = inv;
-  if (gamma) gamma_out[j] = __fmul_rn(gamma[j], inv);
-  if (beta) beta_out[j] = __fmul_rn(beta[j], inv);
+  if (gamma) gamma_out[j] = __fmul_rn(gj, inv);
+  if (beta) beta_out[j] = __fmul_rn(bj, inv);
 }
 
 // w_out[n, j] = fp16(fp32(w[n, j]) * s_j), one 8-element chunk per thread and
