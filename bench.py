@@ -302,9 +302,9 @@ class Plan:
         self.side.wait_stream(main)                    # amax zeroed, previous step done
         for name, fn, args in self.calls:
             if name == "smooth_fold":                  # needs both ranges
-                main.wait_stream(self.side)
-                if allreduce is not None:
+                if allreduce is not None:              # on main after calibrate_x: overlaps calibrate_w
                     allreduce(self.amax_x)
+                main.wait_stream(self.side)
             if name == "quantize_weight":              # needs s
                 self.side.wait_stream(main)
             if name == "w8a8_linear":                  # needs wq and xq
