@@ -271,7 +271,7 @@ class Plan:
                                (name == "ln_quant_act" and act == "tensor") else 1)
                         for name, _, _ in calls}
 
-    def step(self, events=None, allreduce=None):
+    def step(self, events=None, allreduce=None, part=None):
         """Run one step.  With two streams the independent stages overlap:
             main: calibrate_x            | smooth_fold | ln_quant_act    | w8a8_linear
             side:          calibrate_w   |             | quantize_weight |
@@ -279,7 +279,8 @@ class Plan:
         With `events` (one per call + 1), the stages instead run one after the
         other on the main stream timing order (for the per-stage breakdown)."""
         torch = self.torch
-        self.amax.zero_()
+        if part != "rest":  # the rest of a step keeps the calibrated, all-reduced ranges
+            self.amax.zero_()
         if events is not None:  # serialized, one event before each call
             for i, (name, fn, args) in enumerate(self.calls):
                 events[i].record(self.main)
@@ -299,9 +300,13 @@ class Plan:
                 self._call(name, fn, args)
             return
         main = self.cur
-        self.side.wait_stream(main)                    # amax zeroed, previous step done
-        for name, fn, args in self.calls:
-            if name == "smooth_fold":                  # needs both ranges
+        calls = self.calls
+        if part == "rest":  # smooth_fold onwards (the ranges are complete and all-reduced)
+            calls = calls[[c[0] for c in calls].index("smooth_fold"):]
+        else:
+            self.side.wait_stream(main)                # amax zeroed, previous step done
+        for name, fn, args in calls:
+            if name == "smooth_fold" and part != "rest":  # needs both ranges
                 if allreduce is not None:              # on main after calibrate_x: overlaps calibrate_w
                     allreduce(self.amax_x)
                 main.wait_stream(self.side)
@@ -313,8 +318,11 @@ class Plan:
 
     def capture(self, world):
         """Capture the step into CUDA graphs: one graph for N = 1; for N > 1 two
-        graphs around the NCCL all-reduce, which runs eagerly between them."""
+        graphs around the NCCL all-reduce, which runs eagerly between them (with
+        two streams, three: see capture_split)."""
         torch = self.torch
+        if self.two_streams and world > 1:
+            return self.capture_split()
         cap = torch.cuda.Stream()
         cap.wait_stream(self.main)
         names = [c[0] for c in self.calls]
@@ -396,7 +404,47 @@ class Plan:
         self.main.wait_stream(cap)
         return gr
 
+    def capture_split(self):
+        """N > 1 with two streams: [zero the ranges, calibrate_x] and
+        [smooth_fold .. w8a8_linear] (which forks the side stream for the weight
+        quantization) captured for the main stream, [calibrate_w] for the side
+        stream; replay_split runs the range all-reduce eagerly on the main stream
+        between the first and the last while the side graph runs."""
+        torch = self.torch
+        calls = lambda: {c[0]: c for c in self.calls}
+        cap = torch.cuda.Stream()
+        cap.wait_stream(self.main)
+        with torch.cuda.stream(cap):
+            self.bind(cap)
+            g_x = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_x, stream=cap):
+                self.amax.zero_()
+                self._call(*calls()["calibrate_x"])
+            g_rest = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_rest, stream=cap):
+                self.step(part="rest")
+            self.bind(cap, single=True)  # calibrate_w on the capturing stream
+            g_w = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_w, stream=cap):
+                self._call(*calls()["calibrate_w"])
+        self.bind(self.main)
+        self.main.wait_stream(cap)
+        self.graphs = [g_x, g_w, g_rest]
+        self.split = True
+
+    def replay_split(self, allreduce):
+        torch, main = self.torch, self.main
+        self.graphs[0].replay()                # zero the ranges, calibrate_x
+        self.side.wait_stream(main)
+        with torch.cuda.stream(self.side):
+            self.graphs[1].replay()            # calibrate_w
+        allreduce(self.amax_x)                 # main stream: overlaps calibrate_w
+        main.wait_stream(self.side)
+        self.graphs[2].replay()                # smooth_fold .. w8a8_linear
+
     def replay(self, allreduce=None):
+        if getattr(self, "split", False):
+            return self.replay_split(allreduce)
         self.graphs[0].replay()
         if len(self.graphs) > 1:
             allreduce(self.amax_x)
@@ -451,7 +499,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     if sq.sq_poll_status() != 0:
         raise RuntimeError("device wait timed out during warm-up")
-    use_graph = not args.no_graph and (not plan.two_streams or world == 1)
+    use_graph = not args.no_graph
     graph_note = None
     if use_graph:
         try:
@@ -662,8 +710,14 @@ def run_gpu(args):
             "stage_hbm_frac": {k: round(nbytes[k] / (v * 1e-6) / 1e9 / float(peaks["hbm_gbs"]), 3)
                                for k, v in stage_us.items() if v > 0 and (k != "w8a8_linear" or decode)},
             "gpu_launches": plan.launches_per_step * args.steps,
-            "launch": ("the step captured once into a CUDA graph and replayed (the C-ABI calls are "
-                       "capture-safe); every libsq kernel uses programmatic dependent launch"
+            "launch": (("the step captured once into a CUDA graph and replayed (the C-ABI calls are "
+                        "capture-safe); every libsq kernel uses programmatic dependent launch")
+                       if use_graph and world == 1 else
+                       ("the step captured into CUDA graphs replayed around the NCCL all-reduce of the "
+                        "activation ranges, which runs eagerly" +
+                        (" on the main stream while the weight-range graph runs on the side stream"
+                         if plan.two_streams else "") +
+                        "; every libsq kernel uses programmatic dependent launch")
                        if use_graph else "eager C-ABI calls; every libsq kernel uses programmatic "
                        "dependent launch"),
             "clocks": clocks,
