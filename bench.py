@@ -650,7 +650,7 @@ def run_gpu(args):
     gemm_s = gemm_us * 1e-6
     prof = os.path.join(ROOT, "profiles", f"w8a8_linear_{args.workload}{'_m%d' % M if M != wl.M else ''}.md")
     big = M > 128
-    pair = big and wl.K < 16384  # the library's automatic choice (sq_w8a8_linear)
+    pair = big  # the library's automatic choice (sq_w8a8_linear)
     gemm_src = ("k_gemm_splitk.cu" if decode else "k_gemm_pair.cu" if pair else
                 "k_gemm_wide.cu" if big else "k_gemm_tiled.cu")
     gemm_name = ("k_gemm_splitk (swap-AB stream-K)" if decode else

@@ -253,8 +253,8 @@ size_t sq_w8a8_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * M <= SQ_SPLITK_MAX_M runs the weight-streaming stream-K kernel and needs
  * sq_w8a8_workspace_bytes(M, N, K) bytes of workspace; 32 < M <= 128 runs the
  * tiled tensor-core kernel (128 x 256 tiles) and M > 128 a persistent kernel
- * of 256 x 256 tiles: on CTA pairs (tcgen05 cta_group::2) for K < 16384, on
- * single CTAs for longer K; none of these needs a workspace (it may be NULL).
+ * of 256 x 256 tiles on CTA pairs (tcgen05 cta_group::2); none of these needs
+ * a workspace (it may be NULL).
  */
 sq_status sq_w8a8_linear(const int8_t* xq, const float* x_scale, const int8_t* wq,
                          const float* w_scale, const void* bias_f16, void* y_f16, int64_t M,

@@ -160,13 +160,13 @@ sq_status linear_impl(const int8_t* xq, const float* x_scale, const int8_t* wq,
   if (path == SQ_PATH_PAIR) return launched(launch_gemm_pair(g, ctx));
   if (path == SQ_PATH_WIDE) return launched(launch_gemm_wide(g, ctx));
   if (path == SQ_PATH_TILED) return launched(launch_gemm_tiled(g, ctx));
-  // automatic: 256 x 256 tiles once the token count fills them -- on CTA
-  // pairs, whose double-buffered accumulators hide the epilogue, unless K is
-  // so long that the epilogue is a small share of a tile and the single-CTA
-  // kernel's main loop is ahead (K >= 16384 measured 5 % faster on the
-  // OPT-175B FFN-down shape); single-CTA 128-row tiles below 129 tokens
+  // automatic: 256 x 256 tiles on CTA pairs once the token count fills them
+  // (their double-buffered accumulators hide the epilogue; with two K boxes
+  // per stage they also lead the single-CTA 256 x 256 kernel at long K:
+  // 8192 x 12288 x 49152 and 4096 x 12288 x 16384 12-14 % faster);
+  // single-CTA 128-row tiles below 129 tokens
   if (M <= 128) return launched(launch_gemm_tiled(g, ctx));
-  return launched(K >= 16384 ? launch_gemm_wide(g, ctx) : launch_gemm_pair(g, ctx));
+  return launched(launch_gemm_pair(g, ctx));
 }
 
 }  // namespace
