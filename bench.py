@@ -959,14 +959,18 @@ def pick_sample(wl, M, budget_s, level="channel"):
     """Sample sizes whose oracle step takes about budget_s seconds."""
     import oracle
     c_s, n_s, m_s = min(wl.calib, 16), min(wl.N, 128), min(M, 4)
-    st = oracle_stage_times(wl, oracle_sample_inputs(wl, M, c_s, n_s, m_s), level)
-    dt = sum(st.values())
-    grow = max(1.0, budget_s / max(dt, 1e-6))
-    # grow the token and weight samples together (the GEMM is ~ m_s * n_s)
-    f = grow ** 0.5
-    n_s = int(min(wl.N, max(n_s, n_s * f)))
-    m_s = int(min(M, max(m_s, m_s * f)))
-    c_s = int(min(wl.calib, max(c_s, c_s * f)))
+    for _ in range(3):  # a small sample's time is mostly fixed costs: refine twice
+        st = oracle_stage_times(wl, oracle_sample_inputs(wl, M, c_s, n_s, m_s), level)
+        if oracle_full_time(wl, M, st, c_s, n_s, m_s) <= budget_s:  # the whole workload fits the budget
+            return wl.calib, wl.N, M
+        dt = sum(st.values())
+        if dt >= 0.5 * budget_s:
+            break
+        # grow the token and weight samples together (the GEMM is ~ m_s * n_s)
+        f = (budget_s / max(dt, 1e-6)) ** 0.5
+        n_s = int(min(wl.N, max(n_s, n_s * f)))
+        m_s = int(min(M, max(m_s, m_s * f)))
+        c_s = int(min(wl.calib, max(c_s, c_s * f)))
     return c_s, n_s, m_s
 
 
@@ -989,9 +993,11 @@ def oracle_baseline(wl, M, budget_s, level="channel"):
         oracle.set_num_threads(cores)
     full1 = oracle_full_time(wl, M, st1, c1, n1, m1)
     return {"value": round(v, 6), "unit": u, "cores": cores, "kind": "oracle",
-            "sample": (f"{c_s}/{wl.calib} calibration rows, {n_s}/{wl.N} weight rows, {m_s}/{M} tokens; "
-                       f"each stage timed on its sample and scaled linearly to the full workload "
-                       f"({sum(st.values()):.2f} s of CPU work; full step estimated {full:.1f} s)"),
+            "sample": (f"{c_s}/{wl.calib} calibration rows, {n_s}/{wl.N} weight rows, {m_s}/{M} tokens; " +
+                       (f"the whole workload, timed directly ({sum(st.values()):.2f} s of CPU work)"
+                        if (c_s, n_s, m_s) == (wl.calib, wl.N, M) else
+                        f"each stage timed on its sample and scaled linearly to the full workload "
+                        f"({sum(st.values()):.2f} s of CPU work; full step estimated {full:.1f} s)")),
             "single_thread": {"value": round(rate(full1), 6), "unit": u, "cores": 1,
                               "sample": f"{c1} calibration rows, {n1} weight rows, {m1} tokens, scaled linearly"}}
 
