@@ -649,13 +649,10 @@ def run_gpu(args):
     peaks, peak_kind = load_peaks()
     gemm_s = gemm_us * 1e-6
     prof = os.path.join(ROOT, "profiles", f"w8a8_linear_{args.workload}{'_m%d' % M if M != wl.M else ''}.md")
-    big = M > 128
-    pair = big  # the library's automatic choice (sq_w8a8_linear)
-    gemm_src = ("k_gemm_splitk.cu" if decode else "k_gemm_pair.cu" if pair else
-                "k_gemm_wide.cu" if big else "k_gemm_tiled.cu")
+    pair = M > 128  # the library's automatic choice (sq_w8a8_linear): CTA pairs above 128 tokens
+    gemm_src = "k_gemm_splitk.cu" if decode else "k_gemm_pair.cu" if pair else "k_gemm_tiled.cu"
     gemm_name = ("k_gemm_splitk (swap-AB stream-K)" if decode else
                  "k_gemm_pair (tcgen05 cta_group::2 kind::i8, 256x256 tiles)" if pair else
-                 "k_gemm_wide (tcgen05 kind::i8, 256x256 tiles per CTA)" if big else
                  "k_gemm_tiled (tcgen05 kind::i8, 128x256 tiles)")
     src = os.path.join(ROOT, "w8a8_int8_linear_channel_b200", "csrc", gemm_src)
     traffic = traffic_from_profile(src, prof)

@@ -1,7 +1,8 @@
-// k_gemm_wide.cu -- the W8A8 linear for large token counts (M > 128): INT8 x
-// INT8 -> INT32 GEMM on the 5th-generation tensor cores with the dequant
-// epilogue fused (glossary "INT8 GEMM"; section "inference", O1 scales; the
-// quantization tutorial's "multiply the scale back").
+// k_gemm_wide.cu -- the W8A8 linear on single CTAs with 256 x 256 tiles
+// (SQ_PATH_WIDE; the automatic choice for M > 128 is the CTA-pair kernel):
+// INT8 x INT8 -> INT32 GEMM on the 5th-generation tensor cores with the
+// dequant epilogue fused (glossary "INT8 GEMM"; section "inference", O1
+// scales; the quantization tutorial's "multiply the scale back").
 //
 // Persistent: one CTA per SM walks 256 x 256 output tiles.  Per 128-byte K
 // block a 64 KB stage holds 256 token rows of xq and 256 weight rows of wq;
