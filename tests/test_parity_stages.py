@@ -138,8 +138,11 @@ def test_ln_quant_act(sq, M, K, mode):
 
 
 # ------------------------------------------------------------------ GEMM ----
+# K = 496 / 512 / 528: the pair kernel's one-box ring below K = 512, two-box stages from there
+# (528: the last stage's second box lies wholly past K)
 GEMM_SHAPES = [(1, 8, 16), (5, 100, 48), (16, 256, 256), (17, 260, 144), (32, 1000, 4112),
-               (33, 77, 16), (127, 513, 272), (129, 256, 4096), (300, 1000, 2064), (256, 520, 528)]
+               (33, 77, 16), (127, 513, 272), (129, 256, 4096), (300, 1000, 2064), (256, 520, 528),
+               (260, 300, 496), (513, 264, 512)]
 
 
 def _rand_i8(rng, M, N, K):
