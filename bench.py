@@ -636,7 +636,7 @@ def run_gpu(args):
 
     nbytes, ops = stage_bytes_ops(wl, M, args.level)
     step_bytes = sum(nbytes.values())
-    decode = M <= sq.SPLITK_MAX_M
+    decode = M <= sq.DECODE_MAX_M
     if decode:
         value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
         value_warm = world * step_bytes / (warm_ms_per_step * 1e-3) / 1e9
@@ -881,7 +881,7 @@ def run_e2e(plan, sq, torch, world, allreduce, steps, dist):
     ms = float(t.item())
     M, N, K = plan.M, plan.wl.N, plan.wl.K
     nbytes, ops = stage_bytes_ops(plan.wl, M, plan.level)
-    if M <= sq.SPLITK_MAX_M:
+    if M <= sq.DECODE_MAX_M:
         v, u = world * sum(nbytes.values()) * steps / (ms * 1e-3) / 1e9, "GB/s"
     else:
         v, u = world * ops * steps / (ms * 1e-3) / 1e12, "TOPS"

@@ -60,8 +60,12 @@ extern "C" {
 #define SQ_MAX_K 133144
 
 /* Largest token count served by the weight-streaming (swap-AB, stream-K)
- * GEMM path; larger M uses the tiled path. */
-#define SQ_SPLITK_MAX_M 32
+ * GEMM kernel (SQ_PATH_SPLITK: tokens in the MMA's N slot, up to 128). */
+#define SQ_SPLITK_MAX_M 128
+
+/* Token counts up to which sq_w8a8_linear always streams the weight (the
+ * decoding stage), and which the allocation-free entry point serves. */
+#define SQ_DECODE_MAX_M 32
 
 typedef enum sq_status {
   SQ_OK = 0,
@@ -250,11 +254,14 @@ size_t sq_w8a8_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * explainer) is the special case of a w_scale array filled with one value.
  *   xq int8 [M, K]; x_scale fp32 [M]; wq int8 [N, K]; w_scale fp32 [N];
  *   bias fp16 [N] or NULL; y fp16 [M, N]
- * M <= SQ_SPLITK_MAX_M runs the weight-streaming stream-K kernel and needs
- * sq_w8a8_workspace_bytes(M, N, K) bytes of workspace; 32 < M <= 128 runs the
- * tiled tensor-core kernel (128 x 256 tiles) and M > 128 a persistent kernel
- * of 256 x 256 tiles on CTA pairs (tcgen05 cta_group::2); none of these needs
- * a workspace (it may be NULL).
+ * M <= SQ_DECODE_MAX_M runs the weight-streaming stream-K kernel and needs
+ * sq_w8a8_workspace_bytes(M, N, K) bytes of workspace.  For
+ * SQ_DECODE_MAX_M < M <= SQ_SPLITK_MAX_M the stream-K kernel runs when the
+ * workspace given holds sq_w8a8_workspace_bytes(M, N, K) bytes and the layer
+ * is narrow (4 * ceil(N / 256) <= the SM count: the tiled kernel's 128 x 256
+ * tiles would leave most SMs idle), otherwise the tiled tensor-core kernel
+ * (128 x 256 tiles, no workspace; NULL is fine).  M > 128 runs a persistent
+ * kernel of 256 x 256 tiles on CTA pairs (tcgen05 cta_group::2), no workspace.
  */
 sq_status sq_w8a8_linear(const int8_t* xq, const float* x_scale, const int8_t* wq,
                          const float* w_scale, const void* bias_f16, void* y_f16, int64_t M,
@@ -280,7 +287,7 @@ sq_status sq_w8a8_linear(const int8_t* xq, const float* x_scale, const int8_t* w
  *   xq int8 [M, K]; x_scale fp32 [M]; wq int8 [N, K]; w_scale fp32 [N];
  *   bias fp16 [N] or NULL; inv_s_next fp32 [N] or NULL; range_next fp32 [1];
  *   xq_next int8 [M, N]; x_scale_next fp32 [M].  N % 16 == 0 (the next
- *   linear's K).  M <= SQ_SPLITK_MAX_M needs the stream-K workspace.
+ *   linear's K).  M <= SQ_DECODE_MAX_M needs the stream-K workspace.
  */
 sq_status sq_w8a8_linear_quant(const int8_t* xq, const float* x_scale, const int8_t* wq,
                                const float* w_scale, const void* bias_f16, int relu,
@@ -328,7 +335,7 @@ sq_status sq_w8a8_gemm_s32(const int8_t* xq, const int8_t* wq, int32_t* acc, int
                            sq_stream_t stream);
 
 /*
- * Allocation-free variant of sq_w8a8_linear for M <= SQ_SPLITK_MAX_M (the
+ * Allocation-free variant of sq_w8a8_linear for M <= SQ_DECODE_MAX_M (the
  * stream-K decode kernel).  The paper has no counterpart: this entry point
  * exists for callers that cannot allocate device memory -- for example a
  * plug-in inside another runtime that owns every device allocation and hands
@@ -338,7 +345,7 @@ sq_status sq_w8a8_gemm_s32(const int8_t* xq, const int8_t* wq, int32_t* acc, int
  * Instead of a caller workspace it uses one fixed array of
  * SQ_NOALLOC_SCRATCH_BYTES in device global memory, owned by the library;
  * every GPU that loads the library holds that array until the process exits.
- * The call allocates and frees nothing.  Limits: M <= SQ_SPLITK_MAX_M
+ * The call allocates and frees nothing.  Limits: M <= SQ_DECODE_MAX_M
  * (else SQ_ERR_UNSUPPORTED_SHAPE) and at most SQ_NOALLOC_MAX_TILES tiles of
  * 128 output channels, i.e. N <= 524288 (else SQ_ERR_WORKSPACE, the shape
  * needs more scratch than the fixed array holds).  Same numerics and the

@@ -62,7 +62,7 @@ def test_linear_rejects_bad_arguments_on_the_host():
     # misaligned pointer
     assert f(FAKE_ODD, FAKE, FAKE, FAKE, None, FAKE, 64, 64, 64, None, 0, None) == 2
     # forced stream-K path for too many tokens
-    assert L.sq_w8a8_linear_path(FAKE, FAKE, FAKE, FAKE, None, FAKE, 33, 64, 64, FAKE, 1 << 20, 2, None) == 3
+    assert L.sq_w8a8_linear_path(FAKE, FAKE, FAKE, FAKE, None, FAKE, 129, 64, 64, FAKE, 1 << 20, 2, None) == 3
     # unknown path
     assert L.sq_w8a8_linear_path(FAKE, FAKE, FAKE, FAKE, None, FAKE, 8, 64, 64, FAKE, 1 << 20, 7, None) == 1
     del ok
@@ -86,11 +86,14 @@ def test_other_entry_points_reject_bad_arguments():
 
 def test_workspace_size_formula():
     L = _lib()
-    assert L.sq_w8a8_workspace_bytes(64, 4096, 4096) == 0       # tiled path needs none
+    assert L.sq_w8a8_workspace_bytes(129, 4096, 4096) == 0      # beyond stream-K: none
     assert L.sq_w8a8_workspace_bytes(0, 4096, 4096) == 0
     n = L.sq_w8a8_workspace_bytes(32, 49152, 12288)
     # counters for 384 channel tiles (rounded to 256 B) + 2 int32 [128 x 32] slots per SM
     assert n >= 1536 + 2 * 148 * 128 * 32 * 4
+    # 33-64 tokens take the 64-token tile, 65-128 the 128-token tile
+    assert L.sq_w8a8_workspace_bytes(64, 4096, 4096) >= 256 + 2 * 148 * 128 * 64 * 4
+    assert L.sq_w8a8_workspace_bytes(65, 4096, 4096) >= 256 + 2 * 148 * 128 * 128 * 4
 
 
 def _has_gpu():

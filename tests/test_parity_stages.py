@@ -139,10 +139,12 @@ def test_ln_quant_act(sq, M, K, mode):
 
 # ------------------------------------------------------------------ GEMM ----
 # K = 496 / 512 / 528: the pair kernel's one-box ring below K = 512, two-box stages from there
-# (528: the last stage's second box lies wholly past K)
+# (528: the last stage's second box lies wholly past K).  33 / 64 / 127 / 128 tokens: the
+# stream-K kernel's 64- and 128-token tiles; (64, 520, 8208) and (128, 1000, 4112) split
+# their channel tiles between CTAs
 GEMM_SHAPES = [(1, 8, 16), (5, 100, 48), (16, 256, 256), (17, 260, 144), (32, 1000, 4112),
-               (33, 77, 16), (127, 513, 272), (129, 256, 4096), (300, 1000, 2064), (256, 520, 528),
-               (260, 300, 496), (513, 264, 512)]
+               (33, 77, 16), (64, 520, 8208), (127, 513, 272), (128, 1000, 4112), (129, 256, 4096),
+               (300, 1000, 2064), (256, 520, 528), (260, 300, 496), (513, 264, 512)]
 
 
 def _rand_i8(rng, M, N, K):
@@ -163,7 +165,7 @@ _PATHS = {"tiled": lambda m: m.PATH_TILED, "splitk": lambda m: m.PATH_SPLITK,
 @pytest.mark.parametrize("path", ["tiled", "splitk", "pair", "wide"])
 def test_gemm_accumulators_bit_exact(sq, M, N, K, path):
     if path == "splitk" and M > sq.SPLITK_MAX_M:
-        pytest.skip("stream-K path serves M <= 32")
+        pytest.skip("stream-K path serves M <= 128")
     rng = np.random.default_rng(M * 1000003 + N * 101 + K)
     xq, wq, _, _, _ = _rand_i8(rng, M, N, K)
     p = _PATHS[path](sq)
@@ -179,7 +181,7 @@ def test_gemm_accumulators_bit_exact(sq, M, N, K, path):
 @pytest.mark.parametrize("with_bias", [False, True])
 def test_linear_output(sq, M, N, K, path, with_bias):
     if path == "splitk" and M > sq.SPLITK_MAX_M:
-        pytest.skip("stream-K path serves M <= 32")
+        pytest.skip("stream-K path serves M <= 128")
     rng = np.random.default_rng(M * 7919 + N * 31 + K + with_bias)
     xq, wq, sx, sw, bias = _rand_i8(rng, M, N, K)
     bias = bias if with_bias else None

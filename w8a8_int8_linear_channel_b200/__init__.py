@@ -29,14 +29,15 @@ __all__ = [
     "sq_quantize_weight_tensor", "sq_ln_quant_act_tensor", "sq_ln_quant_act_static", "sq_tensor_range",
     "LEVELS", "sq_w8a8_linear_quant", "sq_w8a8_bmm", "sq_row_ranges", "sq_quantize_rows_ranged",
     "sq_dequant",
-    "PATH_AUTO", "PATH_TILED", "PATH_SPLITK", "PATH_PAIR", "PATH_WIDE", "SPLITK_MAX_M", "MAX_K", "library_path",
+    "PATH_AUTO", "PATH_TILED", "PATH_SPLITK", "PATH_PAIR", "PATH_WIDE", "SPLITK_MAX_M", "DECODE_MAX_M", "MAX_K", "library_path",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libsq.so")
 
 PATH_AUTO, PATH_TILED, PATH_SPLITK, PATH_PAIR, PATH_WIDE = 0, 1, 2, 3, 4
-SPLITK_MAX_M = 32
+SPLITK_MAX_M = 128  # the stream-K kernel's largest token count
+DECODE_MAX_M = 32   # sq_w8a8_linear always streams the weight up to here
 MAX_K = 133144
 
 STATUS = {0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_MISALIGNED", 3: "SQ_ERR_UNSUPPORTED_SHAPE",

@@ -1,9 +1,10 @@
 // k_gemm_splitk.cu -- the W8A8 linear for decode-sized token counts
 // (M <= 32), where the layer is bound by streaming the INT8 weight from HBM
-// (the explainer's "decoding stage").
+// (the explainer's "decoding stage"), and for up to 128 tokens on layers too
+// narrow for the tiled kernel's 128 x 256 tiles to cover the SMs.
 //
 // Swap-AB: the MMA's 128-row M slot takes 128 weight rows (output channels)
-// and its N slot takes the BT (16 or 32) zero-padded tokens, so
+// and its N slot takes the BT (16, 32, 64 or 128) zero-padded tokens, so
 //   TMEM lane = output channel n,  TMEM column = token t.
 // Persistent grid of one CTA per SM; a unit is a (channel tile, 256-byte K
 // span).  Each CTA streams its units back to back, so its TMA stream never
@@ -15,9 +16,10 @@
 // the epilogue y = fp16((acc * sx[t]) * sw[n] + bias[n]).  int32 addition is
 // associative, so the result is bit-identical to a single-CTA sum.
 //
-// Roles: warp 0 TMA producer (a 5-deep ring; a stage is two K-consecutive 16 KB weight boxes +
-// BT x 128 B token tiles), warp 1 TMEM owner + MMA issuer (double-buffered
-// accumulators), warps 2-5 epilogue.  All waits are bounded.
+// Roles: warp 0 TMA producer (a 5-deep ring for up to 32 tokens, 4- and 3-deep for 64 and
+// 128; a stage is two K-consecutive 16 KB weight boxes + two BT x 128 B token boxes),
+// warp 1 TMEM owner + MMA issuer (double-buffered accumulators), warps 2-5 epilogue.
+// All waits are bounded.
 #include "sq_internal.h"
 #include "sq_ptx.cuh"
 #include "sq_tmap.h"
@@ -29,13 +31,14 @@ constexpr int BW = 128;  // weight rows (output channels) per tile
 constexpr int BK = 128;  // K bytes per swizzled box
 constexpr int KPS = 2;   // consecutive K boxes per unit (per pipeline stage)
 constexpr int kThreads = 192;
-constexpr int kStages = 5;
 
 template <int BT>
 struct SkLayout {
+  static constexpr int STAGES = BT <= 32 ? 5 : BT == 64 ? 4 : 3;  // about 192-200 KB of ring
   static constexpr int A_BYTES = BW * BK * KPS;  // 2 x 16 KB weight boxes
   static constexpr int B_BYTES = BT * BK * KPS;  // 2 token boxes
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int kStages = STAGES;
   static constexpr int CTRL = kStages * STAGE_BYTES;
   static constexpr int NBARS = 2 * kStages + 5;  // full, empty, acc_full[2], acc_empty[2], drain
   static constexpr int SLOT = CTRL + NBARS * 8;  // TMEM address, abort, last, decision[2]
@@ -43,6 +46,8 @@ struct SkLayout {
   static constexpr int BYTES = SX + BT * 4;
   static constexpr size_t SMEM = BYTES + 1024;
   static constexpr int TMEM_COLS = 2 * BT < 32 ? 32 : 2 * BT;
+  static_assert(BT == 16 || BT == 32 || BT == 64 || BT == 128, "token tile of the MMA's N slot");
+  static_assert(SX + BT * 4 + 1024 <= 232448, "shared memory per CTA");
 };
 
 // Work split.  With T channel tiles on `grid` CTAs, every CTA owns Wt =
@@ -77,6 +82,26 @@ __device__ __forceinline__ void tmem_ld_tokens<16>(uint32_t taddr, uint32_t (&v)
   tmem_ld_32x32b_x16(taddr, v);
 }
 
+// 64 and 128 tokens: 32-column loads, each chunk's registers tied to the wait
+template <>
+__device__ __forceinline__ void tmem_ld_tokens<64>(uint32_t taddr, uint32_t (&v)[64]) {
+  uint32_t(&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+  uint32_t(&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+  tmem_ld_32x32b_x32(taddr, a);
+  tmem_ld_32x32b_x32(taddr + 32u, b);
+  tmem_ld_wait_regs(a);
+  tmem_ld_wait_regs(b);
+}
+
+template <>
+__device__ __forceinline__ void tmem_ld_tokens<128>(uint32_t taddr, uint32_t (&v)[128]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    tmem_ld_32x32b_x32(taddr + 32u * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld_wait_regs(*reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
+}
+
 // EPI: 0 = fp16 y, 1 = int32 accumulators, 2 = the next linear's INT8 codes
 // at its static scale (producer-side quantization).
 template <int BT, int EPI>
@@ -86,6 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   uint32_t* status, uint64_t budget) {
   constexpr bool OUT_I32 = EPI == 1;
   using L = SkLayout<BT>;
+  constexpr int kStages = L::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -414,7 +440,7 @@ cudaError_t launch_bt(const GemmArgs& g, const Ctx& c) {
 
 size_t splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
   (void)K;
-  const int64_t bt = M <= 16 ? 16 : 32;
+  const int64_t bt = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
   const size_t counter_bytes = ((tiles_of(N) * 4 + 255) / 256) * 256;
   return counter_bytes + static_cast<size_t>(2) * num_sms * BW * bt * 4;
 }
@@ -422,7 +448,9 @@ size_t splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
 cudaError_t launch_gemm_splitk(const GemmArgs& g, const Ctx& c) {
   const int epi = g.acc != nullptr ? 1 : g.q_next != nullptr ? 2 : 0;
   if (g.M <= 16) return epi == 1 ? launch_bt<16, 1>(g, c) : epi == 2 ? launch_bt<16, 2>(g, c) : launch_bt<16, 0>(g, c);
-  return epi == 1 ? launch_bt<32, 1>(g, c) : epi == 2 ? launch_bt<32, 2>(g, c) : launch_bt<32, 0>(g, c);
+  if (g.M <= 32) return epi == 1 ? launch_bt<32, 1>(g, c) : epi == 2 ? launch_bt<32, 2>(g, c) : launch_bt<32, 0>(g, c);
+  if (g.M <= 64) return epi == 1 ? launch_bt<64, 1>(g, c) : epi == 2 ? launch_bt<64, 2>(g, c) : launch_bt<64, 0>(g, c);
+  return epi == 1 ? launch_bt<128, 1>(g, c) : epi == 2 ? launch_bt<128, 2>(g, c) : launch_bt<128, 0>(g, c);
 }
 
 }  // namespace sq
@@ -518,7 +546,7 @@ extern "C" sq_status sq_w8a8_linear_noalloc(const int8_t* xq, const float* x_sca
   if (!xq || !x_scale || !wq || !w_scale || !y_f16) return SQ_ERR_INVALID_ARG;
   if (M <= 0 || N <= 0 || K <= 0) return SQ_ERR_INVALID_ARG;
   if (K > SQ_MAX_K) return SQ_ERR_K_OVERFLOW;
-  if (K % 16 != 0 || M > SQ_SPLITK_MAX_M) return SQ_ERR_UNSUPPORTED_SHAPE;
+  if (K % 16 != 0 || M > SQ_DECODE_MAX_M) return SQ_ERR_UNSUPPORTED_SHAPE;
   if (tiles_of(N) > SQ_NOALLOC_MAX_TILES) return SQ_ERR_WORKSPACE;  // beyond the fixed scratch
   if (!a16(xq) || !a16(wq) || !a16(x_scale) || !a16(w_scale) || !a16(y_f16) ||
       (bias_f16 && !a16(bias_f16)))

@@ -132,12 +132,21 @@ sq_status linear_impl(const int8_t* xq, const float* x_scale, const int8_t* wq,
       !opt_aligned(bias_f16) || !opt_aligned(y_f16) || !opt_aligned(acc))
     return SQ_ERR_MISALIGNED;
   if (M > 0x7fffffffLL || N > 0x7fffffffLL) return SQ_ERR_UNSUPPORTED_SHAPE;
-  if (path == SQ_PATH_AUTO && M <= SQ_SPLITK_MAX_M) path = SQ_PATH_SPLITK;
   if (path == SQ_PATH_SPLITK && M > SQ_SPLITK_MAX_M) return SQ_ERR_UNSUPPORTED_SHAPE;
 
   Ctx ctx;
   st = current_ctx(stream, &ctx);
   if (st != SQ_OK) return st;
+  if (path == SQ_PATH_AUTO) {
+    if (M <= SQ_DECODE_MAX_M) {
+      path = SQ_PATH_SPLITK;
+    } else if (M <= SQ_SPLITK_MAX_M && 4 * ((N + 255) / 256) <= ctx.num_sms && workspace != nullptr &&
+               aligned16(workspace) && ws_bytes >= splitk_workspace_bytes(M, N, K, ctx.num_sms)) {
+      // a narrow layer: 128 x 256 tiles would leave most SMs idle, while the
+      // stream-K kernel streams the weight on all of them
+      path = SQ_PATH_SPLITK;
+    }
+  }
 
   GemmArgs g{};
   g.xq = xq;
@@ -521,7 +530,7 @@ sq_status sq_w8a8_linear_quant(const int8_t* xq, const float* x_scale, const int
   g.inv_s_next = inv_s_next;
   g.range_next = range_next;
   g.relu = relu ? 1 : 0;
-  if (M <= SQ_SPLITK_MAX_M) {
+  if (M <= SQ_DECODE_MAX_M) {
     const size_t need = splitk_workspace_bytes(M, N, K, ctx.num_sms);
     if (workspace == nullptr || ws_bytes < need || !aligned16(workspace)) return SQ_ERR_WORKSPACE;
     return launched(launch_gemm_splitk(g, ctx));
