@@ -238,9 +238,11 @@ sq_status sq_quantize_rows_ranged(const void* x_f16, int64_t rows, int64_t K, in
 sq_status sq_dequant(const int32_t* acc, const float* x_scale, const float* w_scale,
                      const void* bias_f16, void* y_f16, int64_t M, int64_t N, sq_stream_t stream);
 
-/* Bytes of workspace sq_w8a8_linear needs for this shape (0 if none).  The
- * workspace holds int32 partial sums and per-tile arrival counters of the
- * stream-K path.  The caller zero-fills it once before its first use; every
+/* Bytes of workspace the stream-K path needs for this shape: nonzero for
+ * M <= SQ_SPLITK_MAX_M (needed up to SQ_DECODE_MAX_M tokens, optional above,
+ * where it lets sq_w8a8_linear stream the weight of a narrow layer), 0 for
+ * larger M or non-positive sizes.  The workspace holds int32 partial sums and
+ * per-tile arrival counters of the stream-K path.  The caller zero-fills it once before its first use; every
  * call that completes leaves the counters at zero again.  After a call that
  * reported SQ_ERR_TIMEOUT, zero-fill it again.  Calls that share a workspace
  * must not overlap on the GPU. */
