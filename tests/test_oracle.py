@@ -556,3 +556,40 @@ def test_nan_values_quantize_to_zero_and_inf_saturates():
     assert np.isinf(sx[1]) and not xq[1].any()
     wq, sw = oracle.quantize_weight(h)
     assert np.array_equal(wq, xq) and np.array_equal(sw, sx)
+
+
+# ------------------------------------------------- quality references ----
+def test_hand_example_quality_references():
+    # naive per-tensor W8A8 and per-token / per-channel W8A8 without smoothing, against the
+    # hand-worked fixture (power-of-two scales, so the fp64 results are exact)
+    g = load("quality_refs_2x3.txt")
+    X, W, bias = g["X"], g["W"], g["bias"]
+    assert np.array_equal(oracle.naive_per_tensor_w8a8(X, W), g["naive_y"])
+    assert np.array_equal(oracle.per_token_per_channel_w8a8(X, W), g["ptpc_y"])
+    assert np.array_equal(oracle.naive_per_tensor_w8a8(X, W, bias), g["naive_y"] + bias[None, :])
+    assert np.array_equal(oracle.per_token_per_channel_w8a8(X, W, bias), g["ptpc_y"] + bias[None, :])
+    # the fixture's own steps hang together: codes -> exact integer sums -> scaled sums
+    assert np.array_equal(g["naive_qx"] @ g["naive_qw"].T, g["naive_acc"])
+    assert np.array_equal(g["naive_acc"] * (2.0 * 2.0), g["naive_y"])
+    assert np.array_equal(g["ptpc_qx"] @ g["ptpc_qw"].T, g["ptpc_acc"])
+    sx, sw = np.array([2.0, 0.5, 0.0]), np.array([1.0, 2.0])
+    assert np.array_equal(g["ptpc_acc"] * sx[:, None] * sw[None, :], g["ptpc_y"])
+    assert np.array_equal(X @ W.T, g["Y"])
+
+
+def test_quality_references_agree_when_every_row_has_one_range():
+    # with the same absmax on every token row and every weight row, one scale per row is one
+    # scale per tensor: the two references take the same codes, so they agree up to the fp64
+    # rounding of their scale products (acc * (sx * sw) against (acc * sx) * sw)
+    rng = np.random.default_rng(5)
+    X = rng.uniform(-2.9, 2.9, (6, 16))
+    W = rng.uniform(-0.49, 0.49, (5, 16))
+    X[np.arange(6), rng.integers(0, 16, 6)] = 3.0 * rng.choice([-1.0, 1.0], 6)
+    W[np.arange(5), rng.integers(0, 16, 5)] = 0.5 * rng.choice([-1.0, 1.0], 5)
+    b = rng.standard_normal(5)
+    assert np.allclose(oracle.naive_per_tensor_w8a8(X, W, b), oracle.per_token_per_channel_w8a8(X, W, b),
+                       rtol=1e-14, atol=1e-14)
+    # and both are the plain product within half a quantization step per operand
+    err = np.abs(oracle.naive_per_tensor_w8a8(X, W) - X @ W.T)
+    bound = 16 * (0.5 * 3.0 / 127 * 0.5 + 0.5 * 0.5 / 127 * 3.0 + 0.25 * (3.0 / 127) * (0.5 / 127))
+    assert (err <= bound).all()

@@ -56,3 +56,53 @@ def test_pins_catch_mutant(name, tmp_path):
                         os.path.join(ROOT, "tests", "test_oracle.py")],
                        env=env, cwd=ROOT, capture_output=True, text=True)
     assert r.returncode != 0, f"mutant {name} passed every pin:\n{r.stdout[-2000:]}"
+
+
+# Mistakes planted in the oracle's numpy quality references (naive per-tensor W8A8 and
+# per-token / per-channel W8A8 without smoothing); the copy of the package runs with the
+# real C library, so only the planted line differs.
+PY_SRC = os.path.join(ROOT, "oracle", "__init__.py")
+PY_MUTANTS = {
+    "naive_scale_per_row": ("    sx = np.abs(x).max() / 127.0\n", "    sx = np.abs(x).max(axis=1, keepdims=True) / 127.0\n"),
+    "naive_weight_truncates": ("qw = np.clip(np.rint(w / sw if sw > 0 else 0 * w), -127, 127)",
+                               "qw = np.clip(np.trunc(w / sw if sw > 0 else 0 * w), -127, 127)"),
+    "naive_scale_128": ("    sw = np.abs(w).max() / 127.0\n", "    sw = np.abs(w).max() / 128.0\n"),
+    "ptpc_ties_away": ("qx = np.clip(np.rint(np.where(sx > 0, x / sx, 0.0)), -127, 127)",
+                       "qx = np.clip(np.sign(x) * np.floor(np.abs(np.where(sx > 0, x / sx, 0.0)) + 0.5), -127, 127)"),
+    "ptpc_drops_sw": ("    y = (qx @ qw.T) * sx * sw.T\n", "    y = (qx @ qw.T) * sx\n"),
+    "ptpc_tensor_scale_for_w": ("    sw = np.abs(w).max(axis=1, keepdims=True) / 127.0\n",
+                                "    sw = np.abs(w).max() / 127.0 + 0.0 * np.abs(w).max(axis=1, keepdims=True)\n"),
+}
+
+
+def _run_pins_on_copy(tmp_path, src_text):
+    """Run test_oracle.py against a copy of the oracle package whose __init__.py is src_text."""
+    import shutil
+
+    from oracle import build as oracle_build
+
+    shutil.copytree(os.path.join(ROOT, "oracle"), tmp_path / "oracle",
+                    ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    (tmp_path / "oracle" / "__init__.py").write_text(src_text)
+    shutil.copytree(os.path.join(ROOT, "tests"), tmp_path / "tests", ignore=shutil.ignore_patterns("__pycache__"))
+    shutil.copy(os.path.join(ROOT, "sq_inputs.py"), tmp_path / "sq_inputs.py")
+    env = dict(os.environ, SQ_ORACLE_LIB=oracle_build.build())
+    return subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                           str(tmp_path / "tests" / "test_oracle.py")],
+                          env=env, cwd=str(tmp_path), capture_output=True, text=True)
+
+
+def test_python_mutant_harness_passes_the_real_oracle(tmp_path):
+    # the copy itself must pass, so a failing mutant run means the planted line was caught
+    r = _run_pins_on_copy(tmp_path, open(PY_SRC).read())
+    assert r.returncode == 0, r.stdout[-2000:]
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_pins_catch_python_mutant(name, tmp_path):
+    old, new = PY_MUTANTS[name]
+    src = open(PY_SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not unique in the oracle package"
+    r = _run_pins_on_copy(tmp_path, src.replace(old, new))
+    assert r.returncode != 0, f"mutant {name} passed every pin:\n{r.stdout[-2000:]}"
+    assert "1 failed" in r.stdout, r.stdout[-2000:]
