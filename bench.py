@@ -37,6 +37,7 @@ import numpy as np  # noqa: E402
 import sq_inputs  # noqa: E402
 
 METRIC = "W8A8 linear TOPS and % of INT8 peak (large M); GB/s % HBM (decode M≤32)"
+DECODE_M = 32  # the metric's decode range: up to this many tokens the step is reported in GB/s
 DESCR = {
     "tiny": "tiny: K=N=256, M=16, calib 128, outliers x60 on channels 3/77",
     "attn": "OPT-6.7B attention projection: K=N=4096, M=2048 tokens, calib 512, 6 outlier channels x40-100, LN folded, alpha 0.5",
@@ -636,7 +637,7 @@ def run_gpu(args):
 
     nbytes, ops = stage_bytes_ops(wl, M, args.level)
     step_bytes = sum(nbytes.values())
-    decode = M <= sq.DECODE_MAX_M
+    decode = M <= DECODE_M
     if decode:
         value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
         value_warm = world * step_bytes / (warm_ms_per_step * 1e-3) / 1e9
@@ -881,7 +882,7 @@ def run_e2e(plan, sq, torch, world, allreduce, steps, dist):
     ms = float(t.item())
     M, N, K = plan.M, plan.wl.N, plan.wl.K
     nbytes, ops = stage_bytes_ops(plan.wl, M, plan.level)
-    if M <= sq.DECODE_MAX_M:
+    if M <= DECODE_M:
         v, u = world * sum(nbytes.values()) * steps / (ms * 1e-3) / 1e9, "GB/s"
     else:
         v, u = world * ops * steps / (ms * 1e-3) / 1e12, "TOPS"
@@ -977,8 +978,8 @@ def oracle_baseline(wl, M, budget_s, level="channel"):
     st = oracle_stage_times(wl, oracle_sample_inputs(wl, M, c_s, n_s, m_s), level)
     full = oracle_full_time(wl, M, st, c_s, n_s, m_s)
     nbytes, ops = stage_bytes_ops(wl, M, level)
-    rate = lambda t: (sum(nbytes.values()) / t / 1e9) if M <= 32 else (ops / t / 1e12)
-    u = "GB/s" if M <= 32 else "TOPS"
+    rate = lambda t: (sum(nbytes.values()) / t / 1e9) if M <= DECODE_M else (ops / t / 1e12)
+    u = "GB/s" if M <= DECODE_M else "TOPS"
     v = rate(full)
     # the same oracle on one thread, on a sample a tenth the size
     cores = oracle.num_threads()
@@ -1022,7 +1023,7 @@ def run_reference(args):
         fulls.append(oracle_full_time(wl, M, st, c_s, n_s, m_s))
     full = sum(fulls) / len(fulls)
     nbytes, ops = stage_bytes_ops(wl, M, args.level)
-    if M <= 32:
+    if M <= DECODE_M:
         v, u = sum(nbytes.values()) / full / 1e9, "GB/s"
     else:
         v, u = ops / full / 1e12, "TOPS"
