@@ -39,7 +39,9 @@ def test_calibrate_absmax_raw(sq, rows, K):
     assert bits_equal(host(amax), want)
 
 
-@pytest.mark.parametrize("rows,K", [(5, 256), (64, 4096), (17, 1040), (9, 16384)])
+# K > 16384 takes the kernel whose CTAs re-read each row from global memory and merge
+# their column maxima with atomics
+@pytest.mark.parametrize("rows,K", [(5, 256), (64, 4096), (17, 1040), (9, 16384), (3, 49152), (2, 65536)])
 def test_calibrate_absmax_layernorm(sq, rows, K):
     rng = np.random.default_rng(rows + K)
     h = rand_h(rng, rows, K, shift=0.3)
