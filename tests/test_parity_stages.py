@@ -39,9 +39,11 @@ def test_calibrate_absmax_raw(sq, rows, K):
     assert bits_equal(host(amax), want)
 
 
-# K > 16384 takes the kernel whose CTAs re-read each row from global memory and merge
-# their column maxima with atomics
-@pytest.mark.parametrize("rows,K", [(5, 256), (64, 4096), (17, 1040), (9, 16384), (3, 49152), (2, 65536)])
+# one case per kernel shape: a warp per row with 1, 2 or 4 chunks (K <= 256, 512, 1024), CTA
+# rows of 64, 128 or 256 threads (K <= 2048, 4096, 8192, 16384), and above 16384 the kernel
+# whose CTAs re-read each row from global memory and merge their column maxima with atomics
+@pytest.mark.parametrize("rows,K", [(5, 256), (6, 512), (64, 4096), (17, 1040), (12, 8192), (9, 16384),
+                                    (3, 49152), (2, 65536)])
 def test_calibrate_absmax_layernorm(sq, rows, K):
     rng = np.random.default_rng(rows + K)
     h = rand_h(rng, rows, K, shift=0.3)
@@ -100,8 +102,9 @@ def test_fold_weight_in_place(sq):
 
 
 # --------------------------------------------------------- weight quantize ----
-@pytest.mark.parametrize("N,K,fold", [(1, 16, False), (77, 48, True), (300, 4112, True),
-                                      (256, 256, False), (40, 16400, True), (13, 49152, True)])
+@pytest.mark.parametrize("N,K,fold", [(1, 16, False), (77, 48, True), (11, 512, True), (21, 2048, True),
+                                      (300, 4112, True), (256, 256, False), (5, 16384, False),
+                                      (40, 16400, True), (13, 49152, True)])
 def test_quantize_weight(sq, N, K, fold):
     rng = np.random.default_rng(N + K)
     w = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
@@ -117,9 +120,10 @@ def test_quantize_weight(sq, N, K, fold):
 
 
 # ---------------------------------------------------------- LN + quantize ----
-@pytest.mark.parametrize("M,K,mode", [(1, 16, "plain"), (16, 256, "inv_s"), (33, 4096, "ln"),
-                                      (129, 1040, "ln_inv_s"), (7, 12288, "ln"),
-                                      (5, 49152, "inv_s"), (3, 65536, "inv_s"), (2, 49152, "ln")])
+@pytest.mark.parametrize("M,K,mode", [(1, 16, "plain"), (16, 256, "inv_s"), (9, 512, "ln"), (33, 4096, "ln"),
+                                      (129, 1040, "ln_inv_s"), (6, 8192, "inv_s"), (7, 12288, "ln"),
+                                      (3, 16384, "ln_inv_s"), (5, 49152, "inv_s"), (3, 65536, "inv_s"),
+                                      (2, 49152, "ln")])
 def test_ln_quant_act(sq, M, K, mode):
     rng = np.random.default_rng(M * K)
     h = rand_h(rng, M, K, outliers=(2, K - 3), shift=0.2)
