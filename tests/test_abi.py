@@ -106,3 +106,24 @@ def test_valid_call_without_a_device_reports_cuda_error():
     L = _lib()
     r = L.sq_w8a8_linear(FAKE, FAKE, FAKE, FAKE, None, FAKE, 64, 64, 64, None, 0, None)
     assert r == 7  # SQ_ERR_CUDA: no device; nothing was launched
+
+
+def test_binding_refuses_host_tensors():
+    # a host tensor must never reach a kernel as a device address: the binding refuses it
+    # before calling the library
+    import torch
+
+    import w8a8_int8_linear_channel_b200 as sq
+    xq = torch.zeros((4, 16), dtype=torch.int8)
+    wq = torch.zeros((8, 16), dtype=torch.int8)
+    sx, sw = torch.zeros(4), torch.zeros(8)
+    y = torch.empty((4, 8), dtype=torch.float16)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        sq.sq_w8a8_linear(xq, sx, wq, sw, y)
+    h = torch.zeros((4, 16), dtype=torch.float16)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        sq.sq_ln_quant_act(h, xq, sx)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        sq.sq_calibrate_absmax(h, torch.zeros(16))
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        sq.sq_w8a8_bmm(xq[None], sx[None], wq[None], sw[None], y[None])

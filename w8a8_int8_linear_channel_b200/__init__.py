@@ -103,7 +103,18 @@ def _check(status: int, where: str) -> None:
 
 
 def _p(t: Optional[torch.Tensor]):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a tensor argument.  The C ABI takes pointers on the
+    current CUDA device: a host tensor, or one on another GPU, is refused here
+    with an error instead of reaching a kernel as a wrong address."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"libsq takes CUDA tensors on the current device; got a tensor on {t.device}")
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"a tensor on {t.device} while the current device is cuda:{cur} "
+                         "(libsq runs on the current device: call torch.cuda.set_device first)")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream) -> ctypes.c_void_p:
