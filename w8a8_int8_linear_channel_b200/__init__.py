@@ -495,14 +495,18 @@ class SmoothQuantLinear:
                    act_range=act_range)
 
     def workspace(self, M: int) -> Optional[torch.Tensor]:
+        """The stream-K workspace for M tokens (None where no kernel needs one).  Calls that share
+        a workspace must not overlap on the GPU, so the layer keeps one per stream: forward calls
+        issued on different streams may run concurrently."""
         N, K = self.wq.shape
         need = sq_w8a8_workspace_bytes(M, N, K)
         if need == 0:
             return None
-        ws = self._ws.get(self.wq.device)
+        key = torch.cuda.current_stream(self.wq.device).cuda_stream
+        ws = self._ws.get(key)
         if ws is None or ws.numel() < need:
             ws = torch.zeros(need, dtype=torch.uint8, device=self.wq.device)
-            self._ws[self.wq.device] = ws
+            self._ws[key] = ws
         return ws
 
     def quantize_input(self, h: torch.Tensor, xq=None, x_scale=None):
