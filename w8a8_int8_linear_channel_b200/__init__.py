@@ -496,8 +496,9 @@ class SmoothQuantLinear:
 
     def workspace(self, M: int) -> Optional[torch.Tensor]:
         """The stream-K workspace for M tokens (None where no kernel needs one).  Calls that share
-        a workspace must not overlap on the GPU, so the layer keeps one per stream: forward calls
-        issued on different streams may run concurrently."""
+        a workspace must not overlap on the GPU, so the layer keeps one per stream.  (At level O2
+        every forward also writes the layer's one batch-range buffer, ``act_range``, so O2
+        forwards on different streams must still not overlap.)"""
         N, K = self.wq.shape
         need = sq_w8a8_workspace_bytes(M, N, K)
         if need == 0:
