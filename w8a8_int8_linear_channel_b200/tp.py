@@ -174,7 +174,10 @@ class RowParallelSmoothQuantLinear:
     def from_float(cls, w_shard, calib_shard, alpha: float = 0.5, bias=None, ops=None, comm=None):
         """w_shard: fp16 [N, K_rank] (all output channels, this rank's input
         channels); calib_shard: [T, K_rank], this rank's slice of the layer's
-        calibration input; bias [N] is added once, after the reduction."""
+        calibration input; bias [N] is added once, after the reduction.  The
+        layer's whole K (the sum of K_rank over ranks) must be at most MAX_K,
+        the bound under which the all-reduced int32 sums of 127 x 127 products
+        cannot overflow; each rank can only check its own slice."""
         ops = ops or LibsqOps()
         comm = comm or DistComm()
         amax_x = ops.col_absmax(calib_shard)  # channel j lives on one rank only
