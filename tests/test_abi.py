@@ -127,3 +127,15 @@ def test_binding_refuses_host_tensors():
         sq.sq_calibrate_absmax(h, torch.zeros(16))
     with pytest.raises(ValueError, match="CUDA tensors"):
         sq.sq_w8a8_bmm(xq[None], sx[None], wq[None], sw[None], y[None])
+
+
+def test_layer_forward_refuses_a_host_input():
+    # SmoothQuantLinear.forward on a host tensor must fail before any kernel is launched
+    import torch
+
+    import w8a8_int8_linear_channel_b200 as sq
+    K, N = 16, 8
+    layer = sq.SmoothQuantLinear(torch.zeros((N, K), dtype=torch.int8), torch.zeros(N), None, None, None,
+                                 torch.ones(K), torch.ones(K), 1e-5)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        layer(torch.zeros((3, K), dtype=torch.float16))
