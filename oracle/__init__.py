@@ -26,8 +26,9 @@ Sources, cited by page title and section:
 
 Beyond the per-token / per-channel layer: the explainer's quantization
 levels O1-O3 (``quantize_weight_tensor``, ``ln_quant_act_tensor``,
-``ln_quant_act_static``, ``tensor_range``), producer-side quantization
-(``w8a8_linear_quant_static``) and the INT8 BMM (``w8a8_bmm``).
+``ln_quant_act_static``, ``tensor_range``), producer-side quantization at a
+static scale (``w8a8_linear_quant_static``) and at the per-token dynamic
+scale (``w8a8_linear_quant_dynamic``), and the INT8 BMM (``w8a8_bmm``).
 
 Parity status: every function here is pinned by ``tests/test_oracle.py``,
 including the two unsmoothed quality references (``naive_per_tensor_w8a8``,
@@ -342,6 +343,18 @@ def w8a8_linear_quant_static(xq, sx, wq, sw, bias=None, relu=False, inv_s_next=N
                                           _ptr(inv_s_next), float(np.float32(range_next)), M, N, K,
                                           _ptr(q), _ptr(s_next))
     return q, s_next
+
+
+def w8a8_linear_quant_dynamic(xq, sx, wq, sw, bias=None, relu=False, inv_s_next=None):
+    """[SQ] producer-side quantization at the next linear's default level (per-token dynamic
+    scale, "inference" O1): the linear, an optional ReLU, the next linear's 1/s, then the
+    per-token quantizer -- written as the composition of the pinned steps, so it is exactly
+    w8a8_linear, then max(a, 0) on the fp16 values (a NaN becomes 0, as ``y > 0 ? y : 0``),
+    then ln_quant_act with inv_s only.  Returns (q_next [M, N] int8, sx_next [M] fp32)."""
+    y = w8a8_linear(xq, sx, wq, sw, bias)
+    if relu:
+        y = np.where(y > 0, y, np.float16(0)).astype(np.float16)
+    return ln_quant_act(y, None, None, inv_s_next)
 
 
 def w8a8_bmm(a, a_scale, b, b_scale) -> np.ndarray:

@@ -482,6 +482,64 @@ def test_producer_quant_is_linear_then_static_quant(relu):
     assert (np.abs(q) == 127).any()
 
 
+def test_hand_example_producer_dynamic():
+    g = load("producer_dyn_3x3.txt")
+    args = (g["xq"].astype(np.int8), g["sx"], g["wq"].astype(np.int8), g["sw"], f16(g["bias"]))
+    q, s = oracle.w8a8_linear_quant_dynamic(*args, relu=True, inv_s_next=g["inv_s"])
+    assert np.array_equal(q, g["q_relu"]) and np.array_equal(s, g["sx_relu"].astype(np.float32))
+    q, s = oracle.w8a8_linear_quant_dynamic(*args, relu=False, inv_s_next=g["inv_s"])
+    assert np.array_equal(q, g["q_plain"])
+    assert np.array_equal(s[:2], g["sx_plain_rows01"].astype(np.float32))
+    assert s[2] == np.float32(0.375) / np.float32(127)
+
+
+@pytest.mark.parametrize("relu", [False, True])
+def test_producer_dynamic_is_linear_then_per_token_quant(relu):
+    """Independent restatement in numpy float32 of everything after the (separately pinned)
+    fp16 linear output: ReLU, times 1/s, per-token absmax scale, round half to even."""
+    rng = np.random.default_rng(77 + relu)
+    M, N, K = 11, 48, 64
+    xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    wq = rng.integers(-127, 128, (N, K)).astype(np.int8)
+    sx = rng.uniform(1e-3, 1e-2, M).astype(np.float32)
+    sx[3] = 0.0  # a zero row: y = bias
+    sw = rng.uniform(1e-3, 1e-2, N).astype(np.float32)
+    bias = f16(rng.standard_normal(N) * 0.1)
+    inv = rng.uniform(0.1, 3.0, N).astype(np.float32)
+    y = oracle.w8a8_linear(xq, sx, wq, sw, bias).astype(np.float32)
+    a = np.where(y > 0, y, np.float32(0)) if relu else y
+    x = (a * inv[None, :]).astype(np.float32)
+    sc = (np.abs(x).max(axis=1) / np.float32(127)).astype(np.float32)
+    rcp = np.where(sc > 0, np.float32(1) / np.where(sc > 0, sc, 1), 0).astype(np.float32)
+    codes = np.clip(np.rint((x * rcp[:, None]).astype(np.float32)), -127, 127).astype(np.int8)
+    q, s = oracle.w8a8_linear_quant_dynamic(xq, sx, wq, sw, bias, relu=relu, inv_s_next=inv)
+    assert np.array_equal(s, sc) and np.array_equal(q, codes)
+    # the row maxima hit 127 exactly: the dynamic scale is each row's own range
+    assert np.all(np.abs(q).max(axis=1)[sc > 0] == 127)
+
+
+def test_producer_dynamic_equals_static_when_rows_share_a_range():
+    """When every row's range equals one static range, the per-token and the static
+    (level O3) producer quantizations coincide."""
+    rng = np.random.default_rng(5)
+    M, N, K = 6, 32, 32
+    xq = rng.integers(-20, 21, (M, K)).astype(np.int8)
+    wq = rng.integers(-20, 21, (N, K)).astype(np.int8)
+    xq[:, 0] = 100  # channel 0 of every output gets one large, equal value per row
+    wq[:, 0] = 0
+    wq[0, :] = 0
+    wq[0, 0] = 127
+    sx = np.full(M, 0.01, np.float32)
+    sw = np.full(N, 0.01, np.float32)
+    inv = np.ones(N, np.float32)
+    y = oracle.w8a8_linear(xq, sx, wq, sw).astype(np.float32)
+    r = np.abs(y).max(axis=1)
+    assert np.all(r == r[0])  # the same range in every row (output 0 dominates)
+    qd, sd = oracle.w8a8_linear_quant_dynamic(xq, sx, wq, sw, inv_s_next=inv)
+    qs, ss = oracle.w8a8_linear_quant_static(xq, sx, wq, sw, inv_s_next=inv, range_next=r[0])
+    assert np.array_equal(qd, qs) and np.array_equal(sd, ss)
+
+
 # ------------------------------------------------------------------ INT8 BMM --
 def test_hand_example_bmm():
     g = load("bmm_2x2x2.txt")

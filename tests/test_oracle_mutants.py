@@ -72,6 +72,12 @@ PY_MUTANTS = {
     "ptpc_drops_sw": ("    y = (qx @ qw.T) * sx * sw.T\n", "    y = (qx @ qw.T) * sx\n"),
     "ptpc_tensor_scale_for_w": ("    sw = np.abs(w).max(axis=1, keepdims=True) / 127.0\n",
                                 "    sw = np.abs(w).max() / 127.0 + 0.0 * np.abs(w).max(axis=1, keepdims=True)\n"),
+    # the per-token producer-side quantization (a composition of pinned steps)
+    "dyn_relu_dropped": ("        y = np.where(y > 0, y, np.float16(0)).astype(np.float16)\n",
+                         "        y = y.astype(np.float16)\n"),
+    "dyn_inv_s_dropped": ("    return ln_quant_act(y, None, None, inv_s_next)\n", "    return ln_quant_act(y, None, None, None)\n"),
+    "dyn_relu_abs": ("        y = np.where(y > 0, y, np.float16(0)).astype(np.float16)\n",
+                     "        y = np.abs(y).astype(np.float16)\n"),
 }
 
 
