@@ -94,18 +94,34 @@ def outlier_gains(wl: Workload) -> np.ndarray:
 
 
 def _normal_rows(seed: int, tag: str, K: int, row0: int, rows: int, std: float) -> np.ndarray:
-    """Rows [row0, row0+rows) of an fp16 matrix whose ROW_BLOCK-row blocks are independent streams."""
+    """Rows [row0, row0+rows) of an fp16 matrix whose ROW_BLOCK-row blocks are independent streams.
+    Blocks are drawn on a thread pool when there are many of them (each block is its own stream,
+    so the values do not depend on the number of threads)."""
     out = np.empty((rows, K), np.float16)
+    spans = []
     r = row0
     while r < row0 + rows:
         blk = r // ROW_BLOCK
         b0 = blk * ROW_BLOCK
         take = min(b0 + ROW_BLOCK, row0 + rows) - r
+        spans.append((blk, r - b0, r - row0, take))
+        r += take
+
+    def fill(span):
+        blk, src, dst, take = span
         g = _rng(seed, tag, blk).standard_normal((ROW_BLOCK, K), dtype=np.float32)
         if std != 1.0:
             g *= np.float32(std)
-        out[r - row0:r - row0 + take] = g[r - b0:r - b0 + take].astype(np.float16)
-        r += take
+        out[dst:dst + take] = g[src:src + take].astype(np.float16)
+
+    if len(spans) < 2 or rows * K < (1 << 22):
+        for sp in spans:
+            fill(sp)
+    else:
+        import os
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max(1, min(len(spans), os.cpu_count() or 1, 32))) as ex:
+            list(ex.map(fill, spans))
     return out
 
 

@@ -40,6 +40,60 @@ def test_smoothquant_beats_naive_per_tensor(name):
     assert e_sq < 0.05
 
 
+# The four OPT-shaped outlier workloads, on sampled token rows.  The two largest weights
+# (49152 x 12288 and 12288 x 49152) are cut to their first output rows here, i.e. the same
+# layer with fewer outputs (every output row is independent, and the smoothing then sees the
+# weight ranges of those rows); tests/test_quality_gpu.py runs the full layers on the GPU.
+OUTLIER_CASES = [("attn", 4096, 32), ("ffn_up", 16384, 16), ("decode", 2048, 32), ("ffn_down", 1024, 16)]
+
+
+def _case(name, n_rows, m_rows, alpha=None):
+    wl = sq_inputs.WORKLOADS[name]
+    if alpha is not None:
+        wl = sq_inputs.with_(wl, alpha=alpha)
+    w = sq_inputs.weight(wl, 0, n_rows)
+    b16 = sq_inputs.bias(wl)
+    b16 = None if b16 is None else b16[:n_rows]
+    return wl, sq_inputs.calib_rows(wl), sq_inputs.run_rows(wl, 0, m_rows), w, b16
+
+
+def _errors(wl, calib, h, w, b16):
+    r = oracle.run_step(calib, w, h, sq_inputs.gamma(wl), sq_inputs.beta(wl), b16, wl.alpha)
+    X = _x_fp64(wl, h)
+    bias = None if b16 is None else b16.astype(np.float64)
+    w64 = w.astype(np.float64)
+    y64 = oracle.linear_fp64(X, w64, bias)
+    return (_rel(r["y"].astype(np.float64), y64), _rel(oracle.naive_per_tensor_w8a8(X, w64, bias), y64),
+            _rel(oracle.per_token_per_channel_w8a8(X, w64, bias), y64))
+
+
+@pytest.mark.parametrize("name,n_rows,m_rows", OUTLIER_CASES)
+def test_smoothquant_beats_naive_on_outlier_workloads(name, n_rows, m_rows):
+    """The explainer's prediction ("challenge", "why activations are hard to quantize"): with
+    persistent outlier channels naive per-tensor W8A8 loses far more than SmoothQuant."""
+    e_sq, e_naive, e_tok = _errors(*_case(name, n_rows, m_rows))
+    assert e_sq < e_naive, (name, e_sq, e_naive)
+    assert e_sq < e_tok, (name, e_sq, e_tok)
+
+
+def test_ffn_down_alpha_sweep():
+    """The FFN-down alpha sweep {0, .25, .5, .75, .85, 1}: every value is reported as computed;
+    the configured alpha (0.5) beats naive W8A8, and a middle alpha beats both ends (all
+    difficulty left on the activations at alpha 0, all moved to the weights at alpha 1)."""
+    wl, calib, h, w, b16 = _case("ffn_down", 512, 8)
+    assert b16 is None and not wl.ln
+    amax_x = oracle.calibrate_absmax(calib)
+    X, w64 = h.astype(np.float64), w.astype(np.float64)
+    y64 = oracle.linear_fp64(X, w64)
+    naive = _rel(oracle.naive_per_tensor_w8a8(X, w64), y64)
+    errs = {}
+    for a in sq_inputs.FFN_DOWN_ALPHAS:
+        r = oracle.run_step(calib, w, h, alpha=a, amax_x=amax_x)
+        errs[a] = _rel(r["y"].astype(np.float64), y64)
+    assert errs[0.5] < naive, errs
+    assert min(errs[0.25], errs[0.5], errs[0.75]) < min(errs[0.0], errs[1.0]), errs
+
+
 def test_alpha_moves_difficulty_to_weights():
     # "smoothing factor": a larger alpha flattens activations more and loads the weights more.
     wl = sq_inputs.WORKLOADS["tiny"]
