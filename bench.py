@@ -80,6 +80,7 @@ def stage_bytes_ops(wl, M, level="channel"):
     K, N, C = wl.K, wl.N, wl.calib
     act, wgt = LEVELS[level]
     b = {
+        "calib_reset": 3 * 4 * K,
         "calibrate_x": 2 * C * K + 4 * K,
         "calibrate_w": 2 * N * K + 4 * K,
         "smooth_fold": 4 * K * 6,
@@ -171,6 +172,22 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def workload_of(args):
+    wl = sq_inputs.WORKLOADS[args.workload]
+    if args.alpha is not None:
+        wl = sq_inputs.with_(wl, alpha=float(args.alpha))
+    return wl
+
+
+def common_config(args, wl, M, world):
+    """The workload keys, identical in the GPU arm and the reference arm."""
+    return {"workload": DESCR[args.workload] + ("" if M == wl.M else f" (M={M})") +
+                        ("" if args.alpha is None else f" (alpha={wl.alpha})"),
+            "M": M, "N": wl.N, "K": wl.K, "calib_tokens": wl.calib, "alpha": wl.alpha,
+            "level": args.level, "granularity": LEVEL_DESCR[args.level], "step": STEP,
+            "parallelism": f"dp{world}"}
+
+
 # ------------------------------------------------------------ GPU arm -------
 class Plan:
     """Device buffers and prepared C-ABI calls of one step (argument
@@ -231,6 +248,7 @@ class Plan:
         runtime_inv_s, ws_bytes = self.runtime_inv_s, self.ws_bytes
         act, wgt = LEVELS[self.level]
         calls = [
+            ("calib_reset", L.sq_calibrate_reset, (p(self.amax), 3 * K, stream)),
             ("calibrate_x", L.sq_calibrate_absmax, (p(self.calib), self.calib_rows, K, K, p(self.gamma),
                                                     p(self.beta), eps, p(self.amax_x), stream)),
             ("calibrate_w", L.sq_calibrate_absmax, (p(self.w), N, K, K, None, None, eps, p(self.amax_w),
@@ -274,14 +292,12 @@ class Plan:
 
     def step(self, events=None, allreduce=None, part=None):
         """Run one step.  With two streams the independent stages overlap:
-            main: calibrate_x            | smooth_fold | ln_quant_act    | w8a8_linear
-            side:          calibrate_w   |             | quantize_weight |
+            main: calib_reset | calibrate_x | smooth_fold | ln_quant_act    | w8a8_linear
+            side:             | calibrate_w |             | quantize_weight |
         with events joining them where a stage needs the other stream's output.
         With `events` (one per call + 1), the stages instead run one after the
         other on the main stream timing order (for the per-stage breakdown)."""
         torch = self.torch
-        if part != "rest":  # the rest of a step keeps the calibrated, all-reduced ranges
-            self.amax.zero_()
         if events is not None:  # serialized, one event before each call
             for i, (name, fn, args) in enumerate(self.calls):
                 events[i].record(self.main)
@@ -304,8 +320,6 @@ class Plan:
         calls = self.calls
         if part == "rest":  # smooth_fold onwards (the ranges are complete and all-reduced)
             calls = calls[[c[0] for c in calls].index("smooth_fold"):]
-        else:
-            self.side.wait_stream(main)                # amax zeroed, previous step done
         for name, fn, args in calls:
             if name == "smooth_fold" and part != "rest":  # needs both ranges
                 if allreduce is not None:              # on main after calibrate_x: overlaps calibrate_w
@@ -316,6 +330,8 @@ class Plan:
             if name == "w8a8_linear":                  # needs wq and xq
                 main.wait_stream(self.side)
             self._call(name, fn, args)                 # calibrate_w / quantize_weight run on side
+            if name == "calib_reset":                  # ranges zeroed (and the previous step done)
+                self.side.wait_stream(main)
 
     def capture(self, world):
         """Capture the step into CUDA graphs: one graph for N = 1; for N > 1 two
@@ -338,8 +354,6 @@ class Plan:
                     if self.two_streams:  # the side stream forks from and joins the capture
                         self.step()
                     else:
-                        if i == 0:
-                            self.amax.zero_()
                         for name, fn, args in self.calls:
                             if name in seg:
                                 self._call(name, fn, args)
@@ -360,7 +374,6 @@ class Plan:
             self.bind(cap, single=True)
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr, stream=cap):
-                self.amax.zero_()
                 for i, (name, fn, args) in enumerate(self.calls):
                     self.sev[i].record(cap)
                     self._call(name, fn, args)
@@ -419,7 +432,7 @@ class Plan:
             self.bind(cap)
             g_x = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g_x, stream=cap):
-                self.amax.zero_()
+                self._call(*calls()["calib_reset"])
                 self._call(*calls()["calibrate_x"])
             g_rest = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g_rest, stream=cap):
@@ -476,7 +489,7 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
 
-    wl = sq_inputs.WORKLOADS[args.workload]
+    wl = workload_of(args)
     M = args.m if args.m else wl.M
     plan = Plan(wl, M, rank, device, sq, torch, two_streams=args.streams == 2, level=args.level)
     allreduce = None
@@ -634,6 +647,16 @@ def run_gpu(args):
 
     producer = run_producer(plan, sq, torch, flush, reps, args) if args.producer and use_graph else None
     bmm = run_bmm(sq, torch, device, flush, args) if args.bmm and use_graph else None
+    # one-GPU extras: the forward alone, the decode half of the metric, reconstruction quality
+    forward = decode_rec = quality = quality_sweep = None
+    if world == 1 and use_graph and not args.no_extras:
+        forward = run_forward(plan, sq, torch, flush, args.burst_iters)
+        quality = run_quality(plan, sq, torch)
+    peaks_early, _ = load_peaks()
+    if world == 1 and use_graph and not args.no_extras and not args.no_decode:
+        decode_rec = run_decode_sweep(sq, torch, device, flush, args.burst_iters, peaks_early)
+    if world == 1 and not args.no_extras and not args.no_quality_sweep:
+        quality_sweep = run_quality_sweep(sq, torch, device, sq_inputs.FFN_DOWN_ALPHAS)
 
     nbytes, ops = stage_bytes_ops(wl, M, args.level)
     step_bytes = sum(nbytes.values())
@@ -673,10 +696,17 @@ def run_gpu(args):
     roof["kernel"] = gemm_name
     roof["per_launch_us"] = round(gemm_us, 2)
     roof["launch_timing"] = gemm_mode
+    if forward is not None:  # the same kernel with its operands coming from HBM (L2 flushed first)
+        cold_us = forward["linear"]["cold_us"]
+        cold_ach = (nbytes["w8a8_linear"] / (cold_us * 1e-6) / 1e9) if decode else (ops / (cold_us * 1e-6) / 1e12)
+        roof["per_launch_us_cold"] = cold_us
+        roof["achieved_cold"] = round(cold_ach, 1)
+        roof["frac_cold"] = round(cold_ach / roof["peak"], 4)
 
-    e2e = None
+    e2e = e2e_fwd = None
     if not args.no_e2e:
         e2e = run_e2e(plan, sq, torch, world, allreduce, min(args.steps, args.e2e_steps), dist)
+        e2e_fwd = run_e2e_forward(plan, sq, torch, world, min(args.steps, 10 * args.e2e_steps), dist)
 
     result = None
     if rank == 0:
@@ -685,18 +715,15 @@ def run_gpu(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
             "data": "synthetic (seeded PCG64, OPT-shaped with persistent outlier channels)",
-            "config": {"workload": DESCR[args.workload] + ("" if M == wl.M else f" (M={M})"),
-                       "M": M, "N": wl.N, "K": wl.K, "calib_tokens": wl.calib, "alpha": wl.alpha,
-                       "level": args.level, "granularity": LEVEL_DESCR[args.level],
-                       "step": STEP, "streams": args.streams, "cuda_graph": use_graph,
-                       **({"cuda_graph_note": graph_note} if graph_note else {}),
-                       "parallelism": f"dp{world}",
-                       "l2": "flushed before every step (256 MiB write, then 256 MiB read so no dirty "
-                             "lines remain), outside the timed events",
-                       "timing": "CUDA events at the boundaries of every step, summed over steps, max over "
-                                 "ranks; stage_us and the roofline's launch time from a second loop with "
-                                 "events around every call (" + ("event nodes in a CUDA graph of the step"
-                                 if stage_mode == "graph" else "eager launches") + ")"},
+            "config": common_config(args, wl, M, world),
+            "run": {"streams": args.streams, "cuda_graph": use_graph,
+                    **({"cuda_graph_note": graph_note} if graph_note else {}),
+                    "l2": "flushed before every step (256 MiB write, then 256 MiB read so no dirty "
+                          "lines remain), outside the timed events",
+                    "timing": "CUDA events at the boundaries of every step, summed over steps, max over "
+                              "ranks; stage_us and the roofline's launch time from a second loop with "
+                              "events around every call (" + ("event nodes in a CUDA graph of the step"
+                              if stage_mode == "graph" else "eager launches") + ")"},
             "roofline": roof,
             "warm_l2": {"value": round(value_warm, 2), "unit": unit, "ms_per_step": round(warm_ms_per_step, 5),
                         "steps": n_warm, "note": "back-to-back steps with no flush between them"},
@@ -720,7 +747,12 @@ def run_gpu(args):
                        "dependent launch"),
             "clocks": clocks,
             "e2e": e2e,
+            "e2e_forward": e2e_fwd,
         }
+        for key, rec in (("forward", forward), ("decode", decode_rec), ("quality", quality),
+                         ("quality_alpha_sweep", quality_sweep)):
+            if rec is not None:
+                result[key] = rec
         if producer is not None:
             result["producer_quant"] = producer
         if bmm is not None:
@@ -756,8 +788,18 @@ def run_producer(plan, sq, torch, flush, reps, args):
                                               M, N, K, p(plan.ws), plan.ws_bytes, st)),
                (L.sq_ln_quant_act_static, lambda st: (p(y), M, N, N, None, None, p(inv_next), ctypes.c_float(1e-5),
                                                       p(rng_next), p(q_next), p(s_next), st))]
+    # the next linear's per-token dynamic scale: the GEMM with a row-maximum epilogue plus the
+    # codes pass, against the linear to fp16 then the per-token quantization (sq_ln_quant_act)
+    ws_dyn = sq.new_quant_dyn_workspace(M, N, K, device=dev)
+    fused_dyn = [(L.sq_w8a8_linear_quant_dyn, lambda st: (p(plan.xq), p(plan.sx), p(plan.wq), p(plan.sw),
+                                                          p(plan.bias), 0, p(inv_next), p(q_next), p(s_next),
+                                                          M, N, K, p(ws_dyn), ws_dyn.numel(), st))]
+    unfused_dyn = [unfused[0],
+                   (L.sq_ln_quant_act, lambda st: (p(y), M, N, N, None, None, p(inv_next), ctypes.c_float(1e-5),
+                                                   p(q_next), p(s_next), st))]
     out = {}
-    for name, calls in (("fused", fused), ("unfused", unfused)):
+    for name, calls in (("fused", fused), ("unfused", unfused), ("dynamic_fused", fused_dyn),
+                        ("dynamic_unfused", unfused_dyn)):
         gr = plan.capture_burst_of(calls, reps)
         flush()
         gr.replay()
@@ -779,7 +821,9 @@ def run_producer(plan, sq, torch, flush, reps, args):
     out["ops"] = 2 * M * N * K
     out["what"] = ("linear + the next linear's static (level O3) input quantization with its 1/s: fused into "
                    "the GEMM epilogue (sq_w8a8_linear_quant) vs sq_w8a8_linear then sq_ln_quant_act_static; "
-                   f"{reps} back-to-back launches per graph, L2 flushed before each replay")
+                   "and at the next linear's per-token dynamic scale: sq_w8a8_linear_quant_dyn (GEMM with a "
+                   "row-maximum epilogue writing fp16, then a codes pass) vs sq_w8a8_linear then "
+                   f"sq_ln_quant_act; {reps} back-to-back launches per graph, L2 flushed before each replay")
     return out
 
 
@@ -833,6 +877,300 @@ def run_bmm(sq, torch, device, flush, args):
     if sq.sq_poll_status() != 0:
         raise RuntimeError("device wait timed out in the BMM loop")
     return out
+
+
+def graph_of(torch, calls, reps):
+    """One CUDA graph of `reps` rounds of the given (fn, args-builder(stream)) C calls,
+    captured on a side stream (consecutive launches overlap through PDL)."""
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        st = ctypes.c_void_p(cap.cuda_stream)
+        bound = [(fn, mk(st)) for fn, mk in calls]
+        for fn, a in bound:  # once eagerly (lazy set-up outside the capture)
+            Plan._call("call", fn, a)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=cap):
+            for _ in range(reps):
+                for fn, a in bound:
+                    Plan._call("call", fn, a)
+    torch.cuda.current_stream().wait_stream(cap)
+    torch.cuda.synchronize()
+    return gr
+
+
+def time_graph(torch, gr, iters, flush, reps=1):
+    """Mean device time (us) of one round of a graph of `reps` rounds: events around each
+    replay on the current stream, the L2 flushed before each replay (outside the events)."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(iters)]
+    flush()
+    gr.replay()
+    for e in ev:
+        flush()
+        e[0].record()
+        gr.replay()
+        e[1].record()
+    torch.cuda.synchronize()
+    return 1e3 * sum(a.elapsed_time(b) for a, b in ev) / iters / reps
+
+
+def cold_warm(torch, calls, flush, iters, warm_reps):
+    """(cold, warm) microseconds per round of `calls`: cold = one round per replay after an L2
+    flush; warm = `warm_reps` back-to-back rounds per replay (operands stay in L2 when they fit)."""
+    cold = time_graph(torch, graph_of(torch, calls, 1), iters, flush)
+    warm = time_graph(torch, graph_of(torch, calls, warm_reps), max(3, iters // 4), flush, warm_reps)
+    return cold, warm
+
+
+def run_forward(plan, sq, torch, flush, iters):
+    """The per-forward part of the step (a6 + a7 + a8: LayerNorm / per-token quantization, the
+    INT8 GEMM and its epilogue) with the weight already quantized, as a model runs it; and
+    the linear (a7 + a8) alone.  Cold: L2 flushed before every forward; warm: back to back."""
+    calls = {name: (fn, args) for name, fn, args in plan.calls}
+    rebind = lambda name: (calls[name][0], lambda st, a=calls[name][1]: a[:-1] + (st,))
+    wl, M = plan.wl, plan.M
+    nbytes, ops = stage_bytes_ops(wl, M, plan.level)
+    fwd_bytes = nbytes["ln_quant_act"] + nbytes["w8a8_linear"]
+    out = {}
+    for key, names in (("forward", ("ln_quant_act", "w8a8_linear")), ("linear", ("w8a8_linear",)),
+                       ("ln_quant_act", ("ln_quant_act",))):
+        cold, warm = cold_warm(torch, [rebind(n) for n in names], flush, iters, 20)
+        rec = {"cold_us": round(cold, 2), "warm_us": round(warm, 2)}
+        b = fwd_bytes if key == "forward" else nbytes[names[0]]
+        rec["gbs_cold"] = round(b / (cold * 1e-6) / 1e9, 1)
+        if key != "ln_quant_act":
+            rec["tops_cold"] = round(ops / (cold * 1e-6) / 1e12, 1)
+            rec["tops_warm"] = round(ops / (warm * 1e-6) / 1e12, 1)
+        else:
+            rec["gbs_warm"] = round(b / (warm * 1e-6) / 1e9, 1)
+        out[key] = rec
+    out["what"] = ("forward = sq_ln_quant_act + sq_w8a8_linear with the weight already quantized; cold: "
+                   "one forward per graph replay after a 256 MiB L2 flush; warm: 20 back-to-back "
+                   "forwards per replay")
+    if sq.sq_poll_status() != 0:
+        raise RuntimeError("device wait timed out in the forward loop")
+    return out
+
+
+def run_decode_sweep(sq, torch, device, flush, iters, peaks):
+    """The metric's decode half: the OPT-175B FFN-up linear (K = 12288, N = 49152) at
+    M in {1, 4, 8, 16, 32}: per-launch time of the stream-K kernel (cold: one launch after an
+    L2 flush; warm: back-to-back launches; the 604 MB weight never fits the 126 MB L2), its
+    algorithmic GB/s and the fraction of the measured copy bandwidth; and the forward
+    (per-token quantization + linear)."""
+    wl = sq_inputs.WORKLOADS["decode"]
+    Mmax = max(sq_inputs.DECODE_M)
+    plan = Plan(wl, Mmax, 0, device, sq, torch)
+    plan.step()
+    torch.cuda.synchronize()
+    L = sq._L
+    K, N = wl.K, wl.N
+    p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    hbm = float(peaks["hbm_gbs"])
+    uuid = ""
+    try:
+        uuid = str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    if sampler:
+        sampler.start()
+    rows = []
+    for M in sq_inputs.DECODE_M:
+        y = plan.y[:M]
+        lin = (L.sq_w8a8_linear, lambda st, M=M, y=y: (p(plan.xq), p(plan.sx), p(plan.wq), p(plan.sw), None,
+                                                      p(y), M, N, K, p(plan.ws), plan.ws_bytes, st))
+        act = (L.sq_ln_quant_act, lambda st, M=M: (p(plan.h), M, K, K, p(plan.gamma_f), p(plan.beta_f), None,
+                                                  ctypes.c_float(1e-5), p(plan.xq), p(plan.sx), st))
+        cold, warm = cold_warm(torch, [lin], flush, iters, 10)
+        fcold, fwarm = cold_warm(torch, [act, lin], flush, iters, 10)
+        b = M * K + N * K + 4 * M + 4 * N + 2 * M * N
+        fb = b + 3 * M * K + 4 * M + 8 * K
+        rows.append({"M": M, "linear_cold_us": round(cold, 2), "linear_warm_us": round(warm, 2),
+                     "gbs_cold": round(b / (cold * 1e-6) / 1e9, 1), "gbs_warm": round(b / (warm * 1e-6) / 1e9, 1),
+                     "hbm_frac_cold": round(b / (cold * 1e-6) / 1e9 / hbm, 4),
+                     "hbm_frac_warm": round(b / (warm * 1e-6) / 1e9 / hbm, 4),
+                     "forward_cold_us": round(fcold, 2), "forward_warm_us": round(fwarm, 2),
+                     "forward_gbs_cold": round(fb / (fcold * 1e-6) / 1e9, 1),
+                     "algorithmic_bytes": b})
+    clocks = sampler.stop() if sampler else None
+    if sq.sq_poll_status() != 0:
+        raise RuntimeError("device wait timed out in the decode sweep")
+    del plan
+    torch.cuda.empty_cache()
+    return {"workload": DESCR["decode"], "kernel": "k_gemm_splitk (swap-AB stream-K, tcgen05 kind::i8)",
+            "peak_gbs": hbm, "peak_source": "measured copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+            "bytes": "M*K + N*K + 4M + 4N + 2MN per linear launch; the forward adds 3MK + 4M + 8K",
+            "timing": "cold: one launch per CUDA-graph replay after a 256 MiB L2 flush; warm: 10 "
+                      f"back-to-back launches per replay; mean of {iters} replays",
+            "sweep": rows, "clocks": clocks}
+
+
+# ------------------------------------------------------------ quality -------
+def layernorm_fp64(torch, h, gamma, beta, eps):
+    """The LayerNorm the linear's input comes from, in fp64 (biased variance)."""
+    x = h.double()
+    mu = x.mean(1, keepdim=True)
+    var = ((x - mu) ** 2).mean(1, keepdim=True)
+    x = (x - mu) / torch.sqrt(var + eps)
+    if gamma is not None:
+        x = x * gamma.double()
+    if beta is not None:
+        x = x + beta.double()
+    return x
+
+
+def product_fp64(torch, X64, w, bias):
+    """Y = X W^T + b in fp64 (W converted in blocks of rows to bound the memory)."""
+    N = w.shape[0]
+    Y = torch.empty((X64.shape[0], N), dtype=torch.float64, device=X64.device)
+    step = 4096
+    for n0 in range(0, N, step):
+        Y[:, n0:n0 + step] = X64 @ w[n0:n0 + step].double().t()
+    if bias is not None:
+        Y += bias.double()
+    return Y
+
+
+def unsmoothed_w8a8(sq, torch, h_s, w, gamma, beta, bias, per_tensor):
+    """W8A8 without smoothing through the library's own entry points: per token and per output
+    channel (sq_ln_quant_act + sq_quantize_weight), or naive, one scale for all of X and one for
+    all of W (level O2 for X, sq_quantize_weight_tensor)."""
+    m, K = h_s.shape
+    N = w.shape[0]
+    dev = h_s.device
+    xq = torch.empty((m, K), dtype=torch.int8, device=dev)
+    sx = torch.empty(m, dtype=torch.float32, device=dev)
+    wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+    sw = torch.empty(N, dtype=torch.float32, device=dev)
+    if per_tensor:
+        rx = torch.zeros(4, dtype=torch.float32, device=dev)
+        rw = torch.zeros(4, dtype=torch.float32, device=dev)
+        sq.sq_ln_quant_act_tensor(h_s, xq, sx, rx[:1], gamma, beta)
+        sq.sq_quantize_weight_tensor(w, wq, sw, rw[:1])
+    else:
+        sq.sq_ln_quant_act(h_s, xq, sx, gamma, beta)
+        sq.sq_quantize_weight(w, wq, sw)
+    y = torch.empty((m, N), dtype=torch.float16, device=dev)
+    sq.sq_w8a8_linear(xq, sx, wq, sw, y, bias, workspace=sq.new_workspace(m, N, K, device=dev))
+    return y
+
+
+def rel_err(torch, y, Y64):
+    return float(torch.linalg.norm(y.double() - Y64) / torch.linalg.norm(Y64))
+
+
+def quality_of(sq, torch, y_sq, h_s, w, gamma, beta, bias, eps=1e-5):
+    """Relative Frobenius error against the unquantized fp64 X W^T (+ b) of the SmoothQuant
+    output y_sq and of the two unsmoothed W8A8 baselines, on the same sampled token rows."""
+    X64 = layernorm_fp64(torch, h_s, gamma, beta, float(np.float32(eps))) if gamma is not None else h_s.double()
+    Y64 = product_fp64(torch, X64, w, bias)
+    out = {"e_sq": rel_err(torch, y_sq, Y64),
+           "e_naive_per_tensor": rel_err(torch, unsmoothed_w8a8(sq, torch, h_s, w, gamma, beta, bias, True), Y64),
+           "e_per_token_per_channel": rel_err(torch, unsmoothed_w8a8(sq, torch, h_s, w, gamma, beta, bias, False),
+                                              Y64)}
+    return {k: round(v, 6) for k, v in out.items()}
+
+
+def sample_rows(M, m):
+    return np.unique(np.linspace(0, M - 1, min(m, M)).astype(np.int64))
+
+
+def run_quality(plan, sq, torch, m=128):
+    """Quality of the step's own output on the step's workload (sampled token rows x all N)."""
+    idx = sample_rows(plan.M, m)
+    it = torch.from_numpy(idx).to(plan.h.device)
+    q = quality_of(sq, torch, plan.y.index_select(0, it), plan.h.index_select(0, it).contiguous(), plan.w,
+                   plan.gamma, plan.beta, plan.bias)
+    q.update({"rows": f"{idx.size} of {plan.M} tokens (evenly spaced) x all {plan.wl.N} outputs",
+              "alpha": plan.wl.alpha, "reference": "fp64 X W^T (+ b), X the fp64 LayerNorm of h where the "
+              "workload has one", "metric": "||y - Y64||_F / ||Y64||_F",
+              "naive_per_tensor": "no smoothing; one scale for all of X (dynamic) and one for all of W",
+              "per_token_per_channel": "no smoothing; one scale per token and per output channel"})
+    return q
+
+
+def run_quality_sweep(sq, torch, device, alphas, m=64, name="ffn_down"):
+    """The alpha sweep on an outlier workload: for each alpha a SmoothQuantLinear built from the
+    full weight and calibration set, run on sampled token rows; the unsmoothed baselines once."""
+    wl = sq_inputs.WORKLOADS[name]
+    T = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    w, calib = T(sq_inputs.weight(wl)), T(sq_inputs.calib_rows(wl))
+    h_s = T(sq_inputs.run_rows(wl, 0, m))
+    g, b, bias = T(sq_inputs.gamma(wl)), T(sq_inputs.beta(wl)), T(sq_inputs.bias(wl))
+    X64 = layernorm_fp64(torch, h_s, g, b, float(np.float32(1e-5))) if g is not None else h_s.double()
+    Y64 = product_fp64(torch, X64, w, bias)
+    base = {"e_naive_per_tensor": round(rel_err(torch, unsmoothed_w8a8(sq, torch, h_s, w, g, b, bias, True), Y64), 6),
+            "e_per_token_per_channel": round(rel_err(torch, unsmoothed_w8a8(sq, torch, h_s, w, g, b, bias, False),
+                                                     Y64), 6)}
+    sweep = []
+    for a in alphas:
+        layer = sq.SmoothQuantLinear.from_float(w, calib, float(a), g, b, bias)
+        sweep.append({"alpha": a, "e_sq": round(rel_err(torch, layer(h_s), Y64), 6)})
+        del layer
+    torch.cuda.synchronize()
+    if sq.sq_poll_status() != 0:
+        raise RuntimeError("device wait timed out in the quality sweep")
+    del w, calib
+    torch.cuda.empty_cache()
+    return {"workload": DESCR[name], "rows": f"the first {m} of {wl.M} tokens x all {wl.N} outputs", **base,
+            "sweep": sweep}
+
+
+def run_e2e_forward(plan, sq, torch, world, steps, dist):
+    """The forward through the public API with the layer resident: every step copies that
+    step's tokens h from pinned host memory, runs SmoothQuantLinear.forward (LayerNorm /
+    per-token quantization + INT8 GEMM) and copies y back to pinned host memory, all inside
+    the timed events; consecutive steps alternate between two streams."""
+    dev = plan.w.device
+    layer = sq.SmoothQuantLinear.from_float(plan.w, plan.calib, plan.wl.alpha, plan.gamma, plan.beta, plan.bias,
+                                            level=plan.level)
+    h_host = torch.from_numpy(np.ascontiguousarray(plan.host["h"])).pin_memory()
+    y_host = [torch.empty(tuple(plan.y.shape), dtype=torch.float16).pin_memory() for _ in range(2)]
+    streams = [torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)]
+    h_dev = [torch.empty_like(h_host, device=dev) for _ in range(2)]
+    y_dev = [torch.empty(tuple(plan.y.shape), dtype=torch.float16, device=dev) for _ in range(2)]
+
+    def one(i):
+        j = i % 2
+        with torch.cuda.stream(streams[j]):
+            h_dev[j].copy_(h_host, non_blocking=True)
+            layer(h_dev[j], y_dev[j])
+            y_host[j].copy_(y_dev[j], non_blocking=True)
+
+    for i in range(4):
+        one(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    main = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    for st in streams:
+        st.wait_stream(main)
+    for i in range(steps):
+        one(i)
+    for st in streams:
+        main.wait_stream(st)
+    e1.record(main)
+    e1.synchronize()
+    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    M, N, K = plan.M, plan.wl.N, plan.wl.K
+    ops = 2 * M * N * K
+    fb = M * K * 2 + M * N * 2
+    if M <= DECODE_M:
+        v, u = world * (M * K * 3 + N * K + 2 * M * N) * steps / (ms * 1e-3) / 1e9, "GB/s"
+    else:
+        v, u = world * ops * steps / (ms * 1e-3) / 1e12, "TOPS"
+    return {"value": round(v, 3), "unit": u, "h2d_bytes_per_step": int(M * K * 2),
+            "d2h_bytes_per_step": int(M * N * 2), "steps": steps, "ms_per_step": round(ms / steps, 4),
+            "api": "SmoothQuantLinear.forward with the quantized layer resident on the device; h in and y out "
+                   "over pinned host memory inside the timed region; consecutive steps on two streams",
+            "pcie_bytes_per_step": fb}
 
 
 def run_e2e(plan, sq, torch, world, allreduce, steps, dist):
@@ -1008,7 +1346,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return None
-    wl = sq_inputs.WORKLOADS[args.workload]
+    wl = workload_of(args)
     M = args.m if args.m else wl.M
     per_step = max(0.02, min(10.0, args.ref_budget / max(1, args.steps + args.warmup)))
     c_s, n_s, m_s = pick_sample(wl, M, per_step, args.level)
@@ -1033,10 +1371,8 @@ def run_reference(args):
             "warmup": args.warmup, "ms_per_step": round(full * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": DESCR[args.workload] + ("" if M == wl.M else f" (M={M})"), "M": M,
-                       "N": wl.N, "K": wl.K, "calib_tokens": wl.calib, "alpha": wl.alpha,
-                       "level": args.level, "granularity": LEVEL_DESCR[args.level], "step": STEP,
-                       "parallelism": "cpu oracle, rank 0"},
+            "config": common_config(args, wl, M, world),
+            "run": {"where": "CPU oracle on the host cores, rank 0 only"},
             "cpu_baseline": {"value": round(v, 6), "unit": u, "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(v, 6), "unit": u, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -1053,6 +1389,11 @@ def main():
     ap.add_argument("--m", type=int, default=0, help="token count override (decode sweep)")
     ap.add_argument("--level", choices=["channel", "O1", "O2", "O3"], default="channel",
                     help="scale granularities (default: per-token activations, per-channel weights)")
+    ap.add_argument("--alpha", type=float, default=None, help="override the workload's smoothing alpha")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the forward, decode-sweep and quality records (N = 1 only anyway)")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode sweep record")
+    ap.add_argument("--no-quality-sweep", action="store_true", help="skip the FFN-down alpha sweep")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--stage-steps", type=int, default=300, help="steps of the per-stage timing loop")

@@ -100,12 +100,22 @@ int sq_abi_version(void);
  * LayerNorm output is what feeds the linear), and on W [N, K] (ln_gamma NULL)
  * to get b.
  *   x           fp16 [rows, ld], first K columns used
- *   amax_inout  fp32 [K]; the caller zero-fills it before the first batch;
- *               max is exact, so the result does not depend on call order
+ *   amax_inout  fp32 [K]; zero-filled before the first batch (by the caller
+ *               or sq_calibrate_reset); max is exact, so the result does not
+ *               depend on call order
  */
 sq_status sq_calibrate_absmax(const void* x_f16, int64_t rows, int64_t K, int64_t ld,
                               const float* ln_gamma, const float* ln_beta, float ln_eps,
                               float* amax_inout, sq_stream_t stream);
+
+/*
+ * The start of a calibration run: amax[0 .. n) = 0 (one or several running
+ * maxima laid out back to back), on `stream`, ordered with the kernels
+ * before and after it like every other call -- the zero-fill that
+ * sq_calibrate_absmax expects before its first batch.
+ *   amax fp32 [n], n >= 1
+ */
+sq_status sq_calibrate_reset(float* amax, int64_t n, sq_stream_t stream);
 
 /*
  * Smoothing factor and offline fold (step 2).
@@ -284,8 +294,8 @@ sq_status sq_w8a8_linear(const int8_t* xq, const float* x_scale, const int8_t* w
  * the next sq_w8a8_linear directly: the fp16 y never reaches memory (1 byte
  * written per output instead of 2 written + 3 moved by a separate
  * quantization pass).  range_next is the next linear's static input range
- * (sq_tensor_range).  A per-token dynamic scale cannot be fused this way:
- * a token's maximum spans every output tile of its row.
+ * (sq_tensor_range).  For the per-token dynamic scale of the next linear
+ * see sq_w8a8_linear_quant_dyn.
  *   xq int8 [M, K]; x_scale fp32 [M]; wq int8 [N, K]; w_scale fp32 [N];
  *   bias fp16 [N] or NULL; inv_s_next fp32 [N] or NULL; range_next fp32 [1];
  *   xq_next int8 [M, N]; x_scale_next fp32 [M].  N % 16 == 0 (the next
@@ -296,6 +306,43 @@ sq_status sq_w8a8_linear_quant(const int8_t* xq, const float* x_scale, const int
                                const float* inv_s_next, const float* range_next, int8_t* xq_next,
                                float* x_scale_next, int64_t M, int64_t N, int64_t K, void* workspace,
                                size_t ws_bytes, sq_stream_t stream);
+
+/*
+ * Producer-side quantization at the next linear's per-token dynamic scale:
+ * the linear, an optional ReLU and the next linear's 1/s, then the next
+ * linear's default input quantization -- one scale per token, taken from the
+ * token's own maximum (the smoothing of the next linear folded into the
+ * layer that produces its input: section "what it does mathematically"; the
+ * per-token dynamic activation scale: section "inference", level O1).  Per
+ * element, in this order:
+ *   y = fp16( (fp32(acc) * x_scale[t]) * w_scale[n] + fp32(bias[n]) )  (as sq_w8a8_linear)
+ *   a = relu ? max(y, 0) : y                     (a NaN becomes 0)
+ *   x = fp32(a) * inv_s_next[n]                  (x = a when inv_s_next is NULL)
+ *   x_scale_next[t] = max_n |x[t, n]| / 127      (NaN ignored, as in sq_ln_quant_act)
+ *   xq_next[t, n]   = clamp(rint(x * (1 / x_scale_next[t])), -127, 127)
+ * -- exactly sq_w8a8_linear, the ReLU, then sq_ln_quant_act with inv_s.  A
+ * token's maximum spans every output tile of its row, so the work runs in
+ * two launches: the GEMM's epilogue writes a (fp16, into the workspace) and,
+ * per token, the maxima of |x| over groups of its columns; a second kernel
+ * takes each token's maximum of its groups and writes the codes (no row
+ * reduction over the data, no second GEMM).
+ *   xq int8 [M, K]; x_scale fp32 [M]; wq int8 [N, K]; w_scale fp32 [N];
+ *   bias fp16 [N] or NULL; inv_s_next fp32 [N] or NULL;
+ *   xq_next int8 [M, N]; x_scale_next fp32 [M]; N % 16 == 0 (the next
+ *   linear's K).  workspace: at least
+ *   sq_w8a8_linear_quant_dyn_workspace_bytes(M, N, K) bytes, 16-byte
+ *   aligned, zero-filled by the caller once before its first use (for
+ *   M <= SQ_DECODE_MAX_M it starts with the stream-K arrival counters, which
+ *   every completed call leaves at zero; after a call that reported
+ *   SQ_ERR_TIMEOUT zero-fill it again).  Calls sharing a workspace must not
+ *   overlap on the GPU.
+ */
+size_t sq_w8a8_linear_quant_dyn_workspace_bytes(int64_t M, int64_t N, int64_t K);
+sq_status sq_w8a8_linear_quant_dyn(const int8_t* xq, const float* x_scale, const int8_t* wq,
+                                   const float* w_scale, const void* bias_f16, int relu,
+                                   const float* inv_s_next, int8_t* xq_next, float* x_scale_next,
+                                   int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes,
+                                   sq_stream_t stream);
 
 /*
  * INT8 BMM (the explainer, section "inference": after smoothing, the linear

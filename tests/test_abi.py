@@ -40,7 +40,7 @@ def test_status_strings():
     assert L.sq_status_string(0) == b"SQ_OK"
     assert L.sq_status_string(8) == b"SQ_ERR_TIMEOUT"
     assert L.sq_status_string(99) == b"SQ_ERR_UNKNOWN"
-    assert L.sq_abi_version() == 104
+    assert L.sq_abi_version() == 105
 
 
 FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
@@ -66,6 +66,26 @@ def test_linear_rejects_bad_arguments_on_the_host():
     # unknown path
     assert L.sq_w8a8_linear_path(FAKE, FAKE, FAKE, FAKE, None, FAKE, 8, 64, 64, FAKE, 1 << 20, 7, None) == 1
     del ok
+
+
+def test_dynamic_producer_rejects_bad_arguments_on_the_host():
+    L = _lib()
+    f = L.sq_w8a8_linear_quant_dyn
+    big = 1 << 30
+    # no workspace / null operand
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 0, None, FAKE, FAKE, 64, 64, 64, None, big, None) == 1
+    assert f(None, FAKE, FAKE, FAKE, None, 0, None, FAKE, FAKE, 64, 64, 64, FAKE, big, None) == 1
+    # N (the next linear's K) must be a multiple of 16; K as everywhere
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 0, None, FAKE, FAKE, 64, 40, 64, FAKE, big, None) == 3
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 0, None, FAKE, FAKE, 64, 64, 40, FAKE, big, None) == 3
+    # misaligned workspace or 1/s
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 0, None, FAKE, FAKE, 64, 64, 64, FAKE_ODD, big, None) == 2
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 0, FAKE_ODD, FAKE, FAKE, 64, 64, 64, FAKE, big, None) == 2
+    # the workspace query: a fp16 copy of the output and the row-group maxima (more for decode)
+    ws = L.sq_w8a8_linear_quant_dyn_workspace_bytes
+    assert ws(300, 4096, 4096) >= 300 * 4096 * 2 + 300 * 32 * 4
+    assert ws(16, 4096, 4096) > 16 * 4096 * 2 + 16 * 128 * 4
+    assert ws(0, 64, 64) == 0 and ws(4, 64, -1) == 0
 
 
 def test_other_entry_points_reject_bad_arguments():

@@ -55,6 +55,23 @@ def test_calibrate_absmax_layernorm(sq, rows, K):
     assert bits_equal(host(amax), oracle.calibrate_absmax(h, gamma=g, beta=b))
 
 
+@pytest.mark.parametrize("n", [1, 300, 3 * 4096])
+def test_calibrate_reset_starts_a_new_run(sq, n):
+    """sq_calibrate_reset zeroes stale maxima (several ranges back to back), so the next
+    calibration equals one from a zero-filled buffer."""
+    rng = np.random.default_rng(n)
+    amax = dev(rng.uniform(10, 100, n).astype(np.float32))
+    sq.sq_calibrate_reset(amax)
+    assert not host(amax).any()
+    if n < 16:
+        return
+    K = 16 * (n // 16)
+    x = rand_h(rng, 33, K)
+    sq.sq_calibrate_absmax(dev(x), amax[:K])
+    assert bits_equal(host(amax)[:K], oracle.calibrate_absmax(x))
+    assert not host(amax)[K:].any()
+
+
 def test_calibrate_strided_rows(sq):
     rng = np.random.default_rng(3)
     full = rand_h(rng, 40, 320)

@@ -75,3 +75,35 @@ def test_two_rank_tensor_parallel_equals_unsharded():
         assert np.array_equal(y_col.view(np.uint16), ref["y"].view(np.uint16))
         assert np.array_equal(sw, ref2["sw"])  # the weight scales span every input channel
         assert np.array_equal(y_row.view(np.uint16), ref2["y"].view(np.uint16))
+
+
+def _worker_k_overflow(rank, world, port, out):
+    import torch
+
+    from tp_oracle_ops import OracleOps
+    from w8a8_int8_linear_channel_b200 import MAX_K
+    from w8a8_int8_linear_channel_b200.tp import DistComm, RowParallelSmoothQuantLinear
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    k_rank = (MAX_K // 2 // 16 + 2) * 16  # each slice fits, their sum does not
+    assert k_rank <= MAX_K < world * k_rank
+    w = torch.zeros((1, k_rank), dtype=torch.float16)
+    try:
+        RowParallelSmoothQuantLinear.from_float(w, w.clone(), 0.5, ops=OracleOps(), comm=DistComm())
+        out[rank] = "no error"
+    except ValueError as e:
+        out[rank] = str(e)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_row_parallel_rejects_total_k_beyond_int32_bound():
+    """Each rank's K slice is within MAX_K but their sum is not: every rank refuses before any
+    compute, since the summed int32 accumulators could wrap."""
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_worker_k_overflow, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
+    for r in range(world):
+        assert "exceeds" in out[r], out[r]

@@ -23,11 +23,12 @@ from typing import Optional
 import torch
 
 __all__ = [
-    "SQError", "sq_calibrate_absmax", "sq_smooth_fold", "sq_quantize_weight", "sq_ln_quant_act",
+    "SQError", "sq_calibrate_absmax", "sq_calibrate_reset", "sq_smooth_fold", "sq_quantize_weight", "sq_ln_quant_act",
     "sq_w8a8_workspace_bytes", "sq_w8a8_linear", "sq_w8a8_linear_path", "sq_w8a8_gemm_s32",
     "sq_poll_status", "sq_set_wait_budget_ns", "sq_selftest_wait_timeout", "SmoothQuantLinear",
     "sq_quantize_weight_tensor", "sq_ln_quant_act_tensor", "sq_ln_quant_act_static", "sq_tensor_range",
-    "LEVELS", "sq_w8a8_linear_quant", "sq_w8a8_bmm", "sq_row_ranges", "sq_quantize_rows_ranged",
+    "LEVELS", "sq_w8a8_linear_quant", "sq_w8a8_linear_quant_dyn", "sq_w8a8_linear_quant_dyn_workspace_bytes",
+    "new_quant_dyn_workspace", "sq_w8a8_bmm", "sq_row_ranges", "sq_quantize_rows_ranged",
     "sq_dequant",
     "PATH_AUTO", "PATH_TILED", "PATH_SPLITK", "PATH_PAIR", "PATH_WIDE", "SPLITK_MAX_M", "DECODE_MAX_M", "MAX_K", "library_path",
 ]
@@ -60,6 +61,7 @@ def _load() -> ctypes.CDLL:
         "sq_status_string": ([S], ctypes.c_char_p),
         "sq_abi_version": ([], S),
         "sq_calibrate_absmax": ([P, I, I, I, P, P, F, P, P], S),
+        "sq_calibrate_reset": ([P, I, P], S),
         "sq_smooth_fold": ([P, P, I, F, P, P, P, P, P, P, P, P, I, P], S),
         "sq_quantize_weight": ([P, I, I, P, P, P, P], S),
         "sq_ln_quant_act": ([P, I, I, I, P, P, P, F, P, P, P], S),
@@ -73,6 +75,8 @@ def _load() -> ctypes.CDLL:
         "sq_w8a8_gemm_s32": ([P, P, P, I, I, I, P, Z, S, P], S),
         "sq_w8a8_linear_noalloc": ([P, P, P, P, P, P, I, I, I, P], S),
         "sq_w8a8_linear_quant": ([P, P, P, P, P, S, P, P, P, P, I, I, I, P, Z, P], S),
+        "sq_w8a8_linear_quant_dyn_workspace_bytes": ([I, I, I], Z),
+        "sq_w8a8_linear_quant_dyn": ([P, P, P, P, P, S, P, P, P, I, I, I, P, Z, P], S),
         "sq_w8a8_bmm": ([P, P, P, P, P, I, I, I, I, P], S),
         "sq_row_ranges": ([P, I, I, I, P, P, P, P, F, P, P], S),
         "sq_quantize_rows_ranged": ([P, I, I, I, P, P, P, P, F, P, P, P, P], S),
@@ -146,6 +150,14 @@ def sq_calibrate_absmax(x: torch.Tensor, amax: torch.Tensor, gamma=None, beta=No
     _vec(beta, K, torch.float32, "beta")
     _check(_L.sq_calibrate_absmax(_p(x), rows, K, ld, _p(gamma), _p(beta), eps, _p(amax),
                                   _stream(stream)), "sq_calibrate_absmax")
+    return amax
+
+
+def sq_calibrate_reset(amax: torch.Tensor, stream=None) -> torch.Tensor:
+    """Start a calibration run: every running maximum in amax (fp32, contiguous) back to 0."""
+    if amax.dtype != torch.float32 or not amax.is_contiguous() or amax.numel() < 1:
+        raise ValueError("amax: need a contiguous fp32 tensor")
+    _check(_L.sq_calibrate_reset(_p(amax), amax.numel(), _stream(stream)), "sq_calibrate_reset")
     return amax
 
 
@@ -311,6 +323,38 @@ def sq_w8a8_linear_quant(xq, x_scale, wq, w_scale, range_next, xq_next, x_scale_
     return xq_next, x_scale_next
 
 
+def sq_w8a8_linear_quant_dyn_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_L.sq_w8a8_linear_quant_dyn_workspace_bytes(M, N, K))
+
+
+def new_quant_dyn_workspace(M: int, N: int, K: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace for sq_w8a8_linear_quant_dyn."""
+    return torch.zeros(sq_w8a8_linear_quant_dyn_workspace_bytes(M, N, K), dtype=torch.uint8,
+                       device=device or "cuda")
+
+
+def sq_w8a8_linear_quant_dyn(xq, x_scale, wq, w_scale, xq_next, x_scale_next, bias=None, relu: bool = False,
+                             inv_s_next=None, workspace=None, stream=None):
+    """The linear with the next linear's per-token dynamic input quantization: optional ReLU,
+    times inv_s_next, per-token scale x_scale_next [M] = max |x| / 127 and INT8 codes
+    xq_next [M, N] (two launches: the GEMM with a row-maximum epilogue, then the codes)."""
+    M, N, K = _gemm_shapes(xq, wq)
+    _vec(x_scale, M, torch.float32, "x_scale")
+    _vec(w_scale, N, torch.float32, "w_scale")
+    _vec(bias, N, torch.float16, "bias")
+    _vec(inv_s_next, N, torch.float32, "inv_s_next")
+    _vec(x_scale_next, M, torch.float32, "x_scale_next")
+    if xq_next.dtype != torch.int8 or tuple(xq_next.shape) != (M, N) or not xq_next.is_contiguous():
+        raise ValueError("xq_next: need a contiguous int8 [M, N] tensor")
+    if workspace is None:
+        workspace = new_quant_dyn_workspace(M, N, K, device=xq.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_L.sq_w8a8_linear_quant_dyn(_p(xq), _p(x_scale), _p(wq), _p(w_scale), _p(bias), int(bool(relu)),
+                                       _p(inv_s_next), _p(xq_next), _p(x_scale_next), M, N, K, _p(workspace),
+                                       ws_bytes, _stream(stream)), "sq_w8a8_linear_quant_dyn")
+    return xq_next, x_scale_next
+
+
 def sq_row_ranges(x, range_out, gamma=None, beta=None, inv_s=None, s_fold=None, eps: float = 1e-5,
                   stream=None):
     """range_out[r] = max |x_hat[r, :]| over this slice's columns (activation transform, or the
@@ -389,7 +433,9 @@ def sq_w8a8_linear_noalloc(xq, x_scale, wq, w_scale, y, bias=None, stream=None):
 
 
 def sq_poll_status(stream=None) -> int:
-    """Synchronize the stream; return the status code of the device's bounded waits (and clear it)."""
+    """Synchronize the stream; return the status code of the device's bounded waits (and clear it).
+    After SQ_ERR_TIMEOUT (8), zero-fill the stream-K workspaces used by the timed-out calls
+    (SmoothQuantLinear.reset_workspaces for a layer's own)."""
     return int(_L.sq_poll_status(_stream(stream)))
 
 
@@ -509,6 +555,14 @@ class SmoothQuantLinear:
             ws = torch.zeros(need, dtype=torch.uint8, device=self.wq.device)
             self._ws[key] = ws
         return ws
+
+    def reset_workspaces(self) -> None:
+        """Zero-fill every stream-K workspace the layer holds.  Needed after a forward whose
+        bounded device wait ran out (sq_poll_status returned SQ_ERR_TIMEOUT): that call may
+        leave per-tile arrival counters non-zero, and a later decode-sized forward on the same
+        stream would then elect the wrong last contributor."""
+        for ws in self._ws.values():
+            ws.zero_()
 
     def quantize_input(self, h: torch.Tensor, xq=None, x_scale=None):
         M, K = h.shape

@@ -194,7 +194,22 @@ __global__ void __launch_bounds__(256) k_dequant(const int32_t* __restrict__ acc
   }
 }
 
+// The start of a calibration run: every running maximum back to 0.
+__global__ void __launch_bounds__(256) k_calib_reset(float* __restrict__ amax, int64_t n) {
+  griddep_wait();  // an earlier kernel may still read the previous ranges
+  griddep_launch_dependents();
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    amax[i] = 0.0f;
+}
+
 }  // namespace
+
+cudaError_t launch_calib_reset(float* amax, int64_t n, const Ctx& c) {
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > c.num_sms) blocks = c.num_sms;
+  return launch_pdl(k_calib_reset, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, c.stream, amax, n);
+}
 
 cudaError_t launch_dequant(const int32_t* acc, const float* sx, const float* sw, const __half* bias, __half* y,
                            int64_t M, int64_t N, const Ctx& c) {

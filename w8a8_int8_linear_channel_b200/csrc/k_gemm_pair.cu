@@ -23,7 +23,9 @@
 //               y = fp16((acc * sx[t]) * sw[n] + bias[n]) and writes 32 x 32
 //               blocks through shared memory with TMA stores -- or, for
 //               producer-side quantization, turns y into the next linear's
-//               INT8 codes at its static scale and writes 32 bytes per row
+//               INT8 codes at its static scale and writes 32 bytes per row,
+//               or (per-token scale) writes fp16 y after the ReLU and each
+//               row's maximum of |y * inv_s_next| over its 128 columns
 // Every mbarrier wait is bounded; a wait that runs out records a timeout,
 // tells the other CTA of the pair to stop, and both CTAs drain what they
 // issued, free TMEM and return.
@@ -71,8 +73,11 @@ constexpr size_t SMEM = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
 static_assert(SMEM <= 232448, "shared memory per CTA");
 constexpr uint32_t TMEM_COLS = 512;
 
-// What the epilogue writes (EPI_BMM: fp16 y of a batched GEMM, 3-D maps).
-enum Epi { EPI_F16 = 0, EPI_I32 = 1, EPI_Q8 = 2, EPI_BMM = 3 };
+// What the epilogue writes (EPI_BMM: fp16 y of a batched GEMM, 3-D maps;
+// EPI_QD: the first phase of the per-token producer-side quantization, fp16
+// a = y (ReLU if asked) plus per-row maxima of |a * inv_s_next| per 128
+// columns).
+enum Epi { EPI_F16 = 0, EPI_I32 = 1, EPI_Q8 = 2, EPI_BMM = 3, EPI_QD = 4 };
 
 // Tile t -> (token tile, channel tile), grouped: groups of kGroupM token
 // tiles walk every channel tile, token tile fastest.  The 74 tiles in flight
@@ -327,6 +332,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (decision[tl & 1]) break;
       tc_fence_after();
 
+      float pmax = 0.0f;  // EPI_QD: this lane's row maximum over the warp's 128 columns
       auto taddr = [&](int c) {
         return tmem + (static_cast<uint32_t>(32 * q) << 16) +
                static_cast<uint32_t>(BN * b + 128 * half + 32 * c);
@@ -444,6 +450,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               *reinterpret_cast<__half2*>(&h[j + 2 * u]) = __floats2half2_rn(f.x, f.y);
             }
           }
+          if constexpr (EPI == EPI_QD) {
+            // a = relu ? max(y, 0) : y on half2 (a NaN becomes 0, as in the
+            // scalar y > 0 ? y : 0), and this row's running maximum of
+            // |fp32(a) * inv_s_next[n]| (NaN-free: fmaxf drops a NaN); the
+            // 1/s of these 32 columns are the same for every lane (broadcast
+            // loads), columns past N contribute 0
+            const __half2 zero2 = __float2half2_rn(0.0f);
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              __half2* h2 = reinterpret_cast<__half2*>(&h[j]);
+              if (g.relu) {
+                h2[0] = __hmax2(h2[0], zero2);
+                h2[1] = __hmax2(h2[1], zero2);
+              }
+              float4 is = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+              if (col0 + j >= g.N) is = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+              else if (g.inv_s_next != nullptr) is = __ldg(reinterpret_cast<const float4*>(g.inv_s_next + col0 + j));
+              const float2 a01 = __half22float2(h2[0]), a23 = __half22float2(h2[1]);
+              pmax = fmaxf(pmax, fabsf(__fmul_rn(a01.x, is.x)));
+              pmax = fmaxf(pmax, fabsf(__fmul_rn(a01.y, is.y)));
+              pmax = fmaxf(pmax, fabsf(__fmul_rn(a23.x, is.z)));
+              pmax = fmaxf(pmax, fabsf(__fmul_rn(a23.y, is.w)));
+            }
+          }
           if constexpr (TMAS) {
             // stage the 32 x 32 block in the 64-byte-swizzled image; one TMA
             // store writes it (rows/columns outside y are skipped); two buffers
@@ -491,6 +521,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       emit(2, va);
       tmem_ld_wait_regs(vb);
       emit(3, vb);
+      if constexpr (EPI == EPI_QD) {
+        const int64_t row = row0 + lane;
+        // every group of the row is written (a group wholly past N holds 0), so the
+        // codes pass never reads a stale maximum
+        if (row < g.M) g.part[row * g.part_n + 2 * tn + half] = pmax;
+      }
       // every epilogue thread of this CTA has read accumulator b: tell the leader
       tc_fence_before();
       named_bar_sync(1, 32 * kEpiWarps);
@@ -603,7 +639,7 @@ cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
   // TMA stores of fp16 y need 16-byte row strides (N % 8 == 0); otherwise
   // row-by-row stores through the staging (always for int32 accumulators;
   // int8 codes are written 32 bytes per row)
-  const bool tma_store = (EPI == EPI_F16 || bmm) && g.N % 8 == 0;
+  const bool tma_store = (EPI == EPI_F16 || EPI == EPI_QD || bmm) && g.N % 8 == 0;
   if (tma_store) {
     const bool ok = bmm ? make_tmap_f16_out_3d(&tmY, g.y, g.N, g.M, items) : make_tmap_f16_out(&tmY, g.y, g.N, g.M);
     if (!ok) return cudaErrorInvalidValue;
@@ -617,11 +653,16 @@ cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
   const int tiles = static_cast<int>(tiles64);
   const int mp = max_pairs(c.device, c.num_sms);
   const int pairs = tiles < mp ? tiles : mp;
-  if (tma_store) {
-    if constexpr (EPI == EPI_F16 || EPI == EPI_BMM)
-      return launch_ring<EPI, true>(g, c, tmA, tmB, tmY, tiles_m, tiles, pairs);
+  if constexpr (EPI == EPI_QD) {  // N % 16 == 0 here: always TMA stores
+    if (!tma_store) return cudaErrorInvalidValue;
+    return launch_ring<EPI, true>(g, c, tmA, tmB, tmY, tiles_m, tiles, pairs);
+  } else {
+    if (tma_store) {
+      if constexpr (EPI == EPI_F16 || EPI == EPI_BMM)
+        return launch_ring<EPI, true>(g, c, tmA, tmB, tmY, tiles_m, tiles, pairs);
+    }
+    return launch_ring<EPI, false>(g, c, tmA, tmB, tmY, tiles_m, tiles, pairs);
   }
-  return launch_ring<EPI, false>(g, c, tmA, tmB, tmY, tiles_m, tiles, pairs);
 }
 
 }  // namespace
@@ -631,6 +672,7 @@ cudaError_t launch_bmm_pair(const GemmArgs& g, const Ctx& c) { return launch_cfg
 cudaError_t launch_gemm_pair(const GemmArgs& g, const Ctx& c) {
   if (g.acc != nullptr) return launch_cfg<EPI_I32>(g, c);
   if (g.q_next != nullptr) return launch_cfg<EPI_Q8>(g, c);
+  if (g.part != nullptr) return launch_cfg<EPI_QD>(g, c);
   return launch_cfg<EPI_F16>(g, c);
 }
 

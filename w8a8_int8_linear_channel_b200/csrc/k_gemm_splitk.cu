@@ -103,7 +103,10 @@ __device__ __forceinline__ void tmem_ld_tokens<128>(uint32_t taddr, uint32_t (&v
 }
 
 // EPI: 0 = fp16 y, 1 = int32 accumulators, 2 = the next linear's INT8 codes
-// at its static scale (producer-side quantization).
+// at its static scale (producer-side quantization), 3 = the first phase of
+// producer-side quantization at the next linear's per-token scale: fp16
+// a = y (ReLU if asked) and per token the maximum of |a * inv_s_next| over
+// each warp's 32 channels.
 template <int BT, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_splitk(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -325,7 +328,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (emit && n < g.N) {
+      if (EPI == 3 && emit) {
+        // a = relu ? max(y, 0) : y (a NaN becomes 0), written as fp16; per
+        // token the maximum of |fp32(a) * inv_s_next[n]| over this warp's 32
+        // channels (NaN-free; channels past N give 0) -> part[m][n / 32]
+        const bool in_n = n < g.N;
+        const float swn = in_n ? g.sw[n] : 0.0f;
+        const bool has_bias = g.bias != nullptr;
+        const float bn = (has_bias && in_n) ? __half2float(g.bias[n]) : 0.0f;
+        const float isn = !in_n ? 0.0f : g.inv_s_next != nullptr ? g.inv_s_next[n] : 1.0f;
+        const int64_t grp = (t * BW + 32 * q) / 32;
+#pragma unroll
+        for (int m = 0; m < BT; ++m) {
+          if (m < g.M) {  // warp-uniform
+            float f = dequant_f32(static_cast<int32_t>(v[m]), sx_s[m], swn);
+            if (has_bias) f = __fadd_rn(f, bn);
+            __half hv = __float2half_rn(f);
+            if (g.relu && !(__half2float(hv) > 0.0f)) hv = __float2half_rn(0.0f);
+            if (in_n) g.y[m * g.N + n] = hv;
+            float p = fabsf(__fmul_rn(__half2float(hv), isn));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) p = fmaxf(p, __shfl_xor_sync(0xffffffffu, p, o));
+            if (lane == 0 && grp < g.part_n) g.part[m * g.part_n + grp] = p;
+          }
+        }
+      } else if (emit && n < g.N) {
         if (OUT_I32) {
           for (int m = 0; m < BT; ++m)
             if (m < g.M) g.acc[m * g.N + n] = static_cast<int32_t>(v[m]);
@@ -446,7 +473,12 @@ size_t splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
 }
 
 cudaError_t launch_gemm_splitk(const GemmArgs& g, const Ctx& c) {
-  const int epi = g.acc != nullptr ? 1 : g.q_next != nullptr ? 2 : 0;
+  const int epi = g.acc != nullptr ? 1 : g.q_next != nullptr ? 2 : g.part != nullptr ? 3 : 0;
+  if (epi == 3) {  // per-token producer-side quantization: decode token counts only
+    if (g.M <= 16) return launch_bt<16, 3>(g, c);
+    if (g.M <= 32) return launch_bt<32, 3>(g, c);
+    return cudaErrorInvalidValue;
+  }
   if (g.M <= 16) return epi == 1 ? launch_bt<16, 1>(g, c) : epi == 2 ? launch_bt<16, 2>(g, c) : launch_bt<16, 0>(g, c);
   if (g.M <= 32) return epi == 1 ? launch_bt<32, 1>(g, c) : epi == 2 ? launch_bt<32, 2>(g, c) : launch_bt<32, 0>(g, c);
   if (g.M <= 64) return epi == 1 ? launch_bt<64, 1>(g, c) : epi == 2 ? launch_bt<64, 2>(g, c) : launch_bt<64, 0>(g, c);
@@ -516,10 +548,15 @@ cudaError_t noalloc_scratch(int dev, uint8_t** out) {
 template <int BT>
 cudaError_t launch_noalloc(const GemmArgs& g, const Ctx& c, uint8_t* scratch) {
   using L = SkLayout<BT>;
-  cudaError_t e = cudaFuncSetAttribute(k_gemm_splitk<BT, 0>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(L::SMEM));
-  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {false};  // once per device, as in launch_bt
+  const int dev = c.device < 64 ? c.device : 63;
+  cudaError_t e;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(k_gemm_splitk<BT, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(L::SMEM));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
   CUtensorMap tmW, tmX;
   if (!make_tmap_i8(&tmW, g.wq, g.K, g.N, BK, BW)) return cudaErrorInvalidValue;
   if (!make_tmap_i8(&tmX, g.xq, g.K, g.M, BK, BT)) return cudaErrorInvalidValue;

@@ -882,6 +882,367 @@ __global__ void __launch_bounds__(kCtaThreads) k_calib_cta_atomic(const RowArgs 
   cta_rows<MODE_CALIB, kCtaThreads, 0, false, 1>(a, sh, none);
 }
 
+// =========================================================================
+// LayerNorm / smoothing + per-token quantization, rows staged by bulk copies.
+//
+// One CTA of T threads per row, persistent over rows (grid-stride).  One
+// thread streams whole rows into a 2-slot shared-memory ring with untiled
+// bulk copies (cp.async.bulk, one instruction per row, completion counted on
+// an mbarrier), so each CTA has the next row in flight while it works on the
+// current one and no register holds prefetched data.  Every thread keeps its
+// NCH chunks of 8 values as fp32 in registers from the one read of shared
+// memory to the codes.  Per element:
+//   statistics  exact sums in fp64: h (a multiple of 2^-24, |h| < 2^16) adds
+//               exactly into one fp64 accumulator per thread; h*h (exact in
+//               fp64) is added to an accumulator biased by 1.5 * 2^43 (unit in
+//               the last place 2^-9, so every partial sum keeps that unit), and
+//               the part the add rounded away, t - ((A + t) - A), which is
+//               exact (Fast2Sum, |A| >= |t|), goes to a second accumulator in
+//               units of 2^-48.  Per thread the three sums become int64 and are
+//               reduced as integers: S1 = sum v and S2 = sum v^2 (v = h * 2^24)
+//               exactly, whatever the order.
+//   transform   ((x - mu) * rstd) * gamma + beta, times inv_s -- packed fp32
+//               pairs (each lane rounded like the scalar op, no FMA)
+//   maximum     three-input NaN-propagating max of absolute values
+//   codes       x * (1 / scale) + 1.5 * 2^23 in packed pairs, low bytes packed
+// Three block barriers per row with a LayerNorm (statistics, mu / rstd, row
+// maximum), one without.  Rows with a non-finite maximum take the NaN-free
+// maximum and the NaN-safe codes, as in the kernels above.  Every wait is
+// bounded; a wait that runs out stops the CTA uniformly (the decision rides on
+// the first barrier of the row), which then waits (bounded) for its copies in
+// flight before returning.
+// =========================================================================
+constexpr double kS2Bias = 13194139533312.0;  // 1.5 * 2^43: unit in the last place 2^-9
+
+__device__ __forceinline__ uint64_t f2_sub_rn(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ float absmax3(float m, float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(m), "f"(fabsf(a)), "f"(fabsf(b)));
+  return d;
+}
+
+__device__ __forceinline__ void bulk_row_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// Bounded wait that records nothing (the caller turns a time-out into a
+// CTA-wide decision at its next barrier).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > budget_ns) return false;
+  }
+  return true;
+}
+
+template <int T>
+struct ActShared {
+  long long s1[2][T / 32], s2h[2][T / 32], s2l[2][T / 32];
+  int bad[2][T / 32];
+  float mx[2][T / 32];
+  float mx2[2][T / 32];
+  float mu[2], rstd[2];
+  alignas(8) uint64_t full[2];
+};
+
+template <int T, int NCH>
+__global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* status, uint64_t budget) {
+  constexpr int W = T / 32;
+  __shared__ ActShared<T> sh;
+  extern __shared__ __align__(128) uint8_t ring[];  // 2 slots of one row (2K bytes each)
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t Kc = a.K >> 3;
+  const uint32_t row_bytes = static_cast<uint32_t>(a.K * 2);
+  const uint32_t slot0 = smem_u32(ring);
+  const uint32_t full0 = smem_u32(&sh.full[0]);
+  const bool use_ln = a.gamma != nullptr;
+  const int64_t G = gridDim.x;
+  if (tid == 0) {
+    mbar_init(full0, 1);
+    mbar_init(full0 + 8, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  griddep_wait();  // h (and gamma / beta / inv_s) come from earlier kernels
+  griddep_launch_dependents();
+
+  // thread 0: issue the copy of the row of iteration j into slot j & 1
+  int64_t issued = 0;  // iterations whose copy has been issued (thread 0)
+  auto issue = [&](int64_t j) {
+    const int64_t row = blockIdx.x + j * G;
+    if (row >= a.rows) return;
+    const uint32_t bar = full0 + 8u * static_cast<uint32_t>(j & 1);
+    mbar_arrive_expect_tx(bar, row_bytes);
+    bulk_row_load(slot0 + static_cast<uint32_t>(j & 1) * row_bytes, a.x + row * a.ld, row_bytes, bar);
+    issued = j + 1;
+  };
+  if (tid == 0) {
+    issue(0);
+    issue(1);
+  }
+  int64_t consumed = 0;  // iterations whose copy has landed
+  bool aborted = false;
+  int par = 0;
+  for (int64_t j = 0;; ++j, par ^= 1) {
+    const int64_t r = blockIdx.x + j * G;
+    if (r >= a.rows) break;
+    const uint32_t s = static_cast<uint32_t>(j & 1);
+    const bool ok = mbar_wait_bounded(full0 + 8u * s, static_cast<uint32_t>((j >> 1) & 1), budget);
+    float x[NCH][8];
+    const uint4* src = reinterpret_cast<const uint4*>(ring + s * row_bytes);
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int64_t c = tid + static_cast<int64_t>(i) * T;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (ok && c < Kc) v = src[c];
+      unpack8(v, x[i]);  // chunks past K are zeros
+    }
+
+    float mu = 0.0f, rstd = 0.0f;
+    bool stop;
+    if (use_ln) {
+      double s1 = 0.0, hi = kS2Bias, lo = 0.0;
+      int bad = 0;
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const double d = static_cast<double>(x[i][jj]);
+          s1 = __dadd_rn(s1, d);
+          const double t = __dmul_rn(d, d);
+          const double hn = __dadd_rn(hi, t);
+          lo = __dadd_rn(lo, __dsub_rn(t, __dsub_rn(hn, hi)));
+          hi = hn;
+        }
+      }
+      bad = !(fabs(s1) <= 1.7976931348623157e308) || !(hi <= 1.7976931348623157e308);
+      long long v1 = bad ? 0 : __double2ll_rn(__dmul_rn(s1, 16777216.0));               // units 2^-24
+      long long v2h = bad ? 0 : __double2ll_rn(__dmul_rn(__dsub_rn(hi, kS2Bias), 512.0));  // units 2^-9
+      long long v2l = bad ? 0 : __double2ll_rn(__dmul_rn(lo, 281474976710656.0));        // units 2^-48
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        v1 += __shfl_xor_sync(0xffffffffu, v1, o);
+        v2h += __shfl_xor_sync(0xffffffffu, v2h, o);
+        v2l += __shfl_xor_sync(0xffffffffu, v2l, o);
+      }
+      bad = __any_sync(0xffffffffu, bad);
+      if (lane == 0) {
+        sh.s1[par][warp] = v1;
+        sh.s2h[par][warp] = v2h;
+        sh.s2l[par][warp] = v2l;
+        sh.bad[par][warp] = bad;
+      }
+      stop = __syncthreads_or(!ok);  // every thread has read slot s
+      if (stop) {
+        aborted = true;
+        break;
+      }
+      consumed = j + 1;
+      if (tid == 0) issue(j + 2);
+      if (warp == 0) {
+        Sums t{0, 0, 0, 0};
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+          t.s1 += sh.s1[par][w];
+          t.s2h += sh.s2h[par][w] * 16;  // units 2^-13
+          t.s2l += sh.s2l[par][w];
+          t.bad |= sh.bad[par][w];
+        }
+        float m_, r_;
+        ln_finalize(t, a.K, a.eps, m_, r_);
+        if (lane == 0) {
+          sh.mu[par] = m_;
+          sh.rstd[par] = r_;
+        }
+      }
+      __syncthreads();
+      mu = sh.mu[par];
+      rstd = sh.rstd[par];
+    }
+
+    // transform in place and the row maximum (NaN-propagating)
+    float amax = 0.0f;
+    {
+      const uint64_t mu2 = f2_pack(mu, mu), r2 = f2_pack(rstd, rstd);
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        const int64_t c = tid + static_cast<int64_t>(i) * T;
+        if (c < Kc) {
+          const int64_t k0 = c * 8;
+          if (use_ln) {
+            const float4 g0 = __ldg(reinterpret_cast<const float4*>(a.gamma + k0));
+            const float4 g1 = __ldg(reinterpret_cast<const float4*>(a.gamma + k0) + 1);
+            const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+            float bb[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (a.beta) {
+              const float4 b0 = __ldg(reinterpret_cast<const float4*>(a.beta + k0));
+              const float4 b1 = __ldg(reinterpret_cast<const float4*>(a.beta + k0) + 1);
+              bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w;
+              bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
+            }
+#pragma unroll
+            for (int jj = 0; jj < 8; jj += 2) {
+              uint64_t v = f2_pack(x[i][jj], x[i][jj + 1]);
+              v = f2_mul_rn(f2_mul_rn(f2_sub_rn(v, mu2), r2), f2_pack(gg[jj], gg[jj + 1]));
+              if (a.beta) v = f2_add_rn(v, f2_pack(bb[jj], bb[jj + 1]));
+              const float2 f = f2_unpack(v);
+              x[i][jj] = f.x;
+              x[i][jj + 1] = f.y;
+            }
+          }
+          if (a.vec) {
+            const float4 i0 = __ldg(reinterpret_cast<const float4*>(a.vec + k0));
+            const float4 i1 = __ldg(reinterpret_cast<const float4*>(a.vec + k0) + 1);
+            const float is[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+#pragma unroll
+            for (int jj = 0; jj < 8; jj += 2) {
+              const float2 f = f2_unpack(f2_mul_rn(f2_pack(x[i][jj], x[i][jj + 1]), f2_pack(is[jj], is[jj + 1])));
+              x[i][jj] = f.x;
+              x[i][jj + 1] = f.y;
+            }
+          }
+#pragma unroll
+          for (int jj = 0; jj < 8; jj += 2) amax = absmax3(amax, x[i][jj], x[i][jj + 1]);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = absmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (lane == 0) sh.mx[par][warp] = amax;
+    if (use_ln) {
+      __syncthreads();
+    } else {
+      stop = __syncthreads_or(!ok);  // every thread has read slot s
+      if (stop) {
+        aborted = true;
+        break;
+      }
+      consumed = j + 1;
+      if (tid == 0) issue(j + 2);
+    }
+    float m = 0.0f;
+#pragma unroll
+    for (int w = 0; w < W; ++w) m = absmax_nan(m, sh.mx[par][w]);
+    const bool safe = !finite_f(m);  // CTA-uniform
+    if (safe) {  // a NaN or an Inf in the row: the range ignores NaN
+      float a2 = 0.0f;
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+        if (tid + static_cast<int64_t>(i) * T < Kc)
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) a2 = fmaxf(a2, fabsf(x[i][jj]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a2 = fmaxf(a2, __shfl_xor_sync(0xffffffffu, a2, o));
+      if (lane == 0) sh.mx2[par][warp] = a2;
+      __syncthreads();
+      m = 0.0f;
+#pragma unroll
+      for (int w = 0; w < W; ++w) m = fmaxf(m, sh.mx2[par][w]);
+    }
+    m = fabsf(m);
+    const float sc = __fdiv_rn(m, 127.0f);
+    const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+    if (tid == 0) a.scale[r] = sc;
+    int8_t* dst = a.q + r * a.K;
+    const uint64_t inv2 = f2_pack(inv, inv);
+    const uint64_t magic2 = f2_pack(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int64_t c = tid + static_cast<int64_t>(i) * T;
+      if (c < Kc) {
+        uint32_t b[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; jj += 2) {
+          const float2 f = f2_unpack(f2_add_rn(f2_mul_rn(f2_pack(x[i][jj], x[i][jj + 1]), inv2), magic2));
+          b[jj] = __float_as_uint(f.x);
+          b[jj + 1] = __float_as_uint(f.y);
+        }
+        if (safe) {
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) b[jj] = min(b[jj], 0x4B400100u);
+        }
+        const uint32_t lo4 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+        const uint32_t hi4 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+        *reinterpret_cast<uint2*>(dst + c * 8) = make_uint2(lo4, hi4);
+      }
+    }
+  }
+  if (aborted) {
+    if (tid == 0) {
+      atomicCAS(status, DEV_OK, DEV_TIMEOUT);
+      // wait (bounded) for the copies still in flight before shared memory is released
+      for (int64_t j = consumed; j < issued; ++j)
+        mbar_drain(full0 + 8u * static_cast<uint32_t>(j & 1), static_cast<uint32_t>((j >> 1) & 1), budget);
+    }
+    __syncthreads();
+  }
+}
+
+// =========================================================================
+// Second phase of producer-side quantization at the next linear's per-token
+// scale.  The producing GEMM wrote a = fp16 y (ReLU applied) and, per row,
+// the maxima of |fp32(a) * inv_s| over groups of columns; here a row's range
+// is the maximum of its groups (exact, order-free), and every element is
+// coded at that scale: x = fp32(a) * inv_s, q = code(x * (1 / scale)) -- the
+// same values and the same codes as the activation kernel's inv_s path.  A
+// warp per row, no block barrier; the codes go through the NaN-safe path
+// (a NaN x is coded 0; an Inf range gives scale Inf, reciprocal 0, codes 0).
+// =========================================================================
+constexpr int kQuantRowUnroll = 4;
+
+__global__ void __launch_bounds__(256) k_quant_partial_rows(const __half* a, int64_t M, int64_t N,
+                                                             const float* part, int64_t part_n,
+                                                             const float* inv_s, int8_t* q, float* scale) {
+  griddep_wait();  // a and the partial maxima come from the GEMM just before
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t Nc = N >> 3;
+  for (int64_t r = wid; r < M; r += nwarps) {
+    float m = 0.0f;
+    for (int64_t i = lane; i < part_n; i += 32) m = fmaxf(m, __ldg(part + r * part_n + i));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float sc = __fdiv_rn(m, 127.0f);
+    const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+    if (lane == 0) scale[r] = sc;
+    const uint4* src = reinterpret_cast<const uint4*>(a + r * N);
+    uint2* dst = reinterpret_cast<uint2*>(q + r * N);
+    for (int64_t c0 = lane; c0 < Nc; c0 += 32 * kQuantRowUnroll) {
+      uint4 v[kQuantRowUnroll];
+#pragma unroll
+      for (int u = 0; u < kQuantRowUnroll; ++u) {
+        const int64_t c = c0 + 32 * u;
+        v[u] = c < Nc ? ld_stream(src + c) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kQuantRowUnroll; ++u) {
+        const int64_t c = c0 + 32 * u;
+        if (c < Nc) {
+          float x[8];
+          unpack8(v[u], x);
+          if (inv_s != nullptr) {
+            float is[8];
+            load8f(inv_s + c * 8, is);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(x[j], is[j]);
+          }
+          dst[c] = pack8<true>(x, inv);
+        }
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------- launch ----
 template <typename Kern>
 int occupancy(Kern k, int threads, size_t smem) {
@@ -965,7 +1326,54 @@ cudaError_t launch_calib_cta(const RowArgs& a, const Ctx& c) {
 
 }  // namespace
 
-cudaError_t launch_ln_quant_act(const RowArgs& a, const Ctx& c) { return launch_mode<MODE_ACT>(a, c); }
+template <int T, int NCH>
+cudaError_t launch_act_bulk(const RowArgs& a, const Ctx& c) {
+  static int occ[64] = {0};
+  static int64_t occ_bytes[64] = {0};
+  const int dev = c.device < 64 ? c.device : 63;
+  const size_t smem = static_cast<size_t>(a.K) * 4;  // two slots of one fp16 row
+  if (occ_bytes[dev] != static_cast<int64_t>(smem)) {
+    cudaError_t e = cudaFuncSetAttribute(k_act_rows_bulk<T, NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    occ[dev] = occupancy(k_act_rows_bulk<T, NCH>, T, smem);
+    occ_bytes[dev] = static_cast<int64_t>(smem);
+  }
+  int64_t grid = static_cast<int64_t>(c.num_sms) * occ[dev];
+  if (grid > a.rows) grid = a.rows;
+  return launch_pdl(k_act_rows_bulk<T, NCH>, dim3(static_cast<unsigned>(grid)), dim3(T), smem, c.stream, a,
+                    c.status, c.budget_ns);
+}
+
+cudaError_t launch_ln_quant_act(const RowArgs& a, const Ctx& c) {
+  // per-token dynamic scales with the row held in registers: rows staged by
+  // bulk copies (the other modes and shapes keep the kernels above)
+  const int64_t Kc = a.K / 8;
+  if (a.range_in == nullptr && a.range_out == nullptr && Kc > 128 && Kc <= 2048) {
+    if (Kc <= 256) return launch_act_bulk<128, 2>(a, c);
+    if (Kc <= 384) return launch_act_bulk<128, 3>(a, c);
+    if (Kc <= 512) return launch_act_bulk<128, 4>(a, c);
+    if (Kc <= 768) return launch_act_bulk<256, 3>(a, c);
+    if (Kc <= 1024) return launch_act_bulk<256, 4>(a, c);
+    if (Kc <= 1280) return launch_act_bulk<256, 5>(a, c);
+    if (Kc <= 1536) return launch_act_bulk<256, 6>(a, c);
+    if (Kc <= 1792) return launch_act_bulk<256, 7>(a, c);
+    return launch_act_bulk<256, 8>(a, c);
+  }
+  return launch_mode<MODE_ACT>(a, c);
+}
+
+cudaError_t launch_quant_partial_rows(const __half* a, int64_t M, int64_t N, const float* part, int64_t part_n,
+                                      const float* inv_s, int8_t* q, float* scale, const Ctx& c) {
+  static int occ[64] = {0};
+  const int dev = c.device < 64 ? c.device : 63;
+  if (occ[dev] == 0) occ[dev] = occupancy(k_quant_partial_rows, 256, 0);
+  int64_t grid = static_cast<int64_t>(c.num_sms) * occ[dev];
+  const int64_t need = (M + 7) / 8;  // 8 row-warps per CTA
+  if (grid > need) grid = need;
+  return launch_pdl(k_quant_partial_rows, dim3(static_cast<unsigned>(grid)), dim3(256), 0, c.stream, a, M, N, part,
+                    part_n, inv_s, q, scale);
+}
 
 cudaError_t launch_quantize_weight(const RowArgs& a, const Ctx& c) {
   return launch_mode<MODE_WEIGHT>(a, c);

@@ -283,7 +283,16 @@ const char* sq_status_string(int status) {
   }
 }
 
-int sq_abi_version(void) { return 104; }
+int sq_abi_version(void) { return 105; }
+
+sq_status sq_calibrate_reset(float* amax, int64_t n, sq_stream_t stream) {
+  if (!amax || n <= 0) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(amax)) return SQ_ERR_MISALIGNED;
+  Ctx ctx;
+  sq_status st = current_ctx(stream, &ctx);
+  if (st != SQ_OK) return st;
+  return launched(launch_calib_reset(amax, n, ctx));
+}
 
 sq_status sq_calibrate_absmax(const void* x_f16, int64_t rows, int64_t K, int64_t ld,
                               const float* ln_gamma, const float* ln_beta, float ln_eps,
@@ -536,6 +545,89 @@ sq_status sq_w8a8_linear_quant(const int8_t* xq, const float* x_scale, const int
     return launched(launch_gemm_splitk(g, ctx));
   }
   return launched(launch_gemm_pair(g, ctx));
+}
+
+namespace {
+
+// Workspace of the per-token producer-side quantization: [the stream-K
+// scratch for M <= SQ_DECODE_MAX_M] [a fp16 M x N] [row-group maxima fp32 M x part_n],
+// each piece 256-byte aligned.
+struct DynLayout {
+  size_t sk, a_off, part_off, total;
+  int64_t part_n;
+};
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+DynLayout dyn_layout(int64_t M, int64_t N, int64_t K, int num_sms) {
+  DynLayout l{};
+  const bool decode = M <= SQ_DECODE_MAX_M;
+  l.sk = decode ? round256(splitk_workspace_bytes(M, N, K, num_sms)) : 0;
+  l.part_n = decode ? (N + 31) / 32 : 2 * ((N + 255) / 256);
+  l.a_off = l.sk;
+  l.part_off = l.a_off + round256(static_cast<size_t>(M) * static_cast<size_t>(N) * 2);
+  l.total = l.part_off + round256(static_cast<size_t>(M) * static_cast<size_t>(l.part_n) * 4);
+  return l;
+}
+
+int sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  return sms;
+}
+
+}  // namespace
+
+size_t sq_w8a8_linear_quant_dyn_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0 || M > 0x7fffffffLL || N > SQ_MAX_K) return 0;
+  return dyn_layout(M, N, K, sm_count()).total;
+}
+
+sq_status sq_w8a8_linear_quant_dyn(const int8_t* xq, const float* x_scale, const int8_t* wq,
+                                   const float* w_scale, const void* bias_f16, int relu,
+                                   const float* inv_s_next, int8_t* xq_next, float* x_scale_next,
+                                   int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes,
+                                   sq_stream_t stream) {
+  if (!xq || !x_scale || !wq || !w_scale || !xq_next || !x_scale_next || !workspace)
+    return SQ_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_k(K);
+  if (st != SQ_OK) return st;
+  // the codes are the next linear's input: its K (= N here) follows the same rule
+  if (N % 16 != 0 || N > SQ_MAX_K) return SQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(xq) || !aligned16(x_scale) || !aligned16(wq) || !aligned16(w_scale) ||
+      !opt_aligned(bias_f16) || !opt_aligned(inv_s_next) || !aligned16(xq_next) ||
+      !aligned16(x_scale_next) || !aligned16(workspace))
+    return SQ_ERR_MISALIGNED;
+  if (M > 0x7fffffffLL) return SQ_ERR_UNSUPPORTED_SHAPE;
+  Ctx ctx;
+  if ((st = current_ctx(stream, &ctx)) != SQ_OK) return st;
+  const DynLayout l = dyn_layout(M, N, K, ctx.num_sms);
+  if (ws_bytes < l.total) return SQ_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  GemmArgs g{};
+  g.xq = xq;
+  g.sx = x_scale;
+  g.wq = wq;
+  g.sw = w_scale;
+  g.bias = static_cast<const __half*>(bias_f16);
+  g.y = reinterpret_cast<__half*>(ws + l.a_off);
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.ws = workspace;
+  g.ws_bytes = l.sk;
+  g.inv_s_next = inv_s_next;
+  g.relu = relu ? 1 : 0;
+  g.part = reinterpret_cast<float*>(ws + l.part_off);
+  g.part_n = l.part_n;
+  cudaError_t e = M <= SQ_DECODE_MAX_M ? launch_gemm_splitk(g, ctx) : launch_gemm_pair(g, ctx);
+  if (e != cudaSuccess) return launched(e);
+  return launched(launch_quant_partial_rows(g.y, M, N, g.part, g.part_n, inv_s_next, xq_next, x_scale_next, ctx));
 }
 
 sq_status sq_w8a8_bmm(const int8_t* a, const float* a_scale, const int8_t* b, const float* b_scale,

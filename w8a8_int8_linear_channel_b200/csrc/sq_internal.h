@@ -62,10 +62,16 @@ cudaError_t launch_dequant(const int32_t* acc, const float* sx, const float* sw,
                            int64_t M, int64_t N, const Ctx& c);
 
 cudaError_t launch_ln_quant_act(const RowArgs& a, const Ctx& c);
+// Second phase of the per-token producer-side quantization: row t's scale is
+// max_g part[t * part_n + g] / 127 and q[t, n] the code of fp32(a[t, n]) *
+// inv_s[n] (inv_s NULL: 1) at that scale; N % 8 == 0.
+cudaError_t launch_quant_partial_rows(const __half* a, int64_t M, int64_t N, const float* part, int64_t part_n,
+                                      const float* inv_s, int8_t* q, float* scale, const Ctx& c);
 cudaError_t launch_quantize_weight(const RowArgs& a, const Ctx& c);
 cudaError_t launch_calibrate_ln(const RowArgs& a, const Ctx& c);
 
 // Column-wise / elementwise kernels (k_cols.cu).
+cudaError_t launch_calib_reset(float* amax, int64_t n, const Ctx& c);
 cudaError_t launch_absmax_cols(const __half* x, int64_t rows, int64_t K, int64_t ld, float* amax,
                                const Ctx& c);
 cudaError_t launch_smooth(const float* amax_x, const float* amax_w, int64_t K, float alpha,
@@ -100,6 +106,14 @@ struct GemmArgs {
   // batched GEMM (INT8 BMM): batch items of [M, K] x [N, K]^T -> [M, N], the
   // scales per (item, row) sx [batch, M] and per (item, column) sw [batch, N]
   int64_t batch;  // 0 = not batched
+  // producer-side quantization at the next linear's per-token dynamic scale,
+  // first phase (part != NULL; y receives a = fp16(y), ReLU if relu): per row
+  // the maxima of |fp32(a) * inv_s_next[n]| over consecutive column groups,
+  // part[row * part_n + group] (groups of 128 columns on the CTA-pair kernel,
+  // 32 on the stream-K kernel); launch_quant_partial_rows then quantizes a
+  // with each row's maximum.
+  float* part;
+  int64_t part_n;
 };
 
 cudaError_t launch_gemm_tiled(const GemmArgs& g, const Ctx& c);  // 128 x 256 tiles

@@ -78,7 +78,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
 }
 
 // Wait used while tearing down after an abort: bounded, records nothing.
+// Copies and MMAs already issued finish in microseconds, so the teardown
+// waits at least 100 ms for them whatever the (possibly tiny) wait budget
+// that ran out: a CTA must not release its shared memory or tensor memory
+// while they are still in flight.
 __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
+  constexpr uint64_t kDrainFloorNs = 100000000ull;
+  if (budget_ns < kDrainFloorNs) budget_ns = kDrainFloorNs;
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() - t0 > budget_ns) return false;

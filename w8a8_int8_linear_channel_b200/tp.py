@@ -30,7 +30,7 @@ from typing import Optional
 
 import torch
 
-from . import (sq_calibrate_absmax, sq_dequant, sq_ln_quant_act, sq_quantize_rows_ranged,
+from . import (MAX_K, sq_calibrate_absmax, sq_dequant, sq_ln_quant_act, sq_quantize_rows_ranged,
                sq_quantize_weight, sq_row_ranges, sq_smooth_fold, sq_w8a8_gemm_s32, sq_w8a8_linear,
                sq_w8a8_workspace_bytes)
 
@@ -177,9 +177,14 @@ class RowParallelSmoothQuantLinear:
         calibration input; bias [N] is added once, after the reduction.  The
         layer's whole K (the sum of K_rank over ranks) must be at most MAX_K,
         the bound under which the all-reduced int32 sums of 127 x 127 products
-        cannot overflow; each rank can only check its own slice."""
+        cannot overflow: one integer all-reduce of the slice widths checks it
+        on every rank (ValueError) before anything is computed."""
         ops = ops or LibsqOps()
         comm = comm or DistComm()
+        k_total = comm.sum_(torch.tensor([w_shard.shape[1]], dtype=torch.int64, device=w_shard.device))
+        if int(k_total.item()) > MAX_K:
+            raise ValueError(f"row-parallel K = {int(k_total.item())} over all ranks exceeds {MAX_K}: the "
+                             "all-reduced int32 accumulators could overflow")
         amax_x = ops.col_absmax(calib_shard)  # channel j lives on one rank only
         amax_w = ops.col_absmax(w_shard)
         s, inv_s, _, _ = ops.smooth(amax_x, amax_w, alpha)
