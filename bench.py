@@ -879,9 +879,10 @@ def run_bmm(sq, torch, device, flush, args):
     return out
 
 
-def graph_of(torch, calls, reps):
+def graph_of(torch, calls, reps, pre=None):
     """One CUDA graph of `reps` rounds of the given (fn, args-builder(stream)) C calls,
-    captured on a side stream (consecutive launches overlap through PDL)."""
+    captured on a side stream (consecutive launches overlap through PDL); `pre` (torch work,
+    e.g. an L2 flush) is captured before every round."""
     cap = torch.cuda.Stream()
     cap.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(cap):
@@ -889,9 +890,13 @@ def graph_of(torch, calls, reps):
         bound = [(fn, mk(st)) for fn, mk in calls]
         for fn, a in bound:  # once eagerly (lazy set-up outside the capture)
             Plan._call("call", fn, a)
+        if pre is not None:
+            pre()
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=cap):
             for _ in range(reps):
+                if pre is not None:
+                    pre()
                 for fn, a in bound:
                     Plan._call("call", fn, a)
     torch.cuda.current_stream().wait_stream(cap)
@@ -914,11 +919,22 @@ def time_graph(torch, gr, iters, flush, reps=1):
     return 1e3 * sum(a.elapsed_time(b) for a, b in ev) / iters / reps
 
 
-def cold_warm(torch, calls, flush, iters, warm_reps):
-    """(cold, warm) microseconds per round of `calls`: cold = one round per replay after an L2
-    flush; warm = `warm_reps` back-to-back rounds per replay (operands stay in L2 when they fit)."""
-    cold = time_graph(torch, graph_of(torch, calls, 1), iters, flush)
-    warm = time_graph(torch, graph_of(torch, calls, warm_reps), max(3, iters // 4), flush, warm_reps)
+COLD_REPS = 10
+
+
+def cold_warm(torch, calls, flush, iters, warm_reps, flush_graph=None):
+    """(cold, warm) microseconds per round of `calls`.  Cold: a graph of COLD_REPS x [L2 flush,
+    round] minus a graph of COLD_REPS x [L2 flush] (so neither the flush nor an event pair around
+    a single short launch enters the figure), divided by COLD_REPS; every round starts with its
+    operands in HBM.  Warm: `warm_reps` back-to-back rounds per replay (operands stay in L2 when
+    they fit)."""
+    with_flush = graph_of(torch, calls, COLD_REPS, pre=flush)
+    if flush_graph is None:
+        flush_graph = graph_of(torch, [], COLD_REPS, pre=flush)
+    nrep = max(3, iters // 4)
+    cold = (time_graph(torch, with_flush, nrep, flush, COLD_REPS)
+            - time_graph(torch, flush_graph, nrep, flush, COLD_REPS))
+    warm = time_graph(torch, graph_of(torch, calls, warm_reps), nrep, flush, warm_reps)
     return cold, warm
 
 
@@ -944,9 +960,9 @@ def run_forward(plan, sq, torch, flush, iters):
         else:
             rec["gbs_warm"] = round(b / (warm * 1e-6) / 1e9, 1)
         out[key] = rec
-    out["what"] = ("forward = sq_ln_quant_act + sq_w8a8_linear with the weight already quantized; cold: "
-                   "one forward per graph replay after a 256 MiB L2 flush; warm: 20 back-to-back "
-                   "forwards per replay")
+    out["what"] = ("forward = sq_ln_quant_act + sq_w8a8_linear with the weight already quantized; cold: a "
+                   f"graph of {COLD_REPS} x [256 MiB L2 flush, forward] minus a graph of the flushes alone, per "
+                   "forward; warm: 20 back-to-back forwards per replay")
     if sq.sq_poll_status() != 0:
         raise RuntimeError("device wait timed out in the forward loop")
     return out
@@ -1001,8 +1017,8 @@ def run_decode_sweep(sq, torch, device, flush, iters, peaks):
     return {"workload": DESCR["decode"], "kernel": "k_gemm_splitk (swap-AB stream-K, tcgen05 kind::i8)",
             "peak_gbs": hbm, "peak_source": "measured copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
             "bytes": "M*K + N*K + 4M + 4N + 2MN per linear launch; the forward adds 3MK + 4M + 8K",
-            "timing": "cold: one launch per CUDA-graph replay after a 256 MiB L2 flush; warm: 10 "
-                      f"back-to-back launches per replay; mean of {iters} replays",
+            "timing": f"cold: a graph of {COLD_REPS} x [256 MiB L2 flush, launch] minus a graph of the flushes "
+                      "alone, per launch; warm: 10 back-to-back launches per replay",
             "sweep": rows, "clocks": clocks}
 
 

@@ -366,8 +366,7 @@ typedef enum sq_gemm_path {
   SQ_PATH_AUTO = 0,   /* what sq_w8a8_linear does */
   SQ_PATH_TILED = 1,  /* tiled tcgen05 kernel, any M */
   SQ_PATH_SPLITK = 2, /* weight-streaming stream-K kernel, M <= SQ_SPLITK_MAX_M */
-  SQ_PATH_PAIR = 3,   /* 256 x 256 tiles on CTA pairs (tcgen05 cta_group::2), any M */
-  SQ_PATH_WIDE = 4    /* 256 x 256 tiles on single CTAs, any M */
+  SQ_PATH_PAIR = 3    /* 256 x 256 tiles on CTA pairs (tcgen05 cta_group::2), any M */
 } sq_gemm_path;
 
 /* sq_w8a8_linear with the kernel chosen by the caller (testing and

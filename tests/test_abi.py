@@ -40,7 +40,7 @@ def test_status_strings():
     assert L.sq_status_string(0) == b"SQ_OK"
     assert L.sq_status_string(8) == b"SQ_ERR_TIMEOUT"
     assert L.sq_status_string(99) == b"SQ_ERR_UNKNOWN"
-    assert L.sq_abi_version() == 105
+    assert L.sq_abi_version() == 200
 
 
 FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
@@ -63,8 +63,9 @@ def test_linear_rejects_bad_arguments_on_the_host():
     assert f(FAKE_ODD, FAKE, FAKE, FAKE, None, FAKE, 64, 64, 64, None, 0, None) == 2
     # forced stream-K path for too many tokens
     assert L.sq_w8a8_linear_path(FAKE, FAKE, FAKE, FAKE, None, FAKE, 129, 64, 64, FAKE, 1 << 20, 2, None) == 3
-    # unknown path
+    # unknown path (4 named single-CTA 256 x 256 tiles before ABI 2.0)
     assert L.sq_w8a8_linear_path(FAKE, FAKE, FAKE, FAKE, None, FAKE, 8, 64, 64, FAKE, 1 << 20, 7, None) == 1
+    assert L.sq_w8a8_linear_path(FAKE, FAKE, FAKE, FAKE, None, FAKE, 300, 64, 64, None, 0, 4, None) == 1
     del ok
 
 

@@ -56,12 +56,12 @@ def f32(a):
     return np.asarray(a, np.float32).ravel()
 
 
-PATHS = ("tiled", "splitk", "pair", "wide", "auto")
+PATHS = ("tiled", "splitk", "pair", "auto")
 
 
 def path_id(sq, name):
     return {"tiled": sq.PATH_TILED, "splitk": sq.PATH_SPLITK, "pair": sq.PATH_PAIR,
-            "wide": sq.PATH_WIDE, "auto": sq.PATH_AUTO}[name]
+            "auto": sq.PATH_AUTO}[name]
 
 
 def act_quant(sq, h, gamma=None, beta=None, inv_s=None):

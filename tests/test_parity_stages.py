@@ -181,11 +181,11 @@ def _rand_i8(rng, M, N, K):
 
 
 _PATHS = {"tiled": lambda m: m.PATH_TILED, "splitk": lambda m: m.PATH_SPLITK,
-          "pair": lambda m: m.PATH_PAIR, "wide": lambda m: m.PATH_WIDE}
+          "pair": lambda m: m.PATH_PAIR}
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
-@pytest.mark.parametrize("path", ["tiled", "splitk", "pair", "wide"])
+@pytest.mark.parametrize("path", ["tiled", "splitk", "pair"])
 def test_gemm_accumulators_bit_exact(sq, M, N, K, path):
     if path == "splitk" and M > sq.SPLITK_MAX_M:
         pytest.skip("stream-K path serves M <= 128")
@@ -200,7 +200,7 @@ def test_gemm_accumulators_bit_exact(sq, M, N, K, path):
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
-@pytest.mark.parametrize("path", ["tiled", "splitk", "pair", "wide"])
+@pytest.mark.parametrize("path", ["tiled", "splitk", "pair"])
 @pytest.mark.parametrize("with_bias", [False, True])
 def test_linear_output(sq, M, N, K, path, with_bias):
     if path == "splitk" and M > sq.SPLITK_MAX_M:
@@ -218,6 +218,25 @@ def test_linear_output(sq, M, N, K, path, with_bias):
     assert bits_equal(got, ref)
 
 
+# The CTA-pair kernel's persistent walk: fewer tiles than pairs, a partial last wave (the
+# attention shape: 128 tiles on 74 pairs), ragged N and M, and more than two waves in grouped
+# order.
+@pytest.mark.parametrize("M,N,K", [(512, 4160, 272), (2048, 4096, 528), (300, 2000, 1040),
+                                   (2100, 8200, 272)])
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_pair_kernel_persistent_walks(sq, M, N, K, with_bias):
+    rng = np.random.default_rng(M + N + K + with_bias)
+    xq, wq, sx, sw, bias = _rand_i8(rng, M, N, K)
+    bias = bias if with_bias else None
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    sq.sq_w8a8_gemm_s32(dev(xq), dev(wq), acc, path=sq.PATH_PAIR)
+    assert np.array_equal(host(acc), oracle.int_gemm(xq, wq))
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    sq.sq_w8a8_linear(dev(xq), dev(sx), dev(wq), dev(sw), y, dev(bias), path=sq.PATH_PAIR)
+    assert bits_equal(host(y), oracle.w8a8_linear(xq, sx, wq, sw, bias))
+    assert sq.sq_poll_status() == 0
+
+
 def test_splitk_many_contributors_per_tile(sq):
     # few channel tiles, long K: every tile is shared by many CTAs
     rng = np.random.default_rng(11)
@@ -232,7 +251,7 @@ def test_splitk_many_contributors_per_tile(sq):
     assert sq.sq_poll_status() == 0
 
 
-@pytest.mark.parametrize("path", ["tiled", "splitk", "pair", "wide"])
+@pytest.mark.parametrize("path", ["tiled", "splitk", "pair"])
 def test_linear_large_accumulators(sq, path):
     # rows of +-127 codes against +-127 weight rows make |acc| = 127^2 K, far
     # above 2^22 (beyond exact conversion through 1.5 * 2^23 + acc); the other
@@ -263,7 +282,7 @@ def test_extreme_codes_do_not_wrap(sq):
     xq[1] = -127
     wq = np.full((3, K), 127, np.int8)
     wq[2] = -127
-    for path in (sq.PATH_TILED, sq.PATH_SPLITK, sq.PATH_PAIR, sq.PATH_WIDE):
+    for path in (sq.PATH_TILED, sq.PATH_SPLITK, sq.PATH_PAIR):
         acc = torch.empty((2, 3), dtype=torch.int32, device="cuda")
         ws = sq.new_workspace(2, 3, K)
         sq.sq_w8a8_gemm_s32(dev(xq), dev(wq), acc, workspace=ws, path=path)

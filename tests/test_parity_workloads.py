@@ -145,10 +145,10 @@ def test_full_size_ffn_down(sq, alpha):
     _check(r, wl, wl.M, alpha, tokens, _weight_sample(wl.N, per_tile=2, seed=3))
 
 
-@pytest.mark.parametrize("path", ["auto", "pair", "wide"])
+@pytest.mark.parametrize("path", ["auto", "pair"])
 def test_persistent_gemm_more_tiles_than_sms(sq, path):
     # 6 x 26 = 156 tiles of 256 x 256 on 148 SMs (74 CTA pairs), ragged M, N and K
-    p = {"auto": sq.PATH_AUTO, "pair": sq.PATH_PAIR, "wide": sq.PATH_WIDE}[path]
+    p = {"auto": sq.PATH_AUTO, "pair": sq.PATH_PAIR}[path]
     rng = np.random.default_rng(99)
     M, N, K = 1300, 6500, 272
     xq = rng.integers(-127, 128, (M, K)).astype(np.int8)

@@ -74,7 +74,7 @@ def _rand_i8(rng, M, N, K):
 # ragged in M, N and K; 33-128 tokens take the stream-K kernel's 64- and 128-token tiles
 LINEAR_SHAPES = [(5, 100, 48), (33, 77, 16), (64, 520, 8208), (127, 513, 272), (128, 1000, 4112),
                  (300, 1000, 2064), (256, 520, 528), (513, 264, 512)]
-PATHS = {"tiled": "PATH_TILED", "splitk": "PATH_SPLITK", "pair": "PATH_PAIR", "wide": "PATH_WIDE"}
+PATHS = {"tiled": "PATH_TILED", "splitk": "PATH_SPLITK", "pair": "PATH_PAIR"}
 
 
 @pytest.mark.gpu

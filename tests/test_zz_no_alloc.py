@@ -64,3 +64,56 @@ def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_device):
     assert lib.sq_w8a8_linear_noalloc(fake, fake, fake, fake, None, fake, 33, 128, 128, None) == 3
     # more output channels than the fixed array has counters for (4096 tiles of 128)
     assert lib.sq_w8a8_linear_noalloc(fake, fake, fake, fake, None, fake, 8, 4096 * 128 + 1, 128, None) == 5
+
+
+def test_noalloc_calls_allocate_no_device_memory(cuda_device):
+    """The defining property: once the library is loaded and the call has run once per shape
+    (module and scratch-address set-up), further calls change neither the device's free memory
+    nor torch's allocations."""
+    import w8a8_int8_linear_channel_b200 as sq
+    lib = sq._L
+    rng = np.random.default_rng(7)
+    cases = []
+    for (M, N, K) in [(1, 4096, 4096), (16, 1000, 2064), (32, 12288, 512)]:
+        xq, sx, wq, sw, bias = _inputs(rng, M, N, K, True)
+        y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+        cases.append((xq, sx, wq, sw, bias, y))
+        assert _noalloc_via_c_abi(lib, xq, sx, wq, sw, bias, y) == 0  # warm-up of this shape
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    for _ in range(3):
+        for xq, sx, wq, sw, bias, y in cases:
+            assert _noalloc_via_c_abi(lib, xq, sx, wq, sw, bias, y) == 0
+    torch.cuda.synchronize()
+    assert sq.sq_poll_status() == 0
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert torch.cuda.memory_allocated() == alloc0
+
+
+def test_noalloc_clears_counters_left_by_a_timed_out_call(cuda_device):
+    """A call whose bounded waits run out (a 1 us budget: the first weight boxes are still in
+    flight) can leave arrival counters raised in the shared array; the next call clears them
+    before its GEMM, so it is exact again.  The kernel drains what it issued before returning,
+    so the device stays usable."""
+    import w8a8_int8_linear_channel_b200 as sq
+    lib = sq._L
+    rng = np.random.default_rng(11)
+    M, N, K = 16, 4096, 8192
+    xq, sx, wq, sw, bias = _inputs(rng, M, N, K, True)
+    y_ref = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    sq.sq_w8a8_linear(xq, sx, wq, sw, y_ref, bias, workspace=sq.new_workspace(M, N, K))
+    assert sq.sq_poll_status() == 0
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    try:
+        sq.sq_set_wait_budget_ns(1000)
+        assert _noalloc_via_c_abi(lib, xq, sx, wq, sw, bias, y) == 0
+        assert sq.sq_poll_status() == 8  # SQ_ERR_TIMEOUT
+    finally:
+        sq.sq_set_wait_budget_ns(2_000_000_000)
+    for _ in range(2):
+        y.fill_(float("nan"))
+        assert _noalloc_via_c_abi(lib, xq, sx, wq, sw, bias, y) == 0
+        assert sq.sq_poll_status() == 0
+        assert bits_equal(y.cpu().numpy(), y_ref.cpu().numpy())

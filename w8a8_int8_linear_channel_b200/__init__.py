@@ -30,13 +30,13 @@ __all__ = [
     "LEVELS", "sq_w8a8_linear_quant", "sq_w8a8_linear_quant_dyn", "sq_w8a8_linear_quant_dyn_workspace_bytes",
     "new_quant_dyn_workspace", "sq_w8a8_bmm", "sq_row_ranges", "sq_quantize_rows_ranged",
     "sq_dequant",
-    "PATH_AUTO", "PATH_TILED", "PATH_SPLITK", "PATH_PAIR", "PATH_WIDE", "SPLITK_MAX_M", "DECODE_MAX_M", "MAX_K", "library_path",
+    "PATH_AUTO", "PATH_TILED", "PATH_SPLITK", "PATH_PAIR", "SPLITK_MAX_M", "DECODE_MAX_M", "MAX_K", "library_path",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libsq.so")
 
-PATH_AUTO, PATH_TILED, PATH_SPLITK, PATH_PAIR, PATH_WIDE = 0, 1, 2, 3, 4
+PATH_AUTO, PATH_TILED, PATH_SPLITK, PATH_PAIR = 0, 1, 2, 3
 SPLITK_MAX_M = 128  # the stream-K kernel's largest token count
 DECODE_MAX_M = 32   # sq_w8a8_linear always streams the weight up to here
 MAX_K = 133144

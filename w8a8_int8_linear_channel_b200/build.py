@@ -25,7 +25,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-fmad=false",
                 "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
 
-SOURCES = ["sq_api.cu", "k_rows.cu", "k_cols.cu", "k_gemm_tiled.cu", "k_gemm_wide.cu", "k_gemm_pair.cu", "k_gemm_splitk.cu"]
+SOURCES = ["sq_api.cu", "k_rows.cu", "k_cols.cu", "k_gemm_tiled.cu", "k_gemm_pair.cu", "k_gemm_splitk.cu"]
 HEADERS = ["sq_internal.h", "sq_ptx.cuh", "sq_tmap.h"]
 
 

@@ -380,8 +380,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint2 b4 = reinterpret_cast<const uint2*>(bv)[j / 4];
                 const float2 b01 = __half22float2(*reinterpret_cast<const __half2*>(&b4.x));
                 const float2 b23 = __half22float2(*reinterpret_cast<const __half2*>(&b4.y));
-                d0 = f2_add_rn(d0, f2_pack(b01.x, b01.y));
-                d1 = f2_add_rn(d1, f2_pack(b23.x, b23.y));
+                // the add stays scalar: a packed add after a packed multiply can be
+                // contracted into a fused multiply-add
+                float2 e0 = f2_unpack(d0), e1 = f2_unpack(d1);
+                d0 = f2_pack(__fadd_rn(e0.x, b01.x), __fadd_rn(e0.y, b01.y));
+                d1 = f2_pack(__fadd_rn(e1.x, b23.x), __fadd_rn(e1.y, b23.y));
               }
               const float2 f0 = f2_unpack(d0), f1 = f2_unpack(d1);
               __half2 h0 = __floats2half2_rn(f0.x, f0.y), h1 = __floats2half2_rn(f1.x, f1.y);
@@ -441,7 +444,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
                 const float2 bf = __half22float2(*reinterpret_cast<const __half2*>(&bw[u]));
-                p[u] = f2_add_rn(p[u], f2_pack(bf.x, bf.y));
+                const float2 e = f2_unpack(p[u]);  // scalar adds: never contracted with the multiply
+                p[u] = f2_pack(__fadd_rn(e.x, bf.x), __fadd_rn(e.y, bf.y));
               }
             }
 #pragma unroll

@@ -119,8 +119,12 @@ __device__ __forceinline__ void warp_sum(Sums& s) {
 
 // mu and rstd from the exact sums S1 = s1 and S2 = s2h * 2^35 + s2l, by the
 // fixed sequence of correctly rounded fp64 operations documented in sq.h.
+// k_log2 >= 0 when K is a power of two: the divisions by K * 2^24 and K * 2^48
+// are then exact scalings, done as multiplications by the (exact) reciprocal
+// power of two -- the same correctly rounded results, without the division
+// sequences.
 __device__ __forceinline__ void ln_finalize(const Sums& s, int64_t K, float eps, float& mu,
-                                            float& rstd) {
+                                            float& rstd, int k_log2 = -1) {
   if (s.bad) {  // a row with an Inf or a NaN: NaN statistics
     mu = __int_as_float(0x7fc00000);
     rstd = mu;
@@ -134,8 +138,16 @@ __device__ __forceinline__ void ln_finalize(const Sums& s, int64_t K, float eps,
       __dmul_rn(__ull2double_rn(static_cast<unsigned long long>(S2 >> 64)), two64),
       __ull2double_rn(static_cast<unsigned long long>(S2)));
   const double Kd = static_cast<double>(K);
-  const double mean = __ddiv_rn(d1, __dmul_rn(Kd, 16777216.0));
-  const double ex2 = __ddiv_rn(d2, __dmul_rn(Kd, 281474976710656.0));
+  double mean, ex2;
+  if (k_log2 >= 0) {
+    const double r1 = __longlong_as_double(static_cast<long long>(1023 - 24 - k_log2) << 52);  // 2^-(24+log2 K)
+    const double r2 = __longlong_as_double(static_cast<long long>(1023 - 48 - k_log2) << 52);  // 2^-(48+log2 K)
+    mean = __dmul_rn(d1, r1);
+    ex2 = __dmul_rn(d2, r2);
+  } else {
+    mean = __ddiv_rn(d1, __dmul_rn(Kd, 16777216.0));
+    ex2 = __ddiv_rn(d2, __dmul_rn(Kd, 281474976710656.0));
+  }
   double var = __dsub_rn(ex2, __dmul_rn(mean, mean));
   if (var < 0.0) var = 0.0;
   const double r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(var, static_cast<double>(eps))));
@@ -893,18 +905,22 @@ __global__ void __launch_bounds__(kCtaThreads) k_calib_cta_atomic(const RowArgs 
 // NCH chunks of 8 values as fp32 in registers from the one read of shared
 // memory to the codes.  Per element:
 //   statistics  exact sums in fp64: h (a multiple of 2^-24, |h| < 2^16) adds
-//               exactly into one fp64 accumulator per thread; h*h (exact in
-//               fp64) is added to an accumulator biased by 1.5 * 2^43 (unit in
-//               the last place 2^-9, so every partial sum keeps that unit), and
-//               the part the add rounded away, t - ((A + t) - A), which is
-//               exact (Fast2Sum, |A| >= |t|), goes to a second accumulator in
-//               units of 2^-48.  Per thread the three sums become int64 and are
-//               reduced as integers: S1 = sum v and S2 = sum v^2 (v = h * 2^24)
-//               exactly, whatever the order.
-//   transform   ((x - mu) * rstd) * gamma + beta, times inv_s -- packed fp32
-//               pairs (each lane rounded like the scalar op, no FMA)
+//               exactly into an fp64 accumulator; h*h (exact in fp64) goes
+//               into an accumulator A biased by 1.5 * 2^43 (unit in the last
+//               place 2^-9 for every partial sum) with one fused multiply-add,
+//               A' = fma(h, h, A), and the part that rounding dropped,
+//               fma(h, h, A - A') (exact: A - A' is exact and so is the
+//               remainder, a multiple of 2^-48 below 2^-10), into a second
+//               accumulator.  Two independent sets per thread (even / odd
+//               elements).  The three sums become int64 and are reduced as
+//               integers: S1 = sum v and S2 = sum v^2 (v = h * 2^24) exactly,
+//               whatever the order.
+//   transform   (x - mu) * rstd, then * gamma, in packed fp32 pairs (each lane
+//               rounded like the scalar op), + beta in scalar adds (a packed add
+//               after a packed multiply can be contracted into a fused
+//               multiply-add; a scalar one is not), times inv_s packed
 //   maximum     three-input NaN-propagating max of absolute values
-//   codes       x * (1 / scale) + 1.5 * 2^23 in packed pairs, low bytes packed
+//   codes       x * (1 / scale) packed, + 1.5 * 2^23 scalar, low bytes packed
 // Three block barriers per row with a LayerNorm (statistics, mu / rstd, row
 // maximum), one without.  Rows with a non-finite maximum take the NaN-free
 // maximum and the NaN-safe codes, as in the kernels above.  Every wait is
@@ -914,6 +930,7 @@ __global__ void __launch_bounds__(kCtaThreads) k_calib_cta_atomic(const RowArgs 
 // =========================================================================
 constexpr double kS2Bias = 13194139533312.0;  // 1.5 * 2^43: unit in the last place 2^-9
 
+// x - mu lane-wise (a subtraction feeding a multiply: nothing to contract)
 __device__ __forceinline__ uint64_t f2_sub_rn(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
@@ -964,6 +981,7 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
   const uint32_t slot0 = smem_u32(ring);
   const uint32_t full0 = smem_u32(&sh.full[0]);
   const bool use_ln = a.gamma != nullptr;
+  const int k_log2 = (a.K & (a.K - 1)) == 0 ? __ffsll(a.K) - 1 : -1;  // K a power of two: its log2
   const int64_t G = gridDim.x;
   if (tid == 0) {
     mbar_init(full0, 1);
@@ -1009,24 +1027,27 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
     float mu = 0.0f, rstd = 0.0f;
     bool stop;
     if (use_ln) {
-      double s1 = 0.0, hi = kS2Bias, lo = 0.0;
+      double s1[2] = {0.0, 0.0}, hi[2] = {kS2Bias, kS2Bias}, lo[2] = {0.0, 0.0};
       int bad = 0;
 #pragma unroll
       for (int i = 0; i < NCH; ++i) {
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
+          const int u = jj & 1;
           const double d = static_cast<double>(x[i][jj]);
-          s1 = __dadd_rn(s1, d);
-          const double t = __dmul_rn(d, d);
-          const double hn = __dadd_rn(hi, t);
-          lo = __dadd_rn(lo, __dsub_rn(t, __dsub_rn(hn, hi)));
-          hi = hn;
+          s1[u] = __dadd_rn(s1[u], d);
+          const double hn = __fma_rn(d, d, hi[u]);
+          lo[u] = __dadd_rn(lo[u], __fma_rn(d, d, __dsub_rn(hi[u], hn)));
+          hi[u] = hn;
         }
       }
-      bad = !(fabs(s1) <= 1.7976931348623157e308) || !(hi <= 1.7976931348623157e308);
-      long long v1 = bad ? 0 : __double2ll_rn(__dmul_rn(s1, 16777216.0));               // units 2^-24
-      long long v2h = bad ? 0 : __double2ll_rn(__dmul_rn(__dsub_rn(hi, kS2Bias), 512.0));  // units 2^-9
-      long long v2l = bad ? 0 : __double2ll_rn(__dmul_rn(lo, 281474976710656.0));        // units 2^-48
+      const double t1 = __dadd_rn(s1[0], s1[1]);
+      const double t2h = __dadd_rn(__dsub_rn(hi[0], kS2Bias), __dsub_rn(hi[1], kS2Bias));
+      const double t2l = __dadd_rn(lo[0], lo[1]);
+      bad = !(fabs(t1) <= 1.7976931348623157e308) || !(fabs(t2h) <= 1.7976931348623157e308);
+      long long v1 = bad ? 0 : __double2ll_rn(__dmul_rn(t1, 16777216.0));            // units 2^-24
+      long long v2h = bad ? 0 : __double2ll_rn(__dmul_rn(t2h, 512.0));               // units 2^-9
+      long long v2l = bad ? 0 : __double2ll_rn(__dmul_rn(t2l, 281474976710656.0));   // units 2^-48
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         v1 += __shfl_xor_sync(0xffffffffu, v1, o);
@@ -1057,7 +1078,7 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
           t.bad |= sh.bad[par][w];
         }
         float m_, r_;
-        ln_finalize(t, a.K, a.eps, m_, r_);
+        ln_finalize(t, a.K, a.eps, m_, r_, k_log2);
         if (lane == 0) {
           sh.mu[par] = m_;
           sh.rstd[par] = r_;
@@ -1088,14 +1109,19 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
               bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w;
               bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
             }
+            // ((x - mu) * rstd) * gamma in packed pairs; the add of beta stays
+            // scalar (a packed add right after a packed multiply was seen
+            // contracted into one fused multiply-add)
 #pragma unroll
             for (int jj = 0; jj < 8; jj += 2) {
-              uint64_t v = f2_pack(x[i][jj], x[i][jj + 1]);
-              v = f2_mul_rn(f2_mul_rn(f2_sub_rn(v, mu2), r2), f2_pack(gg[jj], gg[jj + 1]));
-              if (a.beta) v = f2_add_rn(v, f2_pack(bb[jj], bb[jj + 1]));
-              const float2 f = f2_unpack(v);
+              const float2 f = f2_unpack(f2_mul_rn(f2_mul_rn(f2_sub_rn(f2_pack(x[i][jj], x[i][jj + 1]), mu2), r2),
+                                                   f2_pack(gg[jj], gg[jj + 1])));
               x[i][jj] = f.x;
               x[i][jj + 1] = f.y;
+            }
+            if (a.beta) {
+#pragma unroll
+              for (int jj = 0; jj < 8; ++jj) x[i][jj] = __fadd_rn(x[i][jj], bb[jj]);
             }
           }
           if (a.vec) {
@@ -1153,17 +1179,17 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
     if (tid == 0) a.scale[r] = sc;
     int8_t* dst = a.q + r * a.K;
     const uint64_t inv2 = f2_pack(inv, inv);
-    const uint64_t magic2 = f2_pack(12582912.0f, 12582912.0f);  // 1.5 * 2^23
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int64_t c = tid + static_cast<int64_t>(i) * T;
       if (c < Kc) {
         uint32_t b[8];
+        // x * (1 / scale) in packed pairs, then + 1.5 * 2^23 in scalar adds (each rounded)
 #pragma unroll
         for (int jj = 0; jj < 8; jj += 2) {
-          const float2 f = f2_unpack(f2_add_rn(f2_mul_rn(f2_pack(x[i][jj], x[i][jj + 1]), inv2), magic2));
-          b[jj] = __float_as_uint(f.x);
-          b[jj + 1] = __float_as_uint(f.y);
+          const float2 p = f2_unpack(f2_mul_rn(f2_pack(x[i][jj], x[i][jj + 1]), inv2));
+          b[jj] = __float_as_uint(__fadd_rn(p.x, 12582912.0f));
+          b[jj + 1] = __float_as_uint(__fadd_rn(p.y, 12582912.0f));
         }
         if (safe) {
 #pragma unroll
@@ -1192,52 +1218,60 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
 // the maxima of |fp32(a) * inv_s| over groups of columns; here a row's range
 // is the maximum of its groups (exact, order-free), and every element is
 // coded at that scale: x = fp32(a) * inv_s, q = code(x * (1 / scale)) -- the
-// same values and the same codes as the activation kernel's inv_s path.  A
-// warp per row, no block barrier; the codes go through the NaN-safe path
-// (a NaN x is coded 0; an Inf range gives scale Inf, reciprocal 0, codes 0).
+// same values and the same codes as the activation kernel's inv_s path.  One
+// CTA per (row, segment of kQSeg columns); each thread issues the loads of its
+// kQChunks chunks of 8 columns (16 bytes of a each) before it reduces the row's
+// few group maxima (one barrier per row), so the data is in flight meanwhile.
+// The codes go through the NaN-safe path (a NaN x is coded 0; an Inf range
+// gives scale Inf, reciprocal 0, codes 0).
 // =========================================================================
-constexpr int kQuantRowUnroll = 4;
+constexpr int kQThreads = 256;
+constexpr int kQChunks = 4;                          // 8-column chunks per thread
+constexpr int64_t kQSeg = 8 * kQChunks * kQThreads;  // columns per CTA
 
-__global__ void __launch_bounds__(256) k_quant_partial_rows(const __half* a, int64_t M, int64_t N,
-                                                             const float* part, int64_t part_n,
-                                                             const float* inv_s, int8_t* q, float* scale) {
+__global__ void __launch_bounds__(kQThreads) k_quant_partial_rows(const __half* a, int64_t M, int64_t N,
+                                                                   const float* part, int64_t part_n,
+                                                                   const float* inv_s, int8_t* q, float* scale) {
+  __shared__ float wmax[kQThreads / 32];
   griddep_wait();  // a and the partial maxima come from the GEMM just before
   griddep_launch_dependents();
-  const int lane = threadIdx.x & 31;
-  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t Nc = N >> 3;
-  for (int64_t r = wid; r < M; r += nwarps) {
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * (kQSeg / 8) + tid;  // chunks c0 + i * kQThreads
+  for (int64_t r = blockIdx.y; r < M; r += gridDim.y) {
+    // this thread's data first (all its loads in flight), then the row's range
+    uint4 v[kQChunks];
+    float is[kQChunks][8];
+#pragma unroll
+    for (int i = 0; i < kQChunks; ++i) {
+      const int64_t c = c0 + static_cast<int64_t>(i) * kQThreads;
+      v[i] = c < Nc ? ld_stream(reinterpret_cast<const uint4*>(a + r * N) + c) : make_uint4(0, 0, 0, 0);
+      if (inv_s != nullptr && c < Nc) load8f(inv_s + c * 8, is[i]);
+    }
     float m = 0.0f;
-    for (int64_t i = lane; i < part_n; i += 32) m = fmaxf(m, __ldg(part + r * part_n + i));
+    for (int64_t i = tid; i < part_n; i += kQThreads) m = fmaxf(m, __ldg(part + r * part_n + i));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    __syncthreads();  // the previous row's reads of wmax are done
+    if (lane == 0) wmax[warp] = m;
+    __syncthreads();
+    m = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kQThreads / 32; ++w) m = fmaxf(m, wmax[w]);
     const float sc = __fdiv_rn(m, 127.0f);
     const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
-    if (lane == 0) scale[r] = sc;
-    const uint4* src = reinterpret_cast<const uint4*>(a + r * N);
-    uint2* dst = reinterpret_cast<uint2*>(q + r * N);
-    for (int64_t c0 = lane; c0 < Nc; c0 += 32 * kQuantRowUnroll) {
-      uint4 v[kQuantRowUnroll];
+    if (blockIdx.x == 0 && tid == 0) scale[r] = sc;
 #pragma unroll
-      for (int u = 0; u < kQuantRowUnroll; ++u) {
-        const int64_t c = c0 + 32 * u;
-        v[u] = c < Nc ? ld_stream(src + c) : make_uint4(0, 0, 0, 0);
-      }
+    for (int i = 0; i < kQChunks; ++i) {
+      const int64_t c = c0 + static_cast<int64_t>(i) * kQThreads;
+      if (c < Nc) {
+        float x[8];
+        unpack8(v[i], x);
+        if (inv_s != nullptr) {
 #pragma unroll
-      for (int u = 0; u < kQuantRowUnroll; ++u) {
-        const int64_t c = c0 + 32 * u;
-        if (c < Nc) {
-          float x[8];
-          unpack8(v[u], x);
-          if (inv_s != nullptr) {
-            float is[8];
-            load8f(inv_s + c * 8, is);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(x[j], is[j]);
-          }
-          dst[c] = pack8<true>(x, inv);
+          for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(x[j], is[i][j]);
         }
+        *reinterpret_cast<uint2*>(q + r * N + c * 8) = pack8<true>(x, inv);
       }
     }
   }
@@ -1347,32 +1381,25 @@ cudaError_t launch_act_bulk(const RowArgs& a, const Ctx& c) {
 
 cudaError_t launch_ln_quant_act(const RowArgs& a, const Ctx& c) {
   // per-token dynamic scales with the row held in registers: rows staged by
-  // bulk copies (the other modes and shapes keep the kernels above)
+  // bulk copies, 4 to 8 chunks of 8 values per thread and as few threads per
+  // row as that allows (the per-row reductions and the LayerNorm statistics'
+  // finalization are amortized over more elements); the other modes and
+  // shapes keep the kernels above
   const int64_t Kc = a.K / 8;
   if (a.range_in == nullptr && a.range_out == nullptr && Kc > 128 && Kc <= 2048) {
-    if (Kc <= 256) return launch_act_bulk<128, 2>(a, c);
-    if (Kc <= 384) return launch_act_bulk<128, 3>(a, c);
-    if (Kc <= 512) return launch_act_bulk<128, 4>(a, c);
-    if (Kc <= 768) return launch_act_bulk<256, 3>(a, c);
-    if (Kc <= 1024) return launch_act_bulk<256, 4>(a, c);
-    if (Kc <= 1280) return launch_act_bulk<256, 5>(a, c);
-    if (Kc <= 1536) return launch_act_bulk<256, 6>(a, c);
-    if (Kc <= 1792) return launch_act_bulk<256, 7>(a, c);
-    return launch_act_bulk<256, 8>(a, c);
+    if (Kc <= 256) return Kc <= 192 ? launch_act_bulk<32, 6>(a, c) : launch_act_bulk<32, 8>(a, c);
+    if (Kc <= 512) return Kc <= 384 ? launch_act_bulk<64, 6>(a, c) : launch_act_bulk<128, 4>(a, c);
+    if (Kc <= 1024) return Kc <= 768 ? launch_act_bulk<128, 6>(a, c) : launch_act_bulk<128, 8>(a, c);
+    return Kc <= 1536 ? launch_act_bulk<256, 6>(a, c) : launch_act_bulk<256, 8>(a, c);
   }
   return launch_mode<MODE_ACT>(a, c);
 }
 
 cudaError_t launch_quant_partial_rows(const __half* a, int64_t M, int64_t N, const float* part, int64_t part_n,
                                       const float* inv_s, int8_t* q, float* scale, const Ctx& c) {
-  static int occ[64] = {0};
-  const int dev = c.device < 64 ? c.device : 63;
-  if (occ[dev] == 0) occ[dev] = occupancy(k_quant_partial_rows, 256, 0);
-  int64_t grid = static_cast<int64_t>(c.num_sms) * occ[dev];
-  const int64_t need = (M + 7) / 8;  // 8 row-warps per CTA
-  if (grid > need) grid = need;
-  return launch_pdl(k_quant_partial_rows, dim3(static_cast<unsigned>(grid)), dim3(256), 0, c.stream, a, M, N, part,
-                    part_n, inv_s, q, scale);
+  const dim3 grid(static_cast<unsigned>((N + kQSeg - 1) / kQSeg), static_cast<unsigned>(M < 65535 ? M : 65535));
+  return launch_pdl(k_quant_partial_rows, grid, dim3(kQThreads), 0, c.stream, a, M, N, part, part_n, inv_s, q,
+                    scale);
 }
 
 cudaError_t launch_quantize_weight(const RowArgs& a, const Ctx& c) {

@@ -127,7 +127,7 @@ sq_status linear_impl(const int8_t* xq, const float* x_scale, const int8_t* wq,
   if (M <= 0 || N <= 0) return SQ_ERR_INVALID_ARG;
   sq_status st = check_k(K);
   if (st != SQ_OK) return st;
-  if (path < SQ_PATH_AUTO || path > SQ_PATH_WIDE) return SQ_ERR_INVALID_ARG;
+  if (path < SQ_PATH_AUTO || path > SQ_PATH_PAIR) return SQ_ERR_INVALID_ARG;
   if (!aligned16(xq) || !aligned16(wq) || !opt_aligned(x_scale) || !opt_aligned(w_scale) ||
       !opt_aligned(bias_f16) || !opt_aligned(y_f16) || !opt_aligned(acc))
     return SQ_ERR_MISALIGNED;
@@ -167,7 +167,6 @@ sq_status linear_impl(const int8_t* xq, const float* x_scale, const int8_t* wq,
     return launched(launch_gemm_splitk(g, ctx));
   }
   if (path == SQ_PATH_PAIR) return launched(launch_gemm_pair(g, ctx));
-  if (path == SQ_PATH_WIDE) return launched(launch_gemm_wide(g, ctx));
   if (path == SQ_PATH_TILED) return launched(launch_gemm_tiled(g, ctx));
   // automatic: 256 x 256 tiles on CTA pairs once the token count fills them
   // (their double-buffered accumulators hide the epilogue; with two K boxes
@@ -283,7 +282,7 @@ const char* sq_status_string(int status) {
   }
 }
 
-int sq_abi_version(void) { return 105; }
+int sq_abi_version(void) { return 200; }
 
 sq_status sq_calibrate_reset(float* amax, int64_t n, sq_stream_t stream) {
   if (!amax || n <= 0) return SQ_ERR_INVALID_ARG;
@@ -563,6 +562,8 @@ DynLayout dyn_layout(int64_t M, int64_t N, int64_t K, int num_sms) {
   DynLayout l{};
   const bool decode = M <= SQ_DECODE_MAX_M;
   l.sk = decode ? round256(splitk_workspace_bytes(M, N, K, num_sms)) : 0;
+  // one maximum per row and column group: 32 columns (a warp's channels) on the stream-K
+  // kernel, 128 (half a 256-column tile) on the CTA-pair kernel
   l.part_n = decode ? (N + 31) / 32 : 2 * ((N + 255) / 256);
   l.a_off = l.sk;
   l.part_off = l.a_off + round256(static_cast<size_t>(M) * static_cast<size_t>(N) * 2);

@@ -117,7 +117,6 @@ struct GemmArgs {
 };
 
 cudaError_t launch_gemm_tiled(const GemmArgs& g, const Ctx& c);  // 128 x 256 tiles
-cudaError_t launch_gemm_wide(const GemmArgs& g, const Ctx& c);   // 256 x 256 tiles, persistent
 cudaError_t launch_gemm_pair(const GemmArgs& g, const Ctx& c);   // 256 x 256 tiles on CTA pairs
 cudaError_t launch_bmm_pair(const GemmArgs& g, const Ctx& c);    // the same, batched (g.batch items)
 cudaError_t launch_gemm_splitk(const GemmArgs& g, const Ctx& c);

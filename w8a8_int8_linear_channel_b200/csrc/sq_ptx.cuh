@@ -461,8 +461,8 @@ __device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t pa
 
 namespace sq {
 
-// Packed pairs of fp32 (one 64-bit register): lane-wise IEEE multiply / add,
-// each lane rounded to nearest even exactly like __fmul_rn / __fadd_rn.
+// Packed pairs of fp32 (one 64-bit register): lane-wise IEEE multiply, each
+// lane rounded to nearest even exactly like __fmul_rn.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
@@ -481,11 +481,11 @@ __device__ __forceinline__ uint64_t f2_mul_rn(uint64_t a, uint64_t b) {
   return r;
 }
 
-__device__ __forceinline__ uint64_t f2_add_rn(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
+// No packed add is provided: measured on this toolchain, add.rn.f32x2 right
+// after mul.rn.f32x2 is contracted into one fused multiply-add (one rounding
+// instead of two) despite the explicit rounding modifiers, while a scalar
+// __fadd_rn after a packed multiply is not.  Adds that follow a multiply stay
+// scalar.
 
 }  // namespace sq
 
