@@ -921,12 +921,13 @@ __global__ void __launch_bounds__(kCtaThreads) k_calib_cta_atomic(const RowArgs 
 //               multiply-add; a scalar one is not), times inv_s packed
 //   maximum     three-input NaN-propagating max of absolute values
 //   codes       x * (1 / scale) packed, + 1.5 * 2^23 scalar, low bytes packed
-// Three block barriers per row with a LayerNorm (statistics, mu / rstd, row
-// maximum), one without.  Rows with a non-finite maximum take the NaN-free
-// maximum and the NaN-safe codes, as in the kernels above.  Every wait is
-// bounded; a wait that runs out stops the CTA uniformly (the decision rides on
-// the first barrier of the row), which then waits (bounded) for its copies in
-// flight before returning.
+// One thread waits for each row (suspended in the mbarrier try-wait, bounded);
+// the others wait at the row's first barrier, which also turns a time-out into
+// a CTA-wide stop, after which the CTA waits (bounded) for its copies in
+// flight before returning.  Then two more barriers with a LayerNorm
+// (statistics, mu / rstd), and one for the row maximum.  Rows with a
+// non-finite maximum take the NaN-free maximum and the NaN-safe codes, as in
+// the kernels above.
 // =========================================================================
 constexpr double kS2Bias = 13194139533312.0;  // 1.5 * 2^43: unit in the last place 2^-9
 
@@ -954,7 +955,7 @@ __device__ __forceinline__ void bulk_row_load(uint32_t dst, const void* src, uin
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_hint(bar, parity, 2000)) {  // suspended up to 2 us per try, not spinning
     if (globaltimer_ns() - t0 > budget_ns) return false;
   }
   return true;
@@ -1013,19 +1014,25 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
     const int64_t r = blockIdx.x + j * G;
     if (r >= a.rows) break;
     const uint32_t s = static_cast<uint32_t>(j & 1);
-    const bool ok = mbar_wait_bounded(full0 + 8u * s, static_cast<uint32_t>((j >> 1) & 1), budget);
+    // one thread waits for the row (the others wait at the barrier, issuing
+    // nothing); the barrier also makes a time-out a CTA-wide decision
+    bool ok = true;
+    if (tid == 0) ok = mbar_wait_bounded(full0 + 8u * s, static_cast<uint32_t>((j >> 1) & 1), budget);
+    if (__syncthreads_or(!ok)) {
+      aborted = true;
+      break;
+    }
     float x[NCH][8];
     const uint4* src = reinterpret_cast<const uint4*>(ring + s * row_bytes);
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int64_t c = tid + static_cast<int64_t>(i) * T;
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (ok && c < Kc) v = src[c];
+      if (c < Kc) v = src[c];
       unpack8(v, x[i]);  // chunks past K are zeros
     }
 
     float mu = 0.0f, rstd = 0.0f;
-    bool stop;
     if (use_ln) {
       double s1[2] = {0.0, 0.0}, hi[2] = {kS2Bias, kS2Bias}, lo[2] = {0.0, 0.0};
       int bad = 0;
@@ -1061,11 +1068,7 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
         sh.s2l[par][warp] = v2l;
         sh.bad[par][warp] = bad;
       }
-      stop = __syncthreads_or(!ok);  // every thread has read slot s
-      if (stop) {
-        aborted = true;
-        break;
-      }
+      __syncthreads();  // every thread has read slot s
       consumed = j + 1;
       if (tid == 0) issue(j + 2);
       if (warp == 0) {
@@ -1143,14 +1146,8 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = absmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if (lane == 0) sh.mx[par][warp] = amax;
-    if (use_ln) {
-      __syncthreads();
-    } else {
-      stop = __syncthreads_or(!ok);  // every thread has read slot s
-      if (stop) {
-        aborted = true;
-        break;
-      }
+    __syncthreads();  // (without a LayerNorm: every thread has read slot s)
+    if (!use_ln) {
       consumed = j + 1;
       if (tid == 0) issue(j + 2);
     }
