@@ -912,15 +912,20 @@ __global__ void __launch_bounds__(kCtaThreads) k_calib_cta_atomic(const RowArgs 
 //               fma(h, h, A - A') (exact: A - A' is exact and so is the
 //               remainder, a multiple of 2^-48 below 2^-10), into a second
 //               accumulator.  Two independent sets per thread (even / odd
-//               elements).  The three sums become int64 and are reduced as
-//               integers: S1 = sum v and S2 = sum v^2 (v = h * 2^24) exactly,
-//               whatever the order.
+//               elements), added (exactly) into three fp64 partials per
+//               thread.  Warp 0 alone reduces them: per lane the partials of
+//               T / 32 threads in fp64 (exact: at most 512 elements), then as
+//               int64 across the warp: S1 = sum v and S2 = sum v^2
+//               (v = h * 2^24) exactly, whatever the order.
 //   transform   (x - mu) * rstd, then * gamma, in packed fp32 pairs (each lane
 //               rounded like the scalar op), + beta in scalar adds (a packed add
 //               after a packed multiply can be contracted into a fused
 //               multiply-add; a scalar one is not), times inv_s packed
-//   maximum     three-input NaN-propagating max of absolute values
+//   maximum     three-input NaN-propagating max of absolute values; across
+//               lanes and warps an unsigned max of the bit patterns (|x| and a
+//               positive NaN order as their bits: NaN above Inf above finite)
 //   codes       x * (1 / scale) packed, + 1.5 * 2^23 scalar, low bytes packed
+// FULL: K = 8 * NCH * T, every chunk of every thread is inside the row.
 // One thread waits for each row (suspended in the mbarrier try-wait, bounded);
 // the others wait at the row's first barrier, which also turns a time-out into
 // a CTA-wide stop, after which the CTA waits (bounded) for its copies in
@@ -963,15 +968,21 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 
 template <int T>
 struct ActShared {
-  long long s1[2][T / 32], s2h[2][T / 32], s2l[2][T / 32];
-  int bad[2][T / 32];
-  float mx[2][T / 32];
-  float mx2[2][T / 32];
+  double p1[2][T], p2h[2][T], p2l[2][T];  // per-thread statistics partials
+  alignas(16) uint32_t mx[2][T / 32];     // per-warp row maxima (bit patterns)
+  alignas(16) uint32_t mx2[2][T / 32];
   float mu[2], rstd[2];
   alignas(8) uint64_t full[2];
 };
 
-template <int T, int NCH>
+// Unsigned max over the warp (redux.sync).
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
+  uint32_t r;
+  asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
+  return r;
+}
+
+template <int T, int NCH, bool FULL>
 __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* status, uint64_t budget) {
   constexpr int W = T / 32;
   __shared__ ActShared<T> sh;
@@ -1028,14 +1039,14 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
     for (int i = 0; i < NCH; ++i) {
       const int64_t c = tid + static_cast<int64_t>(i) * T;
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (c < Kc) v = src[c];
+      if (FULL || c < Kc) v = src[c];
       unpack8(v, x[i]);  // chunks past K are zeros
     }
 
     float mu = 0.0f, rstd = 0.0f;
     if (use_ln) {
       double s1[2] = {0.0, 0.0}, hi[2] = {kS2Bias, kS2Bias}, lo[2] = {0.0, 0.0};
-      int bad = 0;
+      int bad;
 #pragma unroll
       for (int i = 0; i < NCH; ++i) {
 #pragma unroll
@@ -1048,38 +1059,38 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
           hi[u] = hn;
         }
       }
-      const double t1 = __dadd_rn(s1[0], s1[1]);
-      const double t2h = __dadd_rn(__dsub_rn(hi[0], kS2Bias), __dsub_rn(hi[1], kS2Bias));
-      const double t2l = __dadd_rn(lo[0], lo[1]);
-      bad = !(fabs(t1) <= 1.7976931348623157e308) || !(fabs(t2h) <= 1.7976931348623157e308);
-      long long v1 = bad ? 0 : __double2ll_rn(__dmul_rn(t1, 16777216.0));            // units 2^-24
-      long long v2h = bad ? 0 : __double2ll_rn(__dmul_rn(t2h, 512.0));               // units 2^-9
-      long long v2l = bad ? 0 : __double2ll_rn(__dmul_rn(t2l, 281474976710656.0));   // units 2^-48
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        v1 += __shfl_xor_sync(0xffffffffu, v1, o);
-        v2h += __shfl_xor_sync(0xffffffffu, v2h, o);
-        v2l += __shfl_xor_sync(0xffffffffu, v2l, o);
-      }
-      bad = __any_sync(0xffffffffu, bad);
-      if (lane == 0) {
-        sh.s1[par][warp] = v1;
-        sh.s2h[par][warp] = v2h;
-        sh.s2l[par][warp] = v2l;
-        sh.bad[par][warp] = bad;
-      }
+      // this thread's partials (exact: multiples of 2^-24, 2^-9 and 2^-48 far
+      // inside 53 bits); an Inf or a NaN in the row leaves them non-finite
+      sh.p1[par][tid] = __dadd_rn(s1[0], s1[1]);
+      sh.p2h[par][tid] = __dadd_rn(__dsub_rn(hi[0], kS2Bias), __dsub_rn(hi[1], kS2Bias));
+      sh.p2l[par][tid] = __dadd_rn(lo[0], lo[1]);
       __syncthreads();  // every thread has read slot s
       consumed = j + 1;
       if (tid == 0) issue(j + 2);
       if (warp == 0) {
-        Sums t{0, 0, 0, 0};
+        // pairwise (every partial sum is exact, so any order gives the same)
+        double q1[W], q2h[W], q2l[W];
 #pragma unroll
         for (int w = 0; w < W; ++w) {
-          t.s1 += sh.s1[par][w];
-          t.s2h += sh.s2h[par][w] * 16;  // units 2^-13
-          t.s2l += sh.s2l[par][w];
-          t.bad |= sh.bad[par][w];
+          q1[w] = sh.p1[par][32 * w + lane];
+          q2h[w] = sh.p2h[par][32 * w + lane];
+          q2l[w] = sh.p2l[par][32 * w + lane];
         }
+#pragma unroll
+        for (int st = 1; st < W; st *= 2)
+#pragma unroll
+          for (int w = 0; w + st < W; w += 2 * st) {
+            q1[w] = __dadd_rn(q1[w], q1[w + st]);
+            q2h[w] = __dadd_rn(q2h[w], q2h[w + st]);
+            q2l[w] = __dadd_rn(q2l[w], q2l[w + st]);
+          }
+        const double t1 = q1[0], t2h = q2h[0], t2l = q2l[0];
+        bad = !(fabs(t1) <= 1.7976931348623157e308) || !(fabs(t2h) <= 1.7976931348623157e308);
+        Sums t{bad ? 0 : __double2ll_rn(__dmul_rn(t1, 16777216.0)),          // units 2^-24
+               bad ? 0 : __double2ll_rn(__dmul_rn(t2h, 8192.0)),             // units 2^-13
+               bad ? 0 : __double2ll_rn(__dmul_rn(t2l, 281474976710656.0)),  // units 2^-48
+               bad};
+        warp_sum(t);
         float m_, r_;
         ln_finalize(t, a.K, a.eps, m_, r_, k_log2);
         if (lane == 0) {
@@ -1099,7 +1110,7 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
 #pragma unroll
       for (int i = 0; i < NCH; ++i) {
         const int64_t c = tid + static_cast<int64_t>(i) * T;
-        if (c < Kc) {
+        if (FULL || c < Kc) {
           const int64_t k0 = c * 8;
           if (use_ln) {
             const float4 g0 = __ldg(reinterpret_cast<const float4*>(a.gamma + k0));
@@ -1143,34 +1154,34 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
         }
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = absmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if (lane == 0) sh.mx[par][warp] = amax;
+    // amax is >= 0 or a positive NaN (max.NaN of absolute values)
+    const uint32_t wmax = warp_max_u32(__float_as_uint(amax));
+    if (lane == 0) sh.mx[par][warp] = wmax;
     __syncthreads();  // (without a LayerNorm: every thread has read slot s)
     if (!use_ln) {
       consumed = j + 1;
       if (tid == 0) issue(j + 2);
     }
-    float m = 0.0f;
+    uint32_t mb = 0;
 #pragma unroll
-    for (int w = 0; w < W; ++w) m = absmax_nan(m, sh.mx[par][w]);
+    for (int w = 0; w < W; ++w) mb = max(mb, sh.mx[par][w]);
+    float m = __uint_as_float(mb);
     const bool safe = !finite_f(m);  // CTA-uniform
     if (safe) {  // a NaN or an Inf in the row: the range ignores NaN
       float a2 = 0.0f;
 #pragma unroll
       for (int i = 0; i < NCH; ++i)
-        if (tid + static_cast<int64_t>(i) * T < Kc)
+        if (FULL || tid + static_cast<int64_t>(i) * T < Kc)
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) a2 = fmaxf(a2, fabsf(x[i][jj]));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) a2 = fmaxf(a2, __shfl_xor_sync(0xffffffffu, a2, o));
-      if (lane == 0) sh.mx2[par][warp] = a2;
+      const uint32_t w2 = warp_max_u32(__float_as_uint(a2));  // NaN-free, >= 0
+      if (lane == 0) sh.mx2[par][warp] = w2;
       __syncthreads();
-      m = 0.0f;
+      mb = 0;
 #pragma unroll
-      for (int w = 0; w < W; ++w) m = fmaxf(m, sh.mx2[par][w]);
+      for (int w = 0; w < W; ++w) mb = max(mb, sh.mx2[par][w]);
+      m = __uint_as_float(mb);
     }
-    m = fabsf(m);
     const float sc = __fdiv_rn(m, 127.0f);
     const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
     if (tid == 0) a.scale[r] = sc;
@@ -1179,7 +1190,7 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int64_t c = tid + static_cast<int64_t>(i) * T;
-      if (c < Kc) {
+      if (FULL || c < Kc) {
         uint32_t b[8];
         // x * (1 / scale) in packed pairs, then + 1.5 * 2^23 in scalar adds (each rounded)
 #pragma unroll
@@ -1357,23 +1368,29 @@ cudaError_t launch_calib_cta(const RowArgs& a, const Ctx& c) {
 
 }  // namespace
 
-template <int T, int NCH>
-cudaError_t launch_act_bulk(const RowArgs& a, const Ctx& c) {
+template <int T, int NCH, bool FULL>
+cudaError_t launch_act_bulk_k(const RowArgs& a, const Ctx& c) {
   static int occ[64] = {0};
   static int64_t occ_bytes[64] = {0};
   const int dev = c.device < 64 ? c.device : 63;
   const size_t smem = static_cast<size_t>(a.K) * 4;  // two slots of one fp16 row
   if (occ_bytes[dev] != static_cast<int64_t>(smem)) {
-    cudaError_t e = cudaFuncSetAttribute(k_act_rows_bulk<T, NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = cudaFuncSetAttribute(k_act_rows_bulk<T, NCH, FULL>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    occ[dev] = occupancy(k_act_rows_bulk<T, NCH>, T, smem);
+    occ[dev] = occupancy(k_act_rows_bulk<T, NCH, FULL>, T, smem);
     occ_bytes[dev] = static_cast<int64_t>(smem);
   }
   int64_t grid = static_cast<int64_t>(c.num_sms) * occ[dev];
   if (grid > a.rows) grid = a.rows;
-  return launch_pdl(k_act_rows_bulk<T, NCH>, dim3(static_cast<unsigned>(grid)), dim3(T), smem, c.stream, a,
+  return launch_pdl(k_act_rows_bulk<T, NCH, FULL>, dim3(static_cast<unsigned>(grid)), dim3(T), smem, c.stream, a,
                     c.status, c.budget_ns);
+}
+
+template <int T, int NCH>
+cudaError_t launch_act_bulk(const RowArgs& a, const Ctx& c) {
+  if (a.K == 8 * NCH * T) return launch_act_bulk_k<T, NCH, true>(a, c);
+  return launch_act_bulk_k<T, NCH, false>(a, c);
 }
 
 cudaError_t launch_ln_quant_act(const RowArgs& a, const Ctx& c) {
