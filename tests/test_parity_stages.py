@@ -121,7 +121,8 @@ def test_fold_weight_in_place(sq):
 # --------------------------------------------------------- weight quantize ----
 @pytest.mark.parametrize("N,K,fold", [(1, 16, False), (77, 48, True), (11, 512, True), (21, 2048, True),
                                       (300, 4112, True), (256, 256, False), (5, 16384, False),
-                                      (40, 16400, True), (13, 49152, True)])
+                                      (40, 16400, True), (13, 49152, True), (1100, 4096, True),
+                                      (9, 12288, True), (150, 1552, False)])
 def test_quantize_weight(sq, N, K, fold):
     rng = np.random.default_rng(N + K)
     w = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)

@@ -328,14 +328,6 @@ __device__ __forceinline__ void range_merge(const RowArgs& a, int64_t r, float m
   else atomicMax(reinterpret_cast<int*>(a.range_out), __float_as_int(m));
 }
 
-__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-
 // =========================================================================
 // Warp per row (K <= 32 * 8 * NW).
 // =========================================================================
@@ -895,7 +887,8 @@ __global__ void __launch_bounds__(kCtaThreads) k_calib_cta_atomic(const RowArgs 
 }
 
 // =========================================================================
-// LayerNorm / smoothing + per-token quantization, rows staged by bulk copies.
+// LayerNorm / smoothing + per-token quantization, and fold + per-channel
+// weight quantization, rows staged by bulk copies.
 //
 // One CTA of T threads per row, persistent over rows (grid-stride).  One
 // thread streams whole rows into a 2-slot shared-memory ring with untiled
@@ -920,7 +913,8 @@ __global__ void __launch_bounds__(kCtaThreads) k_calib_cta_atomic(const RowArgs 
 //   transform   (x - mu) * rstd, then * gamma, in packed fp32 pairs (each lane
 //               rounded like the scalar op), + beta in scalar adds (a packed add
 //               after a packed multiply can be contracted into a fused
-//               multiply-add; a scalar one is not), times inv_s packed
+//               multiply-add; a scalar one is not), times inv_s packed; for a
+//               weight row (no statistics) w * s packed, rounded to fp16 pairs
 //   maximum     three-input NaN-propagating max of absolute values; across
 //               lanes and warps an unsigned max of the bit patterns (|x| and a
 //               positive NaN order as their bits: NaN above Inf above finite)
@@ -966,9 +960,10 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   return true;
 }
 
-template <int T>
+template <int T, bool STATS>
 struct ActShared {
-  double p1[2][T], p2h[2][T], p2l[2][T];  // per-thread statistics partials
+  static constexpr int NP = STATS ? T : 1;
+  double p1[2][NP], p2h[2][NP], p2l[2][NP];  // per-thread statistics partials (LayerNorm rows)
   alignas(16) uint32_t mx[2][T / 32];     // per-warp row maxima (bit patterns)
   alignas(16) uint32_t mx2[2][T / 32];
   float mu[2], rstd[2];
@@ -982,17 +977,17 @@ __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
   return r;
 }
 
-template <int T, int NCH, bool FULL>
-__global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* status, uint64_t budget) {
+template <int MODE, int T, int NCH, bool FULL>
+__device__ __forceinline__ void rows_bulk(const RowArgs& a, uint32_t* status, uint64_t budget) {
   constexpr int W = T / 32;
-  __shared__ ActShared<T> sh;
+  __shared__ ActShared<T, MODE == MODE_ACT> sh;
   extern __shared__ __align__(128) uint8_t ring[];  // 2 slots of one row (2K bytes each)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t Kc = a.K >> 3;
   const uint32_t row_bytes = static_cast<uint32_t>(a.K * 2);
   const uint32_t slot0 = smem_u32(ring);
   const uint32_t full0 = smem_u32(&sh.full[0]);
-  const bool use_ln = a.gamma != nullptr;
+  const bool use_ln = MODE == MODE_ACT && a.gamma != nullptr;
   const int k_log2 = (a.K & (a.K - 1)) == 0 ? __ffsll(a.K) - 1 : -1;  // K a power of two: its log2
   const int64_t G = gridDim.x;
   if (tid == 0) {
@@ -1144,7 +1139,9 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
             const float is[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
 #pragma unroll
             for (int jj = 0; jj < 8; jj += 2) {
-              const float2 f = f2_unpack(f2_mul_rn(f2_pack(x[i][jj], x[i][jj + 1]), f2_pack(is[jj], is[jj + 1])));
+              float2 f = f2_unpack(f2_mul_rn(f2_pack(x[i][jj], x[i][jj + 1]), f2_pack(is[jj], is[jj + 1])));
+              // a weight row: x = fp16(w * s), the folded weight rounded once to fp16
+              if (MODE == MODE_WEIGHT) f = __half22float2(__floats2half2_rn(f.x, f.y));
               x[i][jj] = f.x;
               x[i][jj + 1] = f.y;
             }
@@ -1218,6 +1215,18 @@ __global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* 
     }
     __syncthreads();
   }
+}
+
+// Activation rows (LayerNorm and / or 1/s, per-token scales) and weight rows
+// (fold diag(s) rounded to fp16, per-output-channel scales).
+template <int T, int NCH, bool FULL>
+__global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* status, uint64_t budget) {
+  rows_bulk<MODE_ACT, T, NCH, FULL>(a, status, budget);
+}
+
+template <int T, int NCH, bool FULL>
+__global__ void __launch_bounds__(T) k_weight_rows_bulk(const RowArgs a, uint32_t* status, uint64_t budget) {
+  rows_bulk<MODE_WEIGHT, T, NCH, FULL>(a, status, budget);
 }
 
 // =========================================================================
@@ -1368,46 +1377,48 @@ cudaError_t launch_calib_cta(const RowArgs& a, const Ctx& c) {
 
 }  // namespace
 
-template <int T, int NCH, bool FULL>
-cudaError_t launch_act_bulk_k(const RowArgs& a, const Ctx& c) {
+template <int MODE, int T, int NCH, bool FULL>
+cudaError_t launch_rows_bulk_k(const RowArgs& a, const Ctx& c) {
+  constexpr auto kern = MODE == MODE_ACT ? k_act_rows_bulk<T, NCH, FULL> : k_weight_rows_bulk<T, NCH, FULL>;
   static int occ[64] = {0};
   static int64_t occ_bytes[64] = {0};
   const int dev = c.device < 64 ? c.device : 63;
   const size_t smem = static_cast<size_t>(a.K) * 4;  // two slots of one fp16 row
   if (occ_bytes[dev] != static_cast<int64_t>(smem)) {
-    cudaError_t e = cudaFuncSetAttribute(k_act_rows_bulk<T, NCH, FULL>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    occ[dev] = occupancy(k_act_rows_bulk<T, NCH, FULL>, T, smem);
+    occ[dev] = occupancy(kern, T, smem);
     occ_bytes[dev] = static_cast<int64_t>(smem);
   }
   int64_t grid = static_cast<int64_t>(c.num_sms) * occ[dev];
   if (grid > a.rows) grid = a.rows;
-  return launch_pdl(k_act_rows_bulk<T, NCH, FULL>, dim3(static_cast<unsigned>(grid)), dim3(T), smem, c.stream, a,
-                    c.status, c.budget_ns);
+  return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(T), smem, c.stream, a, c.status, c.budget_ns);
 }
 
-template <int T, int NCH>
-cudaError_t launch_act_bulk(const RowArgs& a, const Ctx& c) {
-  if (a.K == 8 * NCH * T) return launch_act_bulk_k<T, NCH, true>(a, c);
-  return launch_act_bulk_k<T, NCH, false>(a, c);
+template <int MODE, int T, int NCH>
+cudaError_t launch_rows_bulk(const RowArgs& a, const Ctx& c) {
+  if (a.K == 8 * NCH * T) return launch_rows_bulk_k<MODE, T, NCH, true>(a, c);
+  return launch_rows_bulk_k<MODE, T, NCH, false>(a, c);
 }
 
-cudaError_t launch_ln_quant_act(const RowArgs& a, const Ctx& c) {
-  // per-token dynamic scales with the row held in registers: rows staged by
-  // bulk copies, 4 to 8 chunks of 8 values per thread and as few threads per
-  // row as that allows (the per-row reductions and the LayerNorm statistics'
-  // finalization are amortized over more elements); the other modes and
-  // shapes keep the kernels above
+// Rows streamed by bulk copies, for per-row dynamic scales (no fixed range, no
+// range pass) and 1024 < K <= 16384: 4 to 8 chunks of 8 values per thread and
+// as few threads per row as that allows (the per-row reductions and the
+// LayerNorm statistics' finalization are amortized over more elements).
+template <int MODE>
+cudaError_t launch_bulk_or(const RowArgs& a, const Ctx& c) {
   const int64_t Kc = a.K / 8;
   if (a.range_in == nullptr && a.range_out == nullptr && Kc > 128 && Kc <= 2048) {
-    if (Kc <= 256) return Kc <= 192 ? launch_act_bulk<32, 6>(a, c) : launch_act_bulk<32, 8>(a, c);
-    if (Kc <= 512) return Kc <= 384 ? launch_act_bulk<64, 6>(a, c) : launch_act_bulk<128, 4>(a, c);
-    if (Kc <= 1024) return Kc <= 768 ? launch_act_bulk<128, 6>(a, c) : launch_act_bulk<128, 8>(a, c);
-    return Kc <= 1536 ? launch_act_bulk<256, 6>(a, c) : launch_act_bulk<256, 8>(a, c);
+    if (Kc <= 256) return Kc <= 192 ? launch_rows_bulk<MODE, 32, 6>(a, c) : launch_rows_bulk<MODE, 32, 8>(a, c);
+    if (Kc <= 512) return Kc <= 384 ? launch_rows_bulk<MODE, 64, 6>(a, c) : launch_rows_bulk<MODE, 128, 4>(a, c);
+    if (Kc <= 1024)
+      return Kc <= 768 ? launch_rows_bulk<MODE, 128, 6>(a, c) : launch_rows_bulk<MODE, 128, 8>(a, c);
+    return Kc <= 1536 ? launch_rows_bulk<MODE, 256, 6>(a, c) : launch_rows_bulk<MODE, 256, 8>(a, c);
   }
-  return launch_mode<MODE_ACT>(a, c);
+  return launch_mode<MODE>(a, c);
 }
+
+cudaError_t launch_ln_quant_act(const RowArgs& a, const Ctx& c) { return launch_bulk_or<MODE_ACT>(a, c); }
 
 cudaError_t launch_quant_partial_rows(const __half* a, int64_t M, int64_t N, const float* part, int64_t part_n,
                                       const float* inv_s, int8_t* q, float* scale, const Ctx& c) {
@@ -1416,9 +1427,7 @@ cudaError_t launch_quant_partial_rows(const __half* a, int64_t M, int64_t N, con
                     scale);
 }
 
-cudaError_t launch_quantize_weight(const RowArgs& a, const Ctx& c) {
-  return launch_mode<MODE_WEIGHT>(a, c);
-}
+cudaError_t launch_quantize_weight(const RowArgs& a, const Ctx& c) { return launch_bulk_or<MODE_WEIGHT>(a, c); }
 
 cudaError_t launch_calibrate_ln(const RowArgs& a, const Ctx& c) {
   const int64_t Kc = a.K / 8;

@@ -477,6 +477,15 @@ namespace sq {
 
 // Packed pairs of fp32 (one 64-bit register): lane-wise IEEE multiply, each
 // lane rounded to nearest even exactly like __fmul_rn.
+// 16-byte streaming load of read-only data (not kept in L1).
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
