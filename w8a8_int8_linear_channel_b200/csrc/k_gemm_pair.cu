@@ -87,14 +87,64 @@ enum Epi { EPI_F16 = 0, EPI_I32 = 1, EPI_Q8 = 2, EPI_BMM = 3, EPI_QD = 4 };
 // token panel from DRAM for each group of channel tiles).
 constexpr int kGroupM = 8;
 
-__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn) {
-  const int g = t / (kGroupM * tiles_n);
-  const int first = g * kGroupM;
-  const int gm = tiles_m - first < kGroupM ? tiles_m - first : kGroupM;
-  const int r = t - g * kGroupM * tiles_n;
-  tm = first + r % gm;
-  tn = r / gm;
-}
+static_assert((kGroupM & (kGroupM - 1)) == 0, "token tiles per group: a power of two");
+
+// n / d for 0 <= n < 2^31 and a divisor d >= 1 fixed for the whole kernel:
+// a multiply-high, a subtract, an add and two shifts instead of a division
+// sequence (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994: the unsigned case with a 33-bit multiplier, m' =
+// floor(2^32 (2^l - d) / d) + 1 and l = ceil(log2 d)).
+// Built on the host and passed as a kernel parameter (read from the constant
+// bank, so it holds no registers).
+struct FastDiv {
+  uint32_t d, m;
+  int l;
+  static FastDiv make(uint32_t d_) {
+    FastDiv f;
+    f.d = d_;
+    f.l = 0;
+    while (f.l < 32 && (static_cast<uint64_t>(1) << f.l) < d_) ++f.l;  // ceil(log2 d)
+    f.m = static_cast<uint32_t>(((static_cast<uint64_t>(1) << 32) * ((static_cast<uint64_t>(1) << f.l) - d_)) / d_ + 1);
+    return f;
+  }
+  __device__ __forceinline__ int div(int n) const {
+    if (l == 0) return n;
+    const uint32_t u = static_cast<uint32_t>(n);
+    const uint32_t t1 = __umulhi(m, u);
+    return static_cast<int>((t1 + ((u - t1) >> 1)) >> (l - 1));
+  }
+};
+
+// Tile t of the grid -> batch item bi (BATCHED only), token tile tm, channel
+// tile tn.
+struct TileMap {
+  FastDiv item;   // tiles per batch item
+  FastDiv group;  // tiles per group of kGroupM token tiles (kGroupM * tiles_n)
+  int tiles_m;
+  static TileMap make(int per_item, int tiles_m_) {
+    TileMap t;
+    t.item = FastDiv::make(static_cast<uint32_t>(per_item));
+    t.group = FastDiv::make(static_cast<uint32_t>(kGroupM * (per_item / tiles_m_)));
+    t.tiles_m = tiles_m_;
+    return t;
+  }
+  template <bool BATCHED>
+  __device__ __forceinline__ void coords(int t, int& bi, int& tm, int& tn) const {
+    bi = BATCHED ? item.div(t) : 0;
+    const int u = BATCHED ? t - bi * static_cast<int>(item.d) : t;
+    const int gi = group.div(u);
+    const int first = gi * kGroupM;
+    const int r = u - gi * static_cast<int>(group.d);
+    if (tiles_m - first >= kGroupM) {
+      tm = first + (r & (kGroupM - 1));
+      tn = r / kGroupM;
+    } else {  // the last, narrower group
+      const int gm = tiles_m - first;
+      tm = first + r % gm;
+      tn = r / gm;
+    }
+  }
+};
 
 // Bounded wait that, when it runs out, also raises the other CTA's abort
 // flag so the pair stops together.  Barriers completed by the other CTA's
@@ -123,7 +173,7 @@ __device__ __forceinline__ bool pair_wait(uint32_t bar, uint32_t parity, bool cl
 template <int EPI, bool TMAS, int KSUB>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmY, const GemmArgs g, int tiles_m, int tiles,
+                const __grid_constant__ CUtensorMap tmY, const GemmArgs g, const TileMap tmap, int tiles,
                 uint32_t* status, uint64_t budget) {
   constexpr int STAGES = Ring<KSUB>::STAGES, STAGE_BYTES = Ring<KSUB>::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
@@ -151,8 +201,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int npairs = static_cast<int>(gridDim.x >> 1);
   const int KB = static_cast<int>((g.K + KSUB * BK - 1) / (KSUB * BK));
   // tiles of one batch item (the whole grid when not batched)
-  const int per_item = EPI == EPI_BMM ? tiles / static_cast<int>(g.batch) : tiles;
-  const int tiles_n = per_item / tiles_m;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -191,9 +239,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int64_t it = 0;
       bool ok = true;
       for (int t = pair; t < tiles && ok; t += npairs) {
-        const int bi = t / per_item;  // batch item (0 when not batched)
-        int tm, tn;
-        tile_coords(t - bi * per_item, tiles_m, tiles_n, tm, tn);
+        int bi, tm, tn;  // batch item (0 when not batched), token tile, channel tile
+        tmap.coords<EPI == EPI_BMM>(t, bi, tm, tn);
         const int32_t m0 = tm * (2 * BM) + static_cast<int32_t>(rank) * BM;
         const int32_t n0 = tn * BN + static_cast<int32_t>(rank) * BNH;
         for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -289,9 +336,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     auto fetch = [&](int t) {
       Vecs v{0.0f, 1.0f, 0.0f, __float2half_rn(0.0f)};
       if (EPI == EPI_I32 || t >= tiles) return v;
-      const int bi = t / per_item;
-      int tm, tn;
-      tile_coords(t - bi * per_item, tiles_m, tiles_n, tm, tn);
+      int bi, tm, tn;
+      tmap.coords<EPI == EPI_BMM>(t, bi, tm, tn);
       const int64_t n = static_cast<int64_t>(tn) * BN + et;
       const int64_t row = static_cast<int64_t>(tm) * (2 * BM) + static_cast<int64_t>(rank) * BM + 32 * q + lane;
       if (n < g.N) {
@@ -306,9 +352,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int tl = 0;
     for (int t = pair; t < tiles; t += npairs, ++tl) {
       const int b = tl & 1;
-      const int bi = t / per_item;  // batch item (0 when not batched)
-      int tm, tn;
-      tile_coords(t - bi * per_item, tiles_m, tiles_n, tm, tn);
+      int bi, tm, tn;  // batch item (0 when not batched), token tile, channel tile
+      tmap.coords<EPI == EPI_BMM>(t, bi, tm, tn);
       const int64_t m0 = static_cast<int64_t>(tm) * (2 * BM) + static_cast<int64_t>(rank) * BM;
       const int64_t n0 = static_cast<int64_t>(tn) * BN;
       const Vecs cur = nxt;
@@ -323,10 +368,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int64_t row = m0 + 32 * q + lane;
         if (tn == 0 && half == 0 && row < g.M) g.sx_next[row] = q_sc;
       }
-      named_bar_sync(1, 32 * kEpiWarps);
       pair_wait(accf_bar(b), static_cast<uint32_t>((tl >> 1) & 1), false, budget, status, abort_flag, peer_abort);
       // one thread decides whether to stop and broadcasts it (double-buffered by
-      // tile parity), so every epilogue thread leaves the loop at the same point
+      // tile parity), so every epilogue thread leaves the loop at the same point.
+      // The same barrier publishes this tile's sw / bias / 1/s above: the
+      // barrier that ends the previous tile (below) came after every read of the
+      // previous tile's entries, so they were free to overwrite.
       if (et == 0) decision[tl & 1] = *abort_flag;
       named_bar_sync(1, 32 * kEpiWarps);
       if (decision[tl & 1]) break;
@@ -617,8 +664,10 @@ cudaError_t launch_kernel(const GemmArgs& g, const Ctx& c, const CUtensorMap& tm
                           const CUtensorMap& tmY, int tiles_m, int tiles, int pairs) {
   cudaError_t e = smem_attr<EPI, TMAS, KSUB>(c.device);
   if (e != cudaSuccess) return e;
+  // tiles of one batch item (the whole grid when not batched)
+  const int per_item = EPI == EPI_BMM ? tiles / static_cast<int>(g.batch) : tiles;
   return launch_pdl(k_gemm_pair<EPI, TMAS, KSUB>, dim3(2 * pairs), dim3(kThreads), SMEM, c.stream, tmA, tmB, tmY,
-                    g, tiles_m, tiles, c.status, c.budget_ns);
+                    g, TileMap::make(per_item, tiles_m), tiles, c.status, c.budget_ns);
 }
 
 template <int EPI, bool TMAS>
