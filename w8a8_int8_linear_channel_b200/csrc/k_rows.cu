@@ -1236,59 +1236,58 @@ __global__ void __launch_bounds__(T) k_weight_rows_bulk(const RowArgs a, uint32_
 // is the maximum of its groups (exact, order-free), and every element is
 // coded at that scale: x = fp32(a) * inv_s, q = code(x * (1 / scale)) -- the
 // same values and the same codes as the activation kernel's inv_s path.  One
-// CTA per (row, segment of kQSeg columns); each thread issues the loads of its
-// kQChunks chunks of 8 columns (16 bytes of a each) before it reduces the row's
-// few group maxima (one barrier per row), so the data is in flight meanwhile.
-// The codes go through the NaN-safe path (a NaN x is coded 0; an Inf range
-// gives scale Inf, reciprocal 0, codes 0).
+// warp per row (grid-stride), no block barrier: each lane issues the loads of
+// up to kQChunks chunks of 8 columns (16 bytes of a each) before the warp
+// reduces the row's group maxima with one unsigned max of their bit patterns
+// (they are >= 0 and NaN-free), so the data is in flight meanwhile; longer
+// rows take further batches.  The codes go through the NaN-safe path (a NaN x
+// is coded 0; an Inf range gives scale Inf, reciprocal 0, codes 0).
 // =========================================================================
-constexpr int kQThreads = 256;
-constexpr int kQChunks = 4;                          // 8-column chunks per thread
-constexpr int64_t kQSeg = 8 * kQChunks * kQThreads;  // columns per CTA
+constexpr int kQWarps = 8;    // rows in flight per CTA
+constexpr int kQChunks = 16;  // 8-column chunks per lane per batch (4096 columns per warp)
 
-__global__ void __launch_bounds__(kQThreads) k_quant_partial_rows(const __half* a, int64_t M, int64_t N,
-                                                                   const float* part, int64_t part_n,
-                                                                   const float* inv_s, int8_t* q, float* scale) {
-  __shared__ float wmax[kQThreads / 32];
+__global__ void __launch_bounds__(32 * kQWarps) k_quant_partial_rows(const __half* a, int64_t M, int64_t N,
+                                                                     const float* part, int64_t part_n,
+                                                                     const float* inv_s, int8_t* q, float* scale) {
   griddep_wait();  // a and the partial maxima come from the GEMM just before
   griddep_launch_dependents();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int lane = threadIdx.x & 31;
   const int64_t Nc = N >> 3;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * (kQSeg / 8) + tid;  // chunks c0 + i * kQThreads
-  for (int64_t r = blockIdx.y; r < M; r += gridDim.y) {
-    // this thread's data first (all its loads in flight), then the row's range
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kQWarps;
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * kQWarps + (threadIdx.x >> 5); r < M; r += nwarps) {
+    const uint4* src = reinterpret_cast<const uint4*>(a + r * N);
+    int8_t* dst = q + r * N;
     uint4 v[kQChunks];
-    float is[kQChunks][8];
+    auto load = [&](int64_t b0) {
 #pragma unroll
-    for (int i = 0; i < kQChunks; ++i) {
-      const int64_t c = c0 + static_cast<int64_t>(i) * kQThreads;
-      v[i] = c < Nc ? ld_stream(reinterpret_cast<const uint4*>(a + r * N) + c) : make_uint4(0, 0, 0, 0);
-      if (inv_s != nullptr && c < Nc) load8f(inv_s + c * 8, is[i]);
-    }
-    float m = 0.0f;
-    for (int64_t i = tid; i < part_n; i += kQThreads) m = fmaxf(m, __ldg(part + r * part_n + i));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    __syncthreads();  // the previous row's reads of wmax are done
-    if (lane == 0) wmax[warp] = m;
-    __syncthreads();
-    m = 0.0f;
-#pragma unroll
-    for (int w = 0; w < kQThreads / 32; ++w) m = fmaxf(m, wmax[w]);
+      for (int i = 0; i < kQChunks; ++i) {
+        const int64_t c = b0 + lane + 32 * i;
+        v[i] = c < Nc ? ld_stream(src + c) : make_uint4(0, 0, 0, 0);
+      }
+    };
+    load(0);
+    uint32_t mb = 0;
+    for (int64_t i = lane; i < part_n; i += 32) mb = max(mb, __float_as_uint(__ldg(part + r * part_n + i)));
+    const float m = __uint_as_float(warp_max_u32(mb));
     const float sc = __fdiv_rn(m, 127.0f);
     const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
-    if (blockIdx.x == 0 && tid == 0) scale[r] = sc;
+    if (lane == 0) scale[r] = sc;
+    for (int64_t b0 = 0; b0 < Nc; b0 += 32 * kQChunks) {
+      if (b0 > 0) load(b0);
 #pragma unroll
-    for (int i = 0; i < kQChunks; ++i) {
-      const int64_t c = c0 + static_cast<int64_t>(i) * kQThreads;
-      if (c < Nc) {
-        float x[8];
-        unpack8(v[i], x);
-        if (inv_s != nullptr) {
+      for (int i = 0; i < kQChunks; ++i) {
+        const int64_t c = b0 + lane + 32 * i;
+        if (c < Nc) {
+          float x[8];
+          unpack8(v[i], x);
+          if (inv_s != nullptr) {
+            float is[8];
+            load8f(inv_s + c * 8, is);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(x[j], is[i][j]);
+            for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(x[j], is[j]);
+          }
+          *reinterpret_cast<uint2*>(dst + c * 8) = pack8<true>(x, inv);
         }
-        *reinterpret_cast<uint2*>(q + r * N + c * 8) = pack8<true>(x, inv);
       }
     }
   }
@@ -1422,9 +1421,11 @@ cudaError_t launch_ln_quant_act(const RowArgs& a, const Ctx& c) { return launch_
 
 cudaError_t launch_quant_partial_rows(const __half* a, int64_t M, int64_t N, const float* part, int64_t part_n,
                                       const float* inv_s, int8_t* q, float* scale, const Ctx& c) {
-  const dim3 grid(static_cast<unsigned>((N + kQSeg - 1) / kQSeg), static_cast<unsigned>(M < 65535 ? M : 65535));
-  return launch_pdl(k_quant_partial_rows, grid, dim3(kQThreads), 0, c.stream, a, M, N, part, part_n, inv_s, q,
-                    scale);
+  int64_t grid = (M + kQWarps - 1) / kQWarps;
+  const int64_t cap = 16 * static_cast<int64_t>(c.num_sms);
+  if (grid > cap) grid = cap;
+  return launch_pdl(k_quant_partial_rows, dim3(static_cast<unsigned>(grid)), dim3(32 * kQWarps), 0, c.stream, a, M,
+                    N, part, part_n, inv_s, q, scale);
 }
 
 cudaError_t launch_quantize_weight(const RowArgs& a, const Ctx& c) { return launch_bulk_or<MODE_WEIGHT>(a, c); }
