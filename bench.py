@@ -657,6 +657,9 @@ def run_gpu(args):
         decode_rec = run_decode_sweep(sq, torch, device, flush, args.burst_iters, peaks_early)
     if world == 1 and not args.no_extras and not args.no_quality_sweep:
         quality_sweep = run_quality_sweep(sq, torch, device, sq_inputs.FFN_DOWN_ALPHAS)
+    gemm_shapes = None
+    if world == 1 and use_graph and not args.no_extras:
+        gemm_shapes = run_gemm_shapes(sq, torch, device, flush, args)
 
     nbytes, ops = stage_bytes_ops(wl, M, args.level)
     step_bytes = sum(nbytes.values())
@@ -750,7 +753,7 @@ def run_gpu(args):
             "e2e_forward": e2e_fwd,
         }
         for key, rec in (("forward", forward), ("decode", decode_rec), ("quality", quality),
-                         ("quality_alpha_sweep", quality_sweep)):
+                         ("quality_alpha_sweep", quality_sweep), ("gemm_shapes", gemm_shapes)):
             if rec is not None:
                 result[key] = rec
         if producer is not None:
@@ -876,6 +879,63 @@ def run_bmm(sq, torch, device, flush, args):
         del a, b, y
     if sq.sq_poll_status() != 0:
         raise RuntimeError("device wait timed out in the BMM loop")
+    return out
+
+
+def run_gemm_shapes(sq, torch, device, flush, args):
+    """The INT8 linear alone on the other large-M configurations (FFN-up of
+    OPT-6.7B and FFN-down of OPT-175B): random codes of the workload's shape,
+    per-token / per-channel scales and a bias; back-to-back launches in one
+    graph with the L2 flushed before each replay (the operands of FFN-down,
+    1 GB, do not fit in L2 anyway).  Tensor-bound: 2MNK against the measured
+    bf16 burst x the nominal INT8:BF16 ratio."""
+    L = sq._L
+    peaks, _ = load_peaks()
+    peak = float(peaks["bf16_tflops"]) * I8_PER_BF16
+    out = {}
+    g = torch.Generator(device="cpu").manual_seed(11)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    for name, reps in (("ffn_up", 10), ("ffn_down", 3)):
+        wl = sq_inputs.WORKLOADS[name]
+        M, N, K = wl.M, wl.N, wl.K
+        xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=device)
+        wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=device)
+        sx = (torch.rand(M, generator=g) * 1e-3).to(device)
+        sw = (torch.rand(N, generator=g) * 1e-3).to(device)
+        bias = (torch.randn(N, generator=g) * 0.1).half().to(device)
+        y = torch.empty((M, N), dtype=torch.float16, device=device)
+        ws_n = int(sq.sq_w8a8_workspace_bytes(M, N, K))
+        ws = torch.zeros(max(ws_n, 16), dtype=torch.uint8, device=device)
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap):
+            st = ctypes.c_void_p(cap.cuda_stream)
+            cargs = (p(xq), p(sx), p(wq), p(sw), p(bias), p(y), M, N, K, p(ws), ws_n, st)
+            for _ in range(2):
+                Plan._call("linear", L.sq_w8a8_linear, cargs)
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=cap):
+                for _ in range(reps):
+                    Plan._call("linear", L.sq_w8a8_linear, cargs)
+        torch.cuda.current_stream().wait_stream(cap)
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(max(3, args.burst_iters // 4))]
+        for e in ev:
+            flush()
+            e[0].record()
+            gr.replay()
+            e[1].record()
+        torch.cuda.synchronize()
+        us = 1e3 * sum(x.elapsed_time(z) for x, z in ev) / len(ev) / reps
+        tops = 2.0 * M * N * K / (us * 1e-6) / 1e12
+        out[name] = {"shape": f"M={M} N={N} K={K}", "us": round(us, 2), "tops": round(tops, 1),
+                     "frac": round(tops / peak, 4), "bound": "tensor", "launches_per_replay": reps}
+        del xq, wq, y, ws, gr
+        torch.cuda.empty_cache()
+    if sq.sq_poll_status() != 0:
+        raise RuntimeError("device wait timed out in the GEMM-shape loop")
+    out["peak_tops"] = round(peak, 1)
+    out["timing"] = "back-to-back launches in one CUDA graph, L2 flushed before each replay"
     return out
 
 

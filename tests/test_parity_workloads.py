@@ -137,7 +137,7 @@ def _check_decode(r, wl, M, cols):
     assert bits_equal(r["y"][:, cols], y_ref)
 
 
-@pytest.mark.parametrize("alpha", [0.0, 0.5, 1.0])
+@pytest.mark.parametrize("alpha", sq_inputs.FFN_DOWN_ALPHAS)
 def test_full_size_ffn_down(sq, alpha):
     wl = sq_inputs.WORKLOADS["ffn_down"]
     r = _run_path(sq, wl, wl.M, alpha)
