@@ -64,6 +64,13 @@ __device__ __forceinline__ uint32_t half_bits(const uint4& v, int j) {
   return (j & 1) ? (w >> 16) : (w & 0xFFFFu);
 }
 
+// fp16 bit pattern (low 16 bits of b) -> fp64, exact.
+__device__ __forceinline__ double half_to_f64(uint32_t b) {
+  double d;
+  asm("cvt.f64.f16 %0, %1;" : "=d"(d) : "h"(static_cast<unsigned short>(b)));
+  return d;
+}
+
 __device__ __forceinline__ float bits_to_f(uint32_t b) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(b)));
 }
@@ -1013,196 +1020,446 @@ __device__ __forceinline__ void rows_bulk(const RowArgs& a, uint32_t* status, ui
     issue(0);
     issue(1);
   }
-  int64_t consumed = 0;  // iterations whose copy has landed
+  int64_t consumed = 0;  // copies whose landing has been waited for (a time-out drains the rest)
   bool aborted = false;
-  int par = 0;
-  for (int64_t j = 0;; ++j, par ^= 1) {
-    const int64_t r = blockIdx.x + j * G;
-    if (r >= a.rows) break;
-    const uint32_t s = static_cast<uint32_t>(j & 1);
-    // one thread waits for the row (the others wait at the barrier, issuing
-    // nothing); the barrier also makes a time-out a CTA-wide decision
-    bool ok = true;
-    if (tid == 0) ok = mbar_wait_bounded(full0 + 8u * s, static_cast<uint32_t>((j >> 1) & 1), budget);
-    if (__syncthreads_or(!ok)) {
-      aborted = true;
-      break;
-    }
-    float x[NCH][8];
-    const uint4* src = reinterpret_cast<const uint4*>(ring + s * row_bytes);
-#pragma unroll
-    for (int i = 0; i < NCH; ++i) {
-      const int64_t c = tid + static_cast<int64_t>(i) * T;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (FULL || c < Kc) v = src[c];
-      unpack8(v, x[i]);  // chunks past K are zeros
-    }
 
-    float mu = 0.0f, rstd = 0.0f;
-    if (use_ln) {
-      double s1[2] = {0.0, 0.0}, hi[2] = {kS2Bias, kS2Bias}, lo[2] = {0.0, 0.0};
-      int bad;
+  if constexpr (W < 8) {
+    // rows of up to four warps, one row at a time: with a LayerNorm the
+    // statistics from the values in registers, one warp finalizes between two
+    // barriers, then the transform, the row maximum and the codes
+    int par = 0;
+    for (int64_t j = 0;; ++j, par ^= 1) {
+      const int64_t r = blockIdx.x + j * G;
+      if (r >= a.rows) break;
+      const uint32_t s = static_cast<uint32_t>(j & 1);
+      // one thread waits for the row (the others wait at the barrier, issuing
+      // nothing); the barrier also makes a time-out a CTA-wide decision
+      bool ok = true;
+      if (tid == 0) ok = mbar_wait_bounded(full0 + 8u * s, static_cast<uint32_t>((j >> 1) & 1), budget);
+      if (__syncthreads_or(!ok)) {
+        aborted = true;
+        break;
+      }
+      float x[NCH][8];
+      const uint4* src = reinterpret_cast<const uint4*>(ring + s * row_bytes);
 #pragma unroll
       for (int i = 0; i < NCH; ++i) {
+        const int64_t c = tid + static_cast<int64_t>(i) * T;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (FULL || c < Kc) v = src[c];
+        unpack8(v, x[i]);  // chunks past K are zeros
+      }
+
+      float mu = 0.0f, rstd = 0.0f;
+      if (use_ln) {
+        double s1[2] = {0.0, 0.0}, hi[2] = {kS2Bias, kS2Bias}, lo[2] = {0.0, 0.0};
+        int bad;
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int u = jj & 1;
+            const double d = static_cast<double>(x[i][jj]);
+            s1[u] = __dadd_rn(s1[u], d);
+            const double hn = __fma_rn(d, d, hi[u]);
+            lo[u] = __dadd_rn(lo[u], __fma_rn(d, d, __dsub_rn(hi[u], hn)));
+            hi[u] = hn;
+          }
+        }
+        // this thread's partials (exact: multiples of 2^-24, 2^-9 and 2^-48 far
+        // inside 53 bits); an Inf or a NaN in the row leaves them non-finite
+        sh.p1[par][tid] = __dadd_rn(s1[0], s1[1]);
+        sh.p2h[par][tid] = __dadd_rn(__dsub_rn(hi[0], kS2Bias), __dsub_rn(hi[1], kS2Bias));
+        sh.p2l[par][tid] = __dadd_rn(lo[0], lo[1]);
+        __syncthreads();  // every thread has read slot s
+        consumed = j + 1;
+        if (tid == 0) issue(j + 2);
+        if (warp == 0) {
+          // pairwise (every partial sum is exact, so any order gives the same)
+          double q1[W], q2h[W], q2l[W];
+#pragma unroll
+          for (int w = 0; w < W; ++w) {
+            q1[w] = sh.p1[par][32 * w + lane];
+            q2h[w] = sh.p2h[par][32 * w + lane];
+            q2l[w] = sh.p2l[par][32 * w + lane];
+          }
+#pragma unroll
+          for (int st = 1; st < W; st *= 2)
+#pragma unroll
+            for (int w = 0; w + st < W; w += 2 * st) {
+              q1[w] = __dadd_rn(q1[w], q1[w + st]);
+              q2h[w] = __dadd_rn(q2h[w], q2h[w + st]);
+              q2l[w] = __dadd_rn(q2l[w], q2l[w + st]);
+            }
+          const double t1 = q1[0], t2h = q2h[0], t2l = q2l[0];
+          bad = !(fabs(t1) <= 1.7976931348623157e308) || !(fabs(t2h) <= 1.7976931348623157e308);
+          Sums t{bad ? 0 : __double2ll_rn(__dmul_rn(t1, 16777216.0)),          // units 2^-24
+                 bad ? 0 : __double2ll_rn(__dmul_rn(t2h, 8192.0)),             // units 2^-13
+                 bad ? 0 : __double2ll_rn(__dmul_rn(t2l, 281474976710656.0)),  // units 2^-48
+                 bad};
+          warp_sum(t);
+          float m_, r_;
+          ln_finalize(t, a.K, a.eps, m_, r_, k_log2);
+          if (lane == 0) {
+            sh.mu[par] = m_;
+            sh.rstd[par] = r_;
+          }
+        }
+        __syncthreads();
+        mu = sh.mu[par];
+        rstd = sh.rstd[par];
+      }
+
+      // transform in place and the row maximum (NaN-propagating)
+      float amax = 0.0f;
+      {
+        const uint64_t mu2 = f2_pack(mu, mu), r2 = f2_pack(rstd, rstd);
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+          const int64_t c = tid + static_cast<int64_t>(i) * T;
+          if (FULL || c < Kc) {
+            const int64_t k0 = c * 8;
+            if (use_ln) {
+              const float4 g0 = __ldg(reinterpret_cast<const float4*>(a.gamma + k0));
+              const float4 g1 = __ldg(reinterpret_cast<const float4*>(a.gamma + k0) + 1);
+              const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+              float bb[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+              if (a.beta) {
+                const float4 b0 = __ldg(reinterpret_cast<const float4*>(a.beta + k0));
+                const float4 b1 = __ldg(reinterpret_cast<const float4*>(a.beta + k0) + 1);
+                bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w;
+                bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
+              }
+              // ((x - mu) * rstd) * gamma in packed pairs; the add of beta stays
+              // scalar (a packed add right after a packed multiply was seen
+              // contracted into one fused multiply-add)
+#pragma unroll
+              for (int jj = 0; jj < 8; jj += 2) {
+                const float2 f = f2_unpack(f2_mul_rn(f2_mul_rn(f2_sub_rn(f2_pack(x[i][jj], x[i][jj + 1]), mu2), r2),
+                                                     f2_pack(gg[jj], gg[jj + 1])));
+                x[i][jj] = f.x;
+                x[i][jj + 1] = f.y;
+              }
+              if (a.beta) {
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) x[i][jj] = __fadd_rn(x[i][jj], bb[jj]);
+              }
+            }
+            if (a.vec) {
+              const float4 i0 = __ldg(reinterpret_cast<const float4*>(a.vec + k0));
+              const float4 i1 = __ldg(reinterpret_cast<const float4*>(a.vec + k0) + 1);
+              const float is[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+#pragma unroll
+              for (int jj = 0; jj < 8; jj += 2) {
+                float2 f = f2_unpack(f2_mul_rn(f2_pack(x[i][jj], x[i][jj + 1]), f2_pack(is[jj], is[jj + 1])));
+                // a weight row: x = fp16(w * s), the folded weight rounded once to fp16
+                if (MODE == MODE_WEIGHT) f = __half22float2(__floats2half2_rn(f.x, f.y));
+                x[i][jj] = f.x;
+                x[i][jj + 1] = f.y;
+              }
+            }
+#pragma unroll
+            for (int jj = 0; jj < 8; jj += 2) amax = absmax3(amax, x[i][jj], x[i][jj + 1]);
+          }
+        }
+      }
+      // amax is >= 0 or a positive NaN (max.NaN of absolute values)
+      const uint32_t wmax = warp_max_u32(__float_as_uint(amax));
+      if (lane == 0) sh.mx[par][warp] = wmax;
+      __syncthreads();  // (without a LayerNorm: every thread has read slot s)
+      if (!use_ln) {
+        consumed = j + 1;
+        if (tid == 0) issue(j + 2);
+      }
+      uint32_t mb = 0;
+#pragma unroll
+      for (int w = 0; w < W; ++w) mb = max(mb, sh.mx[par][w]);
+      float m = __uint_as_float(mb);
+      const bool safe = !finite_f(m);  // CTA-uniform
+      if (safe) {  // a NaN or an Inf in the row: the range ignores NaN
+        float a2 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NCH; ++i)
+          if (FULL || tid + static_cast<int64_t>(i) * T < Kc)
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) a2 = fmaxf(a2, fabsf(x[i][jj]));
+        const uint32_t w2 = warp_max_u32(__float_as_uint(a2));  // NaN-free, >= 0
+        if (lane == 0) sh.mx2[par][warp] = w2;
+        __syncthreads();
+        mb = 0;
+#pragma unroll
+        for (int w = 0; w < W; ++w) mb = max(mb, sh.mx2[par][w]);
+        m = __uint_as_float(mb);
+      }
+      const float sc = __fdiv_rn(m, 127.0f);
+      const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+      if (tid == 0) a.scale[r] = sc;
+      int8_t* dst = a.q + r * a.K;
+      const uint64_t inv2 = f2_pack(inv, inv);
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        const int64_t c = tid + static_cast<int64_t>(i) * T;
+        if (FULL || c < Kc) {
+          uint32_t b[8];
+          // x * (1 / scale) in packed pairs, then + 1.5 * 2^23 in scalar adds (each rounded)
+#pragma unroll
+          for (int jj = 0; jj < 8; jj += 2) {
+            const float2 p = f2_unpack(f2_mul_rn(f2_pack(x[i][jj], x[i][jj + 1]), inv2));
+            b[jj] = __float_as_uint(__fadd_rn(p.x, 12582912.0f));
+            b[jj + 1] = __float_as_uint(__fadd_rn(p.y, 12582912.0f));
+          }
+          if (safe) {
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) b[jj] = min(b[jj], 0x4B400100u);
+          }
+          const uint32_t lo4 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+          const uint32_t hi4 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+          *reinterpret_cast<uint2*>(dst + c * 8) = make_uint2(lo4, hi4);
+        }
+      }
+    }
+  } else {
+    // rows of eight warps
+    // one thread waits for copy j when `has` (the others wait at the barrier,
+    // issuing nothing); the barrier also turns a time-out into a CTA-wide stop
+    auto wait_copy = [&](int64_t j, bool has) {
+      bool ok = true;
+      if (tid == 0 && has)
+        ok = mbar_wait_bounded(full0 + 8u * static_cast<uint32_t>(j & 1), static_cast<uint32_t>((j >> 1) & 1), budget);
+      if (__syncthreads_or(!ok)) return false;
+      if (has) consumed = j + 1;
+      return true;
+    };
+    // this thread's NCH chunks of the row in slot s, as fp32 (chunks past K are zeros)
+    auto load_x = [&](uint32_t s, float (&x)[NCH][8]) {
+      const uint4* src = reinterpret_cast<const uint4*>(ring + s * row_bytes);
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        const int64_t c = tid + static_cast<int64_t>(i) * T;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (FULL || c < Kc) v = src[c];
+        unpack8(v, x[i]);
+      }
+    };
+    // the exact LayerNorm partials of this thread's chunks of the row in slot s
+    // (read again from shared memory, each fp16 value converted once to fp64)
+    // into sh.p*[pp][tid]: exact, multiples of 2^-24, 2^-9 and 2^-48 far inside
+    // 53 bits; an Inf or a NaN in the row leaves them non-finite
+    auto stats = [&](uint32_t s, int pp) {
+      const uint4* src = reinterpret_cast<const uint4*>(ring + s * row_bytes);
+      double s1[2] = {0.0, 0.0}, hi[2] = {kS2Bias, kS2Bias}, lo[2] = {0.0, 0.0};
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        const int64_t c = tid + static_cast<int64_t>(i) * T;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (FULL || c < Kc) v = src[c];
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           const int u = jj & 1;
-          const double d = static_cast<double>(x[i][jj]);
+          const double d = half_to_f64(half_bits(v, jj));
           s1[u] = __dadd_rn(s1[u], d);
           const double hn = __fma_rn(d, d, hi[u]);
           lo[u] = __dadd_rn(lo[u], __fma_rn(d, d, __dsub_rn(hi[u], hn)));
           hi[u] = hn;
         }
       }
-      // this thread's partials (exact: multiples of 2^-24, 2^-9 and 2^-48 far
-      // inside 53 bits); an Inf or a NaN in the row leaves them non-finite
-      sh.p1[par][tid] = __dadd_rn(s1[0], s1[1]);
-      sh.p2h[par][tid] = __dadd_rn(__dsub_rn(hi[0], kS2Bias), __dsub_rn(hi[1], kS2Bias));
-      sh.p2l[par][tid] = __dadd_rn(lo[0], lo[1]);
-      __syncthreads();  // every thread has read slot s
-      consumed = j + 1;
-      if (tid == 0) issue(j + 2);
-      if (warp == 0) {
-        // pairwise (every partial sum is exact, so any order gives the same)
-        double q1[W], q2h[W], q2l[W];
+      sh.p1[pp][tid] = __dadd_rn(s1[0], s1[1]);
+      sh.p2h[pp][tid] = __dadd_rn(__dsub_rn(hi[0], kS2Bias), __dsub_rn(hi[1], kS2Bias));
+      sh.p2l[pp][tid] = __dadd_rn(lo[0], lo[1]);
+    };
+    // one warp: the row's mu / rstd from the partials sh.p*[pp] into sh.mu[pp], sh.rstd[pp]
+    auto finalize = [&](int pp) {
+      // pairwise (every partial sum is exact, so any order gives the same)
+      double q1[W], q2h[W], q2l[W];
 #pragma unroll
-        for (int w = 0; w < W; ++w) {
-          q1[w] = sh.p1[par][32 * w + lane];
-          q2h[w] = sh.p2h[par][32 * w + lane];
-          q2l[w] = sh.p2l[par][32 * w + lane];
+      for (int w = 0; w < W; ++w) {
+        q1[w] = sh.p1[pp][32 * w + lane];
+        q2h[w] = sh.p2h[pp][32 * w + lane];
+        q2l[w] = sh.p2l[pp][32 * w + lane];
+      }
+#pragma unroll
+      for (int st = 1; st < W; st *= 2)
+#pragma unroll
+        for (int w = 0; w + st < W; w += 2 * st) {
+          q1[w] = __dadd_rn(q1[w], q1[w + st]);
+          q2h[w] = __dadd_rn(q2h[w], q2h[w + st]);
+          q2l[w] = __dadd_rn(q2l[w], q2l[w + st]);
         }
+      const double t1 = q1[0], t2h = q2h[0], t2l = q2l[0];
+      const int bad = !(fabs(t1) <= 1.7976931348623157e308) || !(fabs(t2h) <= 1.7976931348623157e308);
+      Sums t{bad ? 0 : __double2ll_rn(__dmul_rn(t1, 16777216.0)),          // units 2^-24
+             bad ? 0 : __double2ll_rn(__dmul_rn(t2h, 8192.0)),             // units 2^-13
+             bad ? 0 : __double2ll_rn(__dmul_rn(t2l, 281474976710656.0)),  // units 2^-48
+             bad};
+      warp_sum(t);
+      float m_, r_;
+      ln_finalize(t, a.K, a.eps, m_, r_, k_log2);
+      if (lane == 0) {
+        sh.mu[pp] = m_;
+        sh.rstd[pp] = r_;
+      }
+    };
+    // this warp's row maximum (bit patterns: amax is >= 0 or a positive NaN)
+    auto publish = [&](float amax, int pp) {
+      const uint32_t wmax = warp_max_u32(__float_as_uint(amax));
+      if (lane == 0) sh.mx[pp][warp] = wmax;
+    };
+    // the transform in place and this thread's row maximum (NaN-propagating)
+    auto transform = [&](float (&x)[NCH][8], float mu, float rstd) {
+      float amax = 0.0f;
+      {
+        const uint64_t mu2 = f2_pack(mu, mu), r2 = f2_pack(rstd, rstd);
 #pragma unroll
-        for (int st = 1; st < W; st *= 2)
+        for (int i = 0; i < NCH; ++i) {
+          const int64_t c = tid + static_cast<int64_t>(i) * T;
+          if (FULL || c < Kc) {
+            const int64_t k0 = c * 8;
+            if (use_ln) {
+              const float4 g0 = __ldg(reinterpret_cast<const float4*>(a.gamma + k0));
+              const float4 g1 = __ldg(reinterpret_cast<const float4*>(a.gamma + k0) + 1);
+              const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+              float bb[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+              if (a.beta) {
+                const float4 b0 = __ldg(reinterpret_cast<const float4*>(a.beta + k0));
+                const float4 b1 = __ldg(reinterpret_cast<const float4*>(a.beta + k0) + 1);
+                bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w;
+                bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
+              }
+              // ((x - mu) * rstd) * gamma in packed pairs; the add of beta stays
+              // scalar (a packed add right after a packed multiply was seen
+              // contracted into one fused multiply-add)
 #pragma unroll
-          for (int w = 0; w + st < W; w += 2 * st) {
-            q1[w] = __dadd_rn(q1[w], q1[w + st]);
-            q2h[w] = __dadd_rn(q2h[w], q2h[w + st]);
-            q2l[w] = __dadd_rn(q2l[w], q2l[w + st]);
+              for (int jj = 0; jj < 8; jj += 2) {
+                const float2 f = f2_unpack(f2_mul_rn(f2_mul_rn(f2_sub_rn(f2_pack(x[i][jj], x[i][jj + 1]), mu2), r2),
+                                                     f2_pack(gg[jj], gg[jj + 1])));
+                x[i][jj] = f.x;
+                x[i][jj + 1] = f.y;
+              }
+              if (a.beta) {
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) x[i][jj] = __fadd_rn(x[i][jj], bb[jj]);
+              }
+            }
+            if (a.vec) {
+              const float4 i0 = __ldg(reinterpret_cast<const float4*>(a.vec + k0));
+              const float4 i1 = __ldg(reinterpret_cast<const float4*>(a.vec + k0) + 1);
+              const float is[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+#pragma unroll
+              for (int jj = 0; jj < 8; jj += 2) {
+                float2 f = f2_unpack(f2_mul_rn(f2_pack(x[i][jj], x[i][jj + 1]), f2_pack(is[jj], is[jj + 1])));
+                // a weight row: x = fp16(w * s), the folded weight rounded once to fp16
+                if (MODE == MODE_WEIGHT) f = __half22float2(__floats2half2_rn(f.x, f.y));
+                x[i][jj] = f.x;
+                x[i][jj + 1] = f.y;
+              }
+            }
+#pragma unroll
+            for (int jj = 0; jj < 8; jj += 2) amax = absmax3(amax, x[i][jj], x[i][jj + 1]);
           }
-        const double t1 = q1[0], t2h = q2h[0], t2l = q2l[0];
-        bad = !(fabs(t1) <= 1.7976931348623157e308) || !(fabs(t2h) <= 1.7976931348623157e308);
-        Sums t{bad ? 0 : __double2ll_rn(__dmul_rn(t1, 16777216.0)),          // units 2^-24
-               bad ? 0 : __double2ll_rn(__dmul_rn(t2h, 8192.0)),             // units 2^-13
-               bad ? 0 : __double2ll_rn(__dmul_rn(t2l, 281474976710656.0)),  // units 2^-48
-               bad};
-        warp_sum(t);
-        float m_, r_;
-        ln_finalize(t, a.K, a.eps, m_, r_, k_log2);
-        if (lane == 0) {
-          sh.mu[par] = m_;
-          sh.rstd[par] = r_;
         }
       }
-      __syncthreads();
-      mu = sh.mu[par];
-      rstd = sh.rstd[par];
-    }
-
-    // transform in place and the row maximum (NaN-propagating)
-    float amax = 0.0f;
-    {
-      const uint64_t mu2 = f2_pack(mu, mu), r2 = f2_pack(rstd, rstd);
+      return amax;
+    };
+    // row r's scale from the warps' maxima in sh.mx[par], then its codes
+    auto codes = [&](int64_t r, float (&x)[NCH][8], int par) {
+      uint32_t mb = 0;
+#pragma unroll
+      for (int w = 0; w < W; ++w) mb = max(mb, sh.mx[par][w]);
+      float m = __uint_as_float(mb);
+      const bool safe = !finite_f(m);  // CTA-uniform
+      if (safe) {  // a NaN or an Inf in the row: the range ignores NaN
+        float a2 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NCH; ++i)
+          if (FULL || tid + static_cast<int64_t>(i) * T < Kc)
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) a2 = fmaxf(a2, fabsf(x[i][jj]));
+        const uint32_t w2 = warp_max_u32(__float_as_uint(a2));  // NaN-free, >= 0
+        if (lane == 0) sh.mx2[par][warp] = w2;
+        __syncthreads();
+        mb = 0;
+#pragma unroll
+        for (int w = 0; w < W; ++w) mb = max(mb, sh.mx2[par][w]);
+        m = __uint_as_float(mb);
+      }
+      const float sc = __fdiv_rn(m, 127.0f);
+      const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
+      if (tid == 0) a.scale[r] = sc;
+      int8_t* dst = a.q + r * a.K;
+      const uint64_t inv2 = f2_pack(inv, inv);
 #pragma unroll
       for (int i = 0; i < NCH; ++i) {
         const int64_t c = tid + static_cast<int64_t>(i) * T;
         if (FULL || c < Kc) {
-          const int64_t k0 = c * 8;
-          if (use_ln) {
-            const float4 g0 = __ldg(reinterpret_cast<const float4*>(a.gamma + k0));
-            const float4 g1 = __ldg(reinterpret_cast<const float4*>(a.gamma + k0) + 1);
-            const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-            float bb[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            if (a.beta) {
-              const float4 b0 = __ldg(reinterpret_cast<const float4*>(a.beta + k0));
-              const float4 b1 = __ldg(reinterpret_cast<const float4*>(a.beta + k0) + 1);
-              bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w;
-              bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
-            }
-            // ((x - mu) * rstd) * gamma in packed pairs; the add of beta stays
-            // scalar (a packed add right after a packed multiply was seen
-            // contracted into one fused multiply-add)
+          uint32_t b[8];
+          // x * (1 / scale) in packed pairs, then + 1.5 * 2^23 in scalar adds (each rounded)
 #pragma unroll
-            for (int jj = 0; jj < 8; jj += 2) {
-              const float2 f = f2_unpack(f2_mul_rn(f2_mul_rn(f2_sub_rn(f2_pack(x[i][jj], x[i][jj + 1]), mu2), r2),
-                                                   f2_pack(gg[jj], gg[jj + 1])));
-              x[i][jj] = f.x;
-              x[i][jj + 1] = f.y;
-            }
-            if (a.beta) {
-#pragma unroll
-              for (int jj = 0; jj < 8; ++jj) x[i][jj] = __fadd_rn(x[i][jj], bb[jj]);
-            }
+          for (int jj = 0; jj < 8; jj += 2) {
+            const float2 p = f2_unpack(f2_mul_rn(f2_pack(x[i][jj], x[i][jj + 1]), inv2));
+            b[jj] = __float_as_uint(__fadd_rn(p.x, 12582912.0f));
+            b[jj + 1] = __float_as_uint(__fadd_rn(p.y, 12582912.0f));
           }
-          if (a.vec) {
-            const float4 i0 = __ldg(reinterpret_cast<const float4*>(a.vec + k0));
-            const float4 i1 = __ldg(reinterpret_cast<const float4*>(a.vec + k0) + 1);
-            const float is[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+          if (safe) {
 #pragma unroll
-            for (int jj = 0; jj < 8; jj += 2) {
-              float2 f = f2_unpack(f2_mul_rn(f2_pack(x[i][jj], x[i][jj + 1]), f2_pack(is[jj], is[jj + 1])));
-              // a weight row: x = fp16(w * s), the folded weight rounded once to fp16
-              if (MODE == MODE_WEIGHT) f = __half22float2(__floats2half2_rn(f.x, f.y));
-              x[i][jj] = f.x;
-              x[i][jj + 1] = f.y;
-            }
+            for (int jj = 0; jj < 8; ++jj) b[jj] = min(b[jj], 0x4B400100u);
           }
-#pragma unroll
-          for (int jj = 0; jj < 8; jj += 2) amax = absmax3(amax, x[i][jj], x[i][jj + 1]);
+          const uint32_t lo4 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+          const uint32_t hi4 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+          *reinterpret_cast<uint2*>(dst + c * 8) = make_uint2(lo4, hi4);
         }
       }
-    }
-    // amax is >= 0 or a positive NaN (max.NaN of absolute values)
-    const uint32_t wmax = warp_max_u32(__float_as_uint(amax));
-    if (lane == 0) sh.mx[par][warp] = wmax;
-    __syncthreads();  // (without a LayerNorm: every thread has read slot s)
+    };
+
     if (!use_ln) {
-      consumed = j + 1;
-      if (tid == 0) issue(j + 2);
-    }
-    uint32_t mb = 0;
-#pragma unroll
-    for (int w = 0; w < W; ++w) mb = max(mb, sh.mx[par][w]);
-    float m = __uint_as_float(mb);
-    const bool safe = !finite_f(m);  // CTA-uniform
-    if (safe) {  // a NaN or an Inf in the row: the range ignores NaN
-      float a2 = 0.0f;
-#pragma unroll
-      for (int i = 0; i < NCH; ++i)
-        if (FULL || tid + static_cast<int64_t>(i) * T < Kc)
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) a2 = fmaxf(a2, fabsf(x[i][jj]));
-      const uint32_t w2 = warp_max_u32(__float_as_uint(a2));  // NaN-free, >= 0
-      if (lane == 0) sh.mx2[par][warp] = w2;
-      __syncthreads();
-      mb = 0;
-#pragma unroll
-      for (int w = 0; w < W; ++w) mb = max(mb, sh.mx2[par][w]);
-      m = __uint_as_float(mb);
-    }
-    const float sc = __fdiv_rn(m, 127.0f);
-    const float inv = sc > 0.0f ? __frcp_rn(sc) : 0.0f;
-    if (tid == 0) a.scale[r] = sc;
-    int8_t* dst = a.q + r * a.K;
-    const uint64_t inv2 = f2_pack(inv, inv);
-#pragma unroll
-    for (int i = 0; i < NCH; ++i) {
-      const int64_t c = tid + static_cast<int64_t>(i) * T;
-      if (FULL || c < Kc) {
-        uint32_t b[8];
-        // x * (1 / scale) in packed pairs, then + 1.5 * 2^23 in scalar adds (each rounded)
-#pragma unroll
-        for (int jj = 0; jj < 8; jj += 2) {
-          const float2 p = f2_unpack(f2_mul_rn(f2_pack(x[i][jj], x[i][jj + 1]), inv2));
-          b[jj] = __float_as_uint(__fadd_rn(p.x, 12582912.0f));
-          b[jj + 1] = __float_as_uint(__fadd_rn(p.y, 12582912.0f));
+      for (int64_t j = 0;; ++j) {
+        const int64_t r = blockIdx.x + j * G;
+        if (r >= a.rows) break;
+        if (!wait_copy(j, true)) {
+          aborted = true;
+          break;
         }
-        if (safe) {
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) b[jj] = min(b[jj], 0x4B400100u);
+        const int pp = static_cast<int>(j & 1);
+        float x[NCH][8];
+        load_x(static_cast<uint32_t>(pp), x);
+        publish(transform(x, 0.0f, 0.0f), pp);
+        __syncthreads();  // every thread has read slot pp; the warps' maxima are in
+        if (tid == 0) issue(j + 2);
+        codes(r, x, pp);
+      }
+    } else {
+      // LayerNorm rows of eight warps, one row deep (the finalization, a reduction
+      // over eight warps' partials, then overlaps the other warps' codes): iteration j takes the partials of row j+1
+      // (its copy waited for at the iteration's first barrier, which also
+      // publishes row j's mu / rstd), transforms row j, and after the second
+      // barrier every warp writes row j's codes, one of them (in turn) then
+      // finalizing row j+1 while the others go on to the next barrier
+      if (static_cast<int64_t>(blockIdx.x) < a.rows) {
+        if (!wait_copy(0, true)) {
+          aborted = true;
+        } else {
+          stats(0u, 0);
+          __syncthreads();
+          if (warp == 0) finalize(0);
         }
-        const uint32_t lo4 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
-        const uint32_t hi4 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
-        *reinterpret_cast<uint2*>(dst + c * 8) = make_uint2(lo4, hi4);
+      }
+      for (int64_t j = 0; !aborted; ++j) {
+        const int64_t r = blockIdx.x + j * G;
+        if (r >= a.rows) break;
+        const bool nxt = r + G < a.rows;
+        const int pp = static_cast<int>(j & 1), pn = pp ^ 1;
+        if (!wait_copy(j + 1, nxt)) {
+          aborted = true;
+          break;
+        }
+        if (nxt) stats(static_cast<uint32_t>(pn), pn);
+        float x[NCH][8];
+        load_x(static_cast<uint32_t>(pp), x);
+        publish(transform(x, sh.mu[pp], sh.rstd[pp]), pp);
+        __syncthreads();  // slot pp read; row j's maxima and row j+1's partials are in
+        if (tid == 0) issue(j + 2);
+        codes(r, x, pp);
+        // (after the codes: the row's values are no longer held meanwhile)
+        if (nxt && warp == static_cast<int>(j % W)) finalize(pn);
       }
     }
   }
@@ -1219,8 +1476,18 @@ __device__ __forceinline__ void rows_bulk(const RowArgs& a, uint32_t* status, ui
 
 // Activation rows (LayerNorm and / or 1/s, per-token scales) and weight rows
 // (fold diag(s) rounded to fp16, per-output-channel scales).
+// CTAs per SM the activation kernel is built for: two for rows of eight warps
+// (at most 128 registers per thread, which the one-row-deep LayerNorm pipeline
+// would otherwise exceed); 0, no bound, otherwise (a bound of one CTA lets the
+// compiler spend more registers on the one-row-at-a-time loop, measured slower).
+template <int T, int NCH>
+constexpr int act_min_ctas() {
+  return T >= 256 ? 2 : 0;
+}
+
 template <int T, int NCH, bool FULL>
-__global__ void __launch_bounds__(T) k_act_rows_bulk(const RowArgs a, uint32_t* status, uint64_t budget) {
+__global__ void __launch_bounds__(T, act_min_ctas<T, NCH>()) k_act_rows_bulk(const RowArgs a, uint32_t* status,
+                                                                              uint64_t budget) {
   rows_bulk<MODE_ACT, T, NCH, FULL>(a, status, budget);
 }
 
