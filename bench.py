@@ -23,6 +23,7 @@ import ctypes
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -106,12 +107,11 @@ def traffic_from_profile(kernel_src: str, profile_md: str):
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
             got[k.strip()] = v.strip().strip("`")
-    if got.get("source_sha256_16") != sha:
+    m = re.search(r"\b[0-9a-f]{16}\b", got.get("source_sha256_16", ""))
+    if m is None or m.group(0) != sha:
         return None
-    try:
-        return int(float(got["dram_bytes_per_launch"]))
-    except (KeyError, ValueError):
-        return None
+    n = re.match(r"[0-9.]+", got.get("dram_bytes_per_launch", ""))
+    return int(float(n.group(0))) if n else None
 
 
 class ClockSampler:
