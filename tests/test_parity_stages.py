@@ -27,7 +27,10 @@ def rand_h(rng, M, K, outliers=(), gain=60.0, shift=0.0):
 
 
 # ------------------------------------------------------------ calibration ----
-@pytest.mark.parametrize("rows,K", [(1, 16), (7, 48), (128, 256), (300, 4112), (33, 2064)])
+# (4100, 4112) and (1030, 12304): several 32-row boxes per band of the streamed
+# kernel, a ragged last box and a partial last block of 256 columns
+@pytest.mark.parametrize("rows,K", [(1, 16), (7, 48), (128, 256), (300, 4112), (33, 2064), (4100, 4112),
+                                    (1030, 12304)])
 def test_calibrate_absmax_raw(sq, rows, K):
     rng = np.random.default_rng(rows * 7 + K)
     x = rand_h(rng, rows, K, outliers=(0, K - 1, K // 3))

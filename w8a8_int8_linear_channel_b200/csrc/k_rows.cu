@@ -956,17 +956,6 @@ __device__ __forceinline__ void bulk_row_load(uint32_t dst, const void* src, uin
                : "memory");
 }
 
-// Bounded wait that records nothing (the caller turns a time-out into a
-// CTA-wide decision at its next barrier).
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait_hint(bar, parity, 2000)) {  // suspended up to 2 us per try, not spinning
-    if (globaltimer_ns() - t0 > budget_ns) return false;
-  }
-  return true;
-}
-
 template <int T, bool STATS>
 struct ActShared {
   static constexpr int NP = STATS ? T : 1;

@@ -71,6 +71,17 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity
   return ok != 0;
 }
 
+// Bounded wait that records nothing (the caller turns a time-out into a
+// CTA-wide decision at its next barrier).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait_hint(bar, parity, 2000)) {  // suspended up to 2 us per try, not spinning
+    if (globaltimer_ns() - t0 > budget_ns) return false;
+  }
+  return true;
+}
+
 // Bounded wait for the phase of `bar` with parity `parity` to complete.
 // Gives up after budget_ns (wall time from %globaltimer) or as soon as
 // *abort becomes non-zero; on running out it records DEV_TIMEOUT in *status
