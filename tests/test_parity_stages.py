@@ -27,8 +27,8 @@ def rand_h(rng, M, K, outliers=(), gain=60.0, shift=0.0):
 
 
 # ------------------------------------------------------------ calibration ----
-# (4100, 4112) and (1030, 12304): several 32-row boxes per band of the streamed
-# kernel, a ragged last box and a partial last block of 256 columns
+# (4100, 4112) and (1030, 12304): many row bands per block of 256 columns, a
+# ragged last band and a partial last column block
 @pytest.mark.parametrize("rows,K", [(1, 16), (7, 48), (128, 256), (300, 4112), (33, 2064), (4100, 4112),
                                     (1030, 12304)])
 def test_calibrate_absmax_raw(sq, rows, K):
