@@ -902,8 +902,8 @@ __global__ void __launch_bounds__(kCtaThreads) k_calib_cta_atomic(const RowArgs 
 // bulk copies (cp.async.bulk, one instruction per row, completion counted on
 // an mbarrier), so each CTA has the next row in flight while it works on the
 // current one and no register holds prefetched data.  Every thread keeps its
-// NCH chunks of 8 values as fp32 in registers from the one read of shared
-// memory to the codes.  Per element:
+// NCH chunks of 8 values as fp32 in registers from its read of shared memory
+// to the codes.  Per element:
 //   statistics  exact sums in fp64: h (a multiple of 2^-24, |h| < 2^16) adds
 //               exactly into an fp64 accumulator; h*h (exact in fp64) goes
 //               into an accumulator A biased by 1.5 * 2^43 (unit in the last
@@ -913,10 +913,10 @@ __global__ void __launch_bounds__(kCtaThreads) k_calib_cta_atomic(const RowArgs 
 //               remainder, a multiple of 2^-48 below 2^-10), into a second
 //               accumulator.  Two independent sets per thread (even / odd
 //               elements), added (exactly) into three fp64 partials per
-//               thread.  Warp 0 alone reduces them: per lane the partials of
-//               T / 32 threads in fp64 (exact: at most 512 elements), then as
-//               int64 across the warp: S1 = sum v and S2 = sum v^2
-//               (v = h * 2^24) exactly, whatever the order.
+//               thread.  One warp alone reduces them: per lane the partials
+//               of T / 32 threads in fp64, pairwise (exact: at most 512
+//               elements), then as int64 across the warp: S1 = sum v and
+//               S2 = sum v^2 (v = h * 2^24) exactly, whatever the order.
 //   transform   (x - mu) * rstd, then * gamma, in packed fp32 pairs (each lane
 //               rounded like the scalar op), + beta in scalar adds (a packed add
 //               after a packed multiply can be contracted into a fused
@@ -930,10 +930,14 @@ __global__ void __launch_bounds__(kCtaThreads) k_calib_cta_atomic(const RowArgs 
 // One thread waits for each row (suspended in the mbarrier try-wait, bounded);
 // the others wait at the row's first barrier, which also turns a time-out into
 // a CTA-wide stop, after which the CTA waits (bounded) for its copies in
-// flight before returning.  Then two more barriers with a LayerNorm
-// (statistics, mu / rstd), and one for the row maximum.  Rows with a
-// non-finite maximum take the NaN-free maximum and the NaN-safe codes, as in
-// the kernels above.
+// flight before returning.  Rows of up to four warps, one at a time: with a
+// LayerNorm two more barriers (statistics from the values in registers, then
+// mu / rstd from warp 0) and one for the row maximum.  Rows of eight warps
+// with a LayerNorm run one row deep instead: the statistics of row j+1 (read
+// again from its slot) and the transform of row j between the same two
+// barriers, the finalization of row j+1 by one warp after row j's codes.
+// Rows with a non-finite maximum take the NaN-free maximum and the NaN-safe
+// codes, as in the kernels above.
 // =========================================================================
 constexpr double kS2Bias = 13194139533312.0;  // 1.5 * 2^43: unit in the last place 2^-9
 
