@@ -49,20 +49,22 @@ constexpr int B_BYTES = BNH * BK;  // 16 KB
 constexpr int RING = 6 * (A_BYTES + B_BYTES);  // 192 KB of pipeline stages
 // The ring as 6 stages of one 128-byte K box (short K) or 3 stages of two
 // (K >= 512: half the barrier round trips and MMA commits per K byte, which
-// measured 5 % faster on 2048 x 4096 x 4096 and 7-8 % on longer grids).
-template <int KSUB>
+// measured 5 % faster on 2048 x 4096 x 4096 and 7-8 % on longer grids).  With
+// tiles TBN = 128 channels wide (the batched product at N <= 128) each CTA
+// loads 64 weight rows per box: 8 stages of one box, 4 of two.
+template <int KSUB, int TBN = BN>
 struct Ring {
-  static constexpr int STAGE_BYTES = KSUB * (A_BYTES + B_BYTES);
+  static constexpr int STAGE_BYTES = KSUB * (A_BYTES + (TBN / 2) * BK);
   static constexpr int STAGES = RING / STAGE_BYTES;
-  static_assert(STAGES * STAGE_BYTES == RING && STAGES >= 2, "ring of whole stages");
+  static_assert(STAGES * STAGE_BYTES == RING && STAGES >= 2 && STAGES <= 8, "ring of whole stages");
 };
 constexpr int STG = RING;                  // per-epilogue-warp output staging
 constexpr int STG_BYTES = 2048;            // one 32 rows x 32 fp16 block, 64-byte swizzle
 constexpr int STG_WARP = 2 * STG_BYTES;    // double-buffered per warp
 constexpr int CTRL = STG + kEpiWarps * STG_WARP;
 // barriers: full[S] (leader: both CTAs' loads landed), empty[S], accf[2],
-// acce[2] (leader: both epilogues done), drain; sized for the 6-stage ring
-constexpr int NBARS = 2 * Ring<1>::STAGES + 5;
+// acce[2] (leader: both epilogues done), drain; sized for the 8-stage ring
+constexpr int NBARS = 2 * 8 + 5;
 // TMEM address, abort flag, decision[2], loads issued by the peer
 constexpr int SLOT = CTRL + NBARS * 8;
 // sw[BN] fp32, bias[BN] fp16 of the current tile, read as 16-byte vectors
@@ -170,12 +172,19 @@ __device__ __forceinline__ bool pair_wait(uint32_t bar, uint32_t parity, bool cl
 // TMAS: fp16 blocks leave through TMA stores (rows 16-byte aligned); without
 // it they go through the warp's staging, row by row (a separate
 // instantiation, so the TMA-store kernel keeps its own registers).
-template <int EPI, bool TMAS, int KSUB>
+// TBN: channels per tile, 256, or 128 for the batched product at N <= 128
+// (P V of attention: a 256-wide tile would be half padding).
+template <int EPI, bool TMAS, int KSUB, int TBN = BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, const GemmArgs g, const TileMap tmap, int tiles,
                 uint32_t* status, uint64_t budget) {
-  constexpr int STAGES = Ring<KSUB>::STAGES, STAGE_BYTES = Ring<KSUB>::STAGE_BYTES;
+  constexpr int STAGES = Ring<KSUB, TBN>::STAGES, STAGE_BYTES = Ring<KSUB, TBN>::STAGE_BYTES;
+  static_assert(TBN == BN || (TBN == BN / 2 && EPI == EPI_BMM), "128-wide tiles: the batched product");
+  constexpr int TNH = TBN / 2;            // weight rows per CTA
+  constexpr int TB_BYTES = TNH * BK;      // one weight box per CTA
+  constexpr int CW = TBN / 2;             // columns of a tile per epilogue warp
+  constexpr int NB = CW / 32;             // 32-column blocks per epilogue warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -242,7 +251,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         int bi, tm, tn;  // batch item (0 when not batched), token tile, channel tile
         tmap.coords<EPI == EPI_BMM>(t, bi, tm, tn);
         const int32_t m0 = tm * (2 * BM) + static_cast<int32_t>(rank) * BM;
-        const int32_t n0 = tn * BN + static_cast<int32_t>(rank) * BNH;
+        const int32_t n0 = tn * TBN + static_cast<int32_t>(rank) * TNH;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = static_cast<int>(it % STAGES);
           const int64_t r = it / STAGES;
@@ -256,7 +265,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < KSUB; ++j) {
             const int32_t x = (kb * KSUB + j) * BK;
-            const uint32_t sa = st + j * A_BYTES, sb = st + KSUB * A_BYTES + j * B_BYTES;
+            const uint32_t sa = st + j * A_BYTES, sb = st + KSUB * A_BYTES + j * TB_BYTES;
             if constexpr (EPI == EPI_BMM) {
               tma_load_3d_pair(sa, &tmA, full_leader0 + 8u * s, x, m0, bi);
               tma_load_3d_pair(sb, &tmB, full_leader0 + 8u * s, x, n0, bi);
@@ -272,7 +281,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // leader: one pair MMA of 256 x 256 x 32 per 32 bytes of K
-      constexpr uint32_t idesc = idesc_i8(2 * BM, BN);
+      constexpr uint32_t idesc = idesc_i8(2 * BM, TBN);
       int64_t it = 0;
       int tl = 0;
       bool ok = true;
@@ -282,7 +291,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             !pair_wait(acce_bar(b), static_cast<uint32_t>(((tl >> 1) - 1) & 1), true, budget, status, abort_flag, peer_abort))
           break;
         tc_fence_after();
-        const uint32_t dacc = tmem + static_cast<uint32_t>(b * BN);
+        const uint32_t dacc = tmem + static_cast<uint32_t>(b * TBN);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = static_cast<int>(it % STAGES);
           const uint32_t par = static_cast<uint32_t>((it / STAGES) & 1);
@@ -296,7 +305,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int j = 0; j < KSUB; ++j) {
             if (j > 0 && static_cast<int64_t>(kb * KSUB + j) * BK >= g.K) break;  // a box wholly past K: zeros
             const uint64_t a = sdesc_k_sw128(st + j * A_BYTES);
-            const uint64_t bd = sdesc_k_sw128(st + KSUB * A_BYTES + j * B_BYTES);
+            const uint64_t bd = sdesc_k_sw128(st + KSUB * A_BYTES + j * TB_BYTES);
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k)
               mma_i8_pair(dacc, a + 2u * k, bd + 2u * k, idesc, (kb | j | k) != 0 ? 1u : 0u);
@@ -311,7 +320,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       griddep_launch_dependents();
     }
   } else {
-    // epilogue: 256 threads over this CTA's 128 rows x 256 columns
+    // epilogue: 256 threads over this CTA's 128 rows x TBN columns
     const int et = threadIdx.x - 64;
     const int q = warp & 3;            // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;  // column half of the tile
@@ -338,9 +347,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (EPI == EPI_I32 || t >= tiles) return v;
       int bi, tm, tn;
       tmap.coords<EPI == EPI_BMM>(t, bi, tm, tn);
-      const int64_t n = static_cast<int64_t>(tn) * BN + et;
+      const int64_t n = static_cast<int64_t>(tn) * TBN + et;
       const int64_t row = static_cast<int64_t>(tm) * (2 * BM) + static_cast<int64_t>(rank) * BM + 32 * q + lane;
-      if (n < g.N) {
+      if (et < TBN && n < g.N) {  // thread et < TBN holds column et's entries
         v.sw = g.sw[static_cast<int64_t>(bi) * g.N + n];
         if (g.bias != nullptr) v.bias = g.bias[n];
         if (EPI == EPI_Q8 && g.inv_s_next != nullptr) v.is = g.inv_s_next[n];
@@ -355,10 +364,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int bi, tm, tn;  // batch item (0 when not batched), token tile, channel tile
       tmap.coords<EPI == EPI_BMM>(t, bi, tm, tn);
       const int64_t m0 = static_cast<int64_t>(tm) * (2 * BM) + static_cast<int64_t>(rank) * BM;
-      const int64_t n0 = static_cast<int64_t>(tn) * BN;
+      const int64_t n0 = static_cast<int64_t>(tn) * TBN;
       const Vecs cur = nxt;
       nxt = fetch(t + npairs);
-      if (EPI != EPI_I32) {
+      if (EPI != EPI_I32 && et < TBN) {
         sw_s[et] = cur.sw;
         bias_s[et] = cur.bias;
         if (EPI == EPI_Q8) inv_s_s[et] = cur.is;
@@ -382,11 +391,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       float pmax = 0.0f;  // EPI_QD: this lane's row maximum over the warp's 128 columns
       auto taddr = [&](int c) {
         return tmem + (static_cast<uint32_t>(32 * q) << 16) +
-               static_cast<uint32_t>(BN * b + 128 * half + 32 * c);
+               static_cast<uint32_t>(TBN * b + CW * half + 32 * c);
       };
       const int64_t row0 = m0 + 32 * q;  // first row of this warp's blocks
       auto emit = [&](int c, uint32_t (&v)[32]) {
-        const int cl = 128 * half + 32 * c;  // column within the tile
+        const int cl = CW * half + 32 * c;  // column within the tile
         const int64_t col0 = n0 + cl;
         // rows / columns of this warp's 32 x 32 block inside the output (warp-uniform)
         const int brows = g.M - row0 < 32 ? static_cast<int>(g.M - row0) : 32;
@@ -565,13 +574,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tmem_ld_32x32b_x32(taddr(1), vb);
       emit(0, va);
       tmem_ld_wait_regs(vb);
-      tmem_ld_32x32b_x32(taddr(2), va);
-      emit(1, vb);
-      tmem_ld_wait_regs(va);
-      tmem_ld_32x32b_x32(taddr(3), vb);
-      emit(2, va);
-      tmem_ld_wait_regs(vb);
-      emit(3, vb);
+      if constexpr (NB == 4) {
+        tmem_ld_32x32b_x32(taddr(2), va);
+        emit(1, vb);
+        tmem_ld_wait_regs(va);
+        tmem_ld_32x32b_x32(taddr(3), vb);
+        emit(2, va);
+        tmem_ld_wait_regs(vb);
+        emit(3, vb);
+      } else {
+        emit(1, vb);
+      }
       if constexpr (EPI == EPI_QD) {
         const int64_t row = row0 + lane;
         // every group of the row is written (a group wholly past N holds 0), so the
@@ -646,35 +659,35 @@ int max_pairs(int device, int num_sms) {
   return n;
 }
 
-template <int EPI, bool TMAS, int KSUB>
+template <int EPI, bool TMAS, int KSUB, int TBN>
 cudaError_t smem_attr(int device) {
   static bool attr_set[64] = {};
   const int dev = device < 64 ? device : 63;
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_pair<EPI, TMAS, KSUB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(SMEM));
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_pair<EPI, TMAS, KSUB, TBN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SMEM));
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   return cudaSuccess;
 }
 
-template <int EPI, bool TMAS, int KSUB>
+template <int EPI, bool TMAS, int KSUB, int TBN>
 cudaError_t launch_kernel(const GemmArgs& g, const Ctx& c, const CUtensorMap& tmA, const CUtensorMap& tmB,
                           const CUtensorMap& tmY, int tiles_m, int tiles, int pairs) {
-  cudaError_t e = smem_attr<EPI, TMAS, KSUB>(c.device);
+  cudaError_t e = smem_attr<EPI, TMAS, KSUB, TBN>(c.device);
   if (e != cudaSuccess) return e;
   // tiles of one batch item (the whole grid when not batched)
   const int per_item = EPI == EPI_BMM ? tiles / static_cast<int>(g.batch) : tiles;
-  return launch_pdl(k_gemm_pair<EPI, TMAS, KSUB>, dim3(2 * pairs), dim3(kThreads), SMEM, c.stream, tmA, tmB, tmY,
-                    g, TileMap::make(per_item, tiles_m), tiles, c.status, c.budget_ns);
+  return launch_pdl(k_gemm_pair<EPI, TMAS, KSUB, TBN>, dim3(2 * pairs), dim3(kThreads), SMEM, c.stream, tmA, tmB,
+                    tmY, g, TileMap::make(per_item, tiles_m), tiles, c.status, c.budget_ns);
 }
 
-template <int EPI, bool TMAS>
+template <int EPI, bool TMAS, int TBN = BN>
 cudaError_t launch_ring(const GemmArgs& g, const Ctx& c, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         const CUtensorMap& tmY, int tiles_m, int tiles, int pairs) {
-  if (g.K >= 512) return launch_kernel<EPI, TMAS, 2>(g, c, tmA, tmB, tmY, tiles_m, tiles, pairs);
-  return launch_kernel<EPI, TMAS, 1>(g, c, tmA, tmB, tmY, tiles_m, tiles, pairs);
+  if (g.K >= 512) return launch_kernel<EPI, TMAS, 2, TBN>(g, c, tmA, tmB, tmY, tiles_m, tiles, pairs);
+  return launch_kernel<EPI, TMAS, 1, TBN>(g, c, tmA, tmB, tmY, tiles_m, tiles, pairs);
 }
 
 template <int EPI>
@@ -682,9 +695,12 @@ cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
   CUtensorMap tmA, tmB, tmY;
   const bool bmm = EPI == EPI_BMM;
   const uint64_t items = bmm ? static_cast<uint64_t>(g.batch) : 1;
+  // the batched product with at most 128 channels (P V): tiles 128 wide
+  const bool narrow = bmm && g.N <= BN / 2;
+  const int tbn = narrow ? BN / 2 : BN;
   if (bmm) {
     if (!make_tmap_i8_3d(&tmA, g.xq, g.K, g.M, items, BK, BM)) return cudaErrorInvalidValue;
-    if (!make_tmap_i8_3d(&tmB, g.wq, g.K, g.N, items, BK, BNH)) return cudaErrorInvalidValue;
+    if (!make_tmap_i8_3d(&tmB, g.wq, g.K, g.N, items, BK, tbn / 2)) return cudaErrorInvalidValue;
   } else {
     if (!make_tmap_i8(&tmA, g.xq, g.K, g.M, BK, BM)) return cudaErrorInvalidValue;
     if (!make_tmap_i8(&tmB, g.wq, g.K, g.N, BK, BNH)) return cudaErrorInvalidValue;
@@ -700,7 +716,7 @@ cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
     memset(&tmY, 0, sizeof(tmY));
   }
   const int tiles_m = static_cast<int>((g.M + 2 * BM - 1) / (2 * BM));
-  const int tiles_n = static_cast<int>((g.N + BN - 1) / BN);
+  const int tiles_n = static_cast<int>((g.N + tbn - 1) / tbn);
   const int64_t tiles64 = static_cast<int64_t>(items) * tiles_m * tiles_n;
   if (tiles64 > 0x7fffffffLL) return cudaErrorInvalidValue;
   const int tiles = static_cast<int>(tiles64);
@@ -710,6 +726,11 @@ cudaError_t launch_cfg(const GemmArgs& g, const Ctx& c) {
     if (!tma_store) return cudaErrorInvalidValue;
     return launch_ring<EPI, true>(g, c, tmA, tmB, tmY, tiles_m, tiles, pairs);
   } else {
+    if constexpr (EPI == EPI_BMM) {
+      if (narrow)
+        return tma_store ? launch_ring<EPI, true, BN / 2>(g, c, tmA, tmB, tmY, tiles_m, tiles, pairs)
+                         : launch_ring<EPI, false, BN / 2>(g, c, tmA, tmB, tmY, tiles_m, tiles, pairs);
+    }
     if (tma_store) {
       if constexpr (EPI == EPI_F16 || EPI == EPI_BMM)
         return launch_ring<EPI, true>(g, c, tmA, tmB, tmY, tiles_m, tiles, pairs);
