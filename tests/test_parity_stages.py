@@ -43,10 +43,11 @@ def test_calibrate_absmax_raw(sq, rows, K):
 
 
 # one case per kernel shape: a warp per row with 1, 2 or 4 chunks (K <= 256, 512, 1024), CTA
-# rows of 64, 128 or 256 threads (K <= 2048, 4096, 8192, 16384), and above 16384 the kernel
-# whose CTAs re-read each row from global memory and merge their column maxima with atomics
+# rows of 64, 128 or 256 threads (K <= 2048, 4096, 8192, 16384; 3000 and 1500 rows: several
+# rows per CTA, one of them with a ragged last chunk), and above 16384 the kernel whose CTAs
+# re-read each row from global memory and merge their column maxima with atomics
 @pytest.mark.parametrize("rows,K", [(5, 256), (6, 512), (64, 4096), (17, 1040), (12, 8192), (9, 16384),
-                                    (3, 49152), (2, 65536)])
+                                    (3, 49152), (2, 65536), (3000, 4096), (1500, 2064)])
 def test_calibrate_absmax_layernorm(sq, rows, K):
     rng = np.random.default_rng(rows + K)
     h = rand_h(rng, rows, K, shift=0.3)
