@@ -5,7 +5,9 @@ has NaN statistics, so its whole output is NaN; a NaN never wins a maximum;
 a NaN product is quantized to 0; an infinite range gives an infinite scale,
 a zero reciprocal and therefore codes 0.  Every row-kernel shape is covered
 (warp per row, register-resident CTA rows, CTA rows held in registers beyond
-eight chunks, CTA rows re-read from global), with calibration, weight
+eight chunks, CTA rows re-read from global, and at 300 x 12288 the bulk-copy
+rows of eight warps, where CTAs take two rows each and the LayerNorm loop runs
+one row deep, a non-finite row next to a finite one), with calibration, weight
 quantization (with and without the fold), the per-tensor levels, the fused
 producer-side quantization and the dequant epilogue."""
 import numpy as np
@@ -17,7 +19,7 @@ from gpu_util import bits_equal, dev, host
 
 pytestmark = pytest.mark.gpu
 
-SHAPES = [(6, 256), (5, 1024), (7, 4096), (5, 20480), (5, 65536)]
+SHAPES = [(6, 256), (5, 1024), (7, 4096), (300, 12288), (5, 20480), (5, 65536)]
 
 
 @pytest.fixture(scope="module")
