@@ -613,6 +613,9 @@ def run_gpu(args):
     if sq.sq_poll_status() != 0:
         raise RuntimeError("device wait timed out in the stage loop")
     stage_us = {c[0]: 1e3 * per_stage[j] / n_stage for j, c in enumerate(plan.calls)}
+    stage_cold = run_stage_cold(plan, torch, flush, args.burst_iters) if use_graph and world == 1 else None
+    if sq.sq_poll_status() != 0:
+        raise RuntimeError("device wait timed out in the cold stage loop")
 
     # the roofline's launch duration: back-to-back launches of the linear in
     # one graph (inputs as the step leaves them: L2-warm for the large-M
@@ -726,17 +729,24 @@ def run_gpu(args):
                     "timing": "CUDA events at the boundaries of every step, summed over steps, max over "
                               "ranks; stage_us and the roofline's launch time from a second loop with "
                               "events around every call (" + ("event nodes in a CUDA graph of the step"
-                              if stage_mode == "graph" else "eager launches") + ")"},
+                              if stage_mode == "graph" else "eager launches") + "); stage_us_cold: each "
+                              "stage alone, a graph of 10 x [L2 flush, stage] minus a graph of the flushes, "
+                              "per stage"},
             "roofline": roof,
             "warm_l2": {"value": round(value_warm, 2), "unit": unit, "ms_per_step": round(warm_ms_per_step, 5),
                         "steps": n_warm, "note": "back-to-back steps with no flush between them"},
             "stage_us": {k: round(v, 2) for k, v in stage_us.items()},
+            # each stage alone with its operands in HBM (flush-difference method,
+            # no event pair in the figure); the bandwidth figures use these when
+            # they exist, else the event-pair stage times (which read low)
+            "stage_us_cold": ({k: round(v, 2) for k, v in stage_cold.items()} if stage_cold else None),
             # side kernels are HBM-bound: algorithmic bytes / stage time, and its
-            # share of the measured copy bandwidth (stage times carry the event
-            # pair's few microseconds, so small stages read low)
-            "stage_gbs": {k: round(nbytes[k] / (v * 1e-6) / 1e9, 1) for k, v in stage_us.items() if v > 0},
+            # share of the measured copy bandwidth
+            "stage_gbs": {k: round(nbytes[k] / (v * 1e-6) / 1e9, 1) for k, v in (stage_cold or stage_us).items()
+                          if v > 0},
             "stage_hbm_frac": {k: round(nbytes[k] / (v * 1e-6) / 1e9 / float(peaks["hbm_gbs"]), 3)
-                               for k, v in stage_us.items() if v > 0 and (k != "w8a8_linear" or decode)},
+                               for k, v in (stage_cold or stage_us).items()
+                               if v > 0 and (k != "w8a8_linear" or decode)},
             "gpu_launches": plan.launches_per_step * args.steps,
             "launch": (("the step captured once into a CUDA graph and replayed (the C-ABI calls are "
                         "capture-safe); every libsq kernel uses programmatic dependent launch")
@@ -996,6 +1006,18 @@ def cold_warm(torch, calls, flush, iters, warm_reps, flush_graph=None):
             - time_graph(torch, flush_graph, nrep, flush, COLD_REPS))
     warm = time_graph(torch, graph_of(torch, calls, warm_reps), nrep, flush, warm_reps)
     return cold, warm
+
+
+def run_stage_cold(plan, torch, flush, iters):
+    """Each stage of the step alone, cold: a graph of COLD_REPS x [L2 flush, stage] minus a
+    graph of the flushes, per stage (the stages are idempotent on the step's own buffers:
+    ranges max-merged into themselves, the same factors, codes and output rewritten)."""
+    flush_graph = graph_of(torch, [], COLD_REPS, pre=flush)
+    out = {}
+    for name, fn, args in plan.calls:
+        call = (fn, lambda st, a=args: a[:-1] + (st,))
+        out[name] = cold_warm(torch, [call], flush, iters, 2, flush_graph)[0]
+    return out
 
 
 def run_forward(plan, sq, torch, flush, iters):
