@@ -34,7 +34,11 @@ def _case(B, M, N, K, seed, per_head=False):
 
 
 @pytest.mark.parametrize("B,M,N,K", [(1, 1, 16, 16), (3, 37, 40, 48), (3, 37, 36, 48), (4, 300, 272, 144),
-                                     (2, 256, 256, 256), (5, 129, 513, 1040), (32, 64, 64, 128)])
+                                     (2, 256, 256, 256), (5, 129, 513, 1040), (32, 64, 64, 128),
+                                     # 128-channel tiles (N <= 128) with two K boxes per stage:
+                                     # ragged N and M, a last stage whose second box lies past K,
+                                     # N % 8 != 0 (row stores), and N = 128 exactly
+                                     (3, 300, 72, 1040), (2, 200, 100, 528), (2, 130, 128, 640)])
 @pytest.mark.parametrize("per_head", [False, True])
 def test_bmm(sq, B, M, N, K, per_head):
     a, sa, b, sb = _case(B, M, N, K, B * 7 + M + N + K + per_head, per_head)
