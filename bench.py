@@ -1408,6 +1408,19 @@ def pick_sample(wl, M, budget_s, level="channel"):
     return c_s, n_s, m_s
 
 
+def host_cpu_model():
+    """The host CPU's model name from /proc/cpuinfo, or None where it cannot be read."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                key, sep, val = line.partition(":")
+                if sep and key.strip() == "model name":
+                    return val.strip()
+    except OSError:
+        pass
+    return None
+
+
 def oracle_baseline(wl, M, budget_s, level="channel"):
     import oracle
     c_s, n_s, m_s = pick_sample(wl, M, budget_s, level)
@@ -1426,7 +1439,7 @@ def oracle_baseline(wl, M, budget_s, level="channel"):
     finally:
         oracle.set_num_threads(cores)
     full1 = oracle_full_time(wl, M, st1, c1, n1, m1)
-    return {"value": round(v, 6), "unit": u, "cores": cores, "kind": "oracle",
+    return {"value": round(v, 6), "unit": u, "cores": cores, "kind": "oracle", "cpu_model": host_cpu_model(),
             "sample": (f"{c_s}/{wl.calib} calibration rows, {n_s}/{wl.N} weight rows, {m_s}/{M} tokens; " +
                        (f"the whole workload, timed directly ({sum(st.values()):.2f} s of CPU work)"
                         if (c_s, n_s, m_s) == (wl.calib, wl.N, M) else
@@ -1472,7 +1485,7 @@ def run_reference(args):
             "config": common_config(args, wl, M, world),
             "run": {"where": "CPU oracle on the host cores, rank 0 only"},
             "cpu_baseline": {"value": round(v, 6), "unit": u, "cores": oracle.num_threads(),
-                             "kind": "oracle", "sample": sample},
+                             "kind": "oracle", "cpu_model": host_cpu_model(), "sample": sample},
             "e2e": {"value": round(v, 6), "unit": u, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "cpu_seconds": round(work, 2)}
 
