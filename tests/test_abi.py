@@ -105,6 +105,77 @@ def test_other_entry_points_reject_bad_arguments():
     assert L.sq_w8a8_gemm_s32(FAKE, FAKE, None, 8, 8, 64, None, 0, 0, None) == 1
 
 
+def test_remaining_entry_points_reject_bad_arguments_on_the_host():
+    """Every other entry point: null or non-positive arguments (1), misaligned
+    pointers or leading dimensions (2), K or N outside the shape rules (3), K
+    past SQ_MAX_K (4), a shape beyond the fixed scratch (5) -- each returned
+    before any device is touched."""
+    L = _lib()
+    big = 1 << 30
+    # the range reset
+    assert L.sq_calibrate_reset(None, 16, None) == 1
+    assert L.sq_calibrate_reset(FAKE, 0, None) == 1
+    assert L.sq_calibrate_reset(FAKE_ODD, 16, None) == 2
+    # per-tensor weight scale (O1-O3): the range output is required
+    f = L.sq_quantize_weight_tensor
+    assert f(FAKE, 8, 64, None, FAKE, FAKE, None, None) == 1
+    assert f(FAKE, 8, 24, None, FAKE, FAKE, FAKE, None) == 3
+    assert f(FAKE, 8, 133152, None, FAKE, FAKE, FAKE, None) == 4
+    assert f(FAKE, 8, 64, None, FAKE, FAKE, FAKE_ODD, None) == 2
+    assert f(FAKE, 8, 64, FAKE_ODD, FAKE, FAKE, FAKE, None) == 2
+    # per-tensor dynamic (O2) and static (O3) activation scales
+    for g in (L.sq_ln_quant_act_tensor, L.sq_ln_quant_act_static):
+        assert g(FAKE, 8, 64, 64, None, None, None, 1e-5, FAKE, FAKE, None, None) == 1   # no range
+        assert g(FAKE, 0, 64, 64, None, None, None, 1e-5, FAKE, FAKE, FAKE, None) == 1   # M = 0
+        assert g(FAKE, 8, 64, 64, None, FAKE, None, 1e-5, FAKE, FAKE, FAKE, None) == 1   # beta w/o gamma
+        assert g(FAKE, 8, 64, 56, None, None, None, 1e-5, FAKE, FAKE, FAKE, None) == 1   # ld < K
+        assert g(FAKE, 8, 64, 68, None, None, None, 1e-5, FAKE, FAKE, FAKE, None) == 2   # ld % 8
+        assert g(FAKE, 8, 64, 64, None, None, None, 1e-5, FAKE, FAKE, FAKE_ODD, None) == 2
+        assert g(FAKE, 8, 40, 40, None, None, None, 1e-5, FAKE, FAKE, FAKE, None) == 3
+    # the tensor range from calibrated column maxima (any K up to SQ_MAX_K)
+    assert L.sq_tensor_range(None, None, 64, FAKE, None) == 1
+    assert L.sq_tensor_range(FAKE, None, 0, FAKE, None) == 1
+    assert L.sq_tensor_range(FAKE, None, 133152, FAKE, None) == 4
+    assert L.sq_tensor_range(FAKE, FAKE_ODD, 64, FAKE, None) == 2
+    # per-row ranges and quantization against them: the weight fold (s_fold)
+    # excludes the activation transform (LayerNorm, 1/s)
+    f = L.sq_row_ranges
+    assert f(FAKE, 8, 64, 64, FAKE, None, None, FAKE, 1e-5, FAKE, None) == 1
+    assert f(FAKE, 8, 64, 64, None, None, FAKE, FAKE, 1e-5, FAKE, None) == 1
+    assert f(FAKE, 8, 64, 64, None, None, None, None, 1e-5, None, None) == 1
+    assert f(FAKE, 8, 64, 64, None, None, None, None, 1e-5, FAKE_ODD, None) == 2
+    assert f(FAKE, 8, 40, 40, None, None, None, None, 1e-5, FAKE, None) == 3
+    f = L.sq_quantize_rows_ranged
+    assert f(FAKE, 8, 64, 64, None, None, None, None, 1e-5, None, FAKE, FAKE, None) == 1
+    assert f(FAKE, 8, 64, 64, None, None, None, None, 1e-5, FAKE, FAKE_ODD, FAKE, None) == 2
+    # the row-parallel layer's dequantization: N % 4 == 0
+    assert L.sq_dequant(None, FAKE, FAKE, None, FAKE, 8, 8, None) == 1
+    assert L.sq_dequant(FAKE, FAKE, FAKE, None, FAKE, 0, 8, None) == 1
+    assert L.sq_dequant(FAKE, FAKE, FAKE, None, FAKE, 8, 6, None) == 3
+    assert L.sq_dequant(FAKE, FAKE, FAKE, FAKE_ODD, FAKE, 8, 8, None) == 2
+    # the static producer-side quantization: N is the next linear's K
+    f = L.sq_w8a8_linear_quant
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 0, None, None, FAKE, FAKE, 64, 64, 64, FAKE, big, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 0, None, FAKE, FAKE, FAKE, 64, 40, 64, FAKE, big, None) == 3
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 0, None, FAKE, FAKE, FAKE, 64, 64, 40, FAKE, big, None) == 3
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 0, None, FAKE, FAKE_ODD, FAKE, 64, 64, 64, FAKE, big, None) == 2
+    # the INT8 BMM
+    f = L.sq_w8a8_bmm
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 64, 64, 64, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 2, 64, 64, 64, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 64, 64, 40, None) == 3
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 64, 64, 133152, None) == 4
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE_ODD, 2, 64, 64, 64, None) == 2
+    # the allocation-free decode entry: M <= 32, at most 4096 tiles of 128 channels
+    f = L.sq_w8a8_linear_noalloc
+    assert f(None, FAKE, FAKE, FAKE, None, FAKE, 8, 64, 64, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, None, FAKE, 33, 64, 64, None) == 3
+    assert f(FAKE, FAKE, FAKE, FAKE, None, FAKE, 8, 64, 40, None) == 3
+    assert f(FAKE, FAKE, FAKE, FAKE, None, FAKE, 8, 64, 133152, None) == 4
+    assert f(FAKE, FAKE, FAKE, FAKE, None, FAKE, 8, 128 * 4096 + 1, 64, None) == 5
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE_ODD, FAKE, 8, 64, 64, None) == 2
+
+
 def test_workspace_size_formula():
     L = _lib()
     assert L.sq_w8a8_workspace_bytes(129, 4096, 4096) == 0      # beyond stream-K: none
